@@ -1,0 +1,220 @@
+"""ctypes front end of the fp64 CPU oracle (oracle/ecasq_oracle.cpp).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by __graft_entry__.smoke() and by
+bench.py's cpu_baseline / reference leg. The product package never imports it.
+
+Every function takes and returns numpy arrays. Definitions follow the ECASQ
+technical summary (gist.science/pt/paper/2608.18147), §1 (problem), §2.1
+(Lagrangian relaxation, time-sharing) and §2.2 (the pair-state DP over a
+permissible set P); the C++ source states each one.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        from . import build as _build  # type: ignore
+
+        path = _build.build()
+        L = C.CDLL(path)
+        f32p = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
+        f64p = np.ctypeslib.ndpointer(np.float64, flags="C_CONTIGUOUS")
+        i64p = np.ctypeslib.ndpointer(np.int64, flags="C_CONTIGUOUS")
+        i32p = np.ctypeslib.ndpointer(np.int32, flags="C_CONTIGUOUS")
+        u8p = np.ctypeslib.ndpointer(np.uint8, flags="C_CONTIGUOUS")
+        u32p = np.ctypeslib.ndpointer(np.uint32, flags="C_CONTIGUOUS")
+        u64p = np.ctypeslib.ndpointer(np.uint64, flags="C_CONTIGUOUS")
+        I, I64, D, U64 = C.c_int, C.c_int64, C.c_double, C.c_uint64
+        sig = {
+            "eo_uniform_grid": (I, [f32p, I64, I, f64p]),
+            "eo_bucket": (I, [f32p, I64, f64p, I, i64p, f64p, f64p]),
+            "eo_tables": (None, [i64p, f64p, f64p, f64p, I, f64p, f64p, f64p]),
+            "eo_eval_tables": (None, [f64p, f64p, f64p, I, I64, i32p, I, C.POINTER(D), C.POINTER(D), C.c_void_p]),
+            "eo_eval_raw": (I, [f32p, I64, f64p, I, C.POINTER(D), C.POINTER(D), C.c_void_p]),
+            "eo_dp": (I, [f64p, f64p, f64p, I, I, I64, D, i32p, C.POINTER(C.c_int32), C.POINTER(D)]),
+            "eo_philox4x32_10": (None, [u32p, u32p, u32p]),
+            "eo_philox4x64_10": (None, [u64p, u64p, u64p]),
+            "eo_entropy": (D, [i64p, I]),
+            "eo_threads": (I, []),
+            "eo_solve_batch": (I, [f32p, I, I64, f64p, I, I, f64p, I, i32p, i32p, f64p, f64p, f64p, i32p]),
+            "eo_solve_budget_batch": (I, [f32p, I, I64, f64p, I, I, D, I, i32p, i32p, i32p, i32p,
+                                          f64p, f64p, f64p, f64p, f64p, f64p, f64p, i32p]),
+            "eo_encode_batch": (I, [f32p, I, I64, f64p, I, i32p, i32p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                    I, U64, u8p, i64p, i32p]),
+            "eo_grid_batch": (I, [f32p, I, I64, I, f64p, i32p]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _f32(x):
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def _f64(x):
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def threads() -> int:
+    return int(lib().eo_threads())
+
+
+# -- single-vector building blocks -------------------------------------------
+
+def uniform_grid(x, p):
+    x = _f32(x).ravel()
+    P = np.empty(p, np.float64)
+    st = lib().eo_uniform_grid(x, x.size, p, P)
+    return P, st
+
+
+def bucket(x, P):
+    x = _f32(x).ravel()
+    P = _f64(P)
+    p = P.size
+    cnt = np.zeros(p - 1, np.int64)
+    A = np.zeros(p - 1, np.float64)
+    B = np.zeros(p - 1, np.float64)
+    st = lib().eo_bucket(x, x.size, P, p, cnt, A, B)
+    return cnt, A, B, st
+
+
+def tables(cnt, A, B, P):
+    P = _f64(P)
+    p = P.size
+    V = np.zeros((p, p))
+    R = np.zeros((p, p))
+    L = np.zeros((p, p))
+    lib().eo_tables(np.ascontiguousarray(cnt, np.int64), _f64(A), _f64(B), P, p, V, R, L)
+    return V, R, L
+
+
+def eval_tables(V, R, L, d, Q):
+    Q = np.ascontiguousarray(Q, np.int32)
+    p = V.shape[0]
+    mse, H = C.c_double(), C.c_double()
+    mu = np.zeros(max(Q.size, 1))
+    lib().eo_eval_tables(_f64(V), _f64(R), _f64(L), p, d, Q, Q.size, C.byref(mse), C.byref(H),
+                         mu.ctypes.data_as(C.c_void_p))
+    return mse.value, H.value, mu[: Q.size]
+
+
+def eval_raw(x, qvals):
+    x = _f32(x).ravel()
+    q = _f64(qvals)
+    mse, H = C.c_double(), C.c_double()
+    mu = np.zeros(max(q.size, 1))
+    st = lib().eo_eval_raw(x, x.size, q, q.size, C.byref(mse), C.byref(H), mu.ctypes.data_as(C.c_void_p))
+    if st:
+        raise ValueError("entry outside the code range")
+    return mse.value, H.value, mu[: q.size]
+
+
+def dp(V, R, L, s, d, lam):
+    p = V.shape[0]
+    Q = np.full(min(s, p), -1, np.int32)
+    m = C.c_int32()
+    J = C.c_double()
+    st = lib().eo_dp(_f64(V), _f64(R), _f64(L), p, s, d, lam, Q, C.byref(m), C.byref(J))
+    if st:
+        raise ValueError("oracle dp failed")
+    return Q[: m.value].copy(), J.value
+
+
+def philox4x32(ctr, key):
+    out = np.zeros(4, np.uint32)
+    lib().eo_philox4x32_10(np.asarray(ctr, np.uint32), np.asarray(key, np.uint32), out)
+    return out
+
+
+def philox4x64(ctr, key):
+    out = np.zeros(4, np.uint64)
+    lib().eo_philox4x64_10(np.asarray(ctr, np.uint64), np.asarray(key, np.uint64), out)
+    return out
+
+
+def entropy(hist, s):
+    return float(lib().eo_entropy(np.ascontiguousarray(hist, np.int64).ravel(), s))
+
+
+# -- batched drivers (OpenMP over vectors) -------------------------------------
+
+def grid_batch(X, p):
+    X = _f32(X)
+    n, d = X.shape
+    P = np.zeros((n, p))
+    st = np.zeros(n, np.int32)
+    lib().eo_grid_batch(X, n, d, p, P, st)
+    return P, st
+
+
+def solve_batch(X, P, s, lam):
+    """lam: [n] or [n, L]. Returns dict of [n, L] arrays (Q is [n, L, s], -1 padded)."""
+    X = _f32(X)
+    n, d = X.shape
+    P = _f64(P)
+    p = P.shape[1]
+    lam = _f64(lam).reshape(n, -1)
+    nl = lam.shape[1]
+    Q = np.full((n, nl, s), -1, np.int32)
+    m = np.zeros((n, nl), np.int32)
+    J = np.zeros((n, nl))
+    mse = np.zeros((n, nl))
+    H = np.zeros((n, nl))
+    st = np.zeros((n, nl), np.int32)
+    thr = lib().eo_solve_batch(X, n, d, P, p, s, lam, nl, Q, m, J, mse, H, st)
+    return dict(Q=Q, m=m, J=J, mse=mse, H=H, status=st, threads=thr)
+
+
+def solve_budget_batch(X, P, s, b, steps=30):
+    X = _f32(X)
+    n, d = X.shape
+    P = _f64(P)
+    p = P.shape[1]
+    out = dict(Q1=np.full((n, s), -1, np.int32), m1=np.zeros(n, np.int32),
+               Q2=np.full((n, s), -1, np.int32), m2=np.zeros(n, np.int32))
+    for k in ("theta", "lam_lo", "lam_hi", "H1", "H2", "mse1", "mse2"):
+        out[k] = np.zeros(n)
+    out["status"] = np.zeros(n, np.int32)
+    thr = lib().eo_solve_budget_batch(X, n, d, P, p, s, float(b), steps, out["Q1"], out["m1"], out["Q2"],
+                                      out["m2"], out["theta"], out["lam_lo"], out["lam_hi"], out["H1"],
+                                      out["H2"], out["mse1"], out["mse2"], out["status"])
+    out["threads"] = thr
+    return out
+
+
+def encode_batch(X, P, Q1, m1, s, seed, Q2=None, m2=None, theta=None):
+    X = _f32(X)
+    n, d = X.shape
+    P = _f64(P)
+    p = P.shape[1]
+    Q1 = np.ascontiguousarray(Q1, np.int32).reshape(n, s)
+    m1 = np.ascontiguousarray(m1, np.int32).reshape(n)
+    idx = np.zeros((n, d), np.uint8)
+    hist = np.zeros((n, 2, s), np.int64)
+    st = np.zeros(n, np.int32)
+    keep = []
+    if Q2 is not None:
+        Q2 = np.ascontiguousarray(Q2, np.int32).reshape(n, s)
+        m2 = np.ascontiguousarray(m2, np.int32).reshape(n)
+        th = _f64(theta).reshape(n)
+        keep = [Q2, m2, th]
+        q2p, m2p, thp = (a.ctypes.data_as(C.c_void_p) for a in keep)
+    else:
+        q2p = m2p = thp = None
+    lib().eo_encode_batch(X, n, d, P, p, Q1, m1, q2p, m2p, thp, s, C.c_uint64(seed), idx, hist, st)
+    del keep
+    return idx, hist, st
