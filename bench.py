@@ -1,0 +1,352 @@
+"""Benchmark of the ECASQ solver hot path on B200.
+
+One step = the whole path on one batch of synthetic vectors already in HBM:
+uniform grid -> bucketing -> DP solves (lambda bisection + time-sharing, or
+fixed lambdas) -> stochastic-rounding encode -> empirical entropy.
+
+Default workload: 4096 x 4096 weight-like rows (0.02 * Student-t, nu = 4),
+p = 128, s = 16, budget b = 3.0 bits/entry, 30 bisection steps.
+
+Metric: DP (k, l, j) triples per second over the whole step (triples counted
+by formula, one solve = every triple the recurrence visits), with entries/s
+and per-kernel roofline fractions alongside. The oracle (fp64 CPU) is timed
+on a bounded sample of the same workload as the CPU baseline.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--fp64]
+  python bench.py --impl reference ...   # the CPU oracle as the reference arm
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from entropy_constrained_unbiased_b200 import workloads as W  # noqa: E402
+
+MUFU_LG2_PER_CLK_PER_SM = 16  # special-function unit results per clock per SM (sm_100)
+B200_SMS = 148
+
+
+def triples_per_solve(p: int, s: int) -> int:
+    """(k, l, j) triples one exact solve evaluates: layer 2 has only k = 0
+    (c_1 = P_0), layers 3 .. S-2 every k < l < j with k >= i-2, and the last
+    layer S-1 only j = p-1."""
+    S = min(s, p)
+    t = 0
+    for i in range(2, S):
+        last = i == S - 1
+        for l in range(i - 1, p - 1):
+            K = 1 if i == 2 else l - i + 2
+            NJ = 1 if last else p - 1 - l
+            t += K * NJ
+    return t
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except OSError:
+        return {}
+
+
+def describe(w: W.Workload) -> str:
+    what = {"budget": f"budget b={w.b} bits/entry, {w.steps}-step lambda bisection + two-way time-sharing",
+            "sweep": f"{w.n_lambda} log-spaced lambdas in [1e-4, 1]",
+            "solve": f"fixed lambda={w.lam}"}[w.mode]
+    return f"{w.name}: {w.n}x{w.d} fp32 ({w.dist}), uniform P p={w.p}, s={w.s}, {what}"
+
+
+def solves_done(w: W.Workload, out) -> int:
+    """DP solves actually executed, read from the solver's outputs."""
+    if w.mode != "budget":
+        return w.n * (w.n_lambda if w.mode == "sweep" else 1)
+    st = out["status"].cpu().numpy()
+    lam_hi = out["lambda_hi"].cpu().numpy()
+    total = 0
+    for r in range(w.n):
+        if st[r] == 1:
+            total += 2
+        elif lam_hi[r] == 0.0:
+            total += 1
+        elif st[r] == 0:
+            total += 2 + w.steps
+    return total
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([c.strip() for c in line.split(",")])
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if len(r) > 5 + i and "Active" in r[5 + i]
+                          and "Not" not in r[5 + i]})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# ---------------------------------------------------------------------------------
+
+def run_ours(args, w: W.Workload, rank: int, world: int):
+    import torch
+    from entropy_constrained_unbiased_b200 import ecasq as E
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    E.load()
+    fp64 = args.fp64
+    X_host = W.make_inputs(w)
+    X = torch.from_numpy(X_host).to(dev)
+    n, d, p, s = w.n, w.d, w.p, w.s
+    lam = torch.from_numpy(w.lambdas()).to(dev) if w.mode != "budget" else None
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    def step(X):
+        P, st = E.uniform_grid(X, p)
+        cnt, A, B, st = E.bucket(X, P)
+        ev_dp0.record(stream)
+        if w.mode == "budget":
+            out = E.solve_budget_stats(cnt, A, B, P, d, s, w.b, w.steps, fp64=fp64)
+            ev_dp1.record(stream)
+            idx, hist, est = E.encode(X, P, s, out["Q1"], out["Q1_len"], w.seed_encode, out["Q2"], out["Q2_len"],
+                                      out["theta"])
+        else:
+            out = E.solve_stats(cnt, A, B, P, d, s, lam, fp64=fp64)
+            ev_dp1.record(stream)
+            Q = out["Q"][:, 0, :].contiguous()
+            idx, hist, est = E.encode(X, P, s, Q, out["Q_len"][:, 0].contiguous(), w.seed_encode)
+        Hemp = E.entropy(hist)
+        return out, idx, hist, Hemp
+
+    ev_dp0 = torch.cuda.Event(enable_timing=True)
+    ev_dp1 = torch.cuda.Event(enable_timing=True)
+    for _ in range(args.warmup):
+        out, idx, hist, Hemp = step(X)
+    torch.cuda.synchronize()
+    n_solves = solves_done(w, out)
+    tps = triples_per_solve(p, s)
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    dp_ms = []
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    E.launch_count(reset=True)
+    with Clocks(dev.index) as clk:
+        for k in range(args.steps):
+            flush.fill_(k & 0xFF)  # evict X and the tables from L2 between steps
+            starts[k].record(stream)
+            out, idx, hist, Hemp = step(X)
+            ends[k].record(stream)
+            torch.cuda.synchronize()
+            dp_ms.append(ev_dp0.elapsed_time(ev_dp1))
+    launches = E.launch_count(reset=True)
+    step_ms = [starts[k].elapsed_time(ends[k]) for k in range(args.steps)]
+    t_ms = float(sum(step_ms))
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([t_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_ms = float(t.item())
+        dist.barrier()
+
+    # e2e: same step through the C ABI with host buffers, copies inside the timed region
+    Xpin = torch.from_numpy(X_host).pin_memory()
+    e2e_ms = []
+    for k in range(max(1, min(args.steps, 3))):
+        flush.fill_(k & 0xFF)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        Xd = Xpin.to(dev, non_blocking=True)
+        o2, idx2, hist2, H2 = step(Xd)
+        res = [idx2.to("cpu", non_blocking=True), H2.to("cpu", non_blocking=True)]
+        if w.mode == "budget":
+            res += [o2[k2].to("cpu", non_blocking=True) for k2 in ("Q1", "Q2", "theta")]
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms.append(e0.elapsed_time(e1))
+    bo = n * d + n * 8 + (n * s * 4 * 2 + n * 8 if w.mode == "budget" else 0)
+
+    peaks = measured_peaks()
+    sm_max = float(peaks.get("sm_max_mhz", 1965.0))
+    mufu_peak = MUFU_LG2_PER_CLK_PER_SM * B200_SMS * sm_max * 1e6
+    dp_avg_ms = float(np.mean(dp_ms))
+    achieved = n_solves * tps / (dp_avg_ms * 1e-3)
+    total_triples = world * n_solves * tps
+    value = total_triples / (t_ms * 1e-3)
+    line = {
+        "metric": "ECASQ DP (k,l,j) triples/s (whole step: grid + bucketing + DP + bisection + encode + entropy)",
+        "value": value,
+        "unit": "triples/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": t_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64" if fp64 else "f32",
+        "data": "synthetic",
+        "config": {"workload": describe(w), "n": n, "d": d, "p": p, "s": s, "l2": "flushed between steps",
+                   "dp_solves_per_step": n_solves, "triples_per_solve": tps,
+                   "entries_per_s": world * n * d / (t_ms * 1e-3 / args.steps),
+                   "parallelism": f"dp{world} (rows sharded, no collective)"},
+        "roofline": {"bound": "alu", "kernel": "k_dp (DP layers + backtrack + bisection)", "achieved": achieved,
+                     "peak": mufu_peak, "unit": "triples/s", "frac": achieved / mufu_peak, "traffic": None,
+                     "peak_basis": f"MUFU lg2 {MUFU_LG2_PER_CLK_PER_SM}/clk/SM x {B200_SMS} SMs x {sm_max:.0f} MHz"},
+        "e2e": {"value": total_triples / (float(np.mean(e2e_ms)) * 1e-3), "unit": "triples/s",
+                "h2d_bytes_per_step": n * d * 4, "d2h_bytes_per_step": bo},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    return line
+
+
+def oracle_sample(w: W.Workload, budget_s: float):
+    """Time the fp64 oracle on a deterministic row sample of the workload."""
+    from oracle import oracle as O
+
+    rows = 1
+    X = W.make_inputs(w, rows=64 if w.n >= 64 else w.n)
+    stride = max(1, X.shape[0] // 64)
+    threads = O.threads()
+    tps = triples_per_solve(w.p, w.s)
+    done_rows, solves, t_tot = 0, 0, 0.0
+    while done_rows < X.shape[0] and t_tot < budget_s:
+        take = min(max(rows, threads), X.shape[0] - done_rows)
+        Xs = np.ascontiguousarray(X[done_rows:done_rows + take])
+        P, _ = O.grid_batch(Xs, w.p)
+        t0 = time.perf_counter()
+        if w.mode == "budget":
+            r = O.solve_budget_batch(Xs, P, w.s, w.b, w.steps)
+            st = r["status"]
+            lam_hi = r["lam_hi"]
+            solves += int(sum(2 if st[i] == 1 else (1 if lam_hi[i] == 0 else 2 + w.steps) for i in range(take)))
+        else:
+            lam = w.lambdas()[:take]
+            O.solve_batch(Xs, P, w.s, lam)
+            solves += take * lam.shape[1]
+        t_tot += time.perf_counter() - t0
+        done_rows += take
+    return {"value": solves * tps / t_tot, "unit": "triples/s", "cores": threads, "kind": "oracle",
+            "sample": f"first {done_rows} rows of {w.n} ({solves} fp64 DP solves, {t_tot:.1f} s)"}
+
+
+def run_reference(args, w: W.Workload, rank: int, world: int):
+    from oracle import oracle as O
+
+    if rank != 0:
+        return None
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(w, per_step / 4)
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(oracle_sample(w, per_step))
+    wall = time.perf_counter() - t0
+    v = float(np.mean([x["value"] for x in vals]))
+    cb = dict(vals[-1])
+    cb["value"] = v
+    return {"impl": "reference", "metric": "ECASQ DP (k,l,j) triples/s (fp64 CPU oracle, row sample)",
+            "value": v, "unit": "triples/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": wall * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": describe(w), "n": w.n, "d": w.d, "p": w.p, "s": w.s},
+            "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": "triples/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="weights", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--fp64", action="store_true", help="fp64 DP layers (parity mode)")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = W.WORKLOADS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if args.impl == "reference":
+        line = run_reference(args, w, rank, world)
+    else:
+        # the oracle's thread pool starts before the first CUDA call
+        cpu = None
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            cpu = oracle_sample(w, args.cpu_seconds)
+        line = run_ours(args, w, rank, world)
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+    if rank == 0 and line is not None:
+        print(json.dumps(line))
+    if world > 1 and args.impl == "ours":
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

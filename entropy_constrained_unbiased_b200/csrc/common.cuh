@@ -1,0 +1,95 @@
+// Device-side helpers shared by the ECASQ kernels (sm_100a).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace ecasq {
+
+constexpr int kWarp = 32;
+constexpr int kMaxP = 512;    // largest alphabet the kernels accept
+constexpr int kMaxS = 255;    // largest code size
+
+// Per-vector status codes written by the device (mirrors include/ecasq.h).
+constexpr int32_t kStatusOk = 0;
+constexpr int32_t kStatusArg = -1;
+constexpr int32_t kStatusRange = -2;
+constexpr int32_t kStatusBudget = 1;
+
+__device__ __forceinline__ int lane_id() { return threadIdx.x & (kWarp - 1); }
+__device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
+
+// log2 on the special-function unit (MUFU.LG2, flush-to-zero; |rel err| ~ 2^-22).
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy
+// as 1, 2, 3", SC'11). Each round maps the counter (c0,c1,c2,c3) with key
+// (k0,k1) through two 32x32->64 multiplications:
+//   (c0,c1,c2,c3) <- (hi(m1*c2) ^ c1 ^ k0, lo(m1*c2), hi(m0*c0) ^ c3 ^ k1, lo(m0*c0))
+// and the key advances by the two Weyl increments between rounds.
+struct Philox4x32 {
+  static constexpr uint32_t kMulA = 0xD2511F53u;  // multiplier applied to c0
+  static constexpr uint32_t kMulB = 0xCD9E8D57u;  // multiplier applied to c2
+  static constexpr uint32_t kWeylA = 0x9E3779B9u; // golden-ratio increment of k0
+  static constexpr uint32_t kWeylB = 0xBB67AE85u; // sqrt(3)-1 increment of k1
+
+  __device__ __forceinline__ static uint4 block(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+      const uint32_t lo0 = kMulA * c.x;
+      const uint32_t hi0 = __umulhi(kMulA, c.x);
+      const uint32_t lo1 = kMulB * c.z;
+      const uint32_t hi1 = __umulhi(kMulB, c.z);
+      c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+      k0 += kWeylA;
+      k1 += kWeylB;
+    }
+    return c;
+  }
+};
+
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Warp-wide argmin: smallest value, ties to the smallest index. All lanes get it.
+template <typename T>
+__device__ __forceinline__ void warp_argmin(T& v, int& i) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const T ov = __shfl_xor_sync(0xffffffffu, v, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, i, o);
+    if (ov < v || (ov == v && oi < i)) {
+      v = ov;
+      i = oi;
+    }
+  }
+}
+
+// Triangle addressing of the pair tables (0 <= k < l < p):
+//   column l holds the entries (k, l), k = 0 .. l-1, at col_off(l) + k;
+//   row l holds the entries (l, j), j = l+1 .. p-1, at row_off(l, p) + (j - l - 1).
+__host__ __device__ __forceinline__ int col_off(int l) { return (l * (l - 1)) >> 1; }
+__host__ __device__ __forceinline__ int row_off(int l, int p) { return l * (p - 1) - ((l * (l - 1)) >> 1); }
+__host__ __device__ __forceinline__ int tri_size(int p) { return (p * (p - 1)) >> 1; }
+
+// Bucket of x on an increasing alphabet P (in shared memory): the largest
+// k <= p-2 with P_k <= x. Starts from the uniform-grid guess and walks; -1 when
+// x is outside [P_0, P_{p-1}] or NaN.
+__device__ __forceinline__ int bucket_of(double x, const double* __restrict__ P, int p, double scale) {
+  if (!(x >= P[0]) || !(x <= P[p - 1])) return -1;
+  int k = static_cast<int>((x - P[0]) * scale);
+  k = k < 0 ? 0 : (k > p - 2 ? p - 2 : k);
+  while (k > 0 && P[k] > x) --k;
+  while (k < p - 2 && P[k + 1] <= x) ++k;
+  return k;
+}
+
+}  // namespace ecasq

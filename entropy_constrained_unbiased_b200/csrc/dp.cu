@@ -1,0 +1,700 @@
+// The exact ECASQ dynamic programme on B200.
+//
+// ECASQ summary (gist.science/pt/paper/2608.18147):
+//   §2.1 "Relaxação Lagrangiana": minimise MSE(Q,X) + lambda * H(X^).
+//   §2.2 "Programação Dinâmica Ótima": the ASQ DP does not extend because the
+//        entropy term of a value depends on both neighbours, so the state is a
+//        PAIR of consecutive values, dp_OPT(i, l, j); the direct programme costs
+//        O(d^3 s) time over the entries, O(p^3 s) over a permissible set P.
+//
+// Recurrence evaluated here (i = number of values up to and including P_l,
+// counting c_1 = P_0; m = mu/d the normalised mass of a value):
+//   F_1(0, j) = V(0,j)/(lambda d) + h(L(0,j)/d)
+//   F_i(l, j) = V(l,j)/(lambda d) + min_{k} [ F_{i-1}(k,l) + h((R(k,l) + L(l,j))/d) ]
+//   J*/lambda = min_{i,k} F_i(k, p-1) + h(R(k,p-1)/d),   h(m) = -m log2 m.
+// The whole programme is scaled by 1/lambda, so one (k,l,j) triple is one add,
+// one MUFU log2 and one FMA plus the running argmin. lambda = 0 is the
+// separable MSE-only programme (the minimum over k no longer depends on j).
+//
+// Design (this file):
+//   * one CTA per vector, persistent over every solve of that vector (all
+//     lambdas, or the whole bisection), so the pair tables are built once;
+//   * the tables and the two live DP layers sit in shared memory when they fit
+//     (fp32, p <= 128) and in a per-CTA global (L2-resident) slab otherwise;
+//   * one DP layer is a list of tasks (row l, a block of <= 64 j, a k-split of
+//     1..32 lanes) in descending cost order, taken by warps from a shared
+//     counter; each lane keeps 2 j in registers and sweeps k with broadcast
+//     loads; k-splits merge with a warp-shuffle argmin;
+//   * back-pointers go to a per-CTA global slab; the backtrack, the fp64
+//     evaluation of the chosen code and the bisection run in the same kernel.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace ecasq {
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / kWarp;
+constexpr int kTJ = 2;                  // j values held per lane
+constexpr int kTaskJ = kWarp * kTJ;     // j values per full task
+
+__host__ __device__ inline uint32_t pack_task(int l, int j0, int nj, int kslog) {
+  return static_cast<uint32_t>(l) | (static_cast<uint32_t>(j0) << 10) | (static_cast<uint32_t>(nj) << 20) |
+         (static_cast<uint32_t>(kslog) << 28);
+}
+
+template <typename T>
+struct Arith;
+
+template <>
+struct Arith<float> {
+  // Added to every R/d so that a mass is never 0 inside the sweep:
+  // h(2^-100) ~ 8e-29, far below fp32 resolution of any objective.
+  static constexpr float kEps = 0x1p-100f;
+  __device__ static float inf() { return __int_as_float(0x7f800000); }
+  __device__ static float nlog(float m) { return -m * lg2_approx(m); }
+  __device__ static float fold(float g, float m) { return fmaf(-m, lg2_approx(m), g); }
+};
+
+template <>
+struct Arith<double> {
+  static constexpr double kEps = 0.0;
+  __device__ static double inf() { return __longlong_as_double(0x7ff0000000000000ll); }
+  __device__ static double nlog(double m) { return m > 0.0 ? -m * log2(m) : 0.0; }
+  __device__ static double fold(double g, double m) { return m > 0.0 ? fma(-m, log2(m), g) : g; }
+};
+
+template <typename T>
+struct Ctx {
+  int p, S, tri;
+  double dd;
+  T* colG0;  // DP layers (even / odd i), column layout (entry (k,l) at col_off(l)+k)
+  T* colG1;
+  __device__ __forceinline__ T* layer(int i) const { return (i & 1) ? colG1 : colG0; }
+  T* colA;     // R(k,l)/d + eps, column layout
+  T* rowB;     // L(l,j)/d, row layout
+  T* rowV;     // V(l,j)/d, row layout
+  uint16_t* bp;  // [S][tri] back-pointers, row layout
+  double *sP, *sN, *sA, *sB;  // [p] alphabet and bucket statistics
+  double *sR, *sL;            // [S] evaluation scratch
+  T* rmin;                    // [p] row minima (lambda = 0)
+  int* rarg;                  // [p]
+  int* ctr;                   // [S] task counters
+  int* sQ;                    // [S] code of the last solve
+  const uint32_t* tasks;
+  const int32_t* ntasks;
+  int max_tasks;
+};
+
+struct SolveOut {
+  double mse, H, J;
+  int m;
+  int bestI, bestK;
+};
+
+// ---- table build -------------------------------------------------------------
+// For every pair a < c, sums over the buckets a .. c-1 (ascending), with
+// delta_k = P_k - P_a:  N = sum n_k, T1 = sum (A_k + n_k delta_k),
+// T2 = sum (B_k + 2 delta_k A_k + n_k delta_k^2); W = P_c - P_a;
+// V = W T1 - T2 (>= 0), R = T1 / W, L = N - R. One thread per a, running in c.
+template <typename T>
+__device__ __forceinline__ void build_tables(const Ctx<T>& c) {
+  const int p = c.p;
+  for (int a = threadIdx.x; a < p - 1; a += blockDim.x) {
+    double N = 0.0, T1 = 0.0, T2 = 0.0;
+    const double Pa = c.sP[a];
+    const int ro = row_off(a, p) - a - 1;
+    for (int cc = a + 1; cc < p; ++cc) {
+      const int k = cc - 1;
+      const double dk = c.sP[k] - Pa;
+      const double nk = c.sN[k];
+      N += nk;
+      T1 += c.sA[k] + nk * dk;
+      T2 += c.sB[k] + 2.0 * dk * c.sA[k] + nk * dk * dk;
+      const double W = c.sP[cc] - Pa;
+      double V = W * T1 - T2;
+      V = V > 0.0 ? V : 0.0;
+      const double R = T1 / W;
+      double L = N - R;
+      L = L > 0.0 ? L : 0.0;
+      c.colA[col_off(cc) + a] = static_cast<T>(R / c.dd) + Arith<T>::kEps;
+      c.rowB[ro + cc] = static_cast<T>(L / c.dd);
+      c.rowV[ro + cc] = static_cast<T>(V / c.dd);
+    }
+  }
+}
+
+// ---- one layer ---------------------------------------------------------------
+
+// Best (E, i, k) over the finished layer i: E = F_i(k, p-1) + h(R(k,p-1)/d).
+// Warp 0 only. Strict '<' over layers in ascending order keeps the smaller code.
+template <typename T>
+__device__ __forceinline__ void finalize_layer(const Ctx<T>& c, int i, const T* G, bool sep, T* bestE, int* bestI,
+                               int* bestK) {
+  const int p = c.p;
+  const int kb = (i == 1) ? 0 : i - 1;
+  const int ke = (i == 1) ? 0 : p - 2;
+  T best = Arith<T>::inf();
+  int arg = 0x7fffffff;
+  const int co = col_off(p - 1);
+  for (int k = kb + lane_id(); k <= ke; k += kWarp) {
+    T e = G[co + k];
+    if (!sep) e += Arith<T>::nlog(c.colA[co + k]);
+    if (e < best) {
+      best = e;
+      arg = k;
+    }
+  }
+  warp_argmin(best, arg);
+  if (lane_id() == 0 && best < *bestE) {
+    *bestE = best;
+    *bestI = i;
+    *bestK = arg;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void run_task(const Ctx<T>& c, uint32_t desc, int i, const T* __restrict__ Gp,
+                                         T* __restrict__ Gc, uint16_t* __restrict__ bpi, T invl) {
+  const int p = c.p;
+  const int l = desc & 1023;
+  const int j0 = (desc >> 10) & 1023;
+  const int nj = (desc >> 20) & 255;
+  const int kslog = (desc >> 28) & 7;
+  const int KS = 1 << kslog;
+  const int JL = kWarp >> kslog;
+  const int lane = lane_id();
+  const int ks = lane & (KS - 1);
+  const int jl = lane >> kslog;
+  const int kmin = i - 2;
+  const T* __restrict__ gcol = Gp + col_off(l);
+  const T* __restrict__ acol = c.colA + col_off(l);
+  const int ro = row_off(l, p) - l - 1;
+  const int jend = j0 + nj;
+
+  T b[kTJ], best[kTJ];
+  int arg[kTJ], jj[kTJ];
+#pragma unroll
+  for (int u = 0; u < kTJ; ++u) {
+    jj[u] = j0 + jl + JL * u;
+    b[u] = (jj[u] < jend) ? c.rowB[ro + jj[u]] : T(0);
+    best[u] = Arith<T>::inf();
+    arg[u] = kmin;
+  }
+#pragma unroll 4
+  for (int k = kmin + ks; k < l; k += KS) {
+    const T g = gcol[k];
+    const T av = acol[k];
+#pragma unroll
+    for (int u = 0; u < kTJ; ++u) {
+      const T v = Arith<T>::fold(g, av + b[u]);
+      if (v < best[u]) {
+        best[u] = v;
+        arg[u] = k;
+      }
+    }
+  }
+  for (int o = 1; o < KS; o <<= 1) {
+#pragma unroll
+    for (int u = 0; u < kTJ; ++u) {
+      const T ov = __shfl_xor_sync(0xffffffffu, best[u], o);
+      const int oa = __shfl_xor_sync(0xffffffffu, arg[u], o);
+      if (ov < best[u] || (ov == best[u] && oa < arg[u])) {
+        best[u] = ov;
+        arg[u] = oa;
+      }
+    }
+  }
+  if (ks == 0) {
+#pragma unroll
+    for (int u = 0; u < kTJ; ++u) {
+      if (jj[u] < jend) {
+        const int e = ro + jj[u];
+        Gc[col_off(jj[u]) + l] = c.rowV[e] * invl + best[u];
+        bpi[e] = static_cast<uint16_t>(arg[u]);
+      }
+    }
+  }
+}
+
+// One full solve at lambda (all threads). Leaves the code in c.sQ and the fp64
+// evaluation in *out (shared).
+template <typename T>
+__device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out, T* bestE) {
+  const int p = c.p, S = c.S, tri = c.tri;
+  // Below kMinLambda the entropy terms vanish under the precision of T and
+  // 1/lambda would overflow it: the layers then run the MSE-only programme
+  // (the code is still evaluated in fp64 at the true lambda).
+  const double kMinLambda = sizeof(T) == 4 ? 1e-30 : 1e-290;
+  const bool sep = !(lam > kMinLambda);
+  const T invl = sep ? T(1) : static_cast<T>(1.0 / lam);
+  const int tid = threadIdx.x;
+  const int warp = warp_id(), lane = lane_id();
+
+  for (int t = tid; t < S; t += blockDim.x) c.ctr[t] = 0;
+  if (tid == 0) {
+    *bestE = Arith<T>::inf();
+    out->bestI = -1;
+    out->bestK = -1;
+  }
+  // Layer 1: F_1(0, j), written to buffer 1.
+  {
+    T* G1 = c.colG1;
+    for (int j = 1 + tid; j < p; j += blockDim.x) {
+      const int e = j - 1;  // row 0
+      T f = c.rowV[e] * invl;
+      if (!sep) f += Arith<T>::nlog(c.rowB[e] + Arith<T>::kEps);
+      G1[col_off(j)] = f;
+    }
+  }
+  __syncthreads();
+  for (int i = 2; i <= S - 1; ++i) {
+    const T* Gp = c.layer(i - 1);
+    T* Gc = c.layer(i);
+    uint16_t* bpi = c.bp + static_cast<size_t>(i) * tri;
+    const bool last = (i == S - 1);
+    if (warp == 0) finalize_layer(c, i - 1, Gp, sep, bestE, &out->bestI, &out->bestK);
+    if (i == 2) {
+      // Only k = c_1 = 0 precedes the second value.
+      for (int l = 1 + warp; l <= p - 2; l += kWarps) {
+        const T g0 = Gp[col_off(l)];
+        const T a0 = c.colA[col_off(l)];
+        const int ro = row_off(l, p) - l - 1;
+        for (int j = (last ? p - 1 : l + 1) + lane; j <= p - 1; j += kWarp) {
+          const int e = ro + j;
+          const T v = sep ? g0 : Arith<T>::fold(g0, a0 + c.rowB[e]);
+          Gc[col_off(j) + l] = c.rowV[e] * invl + v;
+        }
+      }
+    } else if (sep) {
+      const int kmin = i - 2;
+      for (int l = i - 1 + warp; l <= p - 2; l += kWarps) {
+        T best = Arith<T>::inf();
+        int arg = kmin;
+        for (int k = kmin + lane; k < l; k += kWarp) {
+          const T v = Gp[col_off(l) + k];
+          if (v < best) {
+            best = v;
+            arg = k;
+          }
+        }
+        warp_argmin(best, arg);
+        if (lane == 0) {
+          c.rmin[l] = best;
+          c.rarg[l] = arg;
+        }
+      }
+      __syncthreads();
+      for (int l = i - 1 + warp; l <= p - 2; l += kWarps) {
+        const int ro = row_off(l, p) - l - 1;
+        const T rm = c.rmin[l];
+        const uint16_t ra = static_cast<uint16_t>(c.rarg[l]);
+        for (int j = (last ? p - 1 : l + 1) + lane; j <= p - 1; j += kWarp) {
+          const int e = ro + j;
+          Gc[col_off(j) + l] = c.rowV[e] + rm;
+          bpi[e] = ra;
+        }
+      }
+    } else {
+      const uint32_t* tl = c.tasks + static_cast<size_t>(i) * c.max_tasks;
+      const int nt = c.ntasks[i];
+      for (;;) {
+        int t = 0;
+        if (lane == 0) t = atomicAdd(c.ctr + i, 1);
+        t = __shfl_sync(0xffffffffu, t, 0);
+        if (t >= nt) break;
+        run_task(c, tl[t], i, Gp, Gc, bpi, invl);
+      }
+    }
+    __syncthreads();
+  }
+  if (warp == 0) finalize_layer(c, S - 1, c.layer(S - 1), sep, bestE, &out->bestI, &out->bestK);
+  __syncthreads();
+
+  // Backtrack: c_{i+1} = p-1, c_i = k, c_{ii-1} = bp_ii(c_ii, c_{ii+1}), c_1 = 0.
+  if (tid == 0) {
+    if (out->bestI < 1) {  // no finite candidate (non-finite inputs): fall back to {P_0, P_{p-1}}
+      out->bestI = 1;
+      out->bestK = 0;
+    }
+    const int bi = out->bestI;
+    int l = out->bestK, j = p - 1;
+    c.sQ[bi] = p - 1;
+    c.sQ[bi - 1] = l;
+    for (int ii = bi; ii >= 2; --ii) {
+      const int kk = (ii == 2) ? 0 : static_cast<int>(c.bp[static_cast<size_t>(ii) * tri + row_off(l, p) + j - l - 1]);
+      c.sQ[ii - 2] = kk;
+      j = l;
+      l = kk;
+    }
+    out->m = bi + 1;
+  }
+  __syncthreads();
+
+  // fp64 evaluation of the code from the bucket statistics.
+  if (warp == 0) {
+    const int m = out->m;
+    double vs = 0.0;
+    for (int t = lane; t < m - 1; t += kWarp) {
+      const int a = c.sQ[t], cc = c.sQ[t + 1];
+      double N = 0.0, T1 = 0.0, T2 = 0.0;
+      const double Pa = c.sP[a];
+      for (int k = a; k < cc; ++k) {
+        const double dk = c.sP[k] - Pa;
+        const double nk = c.sN[k];
+        N += nk;
+        T1 += c.sA[k] + nk * dk;
+        T2 += c.sB[k] + 2.0 * dk * c.sA[k] + nk * dk * dk;
+      }
+      const double W = c.sP[cc] - Pa;
+      double V = W * T1 - T2;
+      V = V > 0.0 ? V : 0.0;
+      const double R = T1 / W;
+      c.sR[t] = R;
+      c.sL[t] = N - R;
+      vs += V;
+    }
+    __syncwarp();
+    double hs = 0.0;
+    for (int t = lane; t < m; t += kWarp) {
+      const double mu = (t > 0 ? c.sR[t - 1] : 0.0) + (t < m - 1 ? c.sL[t] : 0.0);
+      if (mu > 0.0) {
+        const double q = mu / c.dd;
+        hs -= q * log2(q);
+      }
+    }
+    vs = warp_sum(vs);
+    hs = warp_sum(hs);
+    if (lane == 0) {
+      out->mse = vs / c.dd;
+      out->H = hs;
+      out->J = out->mse + lam * hs;
+    }
+  }
+  __syncthreads();
+}
+
+template <typename T, bool kSmemTables>
+__global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ SolveOut s_out;
+  __shared__ T s_bestE;
+  __shared__ int s_flag;
+
+  const int p = a.p, S = a.s;
+  const int tri = tri_size(p);
+  Ctx<T> c;
+  c.p = p;
+  c.S = S;
+  c.tri = tri;
+  c.dd = static_cast<double>(a.d);
+  c.tasks = a.tasks;
+  c.ntasks = a.ntasks;
+  c.max_tasks = a.max_tasks;
+
+  unsigned char* sp = smem;
+  auto carve = [&sp](size_t bytes) {
+    unsigned char* r = sp;
+    sp += (bytes + 15) & ~size_t(15);
+    return r;
+  };
+  c.sP = reinterpret_cast<double*>(carve(sizeof(double) * p));
+  c.sN = reinterpret_cast<double*>(carve(sizeof(double) * p));
+  c.sA = reinterpret_cast<double*>(carve(sizeof(double) * p));
+  c.sB = reinterpret_cast<double*>(carve(sizeof(double) * p));
+  c.sR = reinterpret_cast<double*>(carve(sizeof(double) * S));
+  c.sL = reinterpret_cast<double*>(carve(sizeof(double) * S));
+  c.rmin = reinterpret_cast<T*>(carve(sizeof(T) * p));
+  c.rarg = reinterpret_cast<int*>(carve(sizeof(int) * p));
+  c.ctr = reinterpret_cast<int*>(carve(sizeof(int) * S));
+  c.sQ = reinterpret_cast<int*>(carve(sizeof(int) * S));
+  int* sQ1 = reinterpret_cast<int*>(carve(sizeof(int) * S));
+  int* sQ2 = reinterpret_cast<int*>(carve(sizeof(int) * S));
+
+  unsigned char* gs = a.scratch + static_cast<size_t>(blockIdx.x) * a.scratch_per_cta;
+  c.bp = reinterpret_cast<uint16_t*>(gs);
+  gs += (sizeof(uint16_t) * static_cast<size_t>(S) * tri + 255) & ~size_t(255);
+  const size_t tb = (sizeof(T) * static_cast<size_t>(tri) + 15) & ~size_t(15);
+  unsigned char* big = kSmemTables ? sp : gs;
+  c.colG0 = reinterpret_cast<T*>(big);
+  c.colG1 = reinterpret_cast<T*>(big + tb);
+  c.colA = reinterpret_cast<T*>(big + 2 * tb);
+  c.rowB = reinterpret_cast<T*>(big + 3 * tb);
+  c.rowV = reinterpret_cast<T*>(big + 4 * tb);
+
+  const int s_out_stride = a.s_out;
+  for (int r = blockIdx.x; r < a.n; r += gridDim.x) {
+    const double* P = a.P + static_cast<int64_t>(r) * p;
+    const int64_t bo = static_cast<int64_t>(r) * (p - 1);
+    if (threadIdx.x == 0) s_flag = a.in_status ? a.in_status[r] : 0;
+    for (int k = threadIdx.x; k < p; k += blockDim.x) {
+      c.sP[k] = P[k];
+      if (k < p - 1) {
+        c.sN[k] = static_cast<double>(a.cnt[bo + k]);
+        c.sA[k] = a.A[bo + k];
+        c.sB[k] = a.B[bo + k];
+      }
+    }
+    __syncthreads();
+    // P must be strictly increasing; P_0 == P_{p-1} is the constant vector.
+    const bool degenerate = (c.sP[0] == c.sP[p - 1]);
+    int bad = 0;
+    if (!degenerate)
+      for (int k = threadIdx.x; k < p - 1; k += blockDim.x) bad |= !(c.sP[k] < c.sP[k + 1]);
+    bad = __syncthreads_or(bad);
+    int32_t st = s_flag != 0 ? s_flag : (bad ? kStatusArg : kStatusOk);
+
+    if (st != kStatusOk || degenerate) {
+      // Invalid row: -1 codes. Constant row: Q = {P_0}, zero cost.
+      const int qv = (st == kStatusOk) ? 0 : -1;
+      const int ml = (st == kStatusOk) ? 1 : 0;
+      if (a.mode == 0) {
+        for (int t = 0; t < a.n_lambda; ++t) {
+          const int64_t w = static_cast<int64_t>(r) * a.n_lambda + t;
+          for (int q = threadIdx.x; q < s_out_stride; q += blockDim.x) a.Q[w * s_out_stride + q] = (q == 0) ? qv : -1;
+          if (threadIdx.x == 0) {
+            a.Q_len[w] = ml;
+            a.obj[w] = a.mse[w] = a.H[w] = 0.0;
+          }
+        }
+      } else {
+        for (int q = threadIdx.x; q < s_out_stride; q += blockDim.x) {
+          a.Q1[int64_t(r) * s_out_stride + q] = (q == 0) ? qv : -1;
+          a.Q2[int64_t(r) * s_out_stride + q] = (q == 0) ? qv : -1;
+        }
+        if (threadIdx.x == 0) {
+          a.Q1_len[r] = a.Q2_len[r] = ml;
+          a.theta[r] = a.lam_lo[r] = a.lam_hi[r] = 0.0;
+          a.H1[r] = a.H2[r] = a.mse1[r] = a.mse2[r] = 0.0;
+        }
+      }
+      if (threadIdx.x == 0) a.status[r] = st;
+      __syncthreads();
+      continue;
+    }
+
+    build_tables(c);
+    __syncthreads();
+
+    if (a.mode == 0) {
+      for (int t = 0; t < a.n_lambda; ++t) {
+        const int64_t w = static_cast<int64_t>(r) * a.n_lambda + t;
+        const double lam = a.lambda[w];
+        solve(c, lam, &s_out, &s_bestE);
+        for (int q = threadIdx.x; q < s_out_stride; q += blockDim.x)
+          a.Q[w * s_out_stride + q] = (q < s_out.m) ? c.sQ[q] : -1;
+        if (threadIdx.x == 0) {
+          a.Q_len[w] = s_out.m;
+          a.obj[w] = s_out.J;
+          a.mse[w] = s_out.mse;
+          a.H[w] = s_out.H;
+        }
+        __syncthreads();
+      }
+      if (threadIdx.x == 0) a.status[r] = kStatusOk;
+    } else {
+      // Bisection on lambda with two-way time-sharing.
+      double lo = 0.0;
+      double hi = (c.sP[p - 1] - c.sP[0]) * (c.sP[p - 1] - c.sP[0]);
+      double H1 = 0, H2 = 0, M1 = 0, M2 = 0;
+      int m1 = 0, m2 = 0;
+      auto keep = [&](int* dst, int& m, double& Hk, double& Mk) {
+        for (int q = threadIdx.x; q < S; q += blockDim.x) dst[q] = c.sQ[q];
+        m = s_out.m;
+        Hk = s_out.H;
+        Mk = s_out.mse;
+      };
+      int32_t status = kStatusOk;
+      double theta = 0.0;
+      solve(c, 0.0, &s_out, &s_bestE);
+      keep(sQ1, m1, H1, M1);
+      if (s_out.H <= a.budget) {
+        keep(sQ2, m2, H2, M2);
+        hi = 0.0;
+      } else {
+        __syncthreads();
+        solve(c, hi, &s_out, &s_bestE);
+        keep(sQ2, m2, H2, M2);
+        if (s_out.H > a.budget) {
+          status = kStatusBudget;
+        } else {
+          for (int it = 0; it < a.steps; ++it) {
+            const double mid = 0.5 * (lo + hi);
+            __syncthreads();
+            solve(c, mid, &s_out, &s_bestE);
+            if (s_out.H > a.budget) {
+              lo = mid;
+              keep(sQ1, m1, H1, M1);
+            } else {
+              hi = mid;
+              keep(sQ2, m2, H2, M2);
+            }
+          }
+          double th = (a.budget - H2) / (H1 - H2);
+          theta = th < 0.0 ? 0.0 : (th > 1.0 ? 1.0 : th);
+        }
+      }
+      __syncthreads();
+      for (int q = threadIdx.x; q < s_out_stride; q += blockDim.x) {
+        a.Q1[int64_t(r) * s_out_stride + q] = (q < m1) ? sQ1[q] : -1;
+        a.Q2[int64_t(r) * s_out_stride + q] = (q < m2) ? sQ2[q] : -1;
+      }
+      if (threadIdx.x == 0) {
+        a.Q1_len[r] = m1;
+        a.Q2_len[r] = m2;
+        a.theta[r] = theta;
+        a.lam_lo[r] = lo;
+        a.lam_hi[r] = hi;
+        a.H1[r] = H1;
+        a.H2[r] = H2;
+        a.mse1[r] = M1;
+        a.mse2[r] = M2;
+        a.status[r] = status;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// ---- schedule ----------------------------------------------------------------
+// Tasks of layer i >= 3 in descending cost (rows taken outward from the
+// costliest one; row cost K * NJ is unimodal in l). Full tasks cover 64 j with
+// one k-lane; the remainder of a row is split over KS k-lanes so that the warp
+// stays busy. One thread per layer.
+__global__ void k_schedule(int p, int S, int max_tasks, uint32_t* tasks, int32_t* ntasks) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= S) return;
+  if (i < 3) {
+    ntasks[i] = 0;
+    return;
+  }
+  const bool last = (i == S - 1);
+  const int kmin = i - 2;
+  const int r0 = i - 1, r1 = p - 2;
+  auto cost = [&](int l) -> long long {
+    const long long K = l - kmin;
+    const long long NJ = last ? 1 : (p - 1 - l);
+    return K * NJ;
+  };
+  uint32_t* out = tasks + static_cast<size_t>(i) * max_tasks;
+  int n = 0;
+  auto emit = [&](int l) {
+    const int K = l - kmin;
+    const int NJ = last ? 1 : (p - 1 - l);
+    const int j0 = last ? p - 1 : l + 1;
+    const int nfull = NJ / kTaskJ;
+    for (int f = 0; f < nfull; ++f) out[n++] = pack_task(l, j0 + f * kTaskJ, kTaskJ, 0);
+    const int rem = NJ - nfull * kTaskJ;
+    if (rem > 0) {
+      const int need = (rem + kTJ - 1) / kTJ;  // j-lanes needed
+      int jl = 1;
+      while (jl < need) jl <<= 1;
+      int ks = kWarp / jl;
+      while (ks > 1 && ks > K) ks >>= 1;
+      int kslog = 0;
+      while ((1 << kslog) < ks) ++kslog;
+      out[n++] = pack_task(l, j0 + nfull * kTaskJ, rem, kslog);
+    }
+  };
+  if (r0 <= r1) {
+    int pk = r0;
+    for (int l = r0; l <= r1; ++l)
+      if (cost(l) > cost(pk)) pk = l;
+    emit(pk);
+    int lo = pk - 1, hi = pk + 1;
+    while (lo >= r0 || hi <= r1) {
+      if (hi > r1 || (lo >= r0 && cost(lo) >= cost(hi)))
+        emit(lo--);
+      else
+        emit(hi++);
+    }
+  }
+  ntasks[i] = n;
+}
+
+template <typename T, bool kSmem>
+void* dp_kernel_ptr() {
+  return reinterpret_cast<void*>(&k_dp<T, kSmem>);
+}
+
+size_t small_smem(int p, int S, size_t tsz) {
+  auto al = [](size_t b) { return (b + 15) & ~size_t(15); };
+  return al(8 * p) * 4 + al(8 * S) * 2 + al(tsz * p) + al(4 * p) + al(4 * S) * 4;
+}
+
+size_t table_bytes(int p, size_t tsz) { return ((tsz * tri_size(p) + 15) & ~size_t(15)) * 5; }
+
+}  // namespace
+
+int64_t dp_triples(int p, int s) {
+  const int S = s < p ? s : p;
+  int64_t t = 0;
+  for (int i = 2; i <= S - 1; ++i) {
+    const bool last = (i == S - 1);
+    for (int l = i - 1; l <= p - 2; ++l) {
+      const int64_t K = (i == 2) ? 1 : (l - i + 2);
+      const int64_t NJ = last ? 1 : (p - 1 - l);
+      t += K * NJ;
+    }
+  }
+  return t;
+}
+
+size_t dp_schedule_bytes(int p, int s) {
+  const int S = s < p ? s : p;
+  const size_t max_tasks = static_cast<size_t>(p) * ((p + kTaskJ - 1) / kTaskJ + 1);
+  return ((sizeof(uint32_t) * max_tasks * S + 255) & ~size_t(255)) + ((sizeof(int32_t) * S + 255) & ~size_t(255));
+}
+
+bool dp_plan(int n, int p, int s, bool fp64, DpPlan* plan) {
+  if (p < 2 || p > kMaxP || s < 2 || n < 1) return false;
+  const int S = s < p ? s : p;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  int sms = 0, optin = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  const size_t tsz = fp64 ? 8 : 4;
+  const size_t small = small_smem(p, S, tsz);
+  const size_t big = table_bytes(p, tsz);
+  plan->fp64 = fp64;
+  plan->threads = kThreads;
+  plan->smem_tables = (small + big + 1024 <= static_cast<size_t>(optin));
+  plan->smem_bytes = small + (plan->smem_tables ? big : 0);
+  const size_t bp = (sizeof(uint16_t) * static_cast<size_t>(S) * tri_size(p) + 255) & ~size_t(255);
+  plan->scratch_per_cta = (bp + (plan->smem_tables ? 0 : big) + 255) & ~size_t(255);
+  plan->max_tasks = p * ((p + kTaskJ - 1) / kTaskJ + 1);
+  void* fn = fp64 ? (plan->smem_tables ? dp_kernel_ptr<double, true>() : dp_kernel_ptr<double, false>())
+                  : (plan->smem_tables ? dp_kernel_ptr<float, true>() : dp_kernel_ptr<float, false>());
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(plan->smem_bytes)) !=
+      cudaSuccess)
+    return false;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, plan->smem_bytes) != cudaSuccess ||
+      per_sm < 1)
+    return false;
+  const int ctas = sms * per_sm;
+  plan->ctas = n < ctas ? n : ctas;
+  return true;
+}
+
+cudaError_t launch_dp(const DpPlan& plan, DpArgs args, uint32_t* tasks, int32_t* ntasks, cudaStream_t st) {
+  const int S = args.s;
+  args.tasks = tasks;
+  args.ntasks = ntasks;
+  args.max_tasks = plan.max_tasks;
+  k_schedule<<<(S + 63) / 64, 64, 0, st>>>(args.p, S, plan.max_tasks, tasks, ntasks);
+  note_launch();
+  void* fn = plan.fp64 ? (plan.smem_tables ? dp_kernel_ptr<double, true>() : dp_kernel_ptr<double, false>())
+                       : (plan.smem_tables ? dp_kernel_ptr<float, true>() : dp_kernel_ptr<float, false>());
+  void* kargs[] = {&args};
+  cudaError_t e = cudaLaunchKernel(fn, dim3(plan.ctas), dim3(plan.threads), kargs, plan.smem_bytes, st);
+  note_launch();
+  return e;
+}
+
+}  // namespace ecasq

@@ -1,0 +1,292 @@
+// Row statistics, uniform grid and bucketing of X onto the permissible set P.
+//
+// ECASQ summary (gist.science/pt/paper/2608.18147) §2.2 "Generalização": for an
+// arbitrary permissible set P the solver costs O(p^2 s + d); the O(d) part is
+// one pass that buckets every entry onto P and accumulates per-bucket
+// statistics, from which every interval table is built without touching X
+// again. Both kernels here are HBM-bound streams over X (4 bytes per entry).
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace ecasq {
+
+// ---------------------------------------------------------------------------
+// Row min / max / finiteness, one chunk of one row per CTA.
+// partial layout per (row, chunk): float lo, float hi, int bad (3 x 32-bit).
+
+namespace {
+
+constexpr int kGridThreads = 256;
+
+__device__ __forceinline__ void mm_update(float v, float& lo, float& hi, int& bad) {
+  if (!isfinite(v)) bad = 1;
+  lo = fminf(lo, v);
+  hi = fmaxf(hi, v);
+}
+
+__global__ void __launch_bounds__(kGridThreads)
+k_minmax_partial(const float* __restrict__ X, int64_t d, int64_t chunk, int n_chunks,
+                 float* __restrict__ part) {
+  const int r = blockIdx.y;
+  const int c = blockIdx.x;
+  const float* x = X + static_cast<int64_t>(r) * d;
+  const int64_t beg = static_cast<int64_t>(c) * chunk;
+  const int64_t end = beg + chunk < d ? beg + chunk : d;
+  float lo = INFINITY, hi = -INFINITY;
+  int bad = 0;
+  // Vector loads when the chunk start is 16-byte aligned.
+  const bool vec = ((reinterpret_cast<uintptr_t>(x + beg) & 15u) == 0);
+  int64_t t = beg;
+  if (vec) {
+    const int64_t nv = (end - beg) >> 2;
+    const float4* x4 = reinterpret_cast<const float4*>(x + beg);
+    for (int64_t i = threadIdx.x; i < nv; i += blockDim.x) {
+      const float4 v = __ldcs(x4 + i);
+      mm_update(v.x, lo, hi, bad);
+      mm_update(v.y, lo, hi, bad);
+      mm_update(v.z, lo, hi, bad);
+      mm_update(v.w, lo, hi, bad);
+    }
+    t = beg + (nv << 2);
+  }
+  for (int64_t i = t + threadIdx.x; i < end; i += blockDim.x) mm_update(__ldcs(x + i), lo, hi, bad);
+
+  __shared__ float s_lo[kGridThreads / kWarp], s_hi[kGridThreads / kWarp];
+  __shared__ int s_bad[kGridThreads / kWarp];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    bad |= __shfl_xor_sync(0xffffffffu, bad, o);
+  }
+  if (lane_id() == 0) {
+    s_lo[warp_id()] = lo;
+    s_hi[warp_id()] = hi;
+    s_bad[warp_id()] = bad;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < kGridThreads / kWarp; ++w) {
+      lo = fminf(lo, s_lo[w]);
+      hi = fmaxf(hi, s_hi[w]);
+      bad |= s_bad[w];
+    }
+    float* o = part + (static_cast<int64_t>(r) * n_chunks + c) * 3;
+    o[0] = lo;
+    o[1] = hi;
+    o[2] = __int_as_float(bad);
+  }
+}
+
+// P_k = lo + (hi - lo) * k / (p - 1) in IEEE fp64 with round-to-nearest and no
+// contraction; P_{p-1} = hi.
+__global__ void k_grid_finish(const float* __restrict__ part, int n_chunks, int p,
+                              double* __restrict__ P, int32_t* __restrict__ status) {
+  const int r = blockIdx.x;
+  __shared__ float s_lo, s_hi;
+  __shared__ int s_bad;
+  if (threadIdx.x == 0) {
+    float lo = INFINITY, hi = -INFINITY;
+    int bad = 0;
+    for (int c = 0; c < n_chunks; ++c) {
+      const float* o = part + (static_cast<int64_t>(r) * n_chunks + c) * 3;
+      lo = fminf(lo, o[0]);
+      hi = fmaxf(hi, o[1]);
+      bad |= __float_as_int(o[2]);
+    }
+    s_lo = lo;
+    s_hi = hi;
+    s_bad = bad;
+    if (status) status[r] = bad ? kStatusRange : kStatusOk;
+  }
+  __syncthreads();
+  const double lo = s_lo, hi = s_hi;
+  const double span = __dsub_rn(hi, lo);
+  const double den = static_cast<double>(p - 1);
+  for (int k = threadIdx.x; k < p; k += blockDim.x) {
+    double v;
+    if (k == p - 1)
+      v = hi;
+    else
+      v = __dadd_rn(lo, __ddiv_rn(__dmul_rn(span, static_cast<double>(k)), den));
+    P[static_cast<int64_t>(r) * p + k] = s_bad ? __longlong_as_double(0x7ff8000000000000ll) : v;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Bucketing. Sums are fixed point: an entry of bucket k with y = x - P_k adds
+// round(y / D_k * 2^fb) to the first-moment accumulator and
+// round((y / D_k)^2 * 2^fb) to the second, D_k = P_{k+1} - P_k, fb chosen so
+// that d entries cannot overflow 64 bits. Integer sums make the result
+// independent of the order in which CTAs and lanes accumulate, and the shared
+// memory updates are native 64-bit integer atomics. Each lane updates copy
+// (lane % kCopies) of the CTA's histogram, which caps same-address collisions
+// inside a warp at 32 / kCopies.
+
+constexpr int kBucketThreads = 256;
+constexpr int kCopies = 4;
+
+__global__ void __launch_bounds__(kBucketThreads)
+k_bucket(const float* __restrict__ X, int64_t d, int64_t chunk, const double* __restrict__ Pall,
+         int p, int fb, unsigned long long* __restrict__ acc, int32_t* __restrict__ flag) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int r = blockIdx.y;
+  const int nb = p - 1;
+  double* sP = reinterpret_cast<double*>(smem);                 // [p]
+  double* sS = sP + p;                                          // [p-1] 2^fb / D_k
+  unsigned long long* sa = reinterpret_cast<unsigned long long*>(sS + p);  // [kCopies][p]
+  unsigned long long* sb = sa + kCopies * p;                     // [kCopies][p]
+  unsigned int* sc = reinterpret_cast<unsigned int*>(sb + kCopies * p);    // [kCopies][p]
+  __shared__ int s_bad;
+
+  const double* P = Pall + static_cast<int64_t>(r) * p;
+  const double two_fb = ldexp(1.0, fb);
+  for (int k = threadIdx.x; k < p; k += blockDim.x) {
+    sP[k] = P[k];
+    if (k < nb) sS[k] = two_fb / (P[k + 1] - P[k]);
+  }
+  for (int k = threadIdx.x; k < kCopies * p; k += blockDim.x) {
+    sa[k] = 0ull;
+    sb[k] = 0ull;
+    sc[k] = 0u;
+  }
+  if (threadIdx.x == 0) s_bad = 0;
+  __syncthreads();
+
+  const double scale = static_cast<double>(p - 1) / (sP[p - 1] - sP[0]);
+  const double inv_two_fb = ldexp(1.0, -fb);
+  const int copy = lane_id() & (kCopies - 1);
+  unsigned long long* ma = sa + copy * p;
+  unsigned long long* mb = sb + copy * p;
+  unsigned int* mc = sc + copy * p;
+  int bad = 0;
+
+  auto one = [&](float xf) {
+    const double x = static_cast<double>(xf);
+    const int k = bucket_of(x, sP, p, scale);
+    if (k < 0) {
+      bad = 1;
+      return;
+    }
+    const double u = (x - sP[k]) * sS[k];
+    const unsigned long long a = __double2ull_rn(u);
+    const unsigned long long b = __double2ull_rn(u * u * inv_two_fb);
+    atomicAdd(mc + k, 1u);
+    atomicAdd(ma + k, a);
+    atomicAdd(mb + k, b);
+  };
+
+  const float* x = X + static_cast<int64_t>(r) * d;
+  const int64_t beg = static_cast<int64_t>(blockIdx.x) * chunk;
+  const int64_t end = beg + chunk < d ? beg + chunk : d;
+  const bool vec = ((reinterpret_cast<uintptr_t>(x + beg) & 15u) == 0);
+  int64_t t = beg;
+  if (vec) {
+    const int64_t nv = (end - beg) >> 2;
+    const float4* x4 = reinterpret_cast<const float4*>(x + beg);
+    for (int64_t i = threadIdx.x; i < nv; i += blockDim.x) {
+      const float4 v = __ldcs(x4 + i);
+      one(v.x);
+      one(v.y);
+      one(v.z);
+      one(v.w);
+    }
+    t = beg + (nv << 2);
+  }
+  for (int64_t i = t + threadIdx.x; i < end; i += blockDim.x) one(__ldcs(x + i));
+  if (bad) s_bad = 1;
+  __syncthreads();
+
+  unsigned long long* g = acc + static_cast<int64_t>(r) * nb * 3;
+  for (int k = threadIdx.x; k < nb; k += blockDim.x) {
+    unsigned long long c = 0, a = 0, b = 0;
+#pragma unroll
+    for (int q = 0; q < kCopies; ++q) {
+      c += sc[q * p + k];
+      a += sa[q * p + k];
+      b += sb[q * p + k];
+    }
+    if (c) {
+      atomicAdd(g + 3 * k + 0, c);
+      atomicAdd(g + 3 * k + 1, a);
+      atomicAdd(g + 3 * k + 2, b);
+    }
+  }
+  if (threadIdx.x == 0 && s_bad) atomicOr(flag + r, 1);
+}
+
+// Fixed-point accumulators -> cnt (int64), A = sum y, B = sum y^2 (fp64).
+__global__ void k_bucket_finish(const unsigned long long* __restrict__ acc, const double* __restrict__ Pall,
+                                int p, int fb, const int32_t* __restrict__ flag, int64_t* __restrict__ cnt,
+                                double* __restrict__ A, double* __restrict__ B, int32_t* __restrict__ status) {
+  const int r = blockIdx.x;
+  const int nb = p - 1;
+  const double* P = Pall + static_cast<int64_t>(r) * p;
+  const unsigned long long* g = acc + static_cast<int64_t>(r) * nb * 3;
+  const double inv_two_fb = ldexp(1.0, -fb);
+  for (int k = threadIdx.x; k < nb; k += blockDim.x) {
+    const double D = P[k + 1] - P[k];
+    const int64_t o = static_cast<int64_t>(r) * nb + k;
+    cnt[o] = static_cast<int64_t>(g[3 * k + 0]);
+    A[o] = static_cast<double>(g[3 * k + 1]) * inv_two_fb * D;
+    B[o] = static_cast<double>(g[3 * k + 2]) * inv_two_fb * D * D;
+  }
+  if (threadIdx.x == 0 && status) status[r] = flag[r] ? kStatusRange : kStatusOk;
+}
+
+}  // namespace
+
+int bucket_fraction_bits(int64_t d) {
+  int lg = 0;
+  while ((int64_t(1) << lg) < d + 1) ++lg;
+  int fb = 63 - lg - 1;
+  return fb > 50 ? 50 : fb;
+}
+
+int64_t minmax_chunk(int64_t d) { return d < 16384 ? d : 16384; }
+
+cudaError_t launch_uniform_grid(const float* X, int n, int64_t d, int p, double* P, int32_t* status,
+                                float* part, cudaStream_t st) {
+  const int64_t chunk = minmax_chunk(d);
+  const int nc = static_cast<int>((d + chunk - 1) / chunk);
+  k_minmax_partial<<<dim3(nc, n), kGridThreads, 0, st>>>(X, d, chunk, nc, part);
+  note_launch();
+  k_grid_finish<<<n, 128, 0, st>>>(part, nc, p, P, status);
+  note_launch();
+  return cudaGetLastError();
+}
+
+size_t bucket_smem_bytes(int p) {
+  return static_cast<size_t>(p) * 8 * 2 + static_cast<size_t>(kCopies) * p * (8 + 8 + 4);
+}
+
+int64_t bucket_chunk(int64_t d) { return d < 16384 ? d : 16384; }
+
+cudaError_t launch_bucket(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt,
+                          double* A, double* B, int32_t* status, unsigned long long* acc,
+                          int32_t* flag, cudaStream_t st) {
+  const int fb = bucket_fraction_bits(d);
+  cudaError_t e = cudaMemsetAsync(acc, 0, sizeof(unsigned long long) * 3 * (p - 1) * static_cast<size_t>(n), st);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(flag, 0, sizeof(int32_t) * n, st);
+  if (e != cudaSuccess) return e;
+  const int64_t chunk = bucket_chunk(d);
+  const int nc = static_cast<int>((d + chunk - 1) / chunk);
+  const size_t smem = bucket_smem_bytes(p);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(k_bucket, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+    attr_set = true;
+  }
+  k_bucket<<<dim3(nc, n), kBucketThreads, smem, st>>>(X, d, chunk, P, p, fb, acc, flag);
+  note_launch();
+  k_bucket_finish<<<n, 256, 0, st>>>(acc, P, p, fb, flag, cnt, A, B, status);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace ecasq

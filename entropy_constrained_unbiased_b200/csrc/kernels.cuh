@@ -1,0 +1,95 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace ecasq {
+
+// Counts kernel launches issued through the library (per host thread).
+void note_launch();
+
+// ---- grid + bucketing (grid_bucket.cu) ----
+int bucket_fraction_bits(int64_t d);
+int64_t minmax_chunk(int64_t d);
+int64_t bucket_chunk(int64_t d);
+size_t bucket_smem_bytes(int p);
+cudaError_t launch_uniform_grid(const float* X, int n, int64_t d, int p, double* P, int32_t* status,
+                                float* part, cudaStream_t st);
+cudaError_t launch_bucket(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt,
+                          double* A, double* B, int32_t* status, unsigned long long* acc,
+                          int32_t* flag, cudaStream_t st);
+
+// ---- DP solver (dp.cu) ----
+struct DpArgs {
+  // bucket statistics [n][p-1] and alphabet [n][p]
+  const int64_t* cnt;
+  const double* A;
+  const double* B;
+  const double* P;
+  const int32_t* in_status;  // [n] status of the bucketing pass, or null
+  int n, p, s;               // s already clamped to p
+  int64_t d;
+  // mode 0: list of lambdas per vector; mode 1: entropy budget
+  int mode;
+  const double* lambda;  // [n][n_lambda]
+  int n_lambda;
+  double budget;
+  int steps;
+  // mode 0 outputs ([n][n_lambda] and [n][n_lambda][s_out])
+  int32_t* Q;
+  int32_t* Q_len;
+  double* obj;
+  double* mse;
+  double* H;
+  // mode 1 outputs ([n] and [n][s_out])
+  int32_t* Q1;
+  int32_t* Q1_len;
+  int32_t* Q2;
+  int32_t* Q2_len;
+  double* theta;
+  double* lam_lo;
+  double* lam_hi;
+  double* H1;
+  double* H2;
+  double* mse1;
+  double* mse2;
+  int32_t* status;  // [n]
+  int s_out;        // row stride of the Q outputs (the caller's s)
+  // schedule of the DP layers (built by the schedule kernel)
+  const uint32_t* tasks;  // [s][max_tasks]
+  const int32_t* ntasks;  // [s]
+  int max_tasks;
+  // per-CTA global scratch
+  unsigned char* scratch;
+  size_t scratch_per_cta;
+};
+
+struct DpPlan {
+  bool fp64;
+  bool smem_tables;  // pair tables resident in shared memory
+  int threads;
+  int ctas;
+  size_t smem_bytes;
+  size_t scratch_per_cta;
+  int max_tasks;
+};
+
+// Plan for the current device; ok = false when the sizes are out of range.
+bool dp_plan(int n, int p, int s, bool fp64, DpPlan* plan);
+size_t dp_schedule_bytes(int p, int s);
+cudaError_t launch_dp(const DpPlan& plan, DpArgs args, uint32_t* tasks, int32_t* ntasks, cudaStream_t st);
+
+// Exact count of (k, l, j) triples one solve evaluates (host).
+int64_t dp_triples(int p, int s);
+
+// ---- encoder (encode.cu) ----
+cudaError_t launch_encode(const float* X, const double* P, int n, int64_t d, int p, int s,
+                          const int32_t* Q1, const int32_t* Q1_len, const int32_t* Q2,
+                          const int32_t* Q2_len, const double* theta, uint64_t seed, uint8_t* idx,
+                          int64_t* hist, int32_t* status, cudaStream_t st);
+cudaError_t launch_entropy(const int64_t* hist, int n, int s, double* H, cudaStream_t st);
+
+}  // namespace ecasq

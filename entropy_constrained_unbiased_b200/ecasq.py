@@ -1,0 +1,258 @@
+"""Thin ctypes binding of libecasq.so (C ABI in include/ecasq.h).
+
+Argument marshalling only: every step of the solver runs in the library's CUDA
+kernels. torch provides device memory and the current stream. There is no CPU
+fallback: loading raises if the library is missing or no CUDA device exists.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libecasq.so")
+
+OK, ERR_ARG, ERR_RANGE, ERR_WORKSPACE, ERR_CUDA, WARN_BUDGET = 0, -1, -2, -3, -4, 1
+
+EXPORTS = [
+    "ecasq_workspace_size", "ecasq_aux_workspace_size", "ecasq_uniform_grid", "ecasq_bucket",
+    "ecasq_solve", "ecasq_solve_stats", "ecasq_solve_budget", "ecasq_solve_budget_stats",
+    "ecasq_encode", "ecasq_entropy", "ecasq_status_string", "ecasq_launch_count",
+]
+
+
+class EcasqError(RuntimeError):
+    pass
+
+
+class Opts(C.Structure):
+    _fields_ = [("dp_fp64", C.c_int), ("hirschberg", C.c_int), ("bisect_steps", C.c_int),
+                ("reserved", C.c_int)]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load the library and declare its signatures (no CUDA call is made)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise EcasqError(f"libecasq.so not built ({path}); run __graft_entry__.build()")
+    L = C.CDLL(path)
+    P, I, I64, D, SZ, U64 = C.c_void_p, C.c_int, C.c_int64, C.c_double, C.c_size_t, C.c_uint64
+    OP = C.POINTER(Opts)
+    sig = {
+        "ecasq_workspace_size": (SZ, [I, I64, I, I, I, OP]),
+        "ecasq_aux_workspace_size": (SZ, [I, I64, I]),
+        "ecasq_uniform_grid": (I, [P, I, I64, I, P, P, P, SZ, P]),
+        "ecasq_bucket": (I, [P, P, I, I64, I, P, P, P, P, P, SZ, P]),
+        "ecasq_solve": (I, [P, P, I, I64, I, I, P, I, P, P, P, P, P, P, OP, P, SZ, P]),
+        "ecasq_solve_stats": (I, [P, P, P, P, I, I64, I, I, P, I, P, P, P, P, P, P, OP, P, SZ, P]),
+        "ecasq_solve_budget": (I, [P, P, I, I64, I, I, D] + [P] * 12 + [OP, P, SZ, P]),
+        "ecasq_solve_budget_stats": (I, [P, P, P, P, I, I64, I, I, D] + [P] * 12 + [OP, P, SZ, P]),
+        "ecasq_encode": (I, [P, P, I, I64, I, I, P, P, P, P, P, U64, P, P, P, P]),
+        "ecasq_entropy": (I, [P, I, I, P, P]),
+        "ecasq_status_string": (C.c_char_p, [I]),
+        "ecasq_launch_count": (C.c_uint64, [I]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def _need_cuda():
+    if not torch.cuda.is_available():
+        raise EcasqError("ECASQ needs a CUDA device; there is no CPU fallback")
+    return load()
+
+
+def _ptr(t):
+    return C.c_void_p(t.data_ptr()) if t is not None else C.c_void_p(0)
+
+
+def _stream():
+    return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(rc: int, what: str):
+    if rc != OK:
+        msg = load().ecasq_status_string(rc).decode()
+        raise EcasqError(f"{what}: {msg} ({rc})")
+
+
+def _dev(t, dtype, name):
+    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous()):
+        raise EcasqError(f"{name} must be a contiguous CUDA {dtype} tensor")
+    return t
+
+
+_ws_cache: dict = {}
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A cached device buffer of at least nbytes (the library never allocates)."""
+    key = torch.device(device)
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=key)
+        _ws_cache[key] = buf
+    return buf
+
+
+def opts(fp64: bool = False, steps: int = 30, hirschberg: bool = False) -> Opts:
+    return Opts(int(fp64), int(hirschberg), int(steps), 0)
+
+
+def launch_count(reset: bool = False) -> int:
+    return int(load().ecasq_launch_count(int(reset)))
+
+
+def uniform_grid(X: torch.Tensor, p: int):
+    L = _need_cuda()
+    _dev(X, torch.float32, "X")
+    n, d = X.shape
+    P = torch.empty((n, p), dtype=torch.float64, device=X.device)
+    st = torch.empty(n, dtype=torch.int32, device=X.device)
+    ws = workspace(L.ecasq_aux_workspace_size(n, d, p), X.device)
+    _check(L.ecasq_uniform_grid(_ptr(X), n, d, p, _ptr(P), _ptr(st), _ptr(ws), ws.numel(), _stream()),
+           "ecasq_uniform_grid")
+    return P, st
+
+
+def bucket(X: torch.Tensor, P: torch.Tensor):
+    L = _need_cuda()
+    _dev(X, torch.float32, "X")
+    _dev(P, torch.float64, "P")
+    n, d = X.shape
+    p = P.shape[1]
+    cnt = torch.empty((n, p - 1), dtype=torch.int64, device=X.device)
+    A = torch.empty((n, p - 1), dtype=torch.float64, device=X.device)
+    B = torch.empty_like(A)
+    st = torch.empty(n, dtype=torch.int32, device=X.device)
+    ws = workspace(L.ecasq_aux_workspace_size(n, d, p), X.device)
+    _check(L.ecasq_bucket(_ptr(X), _ptr(P), n, d, p, _ptr(cnt), _ptr(A), _ptr(B), _ptr(st), _ptr(ws), ws.numel(),
+                          _stream()), "ecasq_bucket")
+    return cnt, A, B, st
+
+
+def _lam_table(lam, n, device):
+    lam = torch.as_tensor(lam, dtype=torch.float64)
+    if lam.dim() == 0:
+        lam = lam.expand(n, 1)
+    elif lam.dim() == 1:
+        lam = lam.reshape(n, 1) if lam.numel() == n else lam.reshape(1, -1).expand(n, -1)
+    return lam.to(device).contiguous()
+
+
+def _solve_outputs(n, nl, s, device):
+    return dict(Q=torch.empty((n, nl, s), dtype=torch.int32, device=device),
+                Q_len=torch.empty((n, nl), dtype=torch.int32, device=device),
+                objective=torch.empty((n, nl), dtype=torch.float64, device=device),
+                mse=torch.empty((n, nl), dtype=torch.float64, device=device),
+                H=torch.empty((n, nl), dtype=torch.float64, device=device),
+                status=torch.empty(n, dtype=torch.int32, device=device))
+
+
+def solve(X: torch.Tensor, P: torch.Tensor, s: int, lam, fp64: bool = False):
+    """Exact Lagrangian solve of each row at each of its lambdas ([n] or [n, L])."""
+    L = _need_cuda()
+    _dev(X, torch.float32, "X")
+    _dev(P, torch.float64, "P")
+    n, d = X.shape
+    p = P.shape[1]
+    lt = _lam_table(lam, n, X.device)
+    nl = lt.shape[1]
+    o = _solve_outputs(n, nl, s, X.device)
+    op = opts(fp64)
+    ws = workspace(L.ecasq_workspace_size(n, d, p, s, nl, C.byref(op)), X.device)
+    _check(L.ecasq_solve(_ptr(X), _ptr(P), n, d, p, s, _ptr(lt), nl, _ptr(o["Q"]), _ptr(o["Q_len"]),
+                         _ptr(o["objective"]), _ptr(o["mse"]), _ptr(o["H"]), _ptr(o["status"]), C.byref(op),
+                         _ptr(ws), ws.numel(), _stream()), "ecasq_solve")
+    return o
+
+
+def solve_stats(cnt, A, B, P, d: int, s: int, lam, fp64: bool = False):
+    L = _need_cuda()
+    n, p = P.shape
+    lt = _lam_table(lam, n, P.device)
+    nl = lt.shape[1]
+    o = _solve_outputs(n, nl, s, P.device)
+    op = opts(fp64)
+    ws = workspace(L.ecasq_workspace_size(n, d, p, s, nl, C.byref(op)), P.device)
+    _check(L.ecasq_solve_stats(_ptr(cnt), _ptr(A), _ptr(B), _ptr(P), n, d, p, s, _ptr(lt), nl, _ptr(o["Q"]),
+                               _ptr(o["Q_len"]), _ptr(o["objective"]), _ptr(o["mse"]), _ptr(o["H"]),
+                               _ptr(o["status"]), C.byref(op), _ptr(ws), ws.numel(), _stream()),
+           "ecasq_solve_stats")
+    return o
+
+
+def _budget_outputs(n, s, device):
+    o = dict(Q1=torch.empty((n, s), dtype=torch.int32, device=device),
+             Q1_len=torch.empty(n, dtype=torch.int32, device=device),
+             Q2=torch.empty((n, s), dtype=torch.int32, device=device),
+             Q2_len=torch.empty(n, dtype=torch.int32, device=device))
+    for k in ("theta", "lambda_lo", "lambda_hi", "H1", "H2", "mse1", "mse2"):
+        o[k] = torch.empty(n, dtype=torch.float64, device=device)
+    o["status"] = torch.empty(n, dtype=torch.int32, device=device)
+    return o
+
+
+_BUDGET_ORDER = ("Q1", "Q1_len", "Q2", "Q2_len", "theta", "lambda_lo", "lambda_hi", "H1", "H2", "mse1", "mse2",
+                 "status")
+
+
+def solve_budget(X: torch.Tensor, P: torch.Tensor, s: int, b: float, steps: int = 30, fp64: bool = False):
+    """Entropy budget b: lambda bisection plus two-way time-sharing per row."""
+    L = _need_cuda()
+    _dev(X, torch.float32, "X")
+    _dev(P, torch.float64, "P")
+    n, d = X.shape
+    p = P.shape[1]
+    o = _budget_outputs(n, s, X.device)
+    op = opts(fp64, steps)
+    ws = workspace(L.ecasq_workspace_size(n, d, p, s, 1, C.byref(op)), X.device)
+    _check(L.ecasq_solve_budget(_ptr(X), _ptr(P), n, d, p, s, float(b), *[_ptr(o[k]) for k in _BUDGET_ORDER],
+                                C.byref(op), _ptr(ws), ws.numel(), _stream()), "ecasq_solve_budget")
+    return o
+
+
+def solve_budget_stats(cnt, A, B, P, d: int, s: int, b: float, steps: int = 30, fp64: bool = False):
+    L = _need_cuda()
+    n, p = P.shape
+    o = _budget_outputs(n, s, P.device)
+    op = opts(fp64, steps)
+    ws = workspace(L.ecasq_workspace_size(n, d, p, s, 1, C.byref(op)), P.device)
+    _check(L.ecasq_solve_budget_stats(_ptr(cnt), _ptr(A), _ptr(B), _ptr(P), n, d, p, s, float(b),
+                                      *[_ptr(o[k]) for k in _BUDGET_ORDER], C.byref(op), _ptr(ws), ws.numel(),
+                                      _stream()), "ecasq_solve_budget_stats")
+    return o
+
+
+def encode(X: torch.Tensor, P: torch.Tensor, s: int, Q1, Q1_len, seed: int, Q2=None, Q2_len=None, theta=None):
+    """Stochastic rounding onto Q1 (or time-shared Q1/Q2). Returns idx [n,d] u8, hist [n,2,s] i64, status."""
+    L = _need_cuda()
+    _dev(X, torch.float32, "X")
+    _dev(P, torch.float64, "P")
+    n, d = X.shape
+    p = P.shape[1]
+    idx = torch.empty((n, d), dtype=torch.uint8, device=X.device)
+    hist = torch.empty((n, 2, s), dtype=torch.int64, device=X.device)
+    st = torch.empty(n, dtype=torch.int32, device=X.device)
+    _check(L.ecasq_encode(_ptr(X), _ptr(P), n, d, p, s, _ptr(Q1), _ptr(Q1_len), _ptr(Q2), _ptr(Q2_len), _ptr(theta),
+                          C.c_uint64(seed), _ptr(idx), _ptr(hist), _ptr(st), _stream()), "ecasq_encode")
+    return idx, hist, st
+
+
+def entropy(hist: torch.Tensor):
+    L = _need_cuda()
+    n, _, s = hist.shape
+    H = torch.empty(n, dtype=torch.float64, device=hist.device)
+    _check(L.ecasq_entropy(_ptr(hist), n, s, _ptr(H), _stream()), "ecasq_entropy")
+    return H

@@ -1,0 +1,166 @@
+/*
+ * ecasq.h — C ABI of libecasq.so, the B200 (sm_100a) ECASQ solver.
+ *
+ * ECASQ = entropy-constrained adaptive stochastic quantization, as defined in the
+ * technical summary "Entropy-Constrained Adaptive Stochastic Quantization (ECASQ)"
+ * (gist.science/pt/paper/2608.18147):
+ *   §1   "O Problema ECASQ": for a vector X in R^d, a permissible alphabet P
+ *        (p sorted values), a code size s and an entropy budget b, choose
+ *        Q subset of P with |Q| <= s that minimises the MSE of unbiased stochastic
+ *        rounding onto Q (E[X^] = X) subject to H(X^) <= b bits per entry.
+ *   §2.1 "Relaxação Lagrangiana": minimise MSE(Q,X) + lambda * H(X^); varying
+ *        lambda traces the Pareto curve; two-way time-sharing of two quantizers
+ *        on a random partition of the input reaches any budget b.
+ *   §2.2 "Programação Dinâmica Ótima": the exact DP over the pair state
+ *        dp_OPT(i, l, j) (the entropy of a value depends on both neighbours);
+ *        "Generalização": arbitrary P in O(p^2 s + d) after bucketing X onto P.
+ *
+ * Conventions shared by every entry point
+ *   - Every array argument is DEVICE memory owned by the caller (for example a
+ *     torch tensor), row-major and contiguous, unless marked "host". The
+ *     library allocates nothing: scratch comes from the caller's workspace
+ *     (ecasq_workspace_size), which must stay alive until the stream work ends.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream). The return value is a HOST status for
+ *     argument and launch errors only. Errors found by the device (an entry
+ *     outside [P_0, P_{p-1}], a NaN/Inf, a budget that cannot be met) are
+ *     written per vector to the `status` array, which the caller reads after
+ *     the stream work is done.
+ *   - X is float32 [n][d]; P is float64 [n][p], strictly increasing per row,
+ *     with P_0 <= min X and max X <= P_{p-1}. The solver keeps P_0 and P_{p-1}
+ *     in every code (the uniform grid of ecasq_uniform_grid spans exactly
+ *     [min X, max X], so both ends are forced by unbiasedness there).
+ *   - A code Q is returned as ascending indices into the vector's row of P,
+ *     padded with -1 up to s; Q_len holds |Q|.
+ *   - Limits: 2 <= p <= 512, 2 <= s <= 255 (s > p is treated as s = p),
+ *     1 <= d <= 2^31 - 1, n >= 1.
+ *   - Entropies are in bits per entry; the MSE is the per-entry mean
+ *     (1/d) * sum (q_hi - x)(x - q_lo); the objective is MSE + lambda * H.
+ */
+#ifndef ECASQ_H_
+#define ECASQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Host return codes and per-vector device status codes. */
+#define ECASQ_OK 0
+#define ECASQ_ERR_ARG (-1)       /* bad argument (host), or P not increasing (device) */
+#define ECASQ_ERR_RANGE (-2)     /* device: an entry is NaN/Inf or outside [P_0, P_{p-1}] */
+#define ECASQ_ERR_WORKSPACE (-3) /* host: workspace missing or smaller than required */
+#define ECASQ_ERR_CUDA (-4)      /* host: a CUDA launch or runtime call failed */
+#define ECASQ_WARN_BUDGET 1      /* device: H(lambda_hi) > b; result is the code at lambda_hi */
+
+/* Solver options (host struct, may be NULL for the defaults). */
+typedef struct ecasq_opts {
+  int dp_fp64;      /* 0 (default): DP layer values in fp32 with the MUFU log2;
+                       1: fp64 DP (parity mode). The chosen code is always
+                       re-evaluated in fp64. */
+  int hirschberg;   /* 0 (default): store back-pointers; 1: recompute them
+                       (O(p^2) DP memory per vector, §2.2 "Algoritmo de Hirschberg"). */
+  int bisect_steps; /* lambda bisection steps of ecasq_solve_budget (default 30). */
+  int reserved;     /* must be 0 */
+} ecasq_opts;
+
+/* Bytes of workspace that ecasq_solve / ecasq_solve_budget / ecasq_solve_stats /
+ * ecasq_solve_budget_stats need for these sizes on the CURRENT device
+ * (n_lambda = lambdas per vector; 1 for the budget solver). Returns 0 on bad
+ * arguments. ecasq_bucket and ecasq_uniform_grid need ecasq_aux_workspace_size. */
+size_t ecasq_workspace_size(int n, int64_t d, int p, int s, int n_lambda, const ecasq_opts* opts);
+
+/* Workspace of ecasq_uniform_grid and ecasq_bucket for these sizes. */
+size_t ecasq_aux_workspace_size(int n, int64_t d, int p);
+
+/* Uniform permissible set on each row's range (the alphabet of the workloads
+ * above; §2.2 "Generalização" allows any P): P[r][k] = lo + (hi-lo)*k/(p-1)
+ * in fp64 with lo = min X[r], hi = max X[r], and P[r][p-1] = hi exactly.
+ * status[r] = ECASQ_ERR_RANGE when row r holds a NaN or an infinity. */
+int ecasq_uniform_grid(const float* X, int n, int64_t d, int p, double* P, int32_t* status,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* Bucketing of each row onto its alphabet (the "+d" term of §2.2
+ * "Generalização"): bucket k = max{k <= p-2 : P_k <= x}, so the last bucket is
+ * closed; per bucket the count cnt (int64 [n][p-1]) and the shifted moments
+ * A = sum (x - P_k), B = sum (x - P_k)^2 (float64 [n][p-1]).
+ * status[r] = ECASQ_ERR_RANGE when an entry of row r lies outside [P_0, P_{p-1}]
+ * or is NaN. */
+int ecasq_bucket(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt,
+                 double* A, double* B, int32_t* status, void* ws, size_t ws_bytes, void* stream);
+
+/* Exact Lagrangian solve (§2.1 + §2.2) of every row at n_lambda multipliers:
+ * lambda is [n][n_lambda] (>= 0). For row r and multiplier t the code
+ * Q[(r*n_lambda + t)*s ...] minimises MSE + lambda*H over |Q| <= s with
+ * P_0, P_{p-1} in Q; objective/mse/H [n][n_lambda] are its fp64 values.
+ * Ties: smallest |Q|, then smallest indices. Buckets X internally. */
+int ecasq_solve(const float* X, const double* P, int n, int64_t d, int p, int s,
+                const double* lambda, int n_lambda, int32_t* Q, int32_t* Q_len,
+                double* objective, double* mse, double* H, int32_t* status,
+                const ecasq_opts* opts, void* ws, size_t ws_bytes, void* stream);
+
+/* Same, from bucket statistics produced by ecasq_bucket (cnt, A, B as above). */
+int ecasq_solve_stats(const int64_t* cnt, const double* A, const double* B, const double* P,
+                      int n, int64_t d, int p, int s, const double* lambda, int n_lambda,
+                      int32_t* Q, int32_t* Q_len, double* objective, double* mse, double* H,
+                      int32_t* status, const ecasq_opts* opts, void* ws, size_t ws_bytes,
+                      void* stream);
+
+/* Entropy budget b (§1 constraint, §2.1 time-sharing), per row:
+ * bracket [0, (P_{p-1} - P_0)^2], arithmetic bisection (opts->bisect_steps,
+ * default 30) with "H(mid) > b => lambda_lo = mid". Q1 [n][s] is the code at
+ * the final lambda_lo (H1 > b), Q2 the code at lambda_hi (H2 <= b), and
+ * theta [n] = (b - H2)/(H1 - H2) the share of entries coded with Q1, so that
+ * theta*H1 + (1-theta)*H2 = b. If H at lambda = 0 is already <= b: Q1 = Q2 =
+ * that code, theta = 0. If H(lambda_hi) > b: status = ECASQ_WARN_BUDGET,
+ * Q2 = code at lambda_hi, theta = 0. */
+int ecasq_solve_budget(const float* X, const double* P, int n, int64_t d, int p, int s, double b,
+                       int32_t* Q1, int32_t* Q1_len, int32_t* Q2, int32_t* Q2_len, double* theta,
+                       double* lambda_lo, double* lambda_hi, double* H1, double* H2, double* mse1,
+                       double* mse2, int32_t* status, const ecasq_opts* opts, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/* Same, from bucket statistics. */
+int ecasq_solve_budget_stats(const int64_t* cnt, const double* A, const double* B, const double* P,
+                             int n, int64_t d, int p, int s, double b, int32_t* Q1,
+                             int32_t* Q1_len, int32_t* Q2, int32_t* Q2_len, double* theta,
+                             double* lambda_lo, double* lambda_hi, double* H1, double* H2,
+                             double* mse1, double* mse2, int32_t* status,
+                             const ecasq_opts* opts, void* ws, size_t ws_bytes, void* stream);
+
+/* Unbiased stochastic rounding (§1, E[X^] = X) with optional two-way
+ * time-sharing (§2.1), counter-based randomness Philox4x32-10 (Salmon et al.,
+ * SC'11) keyed by seed (low word, high word), counter (j >> 2, r, stream, 0),
+ * output word j & 3, u = word * 2^-32, for entry j of row r:
+ *   - Q2 == NULL: every entry uses Q1 (part 0).
+ *   - Q2 != NULL, 0 < theta[r] < 1: entry uses Q1 iff u(stream 1) < theta[r],
+ *     else Q2 (part 1); theta >= 1: Q1 only; theta <= 0 (or theta NULL): Q2 only.
+ *   - x in [q_i, q_{i+1}] of its code rounds up iff u(stream 0) <
+ *     (x - q_i)/(q_{i+1} - q_i) in IEEE fp64 (two subtractions, one division).
+ * idx [n][d] uint8 = position of the emitted value in the code used (so s <= 256);
+ * hist [n][2][s] int64 counts per part and position (overwritten).
+ * status[r] = ECASQ_ERR_RANGE for an entry outside its code's range. */
+int ecasq_encode(const float* X, const double* P, int n, int64_t d, int p, int s,
+                 const int32_t* Q1, const int32_t* Q1_len, const int32_t* Q2,
+                 const int32_t* Q2_len, const double* theta, uint64_t seed, uint8_t* idx,
+                 int64_t* hist, int32_t* status, void* stream);
+
+/* Empirical entropy of the emitted indices from hist [n][2][s] (§1, H(X^)):
+ * per part H_part = -sum c/d_part log2(c/d_part), combined as
+ * (d_0 H_0 + d_1 H_1)/(d_0 + d_1). H [n] float64. */
+int ecasq_entropy(const int64_t* hist, int n, int s, double* H, void* stream);
+
+/* Static text for a status code. */
+const char* ecasq_status_string(int code);
+
+/* Number of kernel launches issued by the calling host thread through this
+ * library since the last reset (instrumentation for benchmarks). */
+uint64_t ecasq_launch_count(int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ECASQ_H_ */

@@ -1,0 +1,86 @@
+"""The C-ABI library loads and exports every symbol include/ecasq.h declares.
+CPU only: no call here reaches the GPU (argument checks return before any
+CUDA work)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from entropy_constrained_unbiased_b200 import build, ecasq
+    build.build()
+    return ecasq.load()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "ecasq.h")).read()
+    return sorted(set(re.findall(r"\b(ecasq_[a-z_]+)\s*\(", text)))
+
+
+def test_header_lists_the_binding_exports():
+    from entropy_constrained_unbiased_b200 import ecasq
+    assert declared_symbols() == sorted(ecasq.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in (0, -1, -2, -3, -4, 1):
+        assert lib.ecasq_status_string(code)
+    assert lib.ecasq_status_string(99) == b"unknown status"
+
+
+def test_argument_errors_return_before_cuda(lib):
+    null = C.c_void_p(0)
+    # null input / bad sizes: ECASQ_ERR_ARG
+    assert lib.ecasq_uniform_grid(null, 1, 16, 8, null, null, null, 0, null) == -1
+    assert lib.ecasq_bucket(null, null, 1, 16, 1, null, null, null, null, null, 0, null) == -1
+    assert lib.ecasq_aux_workspace_size(0, 16, 8) == 0
+    assert lib.ecasq_aux_workspace_size(4, 16, 600) == 0
+    assert lib.ecasq_aux_workspace_size(4, 1024, 64) > 0
+    assert lib.ecasq_entropy(null, 1, 4, null, null) == -1
+    assert lib.ecasq_encode(null, null, 1, 16, 8, 4, null, null, null, null, null, 1, null, null, null, null) == -1
+
+
+def test_missing_workspace_is_reported(lib):
+    dummy = C.c_void_p(16)  # never dereferenced: the check fails first
+    assert lib.ecasq_uniform_grid(dummy, 1, 16, 8, dummy, dummy, C.c_void_p(0), 0, C.c_void_p(0)) == -3
+
+
+def test_launch_counter(lib):
+    lib.ecasq_launch_count(1)
+    assert lib.ecasq_launch_count(0) == 0
+
+
+def test_product_path_has_no_cpu_fallback(monkeypatch):
+    from entropy_constrained_unbiased_b200 import ecasq
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    with pytest.raises(ecasq.EcasqError):
+        ecasq.uniform_grid(torch.zeros(1, 8), 4)
+
+
+def test_triple_count_matches_enumeration():
+    """Per-solve triple count (bench metric): every (k, l, j) the recurrence
+    visits, counted directly; layer 2 has only k = 0 because c_1 = P_0."""
+    from bench import triples_per_solve
+    for p, s in [(8, 4), (12, 5), (64, 8), (20, 20), (30, 3), (5, 2)]:
+        S = min(s, p)
+        t = 0
+        for i in range(2, S):
+            for l in range(i - 1, p - 1):
+                ks = [0] if i == 2 else range(i - 2, l)
+                js = [p - 1] if i == S - 1 else range(l + 1, p)
+                t += len(list(ks)) * len(list(js))
+        assert triples_per_solve(p, s) == t
+    assert triples_per_solve(64, 8) == 151347
+    assert triples_per_solve(128, 16) == 3522197
