@@ -165,6 +165,7 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
 
     ev_dp0 = torch.cuda.Event(enable_timing=True)
     ev_dp1 = torch.cuda.Event(enable_timing=True)
+    unit_peaks = measure_unit_peaks()
     for _ in range(args.warmup):
         out, idx, hist, Hemp = step(X)
     torch.cuda.synchronize()
@@ -222,8 +223,8 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
     mufu_peak = MUFU_LG2_PER_CLK_PER_SM * B200_SMS * sm_max * 1e6
     dp_avg_ms = float(np.mean(dp_ms))
     achieved = n_solves * tps / (dp_avg_ms * 1e-3)
-    total_triples = world * n_solves * tps
-    value = total_triples / (t_ms * 1e-3)
+    total_triples = world * n_solves * tps  # one step, all ranks
+    value = total_triples * args.steps / (t_ms * 1e-3)
     line = {
         "metric": "ECASQ DP (k,l,j) triples/s (whole step: grid + bucketing + DP + bisection + encode + entropy)",
         "value": value,
@@ -243,13 +244,33 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
                    "parallelism": f"dp{world} (rows sharded, no collective)"},
         "roofline": {"bound": "alu", "kernel": "k_dp (DP layers + backtrack + bisection)", "achieved": achieved,
                      "peak": mufu_peak, "unit": "triples/s", "frac": achieved / mufu_peak, "traffic": None,
-                     "peak_basis": f"MUFU lg2 {MUFU_LG2_PER_CLK_PER_SM}/clk/SM x {B200_SMS} SMs x {sm_max:.0f} MHz"},
+                     "peak_basis": f"MUFU lg2 {MUFU_LG2_PER_CLK_PER_SM}/clk/SM x {B200_SMS} SMs x {sm_max:.0f} MHz "
+                                   "(1 lg2 per triple)",
+                     "measured_lg2_per_s": unit_peaks.get("lg2"),
+                     "frac_of_measured_lg2": (achieved / unit_peaks["lg2"]) if unit_peaks.get("lg2") else None,
+                     "measured_ffma_per_s": unit_peaks.get("ffma")},
         "e2e": {"value": total_triples / (float(np.mean(e2e_ms)) * 1e-3), "unit": "triples/s",
                 "h2d_bytes_per_step": n * d * 4, "d2h_bytes_per_step": bo},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
     }
     return line
+
+
+def measure_unit_peaks():
+    """MUFU lg2 and FFMA rates of this GPU from the microbenchmark library."""
+    import ctypes
+
+    from entropy_constrained_unbiased_b200 import build
+
+    try:
+        L = ctypes.CDLL(build.PEAKS_LIB)
+    except OSError:
+        return {}
+    L.ecasq_peak_lg2_per_s.restype = ctypes.c_double
+    L.ecasq_peak_ffma_per_s.restype = ctypes.c_double
+    out = {"lg2": L.ecasq_peak_lg2_per_s(), "ffma": L.ecasq_peak_ffma_per_s()}
+    return {k: v for k, v in out.items() if v > 0}
 
 
 def oracle_sample(w: W.Workload, budget_s: float):
@@ -317,8 +338,13 @@ def main():
     ap.add_argument("--fp64", action="store_true", help="fp64 DP layers (parity mode)")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rows", type=int, default=0, help="first rows only (profiling runs; not a bench line)")
     args = ap.parse_args()
     w = W.WORKLOADS[args.workload]
+    if args.rows:
+        import dataclasses
+
+        w = dataclasses.replace(w, n=min(args.rows, w.n))
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -39,13 +39,14 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / kWarp;
-constexpr int kTJ = 2;                  // j values held per lane
-constexpr int kTaskJ = kWarp * kTJ;     // j values per full task
+constexpr int kNQ = 4;  // independent k-streams per output (breaks the min/argmin chain)
 
-__host__ __device__ inline uint32_t pack_task(int l, int j0, int nj, int kslog) {
-  return static_cast<uint32_t>(l) | (static_cast<uint32_t>(j0) << 10) | (static_cast<uint32_t>(nj) << 20) |
-         (static_cast<uint32_t>(kslog) << 28);
+// A pair descriptor names two outputs (l, j0) and (l, j0 + 1) of one layer:
+// l in bits 0..9, j0 in bits 10..19, bit 20 set when (l, j0 + 1) is real.
+__host__ __device__ inline uint32_t pack_pair(int l, int j0, bool two) {
+  return static_cast<uint32_t>(l) | (static_cast<uint32_t>(j0) << 10) | (two ? (1u << 20) : 0u);
 }
+__host__ __device__ inline int max_pairs(int p) { return p * (p / 2 + 1); }
 
 template <typename T>
 struct Arith;
@@ -85,9 +86,9 @@ struct Ctx {
   int* rarg;                  // [p]
   int* ctr;                   // [S] task counters
   int* sQ;                    // [S] code of the last solve
-  const uint32_t* tasks;
-  const int32_t* ntasks;
-  int max_tasks;
+  const uint32_t* pairs;   // [S][max_pairs] pair descriptors per layer
+  const int32_t* npairs;   // [S]
+  int max_pairs;
 };
 
 struct SolveOut {
@@ -157,66 +158,95 @@ __device__ __forceinline__ void finalize_layer(const Ctx<T>& c, int i, const T* 
   }
 }
 
+// One task of layer i >= 3: 32 pair descriptors, one per lane. Lane L owns the
+// outputs (l, j0) and (l, j0+1) and sweeps k = i-2 .. l-1 over kNQ interleaved
+// streams (each keeps its own running minimum, so consecutive updates do not
+// wait on one another); the k range common to the warp runs unpredicated.
 template <typename T>
-__device__ __forceinline__ void run_task(const Ctx<T>& c, uint32_t desc, int i, const T* __restrict__ Gp,
-                                         T* __restrict__ Gc, uint16_t* __restrict__ bpi, T invl) {
+__device__ __forceinline__ void run_task(const Ctx<T>& c, int t, int np, const uint32_t* __restrict__ pl, int i,
+                                         const T* __restrict__ Gp, T* __restrict__ Gc, uint16_t* __restrict__ bpi,
+                                         T invl) {
   const int p = c.p;
-  const int l = desc & 1023;
-  const int j0 = (desc >> 10) & 1023;
-  const int nj = (desc >> 20) & 255;
-  const int kslog = (desc >> 28) & 7;
-  const int KS = 1 << kslog;
-  const int JL = kWarp >> kslog;
   const int lane = lane_id();
-  const int ks = lane & (KS - 1);
-  const int jl = lane >> kslog;
+  const int q = t * kWarp + lane;
   const int kmin = i - 2;
+  const bool active = q < np;
+  const uint32_t desc = active ? pl[q] : 0u;
+  const int l = active ? static_cast<int>(desc & 1023) : kmin;  // inactive lanes sweep nothing
+  const int j0 = static_cast<int>((desc >> 10) & 1023);
+  const bool two = (desc >> 20) & 1u;
+  const int lmin = __reduce_min_sync(0xffffffffu, active ? l : 0x7fffffff);
+  const int lmax = __reduce_max_sync(0xffffffffu, l);
   const T* __restrict__ gcol = Gp + col_off(l);
   const T* __restrict__ acol = c.colA + col_off(l);
   const int ro = row_off(l, p) - l - 1;
-  const int jend = j0 + nj;
+  const T b0 = active ? c.rowB[ro + j0] : T(0);
+  const T b1 = two ? c.rowB[ro + j0 + 1] : T(0);
 
-  T b[kTJ], best[kTJ];
-  int arg[kTJ], jj[kTJ];
+  T best0[kNQ], best1[kNQ];
+  int arg0[kNQ], arg1[kNQ];
 #pragma unroll
-  for (int u = 0; u < kTJ; ++u) {
-    jj[u] = j0 + jl + JL * u;
-    b[u] = (jj[u] < jend) ? c.rowB[ro + jj[u]] : T(0);
-    best[u] = Arith<T>::inf();
-    arg[u] = kmin;
+  for (int s = 0; s < kNQ; ++s) {
+    best0[s] = best1[s] = Arith<T>::inf();
+    arg0[s] = arg1[s] = kmin;
   }
-#pragma unroll 4
-  for (int k = kmin + ks; k < l; k += KS) {
-    const T g = gcol[k];
-    const T av = acol[k];
+  int k = kmin;
+#pragma unroll 1
+  for (; k + kNQ <= lmin; k += kNQ) {
 #pragma unroll
-    for (int u = 0; u < kTJ; ++u) {
-      const T v = Arith<T>::fold(g, av + b[u]);
-      if (v < best[u]) {
-        best[u] = v;
-        arg[u] = k;
+    for (int s = 0; s < kNQ; ++s) {
+      const T g = gcol[k + s];
+      const T av = acol[k + s];
+      const T v0 = Arith<T>::fold(g, av + b0);
+      const T v1 = Arith<T>::fold(g, av + b1);
+      if (v0 < best0[s]) {
+        best0[s] = v0;
+        arg0[s] = k;
+      }
+      if (v1 < best1[s]) {
+        best1[s] = v1;
+        arg1[s] = k;
       }
     }
   }
-  for (int o = 1; o < KS; o <<= 1) {
-#pragma unroll
-    for (int u = 0; u < kTJ; ++u) {
-      const T ov = __shfl_xor_sync(0xffffffffu, best[u], o);
-      const int oa = __shfl_xor_sync(0xffffffffu, arg[u], o);
-      if (ov < best[u] || (ov == best[u] && oa < arg[u])) {
-        best[u] = ov;
-        arg[u] = oa;
+#pragma unroll 1
+  for (; k < lmax; ++k) {
+    if (k < l) {
+      const T g = gcol[k];
+      const T av = acol[k];
+      const T v0 = Arith<T>::fold(g, av + b0);
+      const T v1 = Arith<T>::fold(g, av + b1);
+      if (v0 < best0[0]) {
+        best0[0] = v0;
+        arg0[0] = k;
+      }
+      if (v1 < best1[0]) {
+        best1[0] = v1;
+        arg1[0] = k;
       }
     }
   }
-  if (ks == 0) {
+  // Streams hold base indices; stream s saw k = base + s. Merge with the tie
+  // rule (smaller k wins).
 #pragma unroll
-    for (int u = 0; u < kTJ; ++u) {
-      if (jj[u] < jend) {
-        const int e = ro + jj[u];
-        Gc[col_off(jj[u]) + l] = c.rowV[e] * invl + best[u];
-        bpi[e] = static_cast<uint16_t>(arg[u]);
-      }
+  for (int s = 1; s < kNQ; ++s) {
+    const int k0 = arg0[s] + s, k1 = arg1[s] + s;
+    if (best0[s] < best0[0] || (best0[s] == best0[0] && k0 < arg0[0])) {
+      best0[0] = best0[s];
+      arg0[0] = k0;
+    }
+    if (best1[s] < best1[0] || (best1[s] == best1[0] && k1 < arg1[0])) {
+      best1[0] = best1[s];
+      arg1[0] = k1;
+    }
+  }
+  if (active) {
+    const int e = ro + j0;
+    Gc[col_off(j0) + l] = c.rowV[e] * invl + best0[0];
+    bpi[e] = static_cast<uint16_t>(arg0[0]);
+    if (two) {
+      Gc[col_off(j0 + 1) + l] = c.rowV[e + 1] * invl + best1[0];
+      bpi[e + 1] = static_cast<uint16_t>(arg1[0]);
     }
   }
 }
@@ -300,14 +330,16 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
         }
       }
     } else {
-      const uint32_t* tl = c.tasks + static_cast<size_t>(i) * c.max_tasks;
-      const int nt = c.ntasks[i];
+      // Tasks in descending cost: higher rows have longer k sweeps.
+      const uint32_t* pl = c.pairs + static_cast<size_t>(i) * c.max_pairs;
+      const int np = c.npairs[i];
+      const int nt = (np + kWarp - 1) / kWarp;
       for (;;) {
         int t = 0;
         if (lane == 0) t = atomicAdd(c.ctr + i, 1);
         t = __shfl_sync(0xffffffffu, t, 0);
         if (t >= nt) break;
-        run_task(c, tl[t], i, Gp, Gc, bpi, invl);
+        run_task(c, nt - 1 - t, np, pl, i, Gp, Gc, bpi, invl);
       }
     }
     __syncthreads();
@@ -392,9 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
   c.S = S;
   c.tri = tri;
   c.dd = static_cast<double>(a.d);
-  c.tasks = a.tasks;
-  c.ntasks = a.ntasks;
-  c.max_tasks = a.max_tasks;
+  c.pairs = a.tasks;
+  c.npairs = a.ntasks;
+  c.max_pairs = a.max_tasks;
 
   unsigned char* sp = smem;
   auto carve = [&sp](size_t bytes) {
@@ -561,59 +593,33 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
 }
 
 // ---- schedule ----------------------------------------------------------------
-// Tasks of layer i >= 3 in descending cost (rows taken outward from the
-// costliest one; row cost K * NJ is unimodal in l). Full tasks cover 64 j with
-// one k-lane; the remainder of a row is split over KS k-lanes so that the warp
-// stays busy. One thread per layer.
-__global__ void k_schedule(int p, int S, int max_tasks, uint32_t* tasks, int32_t* ntasks) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= S) return;
+// Pair descriptors of layer i >= 3 in row-major order (rows l = i-1 .. p-2,
+// j ascending; the last layer has only j = p-1). One CTA per layer, one thread
+// per row; a row's first pair index is the sum of the pair counts of the rows
+// before it.
+__global__ void k_schedule(int p, int S, int max_pairs_, uint32_t* pairs, int32_t* npairs) {
+  const int i = blockIdx.x;
   if (i < 3) {
-    ntasks[i] = 0;
+    if (threadIdx.x == 0) npairs[i] = 0;
     return;
   }
   const bool last = (i == S - 1);
-  const int kmin = i - 2;
-  const int r0 = i - 1, r1 = p - 2;
-  auto cost = [&](int l) -> long long {
-    const long long K = l - kmin;
-    const long long NJ = last ? 1 : (p - 1 - l);
-    return K * NJ;
-  };
-  uint32_t* out = tasks + static_cast<size_t>(i) * max_tasks;
-  int n = 0;
-  auto emit = [&](int l) {
-    const int K = l - kmin;
-    const int NJ = last ? 1 : (p - 1 - l);
-    const int j0 = last ? p - 1 : l + 1;
-    const int nfull = NJ / kTaskJ;
-    for (int f = 0; f < nfull; ++f) out[n++] = pack_task(l, j0 + f * kTaskJ, kTaskJ, 0);
-    const int rem = NJ - nfull * kTaskJ;
-    if (rem > 0) {
-      const int need = (rem + kTJ - 1) / kTJ;  // j-lanes needed
-      int jl = 1;
-      while (jl < need) jl <<= 1;
-      int ks = kWarp / jl;
-      while (ks > 1 && ks > K) ks >>= 1;
-      int kslog = 0;
-      while ((1 << kslog) < ks) ++kslog;
-      out[n++] = pack_task(l, j0 + nfull * kTaskJ, rem, kslog);
-    }
-  };
-  if (r0 <= r1) {
-    int pk = r0;
-    for (int l = r0; l <= r1; ++l)
-      if (cost(l) > cost(pk)) pk = l;
-    emit(pk);
-    int lo = pk - 1, hi = pk + 1;
-    while (lo >= r0 || hi <= r1) {
-      if (hi > r1 || (lo >= r0 && cost(lo) >= cost(hi)))
-        emit(lo--);
-      else
-        emit(hi++);
+  auto row_pairs = [&](int l) { return last ? 1 : (p - l) / 2; };  // ceil((p-1-l)/2)
+  uint32_t* out = pairs + static_cast<size_t>(i) * max_pairs_;
+  for (int l = i - 1 + threadIdx.x; l <= p - 2; l += blockDim.x) {
+    int o = 0;
+    for (int r = i - 1; r < l; ++r) o += row_pairs(r);
+    if (last) {
+      out[o] = pack_pair(l, p - 1, false);
+    } else {
+      for (int j = l + 1; j <= p - 1; j += 2) out[o++] = pack_pair(l, j, j + 1 <= p - 1);
     }
   }
-  ntasks[i] = n;
+  if (threadIdx.x == 0) {
+    int tot = 0;
+    for (int r = i - 1; r <= p - 2; ++r) tot += row_pairs(r);
+    npairs[i] = tot;
+  }
 }
 
 template <typename T, bool kSmem>
@@ -646,8 +652,8 @@ int64_t dp_triples(int p, int s) {
 
 size_t dp_schedule_bytes(int p, int s) {
   const int S = s < p ? s : p;
-  const size_t max_tasks = static_cast<size_t>(p) * ((p + kTaskJ - 1) / kTaskJ + 1);
-  return ((sizeof(uint32_t) * max_tasks * S + 255) & ~size_t(255)) + ((sizeof(int32_t) * S + 255) & ~size_t(255));
+  return ((sizeof(uint32_t) * static_cast<size_t>(max_pairs(p)) * S + 255) & ~size_t(255)) +
+         ((sizeof(int32_t) * S + 255) & ~size_t(255));
 }
 
 bool dp_plan(int n, int p, int s, bool fp64, DpPlan* plan) {
@@ -667,7 +673,7 @@ bool dp_plan(int n, int p, int s, bool fp64, DpPlan* plan) {
   plan->smem_bytes = small + (plan->smem_tables ? big : 0);
   const size_t bp = (sizeof(uint16_t) * static_cast<size_t>(S) * tri_size(p) + 255) & ~size_t(255);
   plan->scratch_per_cta = (bp + (plan->smem_tables ? 0 : big) + 255) & ~size_t(255);
-  plan->max_tasks = p * ((p + kTaskJ - 1) / kTaskJ + 1);
+  plan->max_tasks = max_pairs(p);
   void* fn = fp64 ? (plan->smem_tables ? dp_kernel_ptr<double, true>() : dp_kernel_ptr<double, false>())
                   : (plan->smem_tables ? dp_kernel_ptr<float, true>() : dp_kernel_ptr<float, false>());
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(plan->smem_bytes)) !=
@@ -687,7 +693,7 @@ cudaError_t launch_dp(const DpPlan& plan, DpArgs args, uint32_t* tasks, int32_t*
   args.tasks = tasks;
   args.ntasks = ntasks;
   args.max_tasks = plan.max_tasks;
-  k_schedule<<<(S + 63) / 64, 64, 0, st>>>(args.p, S, plan.max_tasks, tasks, ntasks);
+  k_schedule<<<S, 128, 0, st>>>(args.p, S, plan.max_tasks, tasks, ntasks);
   note_launch();
   void* fn = plan.fp64 ? (plan.smem_tables ? dp_kernel_ptr<double, true>() : dp_kernel_ptr<double, false>())
                        : (plan.smem_tables ? dp_kernel_ptr<float, true>() : dp_kernel_ptr<float, false>());
