@@ -59,6 +59,7 @@ struct Arith<float> {
   __device__ static float inf() { return __int_as_float(0x7f800000); }
   __device__ static float nlog(float m) { return -m * lg2_approx(m); }
   __device__ static float fold(float g, float m) { return fmaf(-m, lg2_approx(m), g); }
+  __device__ static float vmin(float a, float b) { return fminf(a, b); }
 };
 
 template <>
@@ -67,19 +68,34 @@ struct Arith<double> {
   __device__ static double inf() { return __longlong_as_double(0x7ff0000000000000ll); }
   __device__ static double nlog(double m) { return m > 0.0 ? -m * log2(m) : 0.0; }
   __device__ static double fold(double g, double m) { return m > 0.0 ? fma(-m, log2(m), g) : g; }
+  __device__ static double vmin(double a, double b) { return fmin(a, b); }
 };
+
+// One entry of a live DP layer: the layer value G = F_{i-1}(k, l) and
+// a = R(k, l)/d + eps side by side, so one 8- (16-) byte shared load feeds a
+// whole k step. a is written once per vector into both ping-pong layers.
+template <typename T>
+struct alignas(2 * sizeof(T)) GA {
+  T g, a;
+};
+
+// Every pair table uses the row-triangle layout: entry (k, l), k < l, sits at
+// tix(k, l) = row_off(k) + l - k - 1. In the k sweep the lanes of a warp read
+// row k at their own columns l, which are equal or consecutive, so the loads
+// are broadcasts or conflict-free; the outputs (l, j) of a task are
+// consecutive too.
+__host__ __device__ __forceinline__ int tix(int k, int l, int p) { return row_off(k, p) + l - k - 1; }
 
 template <typename T>
 struct Ctx {
   int p, S, tri;
   double dd;
-  T* colG0;  // DP layers (even / odd i), column layout (entry (k,l) at col_off(l)+k)
-  T* colG1;
-  __device__ __forceinline__ T* layer(int i) const { return (i & 1) ? colG1 : colG0; }
-  T* colA;     // R(k,l)/d + eps, column layout
-  T* rowB;     // L(l,j)/d, row layout
-  T* rowV;     // V(l,j)/d, row layout
-  uint16_t* bp;  // [S][tri] back-pointers, row layout
+  GA<T>* ga0;  // DP layers of even / odd i (with a)
+  GA<T>* ga1;
+  __device__ __forceinline__ GA<T>* layer(int i) const { return (i & 1) ? ga1 : ga0; }
+  T* rowB;     // L(l,j)/d
+  T* rowV;     // V(l,j)/d
+  uint16_t* bp;  // [S][tri] back-pointers
   double *sP, *sN, *sA, *sB;  // [p] alphabet and bucket statistics
   double *sR, *sL;            // [S] evaluation scratch
   T* rmin;                    // [p] row minima (lambda = 0)
@@ -122,7 +138,9 @@ __device__ __forceinline__ void build_tables(const Ctx<T>& c) {
       const double R = T1 / W;
       double L = N - R;
       L = L > 0.0 ? L : 0.0;
-      c.colA[col_off(cc) + a] = static_cast<T>(R / c.dd) + Arith<T>::kEps;
+      const T av = static_cast<T>(R / c.dd) + Arith<T>::kEps;
+      c.ga0[ro + cc].a = av;
+      c.ga1[ro + cc].a = av;
       c.rowB[ro + cc] = static_cast<T>(L / c.dd);
       c.rowV[ro + cc] = static_cast<T>(V / c.dd);
     }
@@ -134,17 +152,17 @@ __device__ __forceinline__ void build_tables(const Ctx<T>& c) {
 // Best (E, i, k) over the finished layer i: E = F_i(k, p-1) + h(R(k,p-1)/d).
 // Warp 0 only. Strict '<' over layers in ascending order keeps the smaller code.
 template <typename T>
-__device__ __forceinline__ void finalize_layer(const Ctx<T>& c, int i, const T* G, bool sep, T* bestE, int* bestI,
-                               int* bestK) {
+__device__ __forceinline__ void finalize_layer(const Ctx<T>& c, int i, const GA<T>* G, bool sep, T* bestE,
+                                               int* bestI, int* bestK) {
   const int p = c.p;
   const int kb = (i == 1) ? 0 : i - 1;
   const int ke = (i == 1) ? 0 : p - 2;
   T best = Arith<T>::inf();
   int arg = 0x7fffffff;
-  const int co = col_off(p - 1);
   for (int k = kb + lane_id(); k <= ke; k += kWarp) {
-    T e = G[co + k];
-    if (!sep) e += Arith<T>::nlog(c.colA[co + k]);
+    const GA<T> ga = G[tix(k, p - 1, p)];
+    T e = ga.g;
+    if (!sep) e += Arith<T>::nlog(ga.a);
     if (e < best) {
       best = e;
       arg = k;
@@ -163,22 +181,16 @@ __device__ __forceinline__ void finalize_layer(const Ctx<T>& c, int i, const T* 
 // streams (each keeps its own running minimum, so consecutive updates do not
 // wait on one another); the k range common to the warp runs unpredicated.
 template <typename T>
-__device__ __forceinline__ void run_task(const Ctx<T>& c, int t, int np, const uint32_t* __restrict__ pl, int i,
-                                         const T* __restrict__ Gp, T* __restrict__ Gc, uint16_t* __restrict__ bpi,
-                                         T invl) {
+__device__ __forceinline__ void run_task(const Ctx<T>& c, uint32_t desc, bool active, int i,
+                                         const GA<T>* __restrict__ Gp, GA<T>* __restrict__ Gc,
+                                         uint16_t* __restrict__ bpi, T invl) {
   const int p = c.p;
-  const int lane = lane_id();
-  const int q = t * kWarp + lane;
   const int kmin = i - 2;
-  const bool active = q < np;
-  const uint32_t desc = active ? pl[q] : 0u;
-  const int l = active ? static_cast<int>(desc & 1023) : kmin;  // inactive lanes sweep nothing
+  const int l = active ? static_cast<int>(desc & 1023) : kmin + 1;  // inactive lanes: any in-range row
   const int j0 = static_cast<int>((desc >> 10) & 1023);
-  const bool two = (desc >> 20) & 1u;
+  const bool two = active && ((desc >> 20) & 1u);
   const int lmin = __reduce_min_sync(0xffffffffu, active ? l : 0x7fffffff);
-  const int lmax = __reduce_max_sync(0xffffffffu, l);
-  const T* __restrict__ gcol = Gp + col_off(l);
-  const T* __restrict__ acol = c.colA + col_off(l);
+  const int lmax = __reduce_max_sync(0xffffffffu, active ? l : 0);
   const int ro = row_off(l, p) - l - 1;
   const T b0 = active ? c.rowB[ro + j0] : T(0);
   const T b1 = two ? c.rowB[ro + j0 + 1] : T(0);
@@ -190,32 +202,33 @@ __device__ __forceinline__ void run_task(const Ctx<T>& c, int t, int np, const u
     best0[s] = best1[s] = Arith<T>::inf();
     arg0[s] = arg1[s] = kmin;
   }
+  // Row k of the layer starts at row_off(k) - k - 1 (+ l); the start moves by
+  // p - 2 - k from row k to row k + 1.
+  int base = row_off(kmin, p) - kmin - 1;
   int k = kmin;
 #pragma unroll 1
   for (; k + kNQ <= lmin; k += kNQ) {
 #pragma unroll
     for (int s = 0; s < kNQ; ++s) {
-      const T g = gcol[k + s];
-      const T av = acol[k + s];
-      const T v0 = Arith<T>::fold(g, av + b0);
-      const T v1 = Arith<T>::fold(g, av + b1);
-      if (v0 < best0[s]) {
-        best0[s] = v0;
-        arg0[s] = k;
-      }
-      if (v1 < best1[s]) {
-        best1[s] = v1;
-        arg1[s] = k;
-      }
+      const GA<T> ga = Gp[base + l];
+      base += p - 2 - (k + s);
+      const T v0 = Arith<T>::fold(ga.g, ga.a + b0);
+      const T v1 = Arith<T>::fold(ga.g, ga.a + b1);
+      // The running minimum is one min op per step; the argmin follows it.
+      const bool lt0 = v0 < best0[s];
+      const bool lt1 = v1 < best1[s];
+      best0[s] = Arith<T>::vmin(best0[s], v0);
+      best1[s] = Arith<T>::vmin(best1[s], v1);
+      arg0[s] = lt0 ? k : arg0[s];
+      arg1[s] = lt1 ? k : arg1[s];
     }
   }
 #pragma unroll 1
   for (; k < lmax; ++k) {
     if (k < l) {
-      const T g = gcol[k];
-      const T av = acol[k];
-      const T v0 = Arith<T>::fold(g, av + b0);
-      const T v1 = Arith<T>::fold(g, av + b1);
+      const GA<T> ga = Gp[base + l];
+      const T v0 = Arith<T>::fold(ga.g, ga.a + b0);
+      const T v1 = Arith<T>::fold(ga.g, ga.a + b1);
       if (v0 < best0[0]) {
         best0[0] = v0;
         arg0[0] = k;
@@ -225,6 +238,7 @@ __device__ __forceinline__ void run_task(const Ctx<T>& c, int t, int np, const u
         arg1[0] = k;
       }
     }
+    base += p - 2 - k;
   }
   // Streams hold base indices; stream s saw k = base + s. Merge with the tie
   // rule (smaller k wins).
@@ -242,10 +256,10 @@ __device__ __forceinline__ void run_task(const Ctx<T>& c, int t, int np, const u
   }
   if (active) {
     const int e = ro + j0;
-    Gc[col_off(j0) + l] = c.rowV[e] * invl + best0[0];
+    Gc[e].g = c.rowV[e] * invl + best0[0];
     bpi[e] = static_cast<uint16_t>(arg0[0]);
     if (two) {
-      Gc[col_off(j0 + 1) + l] = c.rowV[e + 1] * invl + best1[0];
+      Gc[e + 1].g = c.rowV[e + 1] * invl + best1[0];
       bpi[e + 1] = static_cast<uint16_t>(arg1[0]);
     }
   }
@@ -271,33 +285,32 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
     out->bestI = -1;
     out->bestK = -1;
   }
-  // Layer 1: F_1(0, j), written to buffer 1.
+  // Layer 1: F_1(0, j) (row 0), written to buffer 1.
   {
-    T* G1 = c.colG1;
+    GA<T>* G1 = c.ga1;
     for (int j = 1 + tid; j < p; j += blockDim.x) {
-      const int e = j - 1;  // row 0
+      const int e = j - 1;
       T f = c.rowV[e] * invl;
       if (!sep) f += Arith<T>::nlog(c.rowB[e] + Arith<T>::kEps);
-      G1[col_off(j)] = f;
+      G1[e].g = f;
     }
   }
   __syncthreads();
   for (int i = 2; i <= S - 1; ++i) {
-    const T* Gp = c.layer(i - 1);
-    T* Gc = c.layer(i);
+    const GA<T>* Gp = c.layer(i - 1);
+    GA<T>* Gc = c.layer(i);
     uint16_t* bpi = c.bp + static_cast<size_t>(i) * tri;
     const bool last = (i == S - 1);
     if (warp == 0) finalize_layer(c, i - 1, Gp, sep, bestE, &out->bestI, &out->bestK);
     if (i == 2) {
       // Only k = c_1 = 0 precedes the second value.
       for (int l = 1 + warp; l <= p - 2; l += kWarps) {
-        const T g0 = Gp[col_off(l)];
-        const T a0 = c.colA[col_off(l)];
+        const GA<T> ga = Gp[l - 1];  // (0, l)
         const int ro = row_off(l, p) - l - 1;
         for (int j = (last ? p - 1 : l + 1) + lane; j <= p - 1; j += kWarp) {
           const int e = ro + j;
-          const T v = sep ? g0 : Arith<T>::fold(g0, a0 + c.rowB[e]);
-          Gc[col_off(j) + l] = c.rowV[e] * invl + v;
+          const T v = sep ? ga.g : Arith<T>::fold(ga.g, ga.a + c.rowB[e]);
+          Gc[e].g = c.rowV[e] * invl + v;
         }
       }
     } else if (sep) {
@@ -306,7 +319,7 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
         T best = Arith<T>::inf();
         int arg = kmin;
         for (int k = kmin + lane; k < l; k += kWarp) {
-          const T v = Gp[col_off(l) + k];
+          const T v = Gp[tix(k, l, p)].g;
           if (v < best) {
             best = v;
             arg = k;
@@ -325,7 +338,7 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
         const uint16_t ra = static_cast<uint16_t>(c.rarg[l]);
         for (int j = (last ? p - 1 : l + 1) + lane; j <= p - 1; j += kWarp) {
           const int e = ro + j;
-          Gc[col_off(j) + l] = c.rowV[e] + rm;
+          Gc[e].g = c.rowV[e] + rm;
           bpi[e] = ra;
         }
       }
@@ -334,12 +347,29 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
       const uint32_t* pl = c.pairs + static_cast<size_t>(i) * c.max_pairs;
       const int np = c.npairs[i];
       const int nt = (np + kWarp - 1) / kWarp;
-      for (;;) {
-        int t = 0;
-        if (lane == 0) t = atomicAdd(c.ctr + i, 1);
-        t = __shfl_sync(0xffffffffu, t, 0);
-        if (t >= nt) break;
-        run_task(c, nt - 1 - t, np, pl, i, Gp, Gc, bpi, invl);
+      // The next task's index and descriptor are fetched before the current
+      // task runs, so their latency hides behind the sweep.
+      auto fetch = [&](int& t, uint32_t& d, bool& act) {
+        int tt = 0;
+        if (lane == 0) tt = atomicAdd(c.ctr + i, 1);
+        t = __shfl_sync(0xffffffffu, tt, 0);
+        const int q = (nt - 1 - t) * kWarp + lane;
+        act = (t < nt) && q < np;
+        d = act ? pl[q] : 0u;
+      };
+      int t;
+      uint32_t d;
+      bool act;
+      fetch(t, d, act);
+      while (t < nt) {
+        int tn;
+        uint32_t dn;
+        bool an;
+        fetch(tn, dn, an);
+        run_task(c, d, act, i, Gp, Gc, bpi, invl);
+        t = tn;
+        d = dn;
+        act = an;
       }
     }
     __syncthreads();
@@ -452,11 +482,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
   gs += (sizeof(uint16_t) * static_cast<size_t>(S) * tri + 255) & ~size_t(255);
   const size_t tb = (sizeof(T) * static_cast<size_t>(tri) + 15) & ~size_t(15);
   unsigned char* big = kSmemTables ? sp : gs;
-  c.colG0 = reinterpret_cast<T*>(big);
-  c.colG1 = reinterpret_cast<T*>(big + tb);
-  c.colA = reinterpret_cast<T*>(big + 2 * tb);
-  c.rowB = reinterpret_cast<T*>(big + 3 * tb);
-  c.rowV = reinterpret_cast<T*>(big + 4 * tb);
+  c.ga0 = reinterpret_cast<GA<T>*>(big);
+  c.ga1 = reinterpret_cast<GA<T>*>(big + 2 * tb);
+  c.rowB = reinterpret_cast<T*>(big + 4 * tb);
+  c.rowV = reinterpret_cast<T*>(big + 5 * tb);
 
   const int s_out_stride = a.s_out;
   for (int r = blockIdx.x; r < a.n; r += gridDim.x) {
@@ -632,7 +661,7 @@ size_t small_smem(int p, int S, size_t tsz) {
   return al(8 * p) * 4 + al(8 * S) * 2 + al(tsz * p) + al(4 * p) + al(4 * S) * 4;
 }
 
-size_t table_bytes(int p, size_t tsz) { return ((tsz * tri_size(p) + 15) & ~size_t(15)) * 5; }
+size_t table_bytes(int p, size_t tsz) { return ((tsz * tri_size(p) + 15) & ~size_t(15)) * 6; }
 
 }  // namespace
 

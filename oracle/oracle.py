@@ -218,3 +218,25 @@ def encode_batch(X, P, Q1, m1, s, seed, Q2=None, m2=None, theta=None):
     lib().eo_encode_batch(X, n, d, P, p, Q1, m1, q2p, m2p, thp, s, C.c_uint64(seed), idx, hist, st)
     del keep
     return idx, hist, st
+
+
+def encode_row(x, P_row, Q1, m1, s, seed, row, Q2=None, m2=0, theta=0.0):
+    """Encode one vector that is row `row` of its batch (the Philox counter
+    carries the row index). Returns idx [d] u8 and hist [2, s]."""
+    L = lib()
+    fn = L.eo_encode
+    fn.restype = C.c_int
+    fn.argtypes = [C.c_void_p, C.c_int64, C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_int,
+                   C.c_double, C.c_int, C.c_uint64, C.c_uint32, C.c_void_p, C.c_void_p]
+    x = _f32(x).ravel()
+    P_row = _f64(P_row).ravel()
+    q1 = np.ascontiguousarray(Q1, np.int32).ravel()
+    q2 = np.ascontiguousarray(Q2, np.int32).ravel() if Q2 is not None else None
+    idx = np.zeros(x.size, np.uint8)
+    hist = np.zeros(2 * s, np.int64)
+    st = fn(x.ctypes.data, x.size, P_row.ctypes.data, P_row.size, q1.ctypes.data, int(m1),
+            q2.ctypes.data if q2 is not None else None, int(m2), float(theta), s, C.c_uint64(seed), row,
+            idx.ctypes.data, hist.ctypes.data)
+    if st:
+        raise ValueError("oracle encode failed")
+    return idx, hist.reshape(2, s)
