@@ -129,6 +129,13 @@ int ecasq_bucket(const float* X, const double* P, int n, int64_t d, int p, int64
   return cuda_status(launch_bucket(X, P, n, d, p, cnt, A, B, status, acc, flag, static_cast<cudaStream_t>(stream)));
 }
 
+int ecasq_bucket_noalloc(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt, double* A,
+                         double* B, int32_t* status, void* stream) {
+  if (!X || !P || !cnt || !A || !B || !status || !valid_sizes(n, d, p, 2)) return ECASQ_ERR_ARG;
+  if (bucket_noalloc_bytes(n, p) > bucket_noalloc_capacity()) return ECASQ_ERR_WORKSPACE;
+  return cuda_status(launch_bucket_noalloc(X, P, n, d, p, cnt, A, B, status, static_cast<cudaStream_t>(stream)));
+}
+
 static int solve_common(const float* X, const int64_t* cnt, const double* A, const double* B, const double* P, int n,
                         int64_t d, int p, int s, int n_lambda, const ecasq_opts* opts, void* ws, size_t ws_bytes,
                         cudaStream_t st, DpArgs* args, DpPlan* plan, SolveWs* w) {

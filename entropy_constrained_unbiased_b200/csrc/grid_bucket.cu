@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -287,6 +288,62 @@ cudaError_t launch_bucket(const float* X, const double* P, int n, int64_t d, int
   k_bucket_finish<<<n, 256, 0, st>>>(acc, P, p, fb, flag, cnt, A, B, status);
   note_launch();
   return cudaGetLastError();
+}
+
+}  // namespace ecasq
+
+// ---------------------------------------------------------------------------
+// Bucketing for callers that cannot allocate device memory (see
+// ecasq_bucket_noalloc in include/ecasq.h). The accumulators live in a fixed
+// array in this module's device memory instead of a caller workspace. Every
+// GPU that loads the library holds this array until the process exits; all
+// calls on a device share it, so calls that overlap on that GPU race.
+
+namespace ecasq {
+
+namespace {
+constexpr size_t kNoallocScratchBytes = size_t(8) << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
+}  // namespace
+
+size_t bucket_noalloc_bytes(int n, int p) {
+  return round256(sizeof(unsigned long long) * 3 * static_cast<size_t>(n) * (p - 1)) +
+         round256(sizeof(int32_t) * static_cast<size_t>(n));
+}
+
+size_t bucket_noalloc_capacity() { return kNoallocScratchBytes; }
+
+cudaError_t launch_bucket_noalloc(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt, double* A,
+                                  double* B, int32_t* status, cudaStream_t st) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  void* base = nullptr;
+  {
+    // Host code cannot use the array's name as a device address: resolve it
+    // once per device, with that device current.
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* ptr = nullptr;
+      e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+      if (e != cudaSuccess) return e;
+      g_noalloc_ptr[dev] = ptr;
+    }
+    base = g_noalloc_ptr[dev];
+  }
+  unsigned char* b = static_cast<unsigned char*>(base);
+  auto* acc = reinterpret_cast<unsigned long long*>(b);
+  auto* flag = reinterpret_cast<int32_t*>(b + round256(sizeof(unsigned long long) * 3 * static_cast<size_t>(n) * (p - 1)));
+  // launch_bucket clears the accumulators and flags on the stream before use,
+  // so nothing carries over from the previous call.
+  return launch_bucket(X, P, n, d, p, cnt, A, B, status, acc, flag, st);
 }
 
 }  // namespace ecasq

@@ -22,6 +22,11 @@ cudaError_t launch_bucket(const float* X, const double* P, int n, int64_t d, int
                           double* A, double* B, int32_t* status, unsigned long long* acc,
                           int32_t* flag, cudaStream_t st);
 
+size_t bucket_noalloc_bytes(int n, int p);
+size_t bucket_noalloc_capacity();
+cudaError_t launch_bucket_noalloc(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt,
+                                  double* A, double* B, int32_t* status, cudaStream_t st);
+
 // ---- DP solver (dp.cu) ----
 struct DpArgs {
   // bucket statistics [n][p-1] and alphabet [n][p]

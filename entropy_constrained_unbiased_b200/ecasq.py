@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libecasq.so")
 OK, ERR_ARG, ERR_RANGE, ERR_WORKSPACE, ERR_CUDA, WARN_BUDGET = 0, -1, -2, -3, -4, 1
 
 EXPORTS = [
-    "ecasq_workspace_size", "ecasq_aux_workspace_size", "ecasq_uniform_grid", "ecasq_bucket",
+    "ecasq_workspace_size", "ecasq_aux_workspace_size", "ecasq_uniform_grid", "ecasq_bucket", "ecasq_bucket_noalloc",
     "ecasq_solve", "ecasq_solve_stats", "ecasq_solve_budget", "ecasq_solve_budget_stats",
     "ecasq_encode", "ecasq_entropy", "ecasq_status_string", "ecasq_launch_count",
 ]
@@ -50,6 +50,7 @@ def load(path: str = LIB_PATH):
         "ecasq_aux_workspace_size": (SZ, [I, I64, I]),
         "ecasq_uniform_grid": (I, [P, I, I64, I, P, P, P, SZ, P]),
         "ecasq_bucket": (I, [P, P, I, I64, I, P, P, P, P, P, SZ, P]),
+        "ecasq_bucket_noalloc": (I, [P, P, I, I64, I, P, P, P, P, P]),
         "ecasq_solve": (I, [P, P, I, I64, I, I, P, I, P, P, P, P, P, P, OP, P, SZ, P]),
         "ecasq_solve_stats": (I, [P, P, P, P, I, I64, I, I, P, I, P, P, P, P, P, P, OP, P, SZ, P]),
         "ecasq_solve_budget": (I, [P, P, I, I64, I, I, D] + [P] * 12 + [OP, P, SZ, P]),
@@ -139,6 +140,24 @@ def bucket(X: torch.Tensor, P: torch.Tensor):
     ws = workspace(L.ecasq_aux_workspace_size(n, d, p), X.device)
     _check(L.ecasq_bucket(_ptr(X), _ptr(P), n, d, p, _ptr(cnt), _ptr(A), _ptr(B), _ptr(st), _ptr(ws), ws.numel(),
                           _stream()), "ecasq_bucket")
+    return cnt, A, B, st
+
+
+def bucket_noalloc(X: torch.Tensor, P: torch.Tensor):
+    """ecasq_bucket through the workspace-free entry point: the library uses its
+    own fixed device array instead of a workspace (for callers that cannot
+    allocate device memory; calls on one GPU must not overlap)."""
+    L = _need_cuda()
+    _dev(X, torch.float32, "X")
+    _dev(P, torch.float64, "P")
+    n, d = X.shape
+    p = P.shape[1]
+    cnt = torch.empty((n, p - 1), dtype=torch.int64, device=X.device)
+    A = torch.empty((n, p - 1), dtype=torch.float64, device=X.device)
+    B = torch.empty_like(A)
+    st = torch.empty(n, dtype=torch.int32, device=X.device)
+    _check(L.ecasq_bucket_noalloc(_ptr(X), _ptr(P), n, d, p, _ptr(cnt), _ptr(A), _ptr(B), _ptr(st), _stream()),
+           "ecasq_bucket_noalloc")
     return cnt, A, B, st
 
 

@@ -91,6 +91,25 @@ int ecasq_uniform_grid(const float* X, int n, int64_t d, int p, double* P, int32
 int ecasq_bucket(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt,
                  double* A, double* B, int32_t* status, void* ws, size_t ws_bytes, void* stream);
 
+/* ecasq_bucket without a workspace, for callers that cannot allocate device
+ * memory where they bucket: plugins inside a framework whose own caching
+ * allocator owns all device memory, and fixed-budget real-time or embedded
+ * pipelines that forbid cudaMalloc after start-up (it can synchronise the
+ * device and can fail under fragmentation). The ECASQ page has no counterpart;
+ * this is an interface convenience around the same bucketing kernels.
+ * Outputs, layout and status are those of ecasq_bucket.
+ * Scratch: a fixed 8 MiB array in the library's device memory, held by every
+ * GPU that loads the library until the process exits. It must hold
+ * 24*n*(p-1) + 4*n bytes (each term rounded up to 256), e.g. n <= 2750 rows at
+ * p = 128 or n <= 1369 at p = 256; larger sizes return ECASQ_ERR_WORKSPACE
+ * and launch nothing. The call allocates nothing: the first call on a device
+ * resolves the array's device address (with that device current), so make
+ * that first call before any stream capture. Every call on a device shares
+ * the array (the call clears it on the stream before use): calls that overlap
+ * on the same GPU race, so serialise them (one stream, or events). */
+int ecasq_bucket_noalloc(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt,
+                         double* A, double* B, int32_t* status, void* stream);
+
 /* Exact Lagrangian solve (§2.1 + §2.2) of every row at n_lambda multipliers:
  * lambda is [n][n_lambda] (>= 0). For row r and multiplier t the code
  * Q[(r*n_lambda + t)*s ...] minimises MSE + lambda*H over |Q| <= s with
