@@ -79,19 +79,34 @@ struct alignas(2 * sizeof(T)) GA {
   T g, a;
 };
 
-// Every pair table uses the row-triangle layout: entry (k, l), k < l, sits at
-// tix(k, l) = row_off(k) + l - k - 1. In the k sweep the lanes of a warp read
-// row k at their own columns l, which are equal or consecutive, so the loads
-// are broadcasts or conflict-free; the outputs (l, j) of a task are
-// consecutive too.
+// Layouts. The live DP layers (with a) are stored by COLUMN: entry (k, l),
+// k < l, sits at cb[l] + k, so a lane sweeping k for its row l walks
+// consecutive addresses (one pointer, immediate offsets). Column starts are
+// padded so that cb[l] = l (mod 16): lanes that hold 16 consecutive rows l
+// then read 16 distinct 8-byte bank pairs at every k. b = L/d and V/d are read
+// once per output and stay in the row-triangle layout tix(l, j).
 __host__ __device__ __forceinline__ int tix(int k, int l, int p) { return row_off(k, p) + l - k - 1; }
+
+// cb[0..p]: padded column starts; cb[p] = elements of one layer buffer.
+__host__ __device__ inline int next_colbase(int prev_base, int prev_col) {
+  int c = prev_base + prev_col;  // column prev_col holds prev_col entries
+  const int want = (prev_col + 1) & 15;
+  c += (want - (c & 15) + 16) & 15;
+  return c;
+}
+__host__ __device__ inline int layer_elems(int p) {
+  int c = 0;
+  for (int l = 0; l < p; ++l) c = next_colbase(c, l);
+  return c;
+}
 
 template <typename T>
 struct Ctx {
   int p, S, tri;
   double dd;
-  GA<T>* ga0;  // DP layers of even / odd i (with a)
+  GA<T>* ga0;  // DP layers of even / odd i (with a), column layout
   GA<T>* ga1;
+  const int* cb;  // [p+1] padded column starts (shared memory)
   __device__ __forceinline__ GA<T>* layer(int i) const { return (i & 1) ? ga1 : ga0; }
   T* rowB;     // L(l,j)/d
   T* rowV;     // V(l,j)/d
@@ -139,8 +154,8 @@ __device__ __forceinline__ void build_tables(const Ctx<T>& c) {
       double L = N - R;
       L = L > 0.0 ? L : 0.0;
       const T av = static_cast<T>(R / c.dd) + Arith<T>::kEps;
-      c.ga0[ro + cc].a = av;
-      c.ga1[ro + cc].a = av;
+      c.ga0[c.cb[cc] + a].a = av;
+      c.ga1[c.cb[cc] + a].a = av;
       c.rowB[ro + cc] = static_cast<T>(L / c.dd);
       c.rowV[ro + cc] = static_cast<T>(V / c.dd);
     }
@@ -159,8 +174,9 @@ __device__ __forceinline__ void finalize_layer(const Ctx<T>& c, int i, const GA<
   const int ke = (i == 1) ? 0 : p - 2;
   T best = Arith<T>::inf();
   int arg = 0x7fffffff;
+  const GA<T>* col = G + c.cb[p - 1];
   for (int k = kb + lane_id(); k <= ke; k += kWarp) {
-    const GA<T> ga = G[tix(k, p - 1, p)];
+    const GA<T> ga = col[k];
     T e = ga.g;
     if (!sep) e += Arith<T>::nlog(ga.a);
     if (e < best) {
@@ -194,6 +210,7 @@ __device__ __forceinline__ void run_task(const Ctx<T>& c, uint32_t desc, bool ac
   const int ro = row_off(l, p) - l - 1;
   const T b0 = active ? c.rowB[ro + j0] : T(0);
   const T b1 = two ? c.rowB[ro + j0 + 1] : T(0);
+  const GA<T>* __restrict__ col = Gp + c.cb[l];
 
   T best0[kNQ], best1[kNQ];
   int arg0[kNQ], arg1[kNQ];
@@ -202,16 +219,12 @@ __device__ __forceinline__ void run_task(const Ctx<T>& c, uint32_t desc, bool ac
     best0[s] = best1[s] = Arith<T>::inf();
     arg0[s] = arg1[s] = kmin;
   }
-  // Row k of the layer starts at row_off(k) - k - 1 (+ l); the start moves by
-  // p - 2 - k from row k to row k + 1.
-  int base = row_off(kmin, p) - kmin - 1;
   int k = kmin;
 #pragma unroll 1
   for (; k + kNQ <= lmin; k += kNQ) {
 #pragma unroll
     for (int s = 0; s < kNQ; ++s) {
-      const GA<T> ga = Gp[base + l];
-      base += p - 2 - (k + s);
+      const GA<T> ga = col[k + s];
       const T v0 = Arith<T>::fold(ga.g, ga.a + b0);
       const T v1 = Arith<T>::fold(ga.g, ga.a + b1);
       // The running minimum is one min op per step; the argmin follows it.
@@ -226,7 +239,7 @@ __device__ __forceinline__ void run_task(const Ctx<T>& c, uint32_t desc, bool ac
 #pragma unroll 1
   for (; k < lmax; ++k) {
     if (k < l) {
-      const GA<T> ga = Gp[base + l];
+      const GA<T> ga = col[k];
       const T v0 = Arith<T>::fold(ga.g, ga.a + b0);
       const T v1 = Arith<T>::fold(ga.g, ga.a + b1);
       if (v0 < best0[0]) {
@@ -238,7 +251,6 @@ __device__ __forceinline__ void run_task(const Ctx<T>& c, uint32_t desc, bool ac
         arg1[0] = k;
       }
     }
-    base += p - 2 - k;
   }
   // Streams hold base indices; stream s saw k = base + s. Merge with the tie
   // rule (smaller k wins).
@@ -256,10 +268,10 @@ __device__ __forceinline__ void run_task(const Ctx<T>& c, uint32_t desc, bool ac
   }
   if (active) {
     const int e = ro + j0;
-    Gc[e].g = c.rowV[e] * invl + best0[0];
+    Gc[c.cb[j0] + l].g = c.rowV[e] * invl + best0[0];
     bpi[e] = static_cast<uint16_t>(arg0[0]);
     if (two) {
-      Gc[e + 1].g = c.rowV[e + 1] * invl + best1[0];
+      Gc[c.cb[j0 + 1] + l].g = c.rowV[e + 1] * invl + best1[0];
       bpi[e + 1] = static_cast<uint16_t>(arg1[0]);
     }
   }
@@ -292,7 +304,7 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
       const int e = j - 1;
       T f = c.rowV[e] * invl;
       if (!sep) f += Arith<T>::nlog(c.rowB[e] + Arith<T>::kEps);
-      G1[e].g = f;
+      G1[c.cb[j]].g = f;
     }
   }
   __syncthreads();
@@ -305,12 +317,12 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
     if (i == 2) {
       // Only k = c_1 = 0 precedes the second value.
       for (int l = 1 + warp; l <= p - 2; l += kWarps) {
-        const GA<T> ga = Gp[l - 1];  // (0, l)
+        const GA<T> ga = Gp[c.cb[l]];  // (0, l)
         const int ro = row_off(l, p) - l - 1;
         for (int j = (last ? p - 1 : l + 1) + lane; j <= p - 1; j += kWarp) {
           const int e = ro + j;
           const T v = sep ? ga.g : Arith<T>::fold(ga.g, ga.a + c.rowB[e]);
-          Gc[e].g = c.rowV[e] * invl + v;
+          Gc[c.cb[j] + l].g = c.rowV[e] * invl + v;
         }
       }
     } else if (sep) {
@@ -319,7 +331,7 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
         T best = Arith<T>::inf();
         int arg = kmin;
         for (int k = kmin + lane; k < l; k += kWarp) {
-          const T v = Gp[tix(k, l, p)].g;
+          const T v = Gp[c.cb[l] + k].g;
           if (v < best) {
             best = v;
             arg = k;
@@ -338,7 +350,7 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
         const uint16_t ra = static_cast<uint16_t>(c.rarg[l]);
         for (int j = (last ? p - 1 : l + 1) + lane; j <= p - 1; j += kWarp) {
           const int e = ro + j;
-          Gc[e].g = c.rowV[e] + rm;
+          Gc[c.cb[j] + l].g = c.rowV[e] + rm;
           bpi[e] = ra;
         }
       }
@@ -476,16 +488,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
   c.sQ = reinterpret_cast<int*>(carve(sizeof(int) * S));
   int* sQ1 = reinterpret_cast<int*>(carve(sizeof(int) * S));
   int* sQ2 = reinterpret_cast<int*>(carve(sizeof(int) * S));
+  int* cbs = reinterpret_cast<int*>(carve(sizeof(int) * (p + 1)));
+  if (threadIdx.x == 0) {
+    int cc = 0;
+    for (int l = 0; l < p; ++l) {
+      cbs[l] = cc;
+      cc = next_colbase(cc, l);
+    }
+    cbs[p] = cc;
+  }
+  c.cb = cbs;
 
   unsigned char* gs = a.scratch + static_cast<size_t>(blockIdx.x) * a.scratch_per_cta;
   c.bp = reinterpret_cast<uint16_t*>(gs);
   gs += (sizeof(uint16_t) * static_cast<size_t>(S) * tri + 255) & ~size_t(255);
   const size_t tb = (sizeof(T) * static_cast<size_t>(tri) + 15) & ~size_t(15);
+  const size_t gb = (2 * sizeof(T) * static_cast<size_t>(layer_elems(p)) + 15) & ~size_t(15);
   unsigned char* big = kSmemTables ? sp : gs;
   c.ga0 = reinterpret_cast<GA<T>*>(big);
-  c.ga1 = reinterpret_cast<GA<T>*>(big + 2 * tb);
-  c.rowB = reinterpret_cast<T*>(big + 4 * tb);
-  c.rowV = reinterpret_cast<T*>(big + 5 * tb);
+  c.ga1 = reinterpret_cast<GA<T>*>(big + gb);
+  c.rowB = reinterpret_cast<T*>(big + 2 * gb);
+  c.rowV = reinterpret_cast<T*>(big + 2 * gb + tb);
+  __syncthreads();  // cb visible to all threads
 
   const int s_out_stride = a.s_out;
   for (int r = blockIdx.x; r < a.n; r += gridDim.x) {
@@ -658,10 +682,14 @@ void* dp_kernel_ptr() {
 
 size_t small_smem(int p, int S, size_t tsz) {
   auto al = [](size_t b) { return (b + 15) & ~size_t(15); };
-  return al(8 * p) * 4 + al(8 * S) * 2 + al(tsz * p) + al(4 * p) + al(4 * S) * 4;
+  return al(8 * p) * 4 + al(8 * S) * 2 + al(tsz * p) + al(4 * p) + al(4 * S) * 4 + al(4 * (p + 1));
 }
 
-size_t table_bytes(int p, size_t tsz) { return ((tsz * tri_size(p) + 15) & ~size_t(15)) * 6; }
+size_t table_bytes(int p, size_t tsz) {
+  const size_t tb = (tsz * tri_size(p) + 15) & ~size_t(15);
+  const size_t gb = (2 * tsz * static_cast<size_t>(layer_elems(p)) + 15) & ~size_t(15);
+  return 2 * gb + 2 * tb;
+}
 
 }  // namespace
 
