@@ -39,14 +39,15 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / kWarp;
-constexpr int kNQ = 4;  // independent k-streams per output (breaks the min/argmin chain)
+constexpr int kTJ = 4;  // outputs (l, j0 .. j0+3) per lane
+constexpr int kNQ = 2;  // interleaved k-streams per output (kTJ * kNQ independent min chains per lane)
 
-// A pair descriptor names two outputs (l, j0) and (l, j0 + 1) of one layer:
-// l in bits 0..9, j0 in bits 10..19, bit 20 set when (l, j0 + 1) is real.
-__host__ __device__ inline uint32_t pack_pair(int l, int j0, bool two) {
-  return static_cast<uint32_t>(l) | (static_cast<uint32_t>(j0) << 10) | (two ? (1u << 20) : 0u);
+// A group descriptor names up to kTJ outputs (l, j0 .. j0 + n - 1) of one layer:
+// l in bits 0..9, j0 in bits 10..19, n - 1 in bits 20..22.
+__host__ __device__ inline uint32_t pack_group(int l, int j0, int n) {
+  return static_cast<uint32_t>(l) | (static_cast<uint32_t>(j0) << 10) | (static_cast<uint32_t>(n - 1) << 20);
 }
-__host__ __device__ inline int max_pairs(int p) { return p * (p / 2 + 1); }
+__host__ __device__ inline int max_groups(int p) { return p * ((p + kTJ - 1) / kTJ + 1); }
 
 template <typename T>
 struct Arith;
@@ -84,8 +85,7 @@ struct alignas(2 * sizeof(T)) GA {
 // consecutive addresses (one pointer, immediate offsets). Column starts are
 // padded so that cb[l] = l (mod 16): lanes that hold 16 consecutive rows l
 // then read 16 distinct 8-byte bank pairs at every k. b = L/d and V/d are read
-// once per output and stay in the row-triangle layout tix(l, j).
-__host__ __device__ __forceinline__ int tix(int k, int l, int p) { return row_off(k, p) + l - k - 1; }
+// once per output and stay in the row-triangle layout (row_off(l) + j - l - 1).
 
 // cb[0..p]: padded column starts; cb[p] = elements of one layer buffer.
 __host__ __device__ inline int next_colbase(int prev_base, int prev_col) {
@@ -117,9 +117,9 @@ struct Ctx {
   int* rarg;                  // [p]
   int* ctr;                   // [S] task counters
   int* sQ;                    // [S] code of the last solve
-  const uint32_t* pairs;   // [S][max_pairs] pair descriptors per layer
-  const int32_t* npairs;   // [S]
-  int max_pairs;
+  const uint32_t* groups;  // [S][max_groups] group descriptors per layer
+  const int32_t* ngroups;  // [S]
+  int max_groups;
 };
 
 struct SolveOut {
@@ -192,10 +192,12 @@ __device__ __forceinline__ void finalize_layer(const Ctx<T>& c, int i, const GA<
   }
 }
 
-// One task of layer i >= 3: 32 pair descriptors, one per lane. Lane L owns the
-// outputs (l, j0) and (l, j0+1) and sweeps k = i-2 .. l-1 over kNQ interleaved
-// streams (each keeps its own running minimum, so consecutive updates do not
-// wait on one another); the k range common to the warp runs unpredicated.
+// One task of layer i >= 3: 32 group descriptors, one per lane. Lane L owns
+// the outputs (l, j0 .. j0+n-1) and sweeps k = i-2 .. l-1 down its column in
+// kNQ interleaved streams (each output and stream keeps its own running
+// minimum, so consecutive updates do not wait on one another). The k range
+// common to the warp runs unpredicated; the rest masks the layer value to +inf
+// past the lane's own column.
 template <typename T>
 __device__ __forceinline__ void run_task(const Ctx<T>& c, uint32_t desc, bool active, int i,
                                          const GA<T>* __restrict__ Gp, GA<T>* __restrict__ Gc,
@@ -204,75 +206,71 @@ __device__ __forceinline__ void run_task(const Ctx<T>& c, uint32_t desc, bool ac
   const int kmin = i - 2;
   const int l = active ? static_cast<int>(desc & 1023) : kmin + 1;  // inactive lanes: any in-range row
   const int j0 = static_cast<int>((desc >> 10) & 1023);
-  const bool two = active && ((desc >> 20) & 1u);
+  const int nv = active ? static_cast<int>((desc >> 20) & 7) + 1 : 0;
   const int lmin = __reduce_min_sync(0xffffffffu, active ? l : 0x7fffffff);
   const int lmax = __reduce_max_sync(0xffffffffu, active ? l : 0);
   const int ro = row_off(l, p) - l - 1;
-  const T b0 = active ? c.rowB[ro + j0] : T(0);
-  const T b1 = two ? c.rowB[ro + j0 + 1] : T(0);
+  T b[kTJ];
+#pragma unroll
+  for (int u = 0; u < kTJ; ++u) b[u] = (u < nv) ? c.rowB[ro + j0 + u] : T(0);
   const GA<T>* __restrict__ col = Gp + c.cb[l];
 
-  T best0[kNQ], best1[kNQ];
-  int arg0[kNQ], arg1[kNQ];
+  T best[kTJ][kNQ];
+  int arg[kTJ][kNQ];
 #pragma unroll
-  for (int s = 0; s < kNQ; ++s) {
-    best0[s] = best1[s] = Arith<T>::inf();
-    arg0[s] = arg1[s] = kmin;
-  }
+  for (int u = 0; u < kTJ; ++u)
+#pragma unroll
+    for (int s = 0; s < kNQ; ++s) {
+      best[u][s] = Arith<T>::inf();
+      arg[u][s] = kmin;
+    }
   int k = kmin;
-#pragma unroll 1
+#pragma unroll 2
   for (; k + kNQ <= lmin; k += kNQ) {
 #pragma unroll
     for (int s = 0; s < kNQ; ++s) {
       const GA<T> ga = col[k + s];
-      const T v0 = Arith<T>::fold(ga.g, ga.a + b0);
-      const T v1 = Arith<T>::fold(ga.g, ga.a + b1);
-      // The running minimum is one min op per step; the argmin follows it.
-      const bool lt0 = v0 < best0[s];
-      const bool lt1 = v1 < best1[s];
-      best0[s] = Arith<T>::vmin(best0[s], v0);
-      best1[s] = Arith<T>::vmin(best1[s], v1);
-      arg0[s] = lt0 ? k : arg0[s];
-      arg1[s] = lt1 ? k : arg1[s];
+#pragma unroll
+      for (int u = 0; u < kTJ; ++u) {
+        const T v = Arith<T>::fold(ga.g, ga.a + b[u]);
+        // The running minimum is one min op per step; the argmin follows it.
+        const bool lt = v < best[u][s];
+        best[u][s] = Arith<T>::vmin(best[u][s], v);
+        arg[u][s] = lt ? k : arg[u][s];
+      }
     }
   }
 #pragma unroll 1
   for (; k < lmax; ++k) {
-    if (k < l) {
-      const GA<T> ga = col[k];
-      const T v0 = Arith<T>::fold(ga.g, ga.a + b0);
-      const T v1 = Arith<T>::fold(ga.g, ga.a + b1);
-      if (v0 < best0[0]) {
-        best0[0] = v0;
-        arg0[0] = k;
-      }
-      if (v1 < best1[0]) {
-        best1[0] = v1;
-        arg1[0] = k;
-      }
-    }
-  }
-  // Streams hold base indices; stream s saw k = base + s. Merge with the tie
-  // rule (smaller k wins).
+    GA<T> ga = col[k];
+    ga.g = (k < l) ? ga.g : Arith<T>::inf();
 #pragma unroll
-  for (int s = 1; s < kNQ; ++s) {
-    const int k0 = arg0[s] + s, k1 = arg1[s] + s;
-    if (best0[s] < best0[0] || (best0[s] == best0[0] && k0 < arg0[0])) {
-      best0[0] = best0[s];
-      arg0[0] = k0;
-    }
-    if (best1[s] < best1[0] || (best1[s] == best1[0] && k1 < arg1[0])) {
-      best1[0] = best1[s];
-      arg1[0] = k1;
+    for (int u = 0; u < kTJ; ++u) {
+      const T v = Arith<T>::fold(ga.g, ga.a + b[u]);
+      const bool lt = v < best[u][0];
+      best[u][0] = Arith<T>::vmin(best[u][0], v);
+      arg[u][0] = lt ? k : arg[u][0];
     }
   }
-  if (active) {
-    const int e = ro + j0;
-    Gc[c.cb[j0] + l].g = c.rowV[e] * invl + best0[0];
-    bpi[e] = static_cast<uint16_t>(arg0[0]);
-    if (two) {
-      Gc[c.cb[j0 + 1] + l].g = c.rowV[e + 1] * invl + best1[0];
-      bpi[e + 1] = static_cast<uint16_t>(arg1[0]);
+  // Stream s holds base indices (it saw k = base + s); the tail updated stream
+  // 0 with true indices. Merge with the tie rule (smaller k wins).
+#pragma unroll
+  for (int u = 0; u < kTJ; ++u) {
+#pragma unroll
+    for (int s = 1; s < kNQ; ++s) {
+      const int ks = arg[u][s] + s;
+      if (best[u][s] < best[u][0] || (best[u][s] == best[u][0] && ks < arg[u][0])) {
+        best[u][0] = best[u][s];
+        arg[u][0] = ks;
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kTJ; ++u) {
+    if (u < nv) {
+      const int e = ro + j0 + u;
+      Gc[c.cb[j0 + u] + l].g = c.rowV[e] * invl + best[u][0];
+      bpi[e] = static_cast<uint16_t>(arg[u][0]);
     }
   }
 }
@@ -356,8 +354,8 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
       }
     } else {
       // Tasks in descending cost: higher rows have longer k sweeps.
-      const uint32_t* pl = c.pairs + static_cast<size_t>(i) * c.max_pairs;
-      const int np = c.npairs[i];
+      const uint32_t* pl = c.groups + static_cast<size_t>(i) * c.max_groups;
+      const int np = c.ngroups[i];
       const int nt = (np + kWarp - 1) / kWarp;
       // The next task's index and descriptor are fetched before the current
       // task runs, so their latency hides behind the sweep.
@@ -466,9 +464,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
   c.S = S;
   c.tri = tri;
   c.dd = static_cast<double>(a.d);
-  c.pairs = a.tasks;
-  c.npairs = a.ntasks;
-  c.max_pairs = a.max_tasks;
+  c.groups = a.tasks;
+  c.ngroups = a.ntasks;
+  c.max_groups = a.max_tasks;
 
   unsigned char* sp = smem;
   auto carve = [&sp](size_t bytes) {
@@ -646,32 +644,32 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
 }
 
 // ---- schedule ----------------------------------------------------------------
-// Pair descriptors of layer i >= 3 in row-major order (rows l = i-1 .. p-2,
-// j ascending; the last layer has only j = p-1). One CTA per layer, one thread
-// per row; a row's first pair index is the sum of the pair counts of the rows
-// before it.
-__global__ void k_schedule(int p, int S, int max_pairs_, uint32_t* pairs, int32_t* npairs) {
+// Group descriptors of layer i >= 3 in row-major order (rows l = i-1 .. p-2,
+// j ascending in groups of kTJ; the last layer has only j = p-1). One CTA per
+// layer, one thread per row; a row's first group index is the sum of the group
+// counts of the rows before it.
+__global__ void k_schedule(int p, int S, int max_groups_, uint32_t* groups, int32_t* ngroups) {
   const int i = blockIdx.x;
   if (i < 3) {
-    if (threadIdx.x == 0) npairs[i] = 0;
+    if (threadIdx.x == 0) ngroups[i] = 0;
     return;
   }
   const bool last = (i == S - 1);
-  auto row_pairs = [&](int l) { return last ? 1 : (p - l) / 2; };  // ceil((p-1-l)/2)
-  uint32_t* out = pairs + static_cast<size_t>(i) * max_pairs_;
+  auto row_groups = [&](int l) { return last ? 1 : (p - 1 - l + kTJ - 1) / kTJ; };
+  uint32_t* out = groups + static_cast<size_t>(i) * max_groups_;
   for (int l = i - 1 + threadIdx.x; l <= p - 2; l += blockDim.x) {
     int o = 0;
-    for (int r = i - 1; r < l; ++r) o += row_pairs(r);
+    for (int r = i - 1; r < l; ++r) o += row_groups(r);
     if (last) {
-      out[o] = pack_pair(l, p - 1, false);
+      out[o] = pack_group(l, p - 1, 1);
     } else {
-      for (int j = l + 1; j <= p - 1; j += 2) out[o++] = pack_pair(l, j, j + 1 <= p - 1);
+      for (int j = l + 1; j <= p - 1; j += kTJ) out[o++] = pack_group(l, j, min(kTJ, p - j));
     }
   }
   if (threadIdx.x == 0) {
     int tot = 0;
-    for (int r = i - 1; r <= p - 2; ++r) tot += row_pairs(r);
-    npairs[i] = tot;
+    for (int r = i - 1; r <= p - 2; ++r) tot += row_groups(r);
+    ngroups[i] = tot;
   }
 }
 
@@ -709,7 +707,7 @@ int64_t dp_triples(int p, int s) {
 
 size_t dp_schedule_bytes(int p, int s) {
   const int S = s < p ? s : p;
-  return ((sizeof(uint32_t) * static_cast<size_t>(max_pairs(p)) * S + 255) & ~size_t(255)) +
+  return ((sizeof(uint32_t) * static_cast<size_t>(max_groups(p)) * S + 255) & ~size_t(255)) +
          ((sizeof(int32_t) * S + 255) & ~size_t(255));
 }
 
@@ -730,7 +728,7 @@ bool dp_plan(int n, int p, int s, bool fp64, DpPlan* plan) {
   plan->smem_bytes = small + (plan->smem_tables ? big : 0);
   const size_t bp = (sizeof(uint16_t) * static_cast<size_t>(S) * tri_size(p) + 255) & ~size_t(255);
   plan->scratch_per_cta = (bp + (plan->smem_tables ? 0 : big) + 255) & ~size_t(255);
-  plan->max_tasks = max_pairs(p);
+  plan->max_tasks = max_groups(p);
   void* fn = fp64 ? (plan->smem_tables ? dp_kernel_ptr<double, true>() : dp_kernel_ptr<double, false>())
                   : (plan->smem_tables ? dp_kernel_ptr<float, true>() : dp_kernel_ptr<float, false>());
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(plan->smem_bytes)) !=
