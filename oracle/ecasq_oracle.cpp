@@ -27,10 +27,11 @@
 //     "H(lambda_mid) > b  =>  lambda_lo = lambda_mid".
 //   * Time-sharing: a per-entry Bernoulli(theta) selector from Philox stream 1.
 //   * Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): key = seed (lo, hi),
-//     counter = (j >> 2, vector, stream, 0), output word j & 3, u = r * 2^-32.
+//     counter = (j >> 2, vector, stream, 0), output word j & 3, u = r * 2^-32;
+//     an entry rounds up iff u * (q_hi - q_lo) < x - q_lo.
 //
 // Compiled with -O2 -fno-fast-math -ffp-contract=off so that the encoder's
-// rounding probability is two IEEE subtractions and one IEEE division.
+// rounding test is exactly two IEEE subtractions and one IEEE product.
 
 #include <algorithm>
 #include <cmath>
@@ -474,8 +475,10 @@ static uint32_t philox_word(uint64_t seed, int64_t j, uint32_t v, uint32_t strea
 //   * Q2 != null and 0 < theta < 1: Q1 when u_sel(j) < theta (Philox stream 1),
 //     else Q2 (part 1).
 //   * Q2 != null otherwise: theta >= 1 gives Q1 only, theta <= 0 Q2 only.
-// An entry in [q_i, q_{i+1}] rounds up when u(j) < (x - q_i)/(q_{i+1} - q_i)
-// (Philox stream 0). idx[j] is the position in the chosen code and
+// An entry in [q_i, q_{i+1}] rounds up when u(j) * (q_{i+1} - q_i) < x - q_i
+// (Philox stream 0): the test u < (x - q_i)/(q_{i+1} - q_i) with the division
+// moved to the other side, each side a single IEEE operation. x = q_i never
+// rounds up; x = q_{i+1} always does (u <= 1 - 2^-32). idx[j] is the position in the chosen code and
 // hist[part*s + idx] counts entries per part.
 int eo_encode(const float* x, int64_t d, const double* P, int p, const int32_t* Q1, int m1,
               const int32_t* Q2, int m2, double theta, int s, uint64_t seed, uint32_t v,
@@ -506,9 +509,12 @@ int eo_encode(const float* x, int64_t d, const double* P, int p, const int32_t* 
     } else {
       if (!(xv >= q[0]) || !(xv <= q[m - 1])) return -2;
       int i = int(std::upper_bound(q.data(), q.data() + (m - 1), xv) - q.data()) - 1;
-      double prob = (xv - q[i]) / (q[i + 1] - q[i]);
+      // Up with probability (x - q_i)/(q_{i+1} - q_i): u < (x - q_i)/(q_{i+1} - q_i)
+      // tested as u * (q_{i+1} - q_i) < x - q_i, each side one IEEE operation.
+      double y = xv - q[i];
+      double w = q[i + 1] - q[i];
       double u = double(philox_word(seed, j, v, 0u)) * 0x1p-32;
-      out = (u < prob) ? i + 1 : i;
+      out = (u * w < y) ? i + 1 : i;
     }
     idx[j] = uint8_t(out);
     hist[part * s + out] += 1;
