@@ -147,24 +147,33 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
     stream = torch.cuda.current_stream()
 
     def step(X):
+        ev["g0"].record(stream)
         P, st = E.uniform_grid(X, p)
+        ev["g1"].record(stream)
         cnt, A, B, st = E.bucket(X, P)
+        ev["b1"].record(stream)
         ev_dp0.record(stream)
         if w.mode == "budget":
             out = E.solve_budget_stats(cnt, A, B, P, d, s, w.b, w.steps, fp64=fp64)
             ev_dp1.record(stream)
             idx, hist, est = E.encode(X, P, s, out["Q1"], out["Q1_len"], w.seed_encode, out["Q2"], out["Q2_len"],
                                       out["theta"])
+            ev["e1"].record(stream)
         else:
             out = E.solve_stats(cnt, A, B, P, d, s, lam, fp64=fp64)
             ev_dp1.record(stream)
             Q = out["Q"][:, 0, :].contiguous()
-            idx, hist, est = E.encode(X, P, s, Q, out["Q_len"][:, 0].contiguous(), w.seed_encode)
+            Ql = out["Q_len"][:, 0].contiguous()
+            ev["e0"].record(stream)
+            idx, hist, est = E.encode(X, P, s, Q, Ql, w.seed_encode)
+            ev["e1"].record(stream)
         Hemp = E.entropy(hist)
         return out, idx, hist, Hemp
 
     ev_dp0 = torch.cuda.Event(enable_timing=True)
     ev_dp1 = torch.cuda.Event(enable_timing=True)
+    ev = {k: torch.cuda.Event(enable_timing=True) for k in ("g0", "g1", "b1", "e0", "e1")}
+    stage_ms = {"grid": [], "bucket": [], "encode": []}
     unit_peaks = measure_unit_peaks()
     for _ in range(args.warmup):
         out, idx, hist, Hemp = step(X)
@@ -188,6 +197,9 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
             ends[k].record(stream)
             torch.cuda.synchronize()
             dp_ms.append(ev_dp0.elapsed_time(ev_dp1))
+            stage_ms["grid"].append(ev["g0"].elapsed_time(ev["g1"]))
+            stage_ms["bucket"].append(ev["g1"].elapsed_time(ev["b1"]))
+            stage_ms["encode"].append((ev["e0"] if w.mode != "budget" else ev_dp1).elapsed_time(ev["e1"]))
     launches = E.launch_count(reset=True)
     step_ms = [starts[k].elapsed_time(ends[k]) for k in range(args.steps)]
     t_ms = float(sum(step_ms))
@@ -219,6 +231,14 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
     bo = n * d + n * 8 + (n * s * 4 * 2 + n * 8 if w.mode == "budget" else 0)
 
     peaks = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    entries = n * d
+    hbm_kernels = {}
+    for name, bpe in (("grid", 4), ("bucket", 4), ("encode", 5)):
+        ms = float(np.mean(stage_ms[name]))
+        gbs = entries * bpe / (ms * 1e-3) / 1e9
+        hbm_kernels[name] = {"ms": ms, "bytes_per_entry": bpe, "achieved_GBps": gbs, "peak_GBps": hbm,
+                             "frac": gbs / hbm, "entries_per_s": entries / (ms * 1e-3)}
     sm_max = float(peaks.get("sm_max_mhz", 1965.0))
     mufu_peak = MUFU_LG2_PER_CLK_PER_SM * B200_SMS * sm_max * 1e6
     dp_avg_ms = float(np.mean(dp_ms))
@@ -251,6 +271,7 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
                      "measured_ffma_per_s": unit_peaks.get("ffma")},
         "e2e": {"value": total_triples / (float(np.mean(e2e_ms)) * 1e-3), "unit": "triples/s",
                 "h2d_bytes_per_step": n * d * 4, "d2h_bytes_per_step": bo},
+        "hbm_kernels": hbm_kernels,
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
     }

@@ -22,10 +22,13 @@ namespace ecasq {
 namespace {
 
 constexpr int kEncThreads = 256;
+constexpr int kEncWarps = kEncThreads / kWarp;
 constexpr int64_t kEncChunk = 16384;  // entries per CTA (multiple of 4)
-constexpr int kPrivateBins = 32;      // per-thread histograms up to 2*s <= 32 bins
 
-template <bool kPrivate>
+// Rounding test: x in [q_t, q_{t+1}] goes up iff u * (q_{t+1} - q_t) < x - q_t,
+// i.e. u < (x - q_t)/(q_{t+1} - q_t) with the division moved across; each side
+// is one IEEE fp64 operation, so the decision is reproducible on any IEEE
+// machine. x = q_t never goes up, x = q_{t+1} always does.
 __global__ void __launch_bounds__(kEncThreads)
 k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d, int p, int s,
          const int32_t* __restrict__ Q1, const int32_t* __restrict__ Q1_len, const int32_t* __restrict__ Q2,
@@ -35,8 +38,9 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
   const int r = blockIdx.y;
   double* sP = reinterpret_cast<double*>(smem);   // [p]
   double* sq = sP + p;                             // [2][s] code values
-  unsigned char* imap = reinterpret_cast<unsigned char*>(sq + 2 * s);  // [2][p] bucket -> interval
-  unsigned int* sh = reinterpret_cast<unsigned int*>(imap + ((2 * p + 15) & ~15));
+  double* sw = sq + 2 * s;                         // [2][s] interval widths q_{t+1} - q_t
+  unsigned int* sh = reinterpret_cast<unsigned int*>(sw + 2 * s);      // [warps][2s] counts
+  unsigned char* imap = reinterpret_cast<unsigned char*>(sh + kEncWarps * 2 * s);  // [2][p]
   __shared__ int s_m[2];
   __shared__ int s_bad;
 
@@ -45,6 +49,7 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
   const double th = (has2 && theta) ? theta[r] : 0.0;
   const bool mix = has2 && th > 0.0 && th < 1.0;
   const int fixed_part = (!has2 || th >= 1.0) ? 0 : 1;
+  const int nbins = 2 * s;
 
   for (int k = threadIdx.x; k < p; k += blockDim.x) sP[k] = P[k];
   if (threadIdx.x == 0) {
@@ -53,12 +58,7 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
     s_m[1] = has2 ? Q2_len[r] : 0;
   }
   for (int k = threadIdx.x; k < 2 * p; k += blockDim.x) imap[k] = 255;
-  const int nbins = 2 * s;
-  if (kPrivate) {
-    for (int k = threadIdx.x; k < nbins * kEncThreads; k += blockDim.x) sh[k] = 0u;
-  } else {
-    for (int k = threadIdx.x; k < nbins; k += blockDim.x) sh[k] = 0u;
-  }
+  for (int k = threadIdx.x; k < kEncWarps * nbins; k += blockDim.x) sh[k] = 0u;
   __syncthreads();
   // A code must hold 1..s increasing indices into P; anything else marks the
   // row invalid and leaves its outputs untouched.
@@ -82,14 +82,17 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
       return;
     }
   }
-  // Code values and the bucket -> interval map of each part.
+  // Code values, interval widths and the bucket -> interval map of each part.
   for (int part = 0; part < 2; ++part) {
     const int m = s_m[part];
     const int32_t* Q = (part == 0 ? Q1 : Q2);
     const bool used = (part == 0) ? (fixed_part == 0 || mix) : (fixed_part == 1 || mix);
     if (!used) continue;
     const int32_t* q = Q + static_cast<int64_t>(r) * s;
-    for (int t = threadIdx.x; t < m; t += blockDim.x) sq[part * s + t] = sP[q[t]];
+    for (int t = threadIdx.x; t < m; t += blockDim.x) {
+      sq[part * s + t] = sP[q[t]];
+      if (t + 1 < m) sw[part * s + t] = __dsub_rn(sP[q[t + 1]], sP[q[t]]);
+    }
     for (int t = threadIdx.x; t < m - 1; t += blockDim.x)
       for (int k = q[t]; k < q[t + 1]; ++k) imap[part * p + k] = static_cast<unsigned char>(t);
   }
@@ -101,6 +104,7 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
   const float* x = X + static_cast<int64_t>(r) * d;
   uint8_t* o = idx + static_cast<int64_t>(r) * d;
   const bool vec = ((reinterpret_cast<uintptr_t>(x) & 15u) == 0) && ((d & 3) == 0);
+  unsigned int* wh = sh + warp_id() * nbins;
   int bad = 0;
 
   for (int64_t g = beg + 4 * static_cast<int64_t>(threadIdx.x); g < end; g += 4 * kEncThreads) {
@@ -121,40 +125,35 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
     uint4 su = make_uint4(0u, 0u, 0u, 0u);
     if (mix) su = Philox4x32::block(make_uint4(blk, static_cast<uint32_t>(r), 1u, 0u), key0, key1);
     const uint32_t rw[4] = {ru.x, ru.y, ru.z, ru.w};
-    const uint32_t sw[4] = {su.x, su.y, su.z, su.w};
+    const uint32_t sel[4] = {su.x, su.y, su.z, su.w};
     uint32_t packed = 0;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       if (e >= cnt) break;
       const double xd = static_cast<double>(xv[e]);
       int part = fixed_part;
-      if (mix) part = (static_cast<double>(sw[e]) * 0x1p-32 < th) ? 0 : 1;
+      if (mix) part = (static_cast<double>(sel[e]) * 0x1p-32 < th) ? 0 : 1;
       const int m = s_m[part];
-      const double* q = sq + part * s;
       int out = 0;
       if (m == 1) {
-        if (xd != q[0]) bad = 1;
+        if (xd != sq[part * s]) bad = 1;
       } else {
         const int k = bucket_of(xd, sP, p, scale);
         int t = (k >= 0) ? imap[part * p + k] : 255;
         if (t == 255) {
-          if (m >= 2 && xd == q[m - 1])
+          if (xd == sq[part * s + m - 1])
             t = m - 2;
           else
             bad = 1;
         }
         if (t != 255) {
-          const double prob = __ddiv_rn(__dsub_rn(xd, q[t]), __dsub_rn(q[t + 1], q[t]));
+          const double y = __dsub_rn(xd, sq[part * s + t]);
           const double u = static_cast<double>(rw[e]) * 0x1p-32;
-          out = t + ((u < prob) ? 1 : 0);
+          out = t + ((__dmul_rn(u, sw[part * s + t]) < y) ? 1 : 0);
         }
       }
       packed |= static_cast<uint32_t>(out) << (8 * e);
-      const int bin = part * s + out;
-      if (kPrivate)
-        sh[bin * kEncThreads + threadIdx.x] += 1u;
-      else
-        atomicAdd(sh + bin, 1u);
+      atomicAdd(wh + part * s + out, 1u);
     }
     if (cnt == 4 && ((reinterpret_cast<uintptr_t>(o + g) & 3u) == 0)) {
       *reinterpret_cast<uint32_t*>(o + g) = packed;
@@ -167,11 +166,8 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
   unsigned long long* gh = hist + static_cast<int64_t>(r) * nbins;
   for (int b = threadIdx.x; b < nbins; b += blockDim.x) {
     unsigned long long tot = 0;
-    if (kPrivate) {
-      for (int t = 0; t < kEncThreads; ++t) tot += sh[b * kEncThreads + ((t + b) & (kEncThreads - 1))];
-    } else {
-      tot = sh[b];
-    }
+#pragma unroll
+    for (int w = 0; w < kEncWarps; ++w) tot += sh[w * nbins + b];
     if (tot) atomicAdd(gh + b, tot);
   }
   if (threadIdx.x == 0 && s_bad) status[r] = kStatusRange;
@@ -200,10 +196,8 @@ __global__ void k_entropy(const int64_t* __restrict__ hist, int n, int s, double
   if (lane_id() == 0) H[r] = tot > 0.0 ? acc / tot : 0.0;
 }
 
-size_t encode_smem(int p, int s, bool priv) {
-  size_t b = sizeof(double) * (p + 2 * s) + ((2 * p + 15) & ~15);
-  b += priv ? sizeof(unsigned int) * 2 * s * kEncThreads : sizeof(unsigned int) * 2 * s;
-  return b;
+size_t encode_smem(int p, int s) {
+  return sizeof(double) * (p + 4 * s) + sizeof(unsigned int) * kEncWarps * 2 * s + 2 * p;
 }
 
 }  // namespace
@@ -217,27 +211,10 @@ cudaError_t launch_encode(const float* X, const double* P, int n, int64_t d, int
   e = cudaMemsetAsync(status, 0, sizeof(int32_t) * n, st);
   if (e != cudaSuccess) return e;
   const int nc = static_cast<int>((d + kEncChunk - 1) / kEncChunk);
-  const bool priv = (2 * s <= kPrivateBins);
-  const size_t smem = encode_smem(p, s, priv);
+  const size_t smem = encode_smem(p, s);
   const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
-  unsigned long long* h = reinterpret_cast<unsigned long long*>(hist);
-  if (priv) {
-    static bool set = false;
-    if (!set) {
-      cudaFuncSetAttribute(k_encode<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
-      set = true;
-    }
-    k_encode<true><<<dim3(nc, n), kEncThreads, smem, st>>>(X, P, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, k0, k1,
-                                                            idx, h, status);
-  } else {
-    static bool set = false;
-    if (!set) {
-      cudaFuncSetAttribute(k_encode<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
-      set = true;
-    }
-    k_encode<false><<<dim3(nc, n), kEncThreads, smem, st>>>(X, P, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, k0, k1,
-                                                             idx, h, status);
-  }
+  k_encode<<<dim3(nc, n), kEncThreads, smem, st>>>(X, P, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, k0, k1, idx,
+                                                    reinterpret_cast<unsigned long long*>(hist), status);
   note_launch();
   return cudaGetLastError();
 }

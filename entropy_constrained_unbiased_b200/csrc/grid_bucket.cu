@@ -119,102 +119,191 @@ __global__ void k_grid_finish(const float* __restrict__ part, int n_chunks, int 
 }
 
 // ---------------------------------------------------------------------------
-// Bucketing. Sums are fixed point: an entry of bucket k with y = x - P_k adds
-// round(y / D_k * 2^fb) to the first-moment accumulator and
-// round((y / D_k)^2 * 2^fb) to the second, D_k = P_{k+1} - P_k, fb chosen so
-// that d entries cannot overflow 64 bits. Integer sums make the result
-// independent of the order in which CTAs and lanes accumulate, and the shared
-// memory updates are native 64-bit integer atomics. Each lane updates copy
-// (lane % kCopies) of the CTA's histogram, which caps same-address collisions
-// inside a warp at 32 / kCopies.
+// Bucketing. Sums are fixed point: an entry of bucket k with u = (x - P_k)/D_k,
+// D_k = P_{k+1} - P_k, adds round(u * 2^fb) to the first-moment accumulator and
+// round(u^2 * 2^fb) to the second; fb is chosen from d so that no 64-bit sum
+// can overflow. Integer sums make the result independent of the order in
+// which entries are added.
+//
+// Only 32-bit shared-memory atomics are native on this GPU, so the kernel
+// groups entries by bucket with a counting sort per tile instead of adding
+// 64-bit values atomically:
+//   1. each thread buckets 8 entries and claims a slot in its bucket with a
+//      32-bit atomic increment of the tile's bucket count;
+//   2. warp 0 turns the counts into offsets (exclusive scan);
+//   3. entries are scattered to their sorted position (u and the bucket id);
+//   4. warps sweep the sorted tile 32 entries at a time with a segmented
+//      inclusive scan (equal keys are contiguous); the last lane of each
+//      segment adds the segment's sums to the warp's private accumulators.
 
 constexpr int kBucketThreads = 256;
-constexpr int kCopies = 4;
+constexpr int kBucketWarps = kBucketThreads / kWarp;
+constexpr int kPerThread = 8;                             // entries per thread per tile
+constexpr int kTile = kBucketThreads * kPerThread;        // 2048
 
 __global__ void __launch_bounds__(kBucketThreads)
-k_bucket(const float* __restrict__ X, int64_t d, int64_t chunk, const double* __restrict__ Pall,
-         int p, int fb, unsigned long long* __restrict__ acc, int32_t* __restrict__ flag) {
+k_bucket(const float* __restrict__ X, int64_t d, int64_t chunk, const double* __restrict__ Pall, int p, int fb,
+         unsigned long long* __restrict__ acc, int32_t* __restrict__ flag) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int r = blockIdx.y;
-  const int nb = p - 1;
-  double* sP = reinterpret_cast<double*>(smem);                 // [p]
-  double* sS = sP + p;                                          // [p-1] 2^fb / D_k
-  unsigned long long* sa = reinterpret_cast<unsigned long long*>(sS + p);  // [kCopies][p]
-  unsigned long long* sb = sa + kCopies * p;                     // [kCopies][p]
-  unsigned int* sc = reinterpret_cast<unsigned int*>(sb + kCopies * p);    // [kCopies][p]
+  const int nb = p - 1;        // real buckets 0 .. p-2; key nb collects entries that add nothing
+  double* sP = reinterpret_cast<double*>(smem);                                  // [p]
+  double* sS = sP + p;                                                           // [p] 2^fb / D_k
+  double* su = sS + p;                                                           // [kTile] sorted u * 2^fb
+  unsigned long long* wa = reinterpret_cast<unsigned long long*>(su + kTile);    // [warps][p]
+  unsigned long long* wb = wa + kBucketWarps * p;                                // [warps][p]
+  unsigned long long* ccnt = wb + kBucketWarps * p;                              // [p]
+  unsigned int* tcnt = reinterpret_cast<unsigned int*>(ccnt + p);                // [p]
+  unsigned int* toff = tcnt + p;                                                 // [p]
+  unsigned short* skey = reinterpret_cast<unsigned short*>(toff + p);            // [kTile]
   __shared__ int s_bad;
 
   const double* P = Pall + static_cast<int64_t>(r) * p;
   const double two_fb = ldexp(1.0, fb);
   for (int k = threadIdx.x; k < p; k += blockDim.x) {
     sP[k] = P[k];
-    if (k < nb) sS[k] = two_fb / (P[k + 1] - P[k]);
+    sS[k] = (k < nb) ? two_fb / (P[k + 1] - P[k]) : 0.0;
+    ccnt[k] = 0ull;
   }
-  for (int k = threadIdx.x; k < kCopies * p; k += blockDim.x) {
-    sa[k] = 0ull;
-    sb[k] = 0ull;
-    sc[k] = 0u;
+  for (int k = threadIdx.x; k < kBucketWarps * p; k += blockDim.x) {
+    wa[k] = 0ull;
+    wb[k] = 0ull;
   }
   if (threadIdx.x == 0) s_bad = 0;
   __syncthreads();
 
   const double scale = static_cast<double>(p - 1) / (sP[p - 1] - sP[0]);
   const double inv_two_fb = ldexp(1.0, -fb);
-  const int copy = lane_id() & (kCopies - 1);
-  unsigned long long* ma = sa + copy * p;
-  unsigned long long* mb = sb + copy * p;
-  unsigned int* mc = sc + copy * p;
+  const double magic = 0x1p52;  // v + 2^52 keeps round(v) in the low mantissa bits for 0 <= v < 2^52
+  const unsigned long long low52 = (1ull << 52) - 1;
+  const int lane = lane_id();
+  const int w = warp_id();
   int bad = 0;
-
-  auto one = [&](float xf) {
-    const double x = static_cast<double>(xf);
-    const int k = bucket_of(x, sP, p, scale);
-    if (k < 0) {
-      bad = 1;
-      return;
-    }
-    const double u = (x - sP[k]) * sS[k];
-    const unsigned long long a = __double2ull_rn(u);
-    const unsigned long long b = __double2ull_rn(u * u * inv_two_fb);
-    atomicAdd(mc + k, 1u);
-    atomicAdd(ma + k, a);
-    atomicAdd(mb + k, b);
-  };
 
   const float* x = X + static_cast<int64_t>(r) * d;
   const int64_t beg = static_cast<int64_t>(blockIdx.x) * chunk;
   const int64_t end = beg + chunk < d ? beg + chunk : d;
   const bool vec = ((reinterpret_cast<uintptr_t>(x + beg) & 15u) == 0);
-  int64_t t = beg;
-  if (vec) {
-    const int64_t nv = (end - beg) >> 2;
-    const float4* x4 = reinterpret_cast<const float4*>(x + beg);
-    for (int64_t i = threadIdx.x; i < nv; i += blockDim.x) {
-      const float4 v = __ldcs(x4 + i);
-      one(v.x);
-      one(v.y);
-      one(v.z);
-      one(v.w);
+
+  // Entry e of a thread in the tile starting at t0: position t0 + 4*(threadIdx.x + 256*(e/4)) + e%4.
+  auto load_tile = [&](int64_t t0, float* xv) {
+#pragma unroll
+    for (int h = 0; h < kPerThread / 4; ++h) {
+      const int64_t g = t0 + 4 * (threadIdx.x + static_cast<int64_t>(kBucketThreads) * h);
+      const int cnt = g < end ? static_cast<int>(end - g < 4 ? end - g : 4) : 0;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (vec && cnt == 4) {
+        v = __ldcs(reinterpret_cast<const float4*>(x + g));
+      } else {
+        if (cnt > 0) v.x = __ldcs(x + g);
+        if (cnt > 1) v.y = __ldcs(x + g + 1);
+        if (cnt > 2) v.z = __ldcs(x + g + 2);
+        if (cnt > 3) v.w = __ldcs(x + g + 3);
+      }
+      xv[4 * h + 0] = v.x;
+      xv[4 * h + 1] = v.y;
+      xv[4 * h + 2] = v.z;
+      xv[4 * h + 3] = v.w;
     }
-    t = beg + (nv << 2);
+  };
+  auto valid = [&](int64_t t0, int e) {
+    return t0 + 4 * (threadIdx.x + static_cast<int64_t>(kBucketThreads) * (e >> 2)) + (e & 3) < end;
+  };
+
+  float xv[kPerThread];
+  if (beg < end) load_tile(beg, xv);
+  for (int64_t t0 = beg; t0 < end; t0 += kTile) {
+    for (int k = threadIdx.x; k < p; k += blockDim.x) tcnt[k] = 0u;
+    int key[kPerThread];
+#pragma unroll
+    for (int e = 0; e < kPerThread; ++e) {
+      key[e] = nb;
+      if (valid(t0, e)) {
+        const int k = bucket_of(static_cast<double>(xv[e]), sP, p, scale);
+        if (k < 0)
+          bad = 1;
+        else
+          key[e] = k;
+      }
+    }
+    __syncthreads();
+    int slot[kPerThread];
+#pragma unroll
+    for (int e = 0; e < kPerThread; ++e) slot[e] = static_cast<int>(atomicAdd(tcnt + key[e], 1u));
+    __syncthreads();
+    if (w == 0) {  // exclusive scan of the tile's counts; per-CTA counts
+      unsigned int run = 0;
+      for (int base = 0; base < p; base += kWarp) {
+        const int k = base + lane;
+        const unsigned int c = (k < p) ? tcnt[k] : 0u;
+        unsigned int incl = c;
+#pragma unroll
+        for (int o = 1; o < kWarp; o <<= 1) {
+          const unsigned int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        if (k < p) {
+          toff[k] = run + incl - c;
+          ccnt[k] += c;
+        }
+        run += __shfl_sync(0xffffffffu, incl, kWarp - 1);
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < kPerThread; ++e) {
+      const int k = key[e];
+      const int pos = static_cast<int>(toff[k]) + slot[e];
+      su[pos] = (k < nb) ? (static_cast<double>(xv[e]) - sP[k]) * sS[k] : 0.0;
+      skey[pos] = static_cast<unsigned short>(k);
+    }
+    __syncthreads();
+    if (t0 + kTile < end) load_tile(t0 + kTile, xv);  // next tile in flight during the sweep
+    const int nreal = static_cast<int>(toff[nb]);      // entries with a real bucket come first
+    for (int base = w * kWarp; base < nreal; base += kBucketThreads) {
+      const int pos = base + lane;
+      int k = nb;
+      unsigned long long a = 0, b = 0;
+      if (pos < nreal) {
+        k = skey[pos];
+        const double u = su[pos];
+        a = static_cast<unsigned long long>(__double_as_longlong(u + magic)) & low52;
+        b = static_cast<unsigned long long>(__double_as_longlong(fma(u, u * inv_two_fb, magic))) & low52;
+      }
+#pragma unroll
+      for (int o = 1; o < kWarp; o <<= 1) {
+        const int ko = __shfl_up_sync(0xffffffffu, k, o);
+        const unsigned long long ao = __shfl_up_sync(0xffffffffu, a, o);
+        const unsigned long long bo = __shfl_up_sync(0xffffffffu, b, o);
+        if (lane >= o && ko == k) {
+          a += ao;
+          b += bo;
+        }
+      }
+      const int knext = __shfl_down_sync(0xffffffffu, k, 1);
+      if (k < nb && (lane == kWarp - 1 || knext != k)) {
+        wa[w * p + k] += a;
+        wb[w * p + k] += b;
+      }
+    }
+    __syncthreads();
   }
-  for (int64_t i = t + threadIdx.x; i < end; i += blockDim.x) one(__ldcs(x + i));
   if (bad) s_bad = 1;
   __syncthreads();
 
-  unsigned long long* g = acc + static_cast<int64_t>(r) * nb * 3;
+  unsigned long long* gacc = acc + static_cast<int64_t>(r) * nb * 3;
   for (int k = threadIdx.x; k < nb; k += blockDim.x) {
-    unsigned long long c = 0, a = 0, b = 0;
-#pragma unroll
-    for (int q = 0; q < kCopies; ++q) {
-      c += sc[q * p + k];
-      a += sa[q * p + k];
-      b += sb[q * p + k];
-    }
+    const unsigned long long c = ccnt[k];
     if (c) {
-      atomicAdd(g + 3 * k + 0, c);
-      atomicAdd(g + 3 * k + 1, a);
-      atomicAdd(g + 3 * k + 2, b);
+      unsigned long long sa = 0, sb = 0;
+#pragma unroll
+      for (int q = 0; q < kBucketWarps; ++q) {
+        sa += wa[q * p + k];
+        sb += wb[q * p + k];
+      }
+      atomicAdd(gacc + 3 * k + 0, c);
+      atomicAdd(gacc + 3 * k + 1, sa);
+      atomicAdd(gacc + 3 * k + 2, sb);
     }
   }
   if (threadIdx.x == 0 && s_bad) atomicOr(flag + r, 1);
@@ -262,10 +351,12 @@ cudaError_t launch_uniform_grid(const float* X, int n, int64_t d, int p, double*
 }
 
 size_t bucket_smem_bytes(int p) {
-  return static_cast<size_t>(p) * 8 * 2 + static_cast<size_t>(kCopies) * p * (8 + 8 + 4);
+  return static_cast<size_t>(p) * 8 * 2 + static_cast<size_t>(kTile) * 8 +
+         static_cast<size_t>(kBucketWarps) * p * 16 + static_cast<size_t>(p) * 8 + static_cast<size_t>(p) * 8 +
+         static_cast<size_t>(kTile) * 2;
 }
 
-int64_t bucket_chunk(int64_t d) { return d < 16384 ? d : 16384; }
+int64_t bucket_chunk(int64_t d) { return d < 32768 ? d : 32768; }
 
 cudaError_t launch_bucket(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt,
                           double* A, double* B, int32_t* status, unsigned long long* acc,
@@ -280,7 +371,7 @@ cudaError_t launch_bucket(const float* X, const double* P, int n, int64_t d, int
   const size_t smem = bucket_smem_bytes(p);
   static bool attr_set = false;
   if (!attr_set) {
-    cudaFuncSetAttribute(k_bucket, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+    cudaFuncSetAttribute(k_bucket, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
     attr_set = true;
   }
   k_bucket<<<dim3(nc, n), kBucketThreads, smem, st>>>(X, d, chunk, P, p, fb, acc, flag);
