@@ -120,188 +120,101 @@ __global__ void k_grid_finish(const float* __restrict__ part, int n_chunks, int 
 
 // ---------------------------------------------------------------------------
 // Bucketing. Sums are fixed point: an entry of bucket k with u = (x - P_k)/D_k,
-// D_k = P_{k+1} - P_k, adds round(u * 2^fb) to the first-moment accumulator and
-// round(u^2 * 2^fb) to the second; fb is chosen from d so that no 64-bit sum
-// can overflow. Integer sums make the result independent of the order in
-// which entries are added.
+// D_k = P_{k+1} - P_k, adds round(u * 2^36) to the first-moment sum and
+// round(u^2 * 2^36) to the second. Integer sums make the result independent
+// of the order in which entries are added.
 //
-// Only 32-bit shared-memory atomics are native on this GPU, so the kernel
-// groups entries by bucket with a counting sort per tile instead of adding
-// 64-bit values atomically:
-//   1. each thread buckets 8 entries and claims a slot in its bucket with a
-//      32-bit atomic increment of the tile's bucket count;
-//   2. warp 0 turns the counts into offsets (exclusive scan);
-//   3. entries are scattered to their sorted position (u and the bucket id);
-//   4. warps sweep the sorted tile 32 entries at a time with a segmented
-//      inclusive scan (equal keys are contiguous); the last lane of each
-//      segment adds the segment's sums to the warp's private accumulators.
+// Only 32-bit shared-memory atomics are native on this GPU (64-bit and
+// floating-point ones are emulated and collapse when lanes collide, which
+// heavy-tailed inputs make the rule). So each 36-bit value is added as two
+// 18-bit limbs to 32-bit counters. A limb is below 2^18 except the high limb
+// of an entry exactly at the top of its bucket (2^18), so 2^13 entries per CTA
+// keep every counter below 2^31. Per entry: one count and four limb additions,
+// all return-less 32-bit atomics.
 
 constexpr int kBucketThreads = 256;
-constexpr int kBucketWarps = kBucketThreads / kWarp;
-constexpr int kPerThread = 8;                             // entries per thread per tile
-constexpr int kTile = kBucketThreads * kPerThread;        // 2048
+constexpr int kFixBits = 36;
+constexpr int kLimbBits = 18;
+constexpr int64_t kBucketChunk = 8192;  // entries per CTA (see above)
 
 __global__ void __launch_bounds__(kBucketThreads)
 k_bucket(const float* __restrict__ X, int64_t d, int64_t chunk, const double* __restrict__ Pall, int p, int fb,
          unsigned long long* __restrict__ acc, int32_t* __restrict__ flag) {
   extern __shared__ __align__(16) unsigned char smem[];
+  (void)fb;
   const int r = blockIdx.y;
-  const int nb = p - 1;        // real buckets 0 .. p-2; key nb collects entries that add nothing
-  double* sP = reinterpret_cast<double*>(smem);                                  // [p]
-  double* sS = sP + p;                                                           // [p] 2^fb / D_k
-  double* su = sS + p;                                                           // [kTile] sorted u * 2^fb
-  unsigned long long* wa = reinterpret_cast<unsigned long long*>(su + kTile);    // [warps][p]
-  unsigned long long* wb = wa + kBucketWarps * p;                                // [warps][p]
-  unsigned long long* ccnt = wb + kBucketWarps * p;                              // [p]
-  unsigned int* tcnt = reinterpret_cast<unsigned int*>(ccnt + p);                // [p]
-  unsigned int* toff = tcnt + p;                                                 // [p]
-  unsigned short* skey = reinterpret_cast<unsigned short*>(toff + p);            // [kTile]
+  const int nb = p - 1;
+  double* sP = reinterpret_cast<double*>(smem);                    // [p]
+  double* sS = sP + p;                                             // [p] 2^36 / D_k
+  unsigned int* hc = reinterpret_cast<unsigned int*>(sS + p);     // [p] count
+  unsigned int* ha = hc + p;                                       // [2][p] first-moment limbs (lo, hi)
+  unsigned int* hb = ha + 2 * p;                                   // [2][p] second-moment limbs
   __shared__ int s_bad;
 
   const double* P = Pall + static_cast<int64_t>(r) * p;
-  const double two_fb = ldexp(1.0, fb);
+  const double two_f = 0x1p36;
   for (int k = threadIdx.x; k < p; k += blockDim.x) {
     sP[k] = P[k];
-    sS[k] = (k < nb) ? two_fb / (P[k + 1] - P[k]) : 0.0;
-    ccnt[k] = 0ull;
+    sS[k] = (k < nb) ? two_f / (P[k + 1] - P[k]) : 0.0;
   }
-  for (int k = threadIdx.x; k < kBucketWarps * p; k += blockDim.x) {
-    wa[k] = 0ull;
-    wb[k] = 0ull;
-  }
+  for (int k = threadIdx.x; k < 5 * p; k += blockDim.x) hc[k] = 0u;
   if (threadIdx.x == 0) s_bad = 0;
   __syncthreads();
 
   const double scale = static_cast<double>(p - 1) / (sP[p - 1] - sP[0]);
-  const double inv_two_fb = ldexp(1.0, -fb);
+  const double inv_two_f = 0x1p-36;
   const double magic = 0x1p52;  // v + 2^52 keeps round(v) in the low mantissa bits for 0 <= v < 2^52
-  const unsigned long long low52 = (1ull << 52) - 1;
-  const int lane = lane_id();
-  const int w = warp_id();
+  const unsigned int lmask = (1u << kLimbBits) - 1u;
   int bad = 0;
+
+  auto one = [&](float xf) {
+    const double x = static_cast<double>(xf);
+    const int k = bucket_of(x, sP, p, scale);
+    if (k < 0) {
+      bad = 1;
+      return;
+    }
+    const double u = (x - sP[k]) * sS[k];  // in [0, 2^36]
+    const unsigned long long a = static_cast<unsigned long long>(__double_as_longlong(u + magic));
+    const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(fma(u, u * inv_two_f, magic)));
+    atomicAdd(hc + k, 1u);
+    atomicAdd(ha + k, static_cast<unsigned int>(a) & lmask);
+    atomicAdd(ha + p + k, static_cast<unsigned int>(a >> kLimbBits) & ((1u << (kFixBits + 1 - kLimbBits)) - 1u));
+    atomicAdd(hb + k, static_cast<unsigned int>(b) & lmask);
+    atomicAdd(hb + p + k, static_cast<unsigned int>(b >> kLimbBits) & ((1u << (kFixBits + 1 - kLimbBits)) - 1u));
+  };
 
   const float* x = X + static_cast<int64_t>(r) * d;
   const int64_t beg = static_cast<int64_t>(blockIdx.x) * chunk;
-  const int64_t end = beg + chunk < d ? beg + chunk : d;
-  const bool vec = ((reinterpret_cast<uintptr_t>(x + beg) & 15u) == 0);
-
-  // Entry e of a thread in the tile starting at t0: position t0 + 4*(threadIdx.x + 256*(e/4)) + e%4.
-  auto load_tile = [&](int64_t t0, float* xv) {
-#pragma unroll
-    for (int h = 0; h < kPerThread / 4; ++h) {
-      const int64_t g = t0 + 4 * (threadIdx.x + static_cast<int64_t>(kBucketThreads) * h);
-      const int cnt = g < end ? static_cast<int>(end - g < 4 ? end - g : 4) : 0;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (vec && cnt == 4) {
-        v = __ldcs(reinterpret_cast<const float4*>(x + g));
-      } else {
-        if (cnt > 0) v.x = __ldcs(x + g);
-        if (cnt > 1) v.y = __ldcs(x + g + 1);
-        if (cnt > 2) v.z = __ldcs(x + g + 2);
-        if (cnt > 3) v.w = __ldcs(x + g + 3);
-      }
-      xv[4 * h + 0] = v.x;
-      xv[4 * h + 1] = v.y;
-      xv[4 * h + 2] = v.z;
-      xv[4 * h + 3] = v.w;
+  const int len = static_cast<int>((beg + chunk < d ? beg + chunk : d) - beg);
+  const float* xc = x + beg;
+  const bool vec = ((reinterpret_cast<uintptr_t>(xc) & 15u) == 0);
+  int t = 0;
+  if (vec) {
+    const int nv = len >> 2;
+    const float4* x4 = reinterpret_cast<const float4*>(xc);
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+      const float4 v = __ldcs(x4 + i);
+      one(v.x);
+      one(v.y);
+      one(v.z);
+      one(v.w);
     }
-  };
-  auto valid = [&](int64_t t0, int e) {
-    return t0 + 4 * (threadIdx.x + static_cast<int64_t>(kBucketThreads) * (e >> 2)) + (e & 3) < end;
-  };
-
-  float xv[kPerThread];
-  if (beg < end) load_tile(beg, xv);
-  for (int64_t t0 = beg; t0 < end; t0 += kTile) {
-    for (int k = threadIdx.x; k < p; k += blockDim.x) tcnt[k] = 0u;
-    int key[kPerThread];
-#pragma unroll
-    for (int e = 0; e < kPerThread; ++e) {
-      key[e] = nb;
-      if (valid(t0, e)) {
-        const int k = bucket_of(static_cast<double>(xv[e]), sP, p, scale);
-        if (k < 0)
-          bad = 1;
-        else
-          key[e] = k;
-      }
-    }
-    __syncthreads();
-    int slot[kPerThread];
-#pragma unroll
-    for (int e = 0; e < kPerThread; ++e) slot[e] = static_cast<int>(atomicAdd(tcnt + key[e], 1u));
-    __syncthreads();
-    if (w == 0) {  // exclusive scan of the tile's counts; per-CTA counts
-      unsigned int run = 0;
-      for (int base = 0; base < p; base += kWarp) {
-        const int k = base + lane;
-        const unsigned int c = (k < p) ? tcnt[k] : 0u;
-        unsigned int incl = c;
-#pragma unroll
-        for (int o = 1; o < kWarp; o <<= 1) {
-          const unsigned int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        if (k < p) {
-          toff[k] = run + incl - c;
-          ccnt[k] += c;
-        }
-        run += __shfl_sync(0xffffffffu, incl, kWarp - 1);
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int e = 0; e < kPerThread; ++e) {
-      const int k = key[e];
-      const int pos = static_cast<int>(toff[k]) + slot[e];
-      su[pos] = (k < nb) ? (static_cast<double>(xv[e]) - sP[k]) * sS[k] : 0.0;
-      skey[pos] = static_cast<unsigned short>(k);
-    }
-    __syncthreads();
-    if (t0 + kTile < end) load_tile(t0 + kTile, xv);  // next tile in flight during the sweep
-    const int nreal = static_cast<int>(toff[nb]);      // entries with a real bucket come first
-    for (int base = w * kWarp; base < nreal; base += kBucketThreads) {
-      const int pos = base + lane;
-      int k = nb;
-      unsigned long long a = 0, b = 0;
-      if (pos < nreal) {
-        k = skey[pos];
-        const double u = su[pos];
-        a = static_cast<unsigned long long>(__double_as_longlong(u + magic)) & low52;
-        b = static_cast<unsigned long long>(__double_as_longlong(fma(u, u * inv_two_fb, magic))) & low52;
-      }
-#pragma unroll
-      for (int o = 1; o < kWarp; o <<= 1) {
-        const int ko = __shfl_up_sync(0xffffffffu, k, o);
-        const unsigned long long ao = __shfl_up_sync(0xffffffffu, a, o);
-        const unsigned long long bo = __shfl_up_sync(0xffffffffu, b, o);
-        if (lane >= o && ko == k) {
-          a += ao;
-          b += bo;
-        }
-      }
-      const int knext = __shfl_down_sync(0xffffffffu, k, 1);
-      if (k < nb && (lane == kWarp - 1 || knext != k)) {
-        wa[w * p + k] += a;
-        wb[w * p + k] += b;
-      }
-    }
-    __syncthreads();
+    t = nv << 2;
   }
+  for (int i = t + threadIdx.x; i < len; i += blockDim.x) one(__ldcs(xc + i));
   if (bad) s_bad = 1;
   __syncthreads();
 
   unsigned long long* gacc = acc + static_cast<int64_t>(r) * nb * 3;
   for (int k = threadIdx.x; k < nb; k += blockDim.x) {
-    const unsigned long long c = ccnt[k];
+    const unsigned int c = hc[k];
     if (c) {
-      unsigned long long sa = 0, sb = 0;
-#pragma unroll
-      for (int q = 0; q < kBucketWarps; ++q) {
-        sa += wa[q * p + k];
-        sb += wb[q * p + k];
-      }
-      atomicAdd(gacc + 3 * k + 0, c);
+      const unsigned long long sa = static_cast<unsigned long long>(ha[k]) +
+                                    (static_cast<unsigned long long>(ha[p + k]) << kLimbBits);
+      const unsigned long long sb = static_cast<unsigned long long>(hb[k]) +
+                                    (static_cast<unsigned long long>(hb[p + k]) << kLimbBits);
+      atomicAdd(gacc + 3 * k + 0, static_cast<unsigned long long>(c));
       atomicAdd(gacc + 3 * k + 1, sa);
       atomicAdd(gacc + 3 * k + 2, sb);
     }
@@ -331,10 +244,8 @@ __global__ void k_bucket_finish(const unsigned long long* __restrict__ acc, cons
 }  // namespace
 
 int bucket_fraction_bits(int64_t d) {
-  int lg = 0;
-  while ((int64_t(1) << lg) < d + 1) ++lg;
-  int fb = 63 - lg - 1;
-  return fb > 50 ? 50 : fb;
+  (void)d;
+  return kFixBits;
 }
 
 int64_t minmax_chunk(int64_t d) { return d < 16384 ? d : 16384; }
@@ -350,13 +261,9 @@ cudaError_t launch_uniform_grid(const float* X, int n, int64_t d, int p, double*
   return cudaGetLastError();
 }
 
-size_t bucket_smem_bytes(int p) {
-  return static_cast<size_t>(p) * 8 * 2 + static_cast<size_t>(kTile) * 8 +
-         static_cast<size_t>(kBucketWarps) * p * 16 + static_cast<size_t>(p) * 8 + static_cast<size_t>(p) * 8 +
-         static_cast<size_t>(kTile) * 2;
-}
+size_t bucket_smem_bytes(int p) { return static_cast<size_t>(p) * (8 * 2 + 4 * 5); }
 
-int64_t bucket_chunk(int64_t d) { return d < 32768 ? d : 32768; }
+int64_t bucket_chunk(int64_t d) { return d < kBucketChunk ? d : kBucketChunk; }
 
 cudaError_t launch_bucket(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt,
                           double* A, double* B, int32_t* status, unsigned long long* acc,
