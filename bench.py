@@ -160,7 +160,7 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
                                       out["theta"])
             ev["e1"].record(stream)
         else:
-            out = E.solve_stats(cnt, A, B, P, d, s, lam, fp64=fp64)
+            out = E.solve_stats(cnt, A, B, P, d, s, lam, fp64=fp64, hirschberg=w.hirschberg)
             ev_dp1.record(stream)
             Q = out["Q"][:, 0, :].contiguous()
             Ql = out["Q_len"][:, 0].contiguous()

@@ -40,13 +40,11 @@ struct SolveWs {
   double* A;
   double* B;
   int32_t* bstatus;
-  uint32_t* tasks;
-  int32_t* ntasks;
   unsigned char* scratch;
   size_t bytes;
 };
 
-bool solve_ws(void* ws, int n, int p, int s, const DpPlan& plan, SolveWs* w) {
+bool solve_ws(void* ws, int n, int p, const DpPlan& plan, SolveWs* w) {
   Carver c{static_cast<unsigned char*>(ws)};
   const size_t nb = static_cast<size_t>(n) * (p - 1);
   w->acc = c.take<unsigned long long>(3 * nb);
@@ -55,9 +53,6 @@ bool solve_ws(void* ws, int n, int p, int s, const DpPlan& plan, SolveWs* w) {
   w->A = c.take<double>(nb);
   w->B = c.take<double>(nb);
   w->bstatus = c.take<int32_t>(n);
-  const int S = s < p ? s : p;
-  w->tasks = c.take<uint32_t>(static_cast<size_t>(plan.max_tasks) * S);
-  w->ntasks = c.take<int32_t>(S);
   w->scratch = c.take<unsigned char>(plan.scratch_per_cta * plan.ctas);
   w->bytes = c.off;
   return true;
@@ -105,9 +100,9 @@ size_t ecasq_aux_workspace_size(int n, int64_t d, int p) {
 size_t ecasq_workspace_size(int n, int64_t d, int p, int s, int n_lambda, const ecasq_opts* opts) {
   if (!valid_sizes(n, d, p, s) || n_lambda < 1) return 0;
   DpPlan plan;
-  if (!dp_plan(n, p, s, opts && opts->dp_fp64, &plan)) return 0;
+  if (!dp_plan(n, p, s, opts && opts->dp_fp64, opts && opts->hirschberg, &plan)) return 0;
   SolveWs w;
-  solve_ws(nullptr, n, p, s, plan, &w);
+  solve_ws(nullptr, n, p, plan, &w);
   return w.bytes;
 }
 
@@ -140,9 +135,9 @@ static int solve_common(const float* X, const int64_t* cnt, const double* A, con
                         int64_t d, int p, int s, int n_lambda, const ecasq_opts* opts, void* ws, size_t ws_bytes,
                         cudaStream_t st, DpArgs* args, DpPlan* plan, SolveWs* w) {
   if (!P || !valid_sizes(n, d, p, s) || n_lambda < 1) return ECASQ_ERR_ARG;
-  if (opts && (opts->reserved != 0 || opts->bisect_steps < 0 || opts->hirschberg)) return ECASQ_ERR_ARG;
-  if (!dp_plan(n, p, s, opts && opts->dp_fp64, plan)) return ECASQ_ERR_ARG;
-  solve_ws(ws, n, p, s, *plan, w);
+  if (opts && (opts->reserved != 0 || opts->bisect_steps < 0)) return ECASQ_ERR_ARG;
+  if (!dp_plan(n, p, s, opts && opts->dp_fp64, opts && opts->hirschberg, plan)) return ECASQ_ERR_ARG;
+  solve_ws(ws, n, p, *plan, w);
   if (!ws || ws_bytes < w->bytes) return ECASQ_ERR_WORKSPACE;
   DpArgs& a = *args;
   a = DpArgs{};
@@ -191,7 +186,7 @@ static int solve_lambdas(const float* X, const int64_t* cnt, const double* A, co
   a.mse = mse;
   a.H = H;
   a.status = status;
-  return cuda_status(launch_dp(plan, a, w.tasks, w.ntasks, st));
+  return cuda_status(launch_dp(plan, a, st));
 }
 
 static int solve_budget(const float* X, const int64_t* cnt, const double* A, const double* B, const double* P, int n,
@@ -223,7 +218,7 @@ static int solve_budget(const float* X, const int64_t* cnt, const double* A, con
   a.mse1 = mse1;
   a.mse2 = mse2;
   a.status = status;
-  return cuda_status(launch_dp(plan, a, w.tasks, w.ntasks, st));
+  return cuda_status(launch_dp(plan, a, st));
 }
 
 int ecasq_solve(const float* X, const double* P, int n, int64_t d, int p, int s, const double* lambda, int n_lambda,

@@ -5,7 +5,9 @@
 //   §2.2 "Programação Dinâmica Ótima": the ASQ DP does not extend because the
 //        entropy term of a value depends on both neighbours, so the state is a
 //        PAIR of consecutive values, dp_OPT(i, l, j); the direct programme costs
-//        O(d^3 s) time over the entries, O(p^3 s) over a permissible set P.
+//        O(d^3 s) time over the entries, O(p^3 s) over a permissible set P;
+//        "Algoritmo de Hirschberg": divide and conquer that keeps only two DP
+//        layers, O(d^2) (here O(p^2)) memory.
 //
 // Recurrence evaluated here (i = number of values up to and including P_l,
 // counting c_1 = P_0; m = mu/d the normalised mass of a value):
@@ -21,12 +23,17 @@
 //     lambdas, or the whole bisection), so the pair tables are built once;
 //   * the tables and the two live DP layers sit in shared memory when they fit
 //     (fp32, p <= 128) and in a per-CTA global (L2-resident) slab otherwise;
-//   * one DP layer is a list of tasks (row l, a block of <= 64 j, a k-split of
-//     1..32 lanes) in descending cost order, taken by warps from a shared
-//     counter; each lane keeps 2 j in registers and sweeps k with broadcast
-//     loads; k-splits merge with a warp-shuffle argmin;
-//   * back-pointers go to a per-CTA global slab; the backtrack, the fp64
-//     evaluation of the chosen code and the bisection run in the same kernel.
+//   * a DP layer is split into tasks of 32 lanes; a lane owns 4 outputs
+//     (l, j0..j0+3) of one row and sweeps k down the column of l in two
+//     interleaved streams; tasks are decoded in closed form from their index,
+//     longest rows first, and taken by warps from a shared counter;
+//   * store mode keeps back-pointers in a per-CTA global slab and backtracks;
+//     Hirschberg mode keeps none: a forward pass finds the optimum and its last
+//     pair, then the code is recovered by divide and conquer, joining a forward
+//     pass over the left part with a pass over the reflected alphabet
+//     (P'_k = -P_{p-1-k}) for the right part;
+//   * the fp64 evaluation of the chosen code and the bisection run in the same
+//     kernel.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -42,19 +49,12 @@ constexpr int kWarps = kThreads / kWarp;
 constexpr int kTJ = 4;  // outputs (l, j0 .. j0+3) per lane
 constexpr int kNQ = 2;  // interleaved k-streams per output (kTJ * kNQ independent min chains per lane)
 
-// A group descriptor names up to kTJ outputs (l, j0 .. j0 + n - 1) of one layer:
-// l in bits 0..9, j0 in bits 10..19, n - 1 in bits 20..22.
-__host__ __device__ inline uint32_t pack_group(int l, int j0, int n) {
-  return static_cast<uint32_t>(l) | (static_cast<uint32_t>(j0) << 10) | (static_cast<uint32_t>(n - 1) << 20);
-}
-__host__ __device__ inline int max_groups(int p) { return p * ((p + kTJ - 1) / kTJ + 1); }
-
 template <typename T>
 struct Arith;
 
 template <>
 struct Arith<float> {
-  // Added to every R/d so that a mass is never 0 inside the sweep:
+  // Added to every mass so that log2 never sees 0 inside the sweep:
   // h(2^-100) ~ 8e-29, far below fp32 resolution of any objective.
   static constexpr float kEps = 0x1p-100f;
   __device__ static float inf() { return __int_as_float(0x7f800000); }
@@ -72,9 +72,9 @@ struct Arith<double> {
   __device__ static double vmin(double a, double b) { return fmin(a, b); }
 };
 
-// One entry of a live DP layer: the layer value G = F_{i-1}(k, l) and
-// a = R(k, l)/d + eps side by side, so one 8- (16-) byte shared load feeds a
-// whole k step. a is written once per vector into both ping-pong layers.
+// One entry of a live DP layer: the layer value G = F(k, l) and a = R(k, l)/d
+// (+ eps) side by side, so one 8- (16-) byte shared load feeds a whole k step.
+// a is written once per vector into both ping-pong layers.
 template <typename T>
 struct alignas(2 * sizeof(T)) GA {
   T g, a;
@@ -86,8 +86,6 @@ struct alignas(2 * sizeof(T)) GA {
 // padded so that cb[l] = l (mod 16): lanes that hold 16 consecutive rows l
 // then read 16 distinct 8-byte bank pairs at every k. b = L/d and V/d are read
 // once per output and stay in the row-triangle layout (row_off(l) + j - l - 1).
-
-// cb[0..p]: padded column starts; cb[p] = elements of one layer buffer.
 __host__ __device__ inline int next_colbase(int prev_base, int prev_col) {
   int c = prev_base + prev_col;  // column prev_col holds prev_col entries
   const int want = (prev_col + 1) & 15;
@@ -100,35 +98,61 @@ __host__ __device__ inline int layer_elems(int p) {
   return c;
 }
 
+// Groups of kTJ outputs of a layer, counted from the last row upward (rows
+// e0-1, e0-2, ...; a row with n outputs holds ceil(n/4) groups). The rows with
+// 1 .. n outputs hold G(n) = 2m(m+1) + r(m+1) groups, n = 4m + r; a group index
+// inverts G with one square root.
+__host__ __device__ inline int groups_upto(int n) {
+  const int m = n >> 2, r = n & 3;
+  return 2 * m * (m + 1) + r * (m + 1);
+}
+__device__ inline void decode_group(int q, int e0, int& l, int& j0, int& nv) {
+  int n = static_cast<int>(sqrtf(8.f * q + 4.f) - 2.f);
+  n = n < 1 ? 1 : n;
+  while (groups_upto(n) <= q) ++n;
+  while (n > 1 && groups_upto(n - 1) > q) --n;
+  l = e0 - n;
+  j0 = l + 1 + kTJ * (q - groups_upto(n - 1));
+  nv = min(kTJ, e0 - j0 + 1);
+}
+
+// The tables a pass reads: two ping-pong layer buffers (with a) and b, V/d.
+template <typename T>
+struct Tables {
+  GA<T>* buf0;
+  GA<T>* buf1;
+  T* rowB;
+  T* rowV;
+  __device__ __forceinline__ GA<T>* layer(int t) const { return (t & 1) ? buf1 : buf0; }
+};
+
 template <typename T>
 struct Ctx {
   int p, S, tri;
   double dd;
-  GA<T>* ga0;  // DP layers of even / odd i (with a), column layout
-  GA<T>* ga1;
-  const int* cb;  // [p+1] padded column starts (shared memory)
-  __device__ __forceinline__ GA<T>* layer(int i) const { return (i & 1) ? ga1 : ga0; }
-  T* rowB;     // L(l,j)/d
-  T* rowV;     // V(l,j)/d
-  uint16_t* bp;  // [S][tri] back-pointers
+  Tables<T> fw;  // the alphabet as given
+  Tables<T> rf;  // the reflected alphabet (Hirschberg mode)
+  const int* cb;              // [p+1] padded column starts (shared memory)
+  uint16_t* bp;               // [S][tri] back-pointers (store mode)
   double *sP, *sN, *sA, *sB;  // [p] alphabet and bucket statistics
   double *sR, *sL;            // [S] evaluation scratch
   T* rmin;                    // [p] row minima (lambda = 0)
   int* rarg;                  // [p]
   int* ctr;                   // [S] task counters
   int* sQ;                    // [S] code of the last solve
-  const uint32_t* groups;  // [S][max_groups] group descriptors per layer
-  const int32_t* ngroups;  // [S]
-  int max_groups;
+  int* stk;                   // [2S] Hirschberg segment stack
+  bool hirschberg;
 };
 
 struct SolveOut {
   double mse, H, J;
   int m;
   int bestI, bestK;
+  int jx, jy;  // Hirschberg join result
+  int nstk;
 };
 
-// ---- table build -------------------------------------------------------------
+// ---- tables --------------------------------------------------------------------
 // For every pair a < c, sums over the buckets a .. c-1 (ascending), with
 // delta_k = P_k - P_a:  N = sum n_k, T1 = sum (A_k + n_k delta_k),
 // T2 = sum (B_k + 2 delta_k A_k + n_k delta_k^2); W = P_c - P_a;
@@ -154,27 +178,57 @@ __device__ __forceinline__ void build_tables(const Ctx<T>& c) {
       double L = N - R;
       L = L > 0.0 ? L : 0.0;
       const T av = static_cast<T>(R / c.dd) + Arith<T>::kEps;
-      c.ga0[c.cb[cc] + a].a = av;
-      c.ga1[c.cb[cc] + a].a = av;
-      c.rowB[ro + cc] = static_cast<T>(L / c.dd);
-      c.rowV[ro + cc] = static_cast<T>(V / c.dd);
+      c.fw.buf0[c.cb[cc] + a].a = av;
+      c.fw.buf1[c.cb[cc] + a].a = av;
+      c.fw.rowB[ro + cc] = static_cast<T>(L / c.dd);
+      c.fw.rowV[ro + cc] = static_cast<T>(V / c.dd);
     }
   }
 }
 
-// ---- one layer ---------------------------------------------------------------
-
-// Best (E, i, k) over the finished layer i: E = F_i(k, p-1) + h(R(k,p-1)/d).
-// Warp 0 only. Strict '<' over layers in ascending order keeps the smaller code.
+// Reflected tables, from the forward ones: with r(x) = p-1-x,
+//   R'(k', l') = L(r(l'), r(k')),  L'(l', j') = R(r(j'), r(l')),  V'(l', j') = V(r(j'), r(l')).
 template <typename T>
-__device__ __forceinline__ void finalize_layer(const Ctx<T>& c, int i, const GA<T>* G, bool sep, T* bestE,
-                                               int* bestI, int* bestK) {
+__device__ __forceinline__ void build_reflected(const Ctx<T>& c) {
   const int p = c.p;
-  const int kb = (i == 1) ? 0 : i - 1;
-  const int ke = (i == 1) ? 0 : p - 2;
+  for (int l = 1 + threadIdx.x / kWarp; l < p; l += blockDim.x / kWarp) {
+    for (int k = lane_id(); k < l; k += kWarp) {
+      const int rl = p - 1 - l, rk = p - 1 - k;  // rl < rk
+      const T av = c.fw.rowB[row_off(rl, p) + rk - rl - 1] + Arith<T>::kEps;
+      c.rf.buf0[c.cb[l] + k].a = av;
+      c.rf.buf1[c.cb[l] + k].a = av;
+      // (k, l) as a row pair of the reflected problem: row k, column l.
+      const int e = row_off(k, p) + l - k - 1;
+      const int rl2 = p - 1 - l, rk2 = p - 1 - k;  // original interval [rl2, rk2]
+      c.rf.rowB[e] = c.fw.buf0[c.cb[rk2] + rl2].a;
+      c.rf.rowV[e] = c.fw.rowV[row_off(rl2, p) + rk2 - rl2 - 1];
+    }
+  }
+}
+
+// ---- one pass of DP layers ------------------------------------------------------
+// Layers 1 .. T over the values s0 .. e0: layer t holds F_t(l, j), the best cost
+// of t values from s0 up to l, followed by j. Layer 1 is row s0 alone; its
+// value's mass adds `extra` (the share from a fixed left neighbour; < 0 when
+// s0 has none). With last_only the last layer is computed for j = e0 only.
+struct Pass {
+  int s0, e0, T;
+  bool last_only;
+  double extra;
+  bool store_bp;
+  bool finalize;
+};
+
+template <typename T>
+__device__ __forceinline__ void finalize_layer(const Ctx<T>& c, const Tables<T>& tb, int i, int s0, int e0,
+                                               const GA<T>* G, bool sep, T* bestE, int* bestI, int* bestK) {
+  // Best (E, i, k) over the finished layer i: E = F_i(k, e0) + h(R(k, e0)/d).
+  // Warp 0 only. Strict '<' over layers in ascending order keeps the smaller code.
+  const int kb = (i == 1) ? s0 : s0 + i - 1;
+  const int ke = (i == 1) ? s0 : e0 - 1;
   T best = Arith<T>::inf();
   int arg = 0x7fffffff;
-  const GA<T>* col = G + c.cb[p - 1];
+  const GA<T>* col = G + c.cb[e0];
   for (int k = kb + lane_id(); k <= ke; k += kWarp) {
     const GA<T> ga = col[k];
     T e = ga.g;
@@ -190,29 +244,30 @@ __device__ __forceinline__ void finalize_layer(const Ctx<T>& c, int i, const GA<
     *bestI = i;
     *bestK = arg;
   }
+  (void)tb;
 }
 
-// One task of layer i >= 3: 32 group descriptors, one per lane. Lane L owns
-// the outputs (l, j0 .. j0+n-1) and sweeps k = i-2 .. l-1 down its column in
-// kNQ interleaved streams (each output and stream keeps its own running
-// minimum, so consecutive updates do not wait on one another). The k range
-// common to the warp runs unpredicated; the rest masks the layer value to +inf
-// past the lane's own column.
+// One task of a layer: 32 groups, one per lane. The lane owns the outputs
+// (l, j0 .. j0+nv-1) and sweeps k = kmin .. l-1 down its column in kNQ
+// interleaved streams (each output and stream keeps its own running minimum,
+// so consecutive updates do not wait on one another). The k range common to
+// the warp runs unpredicated; the rest masks the layer value to +inf past the
+// lane's own column.
 template <typename T>
-__device__ __forceinline__ void run_task(const Ctx<T>& c, uint32_t desc, bool active, int i,
-                                         const GA<T>* __restrict__ Gp, GA<T>* __restrict__ Gc,
+__device__ __forceinline__ void run_task(const Ctx<T>& c, const Tables<T>& tb, int l, int j0, int nv, bool active,
+                                         int kmin, const GA<T>* __restrict__ Gp, GA<T>* __restrict__ Gc,
                                          uint16_t* __restrict__ bpi, T invl) {
   const int p = c.p;
-  const int kmin = i - 2;
-  const int l = active ? static_cast<int>(desc & 1023) : kmin + 1;  // inactive lanes: any in-range row
-  const int j0 = static_cast<int>((desc >> 10) & 1023);
-  const int nv = active ? static_cast<int>((desc >> 20) & 7) + 1 : 0;
+  if (!active) {
+    l = kmin + 1;  // inactive lanes sweep an in-range column and write nothing
+    nv = 0;
+  }
   const int lmin = __reduce_min_sync(0xffffffffu, active ? l : 0x7fffffff);
   const int lmax = __reduce_max_sync(0xffffffffu, active ? l : 0);
   const int ro = row_off(l, p) - l - 1;
   T b[kTJ];
 #pragma unroll
-  for (int u = 0; u < kTJ; ++u) b[u] = (u < nv) ? c.rowB[ro + j0 + u] : T(0);
+  for (int u = 0; u < kTJ; ++u) b[u] = (u < nv) ? tb.rowB[ro + j0 + u] : T(0);
   const GA<T>* __restrict__ col = Gp + c.cb[l];
 
   T best[kTJ][kNQ];
@@ -269,63 +324,56 @@ __device__ __forceinline__ void run_task(const Ctx<T>& c, uint32_t desc, bool ac
   for (int u = 0; u < kTJ; ++u) {
     if (u < nv) {
       const int e = ro + j0 + u;
-      Gc[c.cb[j0 + u] + l].g = c.rowV[e] * invl + best[u][0];
-      bpi[e] = static_cast<uint16_t>(arg[u][0]);
+      Gc[c.cb[j0 + u] + l].g = tb.rowV[e] * invl + best[u][0];
+      if (bpi) bpi[e] = static_cast<uint16_t>(arg[u][0]);
     }
   }
 }
 
-// One full solve at lambda (all threads). Leaves the code in c.sQ and the fp64
-// evaluation in *out (shared).
+// Runs the pass; all threads. Leaves layer T in tb.layer(T).
 template <typename T>
-__device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out, T* bestE) {
-  const int p = c.p, S = c.S, tri = c.tri;
-  // Below kMinLambda the entropy terms vanish under the precision of T and
-  // 1/lambda would overflow it: the layers then run the MSE-only programme
-  // (the code is still evaluated in fp64 at the true lambda).
-  const double kMinLambda = sizeof(T) == 4 ? 1e-30 : 1e-290;
-  const bool sep = !(lam > kMinLambda);
-  const T invl = sep ? T(1) : static_cast<T>(1.0 / lam);
+__device__ __forceinline__ void run_pass(const Ctx<T>& c, const Tables<T>& tb, const Pass& ps, bool sep, T invl,
+                                         SolveOut* out, T* bestE) {
+  const int p = c.p, tri = c.tri;
+  const int s0 = ps.s0, e0 = ps.e0;
   const int tid = threadIdx.x;
   const int warp = warp_id(), lane = lane_id();
-
-  for (int t = tid; t < S; t += blockDim.x) c.ctr[t] = 0;
-  if (tid == 0) {
-    *bestE = Arith<T>::inf();
-    out->bestI = -1;
-    out->bestK = -1;
-  }
-  // Layer 1: F_1(0, j) (row 0), written to buffer 1.
-  {
-    GA<T>* G1 = c.ga1;
-    for (int j = 1 + tid; j < p; j += blockDim.x) {
-      const int e = j - 1;
-      T f = c.rowV[e] * invl;
-      if (!sep) f += Arith<T>::nlog(c.rowB[e] + Arith<T>::kEps);
-      G1[c.cb[j]].g = f;
+  for (int t = tid; t < c.S; t += blockDim.x) c.ctr[t] = 0;
+  {  // layer 1: row s0
+    GA<T>* G1 = tb.layer(1);
+    const T extra = ps.extra > 0.0 ? static_cast<T>(ps.extra) : T(0);
+    const int ro = row_off(s0, p) - s0 - 1;
+    const int jb = (ps.T == 1 && ps.last_only) ? e0 : s0 + 1;
+    for (int j = jb + tid; j <= e0; j += blockDim.x) {
+      const int e = ro + j;
+      T f = tb.rowV[e] * invl;
+      if (!sep) f += Arith<T>::nlog(tb.rowB[e] + extra + Arith<T>::kEps);
+      G1[c.cb[j] + s0].g = f;
     }
   }
   __syncthreads();
-  for (int i = 2; i <= S - 1; ++i) {
-    const GA<T>* Gp = c.layer(i - 1);
-    GA<T>* Gc = c.layer(i);
-    uint16_t* bpi = c.bp + static_cast<size_t>(i) * tri;
-    const bool last = (i == S - 1);
-    if (warp == 0) finalize_layer(c, i - 1, Gp, sep, bestE, &out->bestI, &out->bestK);
-    if (i == 2) {
-      // Only k = c_1 = 0 precedes the second value.
-      for (int l = 1 + warp; l <= p - 2; l += kWarps) {
-        const GA<T> ga = Gp[c.cb[l]];  // (0, l)
+  for (int t = 2; t <= ps.T; ++t) {
+    const GA<T>* Gp = tb.layer(t - 1);
+    GA<T>* Gc = tb.layer(t);
+    uint16_t* bpi = ps.store_bp ? c.bp + static_cast<size_t>(t) * tri : nullptr;
+    const bool last = ps.last_only && t == ps.T;
+    const int r0 = s0 + t - 1;  // first row of the layer
+    if (ps.finalize && warp == 0) finalize_layer(c, tb, t - 1, s0, e0, Gp, sep, bestE, &out->bestI, &out->bestK);
+    if (t == 2) {
+      // Only k = s0 precedes the second value.
+      for (int l = r0 + warp; l <= e0 - 1; l += kWarps) {
+        const GA<T> ga = Gp[c.cb[l] + s0];  // (s0, l)
         const int ro = row_off(l, p) - l - 1;
-        for (int j = (last ? p - 1 : l + 1) + lane; j <= p - 1; j += kWarp) {
+        for (int j = (last ? e0 : l + 1) + lane; j <= e0; j += kWarp) {
           const int e = ro + j;
-          const T v = sep ? ga.g : Arith<T>::fold(ga.g, ga.a + c.rowB[e]);
-          Gc[c.cb[j] + l].g = c.rowV[e] * invl + v;
+          const T v = sep ? ga.g : Arith<T>::fold(ga.g, ga.a + tb.rowB[e]);
+          Gc[c.cb[j] + l].g = tb.rowV[e] * invl + v;
+          if (bpi) bpi[e] = static_cast<uint16_t>(s0);
         }
       }
     } else if (sep) {
-      const int kmin = i - 2;
-      for (int l = i - 1 + warp; l <= p - 2; l += kWarps) {
+      const int kmin = s0 + t - 2;
+      for (int l = r0 + warp; l <= e0 - 1; l += kWarps) {
         T best = Arith<T>::inf();
         int arg = kmin;
         for (int k = kmin + lane; k < l; k += kWarp) {
@@ -342,111 +390,235 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
         }
       }
       __syncthreads();
-      for (int l = i - 1 + warp; l <= p - 2; l += kWarps) {
+      for (int l = r0 + warp; l <= e0 - 1; l += kWarps) {
         const int ro = row_off(l, p) - l - 1;
         const T rm = c.rmin[l];
         const uint16_t ra = static_cast<uint16_t>(c.rarg[l]);
-        for (int j = (last ? p - 1 : l + 1) + lane; j <= p - 1; j += kWarp) {
+        for (int j = (last ? e0 : l + 1) + lane; j <= e0; j += kWarp) {
           const int e = ro + j;
-          Gc[c.cb[j] + l].g = c.rowV[e] + rm;
-          bpi[e] = ra;
+          Gc[c.cb[j] + l].g = tb.rowV[e] + rm;
+          if (bpi) bpi[e] = ra;
         }
       }
-    } else {
-      // Tasks in descending cost: higher rows have longer k sweeps.
-      const uint32_t* pl = c.groups + static_cast<size_t>(i) * c.max_groups;
-      const int np = c.ngroups[i];
-      const int nt = (np + kWarp - 1) / kWarp;
-      // The next task's index and descriptor are fetched before the current
-      // task runs, so their latency hides behind the sweep.
-      auto fetch = [&](int& t, uint32_t& d, bool& act) {
-        int tt = 0;
-        if (lane == 0) tt = atomicAdd(c.ctr + i, 1);
-        t = __shfl_sync(0xffffffffu, tt, 0);
-        const int q = (nt - 1 - t) * kWarp + lane;
-        act = (t < nt) && q < np;
-        d = act ? pl[q] : 0u;
-      };
-      int t;
-      uint32_t d;
-      bool act;
-      fetch(t, d, act);
-      while (t < nt) {
-        int tn;
-        uint32_t dn;
-        bool an;
-        fetch(tn, dn, an);
-        run_task(c, d, act, i, Gp, Gc, bpi, invl);
-        t = tn;
-        d = dn;
-        act = an;
+    } else if (r0 <= e0 - 1) {
+      const int kmin = s0 + t - 2;
+      const int ng = last ? (e0 - r0) : groups_upto(e0 - r0);
+      const int nt = (ng + kWarp - 1) / kWarp;
+      // Tasks in index order are the longest rows first. The next task index
+      // is fetched before the current task runs.
+      int tn = 0;
+      if (lane == 0) tn = atomicAdd(c.ctr + t, 1);
+      tn = __shfl_sync(0xffffffffu, tn, 0);
+      while (tn < nt) {
+        const int tk = tn;
+        if (lane == 0) tn = atomicAdd(c.ctr + t, 1);
+        tn = __shfl_sync(0xffffffffu, tn, 0);
+        const int q = tk * kWarp + lane;
+        const bool act = q < ng;
+        int l = 0, j0 = 0, nv = 0;
+        if (act) {
+          if (last) {
+            l = e0 - 1 - q;
+            j0 = e0;
+            nv = 1;
+          } else {
+            decode_group(q, e0, l, j0, nv);
+          }
+        }
+        run_task(c, tb, l, j0, nv, act, kmin, Gp, Gc, bpi, invl);
       }
     }
     __syncthreads();
   }
-  if (warp == 0) finalize_layer(c, S - 1, c.layer(S - 1), sep, bestE, &out->bestI, &out->bestK);
+  if (ps.finalize && warp == 0)
+    finalize_layer(c, tb, ps.T, s0, e0, tb.layer(ps.T), sep, bestE, &out->bestI, &out->bestK);
   __syncthreads();
+}
 
-  // Backtrack: c_{i+1} = p-1, c_i = k, c_{ii-1} = bp_ii(c_ii, c_{ii+1}), c_1 = 0.
+// Hirschberg join: the split pair (x, y) minimising
+//   F(x, y) + F'(r(y), r(x)) - V(x, y)/(lambda d)
+// over x in [xlo, xhi], y in [x+1, yhi] (y = yhi only when fixed); ties go to
+// the smaller x, then the smaller y. All threads; result in out->jx, out->jy.
+template <typename T>
+__device__ __forceinline__ void join(const Ctx<T>& c, const GA<T>* Ff, const GA<T>* Fb, int xlo, int xhi, int yhi,
+                                     bool yfixed, T invl, SolveOut* out, T* wbest, int* warg) {
+  const int p = c.p;
+  const int warp = warp_id(), lane = lane_id();
+  T best = Arith<T>::inf();
+  int arg = 0x7fffffff;
+  for (int x = xlo + warp; x <= xhi; x += kWarps) {
+    const int ro = row_off(x, p) - x - 1;
+    const int rx = p - 1 - x;
+    for (int y = (yfixed ? yhi : x + 1) + lane; y <= yhi; y += kWarp) {
+      const T v = Ff[c.cb[y] + x].g + Fb[c.cb[rx] + (p - 1 - y)].g - c.fw.rowV[ro + y] * invl;
+      const int id = x * p + y;
+      if (v < best || (v == best && id < arg)) {
+        best = v;
+        arg = id;
+      }
+    }
+  }
+  warp_argmin(best, arg);
+  if (lane == 0) {
+    wbest[warp] = best;
+    warg[warp] = arg;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    best = lane < kWarps ? wbest[lane] : Arith<T>::inf();
+    arg = lane < kWarps ? warg[lane] : 0x7fffffff;
+    warp_argmin(best, arg);
+    if (lane == 0) {
+      if (arg == 0x7fffffff) arg = xlo * p + (yfixed ? yhi : xlo + 1);  // non-finite values only
+      out->jx = arg / p;
+      out->jy = arg % p;
+    }
+  }
+  __syncthreads();
+}
+
+// fp64 evaluation of the code in c.sQ from the bucket statistics (warp 0).
+template <typename T>
+__device__ __forceinline__ void evaluate(const Ctx<T>& c, double lam, SolveOut* out) {
+  if (warp_id() != 0) return;
+  const int lane = lane_id();
+  const int m = out->m;
+  double vs = 0.0;
+  for (int t = lane; t < m - 1; t += kWarp) {
+    const int a = c.sQ[t], cc = c.sQ[t + 1];
+    double N = 0.0, T1 = 0.0, T2 = 0.0;
+    const double Pa = c.sP[a];
+    for (int k = a; k < cc; ++k) {
+      const double dk = c.sP[k] - Pa;
+      const double nk = c.sN[k];
+      N += nk;
+      T1 += c.sA[k] + nk * dk;
+      T2 += c.sB[k] + 2.0 * dk * c.sA[k] + nk * dk * dk;
+    }
+    const double W = c.sP[cc] - Pa;
+    double V = W * T1 - T2;
+    V = V > 0.0 ? V : 0.0;
+    const double R = T1 / W;
+    c.sR[t] = R;
+    c.sL[t] = N - R;
+    vs += V;
+  }
+  __syncwarp();
+  double hs = 0.0;
+  for (int t = lane; t < m; t += kWarp) {
+    const double mu = (t > 0 ? c.sR[t - 1] : 0.0) + (t < m - 1 ? c.sL[t] : 0.0);
+    if (mu > 0.0) {
+      const double q = mu / c.dd;
+      hs -= q * log2(q);
+    }
+  }
+  vs = warp_sum(vs);
+  hs = warp_sum(hs);
+  if (lane == 0) {
+    out->mse = vs / c.dd;
+    out->H = hs;
+    out->J = out->mse + lam * hs;
+  }
+}
+
+// One full solve at lambda (all threads). Leaves the code in c.sQ and the fp64
+// evaluation in *out (shared).
+template <typename T>
+__device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out, T* bestE, T* wbest, int* warg) {
+  const int p = c.p, S = c.S, tri = c.tri;
+  // Below kMinLambda the entropy terms vanish under the precision of T and
+  // 1/lambda would overflow it: the layers then run the MSE-only programme
+  // (the code is still evaluated in fp64 at the true lambda).
+  const double kMinLambda = sizeof(T) == 4 ? 1e-30 : 1e-290;
+  const bool sep = !(lam > kMinLambda);
+  const T invl = sep ? T(1) : static_cast<T>(1.0 / lam);
+  const int tid = threadIdx.x;
+
+  if (tid == 0) {
+    *bestE = Arith<T>::inf();
+    out->bestI = -1;
+    out->bestK = -1;
+  }
+  __syncthreads();
+  // The whole alphabet, from c_1 = P_0; the last layer needs only j = p-1.
+  Pass full{0, p - 1, S - 1, true, -1.0, !c.hirschberg, true};
+  run_pass(c, c.fw, full, sep, invl, out, bestE);
+
   if (tid == 0) {
     if (out->bestI < 1) {  // no finite candidate (non-finite inputs): fall back to {P_0, P_{p-1}}
       out->bestI = 1;
       out->bestK = 0;
     }
     const int bi = out->bestI;
-    int l = out->bestK, j = p - 1;
     c.sQ[bi] = p - 1;
-    c.sQ[bi - 1] = l;
-    for (int ii = bi; ii >= 2; --ii) {
-      const int kk = (ii == 2) ? 0 : static_cast<int>(c.bp[static_cast<size_t>(ii) * tri + row_off(l, p) + j - l - 1]);
-      c.sQ[ii - 2] = kk;
-      j = l;
-      l = kk;
-    }
+    c.sQ[bi - 1] = out->bestK;
+    c.sQ[0] = 0;
     out->m = bi + 1;
+    if (!c.hirschberg) {
+      // Backtrack: c_{i+1} = p-1, c_i = k, c_{ii-1} = bp_ii(c_ii, c_{ii+1}), c_1 = 0.
+      int l = out->bestK, j = p - 1;
+      for (int ii = bi; ii >= 2; --ii) {
+        const int kk = (ii == 2) ? 0 : static_cast<int>(c.bp[static_cast<size_t>(ii) * tri + row_off(l, p) + j - l - 1]);
+        c.sQ[ii - 2] = kk;
+        j = l;
+        l = kk;
+      }
+      out->nstk = 0;
+    } else {
+      // Segments (lo, hi): c[lo] (with c[lo-1] when lo >= 1) and the pair
+      // (c[hi], c[hi+1]) are known; c[lo+1 .. hi-1] are not.
+      const int m = bi + 1;
+      out->nstk = 0;
+      if (m - 3 >= 1) {
+        c.stk[0] = 0;
+        c.stk[1] = m - 2;
+        out->nstk = 1;
+      }
+    }
   }
   __syncthreads();
 
-  // fp64 evaluation of the code from the bucket statistics.
-  if (warp == 0) {
-    const int m = out->m;
-    double vs = 0.0;
-    for (int t = lane; t < m - 1; t += kWarp) {
-      const int a = c.sQ[t], cc = c.sQ[t + 1];
-      double N = 0.0, T1 = 0.0, T2 = 0.0;
-      const double Pa = c.sP[a];
-      for (int k = a; k < cc; ++k) {
-        const double dk = c.sP[k] - Pa;
-        const double nk = c.sN[k];
-        N += nk;
-        T1 += c.sA[k] + nk * dk;
-        T2 += c.sB[k] + 2.0 * dk * c.sA[k] + nk * dk * dk;
+  while (c.hirschberg && out->nstk > 0) {
+    const int top = out->nstk - 1;
+    const int lo = c.stk[2 * top], hi = c.stk[2 * top + 1];
+    __syncthreads();
+    if (tid == 0) out->nstk = top;
+    const int n = hi - lo - 1;          // unknown values c[lo+1 .. hi-1]
+    const int mid = lo + (n + 1) / 2;   // split pair (c[mid], c[mid+1]); c[mid] unknown
+    const int qlo = c.sQ[lo], qhi = c.sQ[hi], qnext = c.sQ[hi + 1];
+    // Forward: values c[lo] .. c[mid], next c[mid+1], all <= c[hi].
+    double extra_f = -1.0;
+    if (lo >= 1) extra_f = static_cast<double>(c.fw.buf0[c.cb[qlo] + c.sQ[lo - 1]].a);  // R(c[lo-1], c[lo])/d
+    Pass fwp{qlo, qhi, mid - lo + 1, mid + 1 == hi, extra_f, false, false};
+    run_pass(c, c.fw, fwp, sep, invl, out, bestE);
+    // Reflected: values c[hi] .. c[mid+1] (reflected), next c[mid]; the mass of
+    // c[hi] takes L(c[hi], c[hi+1]) from its right neighbour.
+    const double extra_b = static_cast<double>(c.fw.rowB[row_off(qhi, p) + qnext - qhi - 1]);
+    Pass bwp{p - 1 - qhi, p - 1 - qlo, hi - mid, false, extra_b, false, false};
+    run_pass(c, c.rf, bwp, sep, invl, out, bestE);
+    const int xlo = qlo + (mid - lo), xhi = qhi - (hi - mid);
+    const int yhi = qhi - (hi - mid - 1);
+    join(c, c.fw.layer(fwp.T), c.rf.layer(bwp.T), xlo, xhi, yhi, mid + 1 == hi, invl, out, wbest, warg);
+    if (tid == 0) {
+      c.sQ[mid] = out->jx;
+      c.sQ[mid + 1] = out->jy;
+      int ns = out->nstk;
+      if (mid - lo - 1 >= 1) {
+        c.stk[2 * ns] = lo;
+        c.stk[2 * ns + 1] = mid;
+        ++ns;
       }
-      const double W = c.sP[cc] - Pa;
-      double V = W * T1 - T2;
-      V = V > 0.0 ? V : 0.0;
-      const double R = T1 / W;
-      c.sR[t] = R;
-      c.sL[t] = N - R;
-      vs += V;
-    }
-    __syncwarp();
-    double hs = 0.0;
-    for (int t = lane; t < m; t += kWarp) {
-      const double mu = (t > 0 ? c.sR[t - 1] : 0.0) + (t < m - 1 ? c.sL[t] : 0.0);
-      if (mu > 0.0) {
-        const double q = mu / c.dd;
-        hs -= q * log2(q);
+      if (hi - mid - 2 >= 1) {
+        c.stk[2 * ns] = mid + 1;
+        c.stk[2 * ns + 1] = hi;
+        ++ns;
       }
+      out->nstk = ns;
     }
-    vs = warp_sum(vs);
-    hs = warp_sum(hs);
-    if (lane == 0) {
-      out->mse = vs / c.dd;
-      out->H = hs;
-      out->J = out->mse + lam * hs;
-    }
+    __syncthreads();
   }
+
+  evaluate(c, lam, out);
   __syncthreads();
 }
 
@@ -456,6 +628,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
   __shared__ SolveOut s_out;
   __shared__ T s_bestE;
   __shared__ int s_flag;
+  __shared__ T s_wbest[kWarps];
+  __shared__ int s_warg[kWarps];
 
   const int p = a.p, S = a.s;
   const int tri = tri_size(p);
@@ -464,9 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
   c.S = S;
   c.tri = tri;
   c.dd = static_cast<double>(a.d);
-  c.groups = a.tasks;
-  c.ngroups = a.ntasks;
-  c.max_groups = a.max_tasks;
+  c.hirschberg = a.hirschberg != 0;
 
   unsigned char* sp = smem;
   auto carve = [&sp](size_t bytes) {
@@ -486,6 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
   c.sQ = reinterpret_cast<int*>(carve(sizeof(int) * S));
   int* sQ1 = reinterpret_cast<int*>(carve(sizeof(int) * S));
   int* sQ2 = reinterpret_cast<int*>(carve(sizeof(int) * S));
+  c.stk = reinterpret_cast<int*>(carve(sizeof(int) * 2 * S));
   int* cbs = reinterpret_cast<int*>(carve(sizeof(int) * (p + 1)));
   if (threadIdx.x == 0) {
     int cc = 0;
@@ -499,14 +672,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
 
   unsigned char* gs = a.scratch + static_cast<size_t>(blockIdx.x) * a.scratch_per_cta;
   c.bp = reinterpret_cast<uint16_t*>(gs);
-  gs += (sizeof(uint16_t) * static_cast<size_t>(S) * tri + 255) & ~size_t(255);
+  if (!c.hirschberg) gs += (sizeof(uint16_t) * static_cast<size_t>(S) * tri + 255) & ~size_t(255);
   const size_t tb = (sizeof(T) * static_cast<size_t>(tri) + 15) & ~size_t(15);
   const size_t gb = (2 * sizeof(T) * static_cast<size_t>(layer_elems(p)) + 15) & ~size_t(15);
   unsigned char* big = kSmemTables ? sp : gs;
-  c.ga0 = reinterpret_cast<GA<T>*>(big);
-  c.ga1 = reinterpret_cast<GA<T>*>(big + gb);
-  c.rowB = reinterpret_cast<T*>(big + 2 * gb);
-  c.rowV = reinterpret_cast<T*>(big + 2 * gb + tb);
+  c.fw.buf0 = reinterpret_cast<GA<T>*>(big);
+  c.fw.buf1 = reinterpret_cast<GA<T>*>(big + gb);
+  c.fw.rowB = reinterpret_cast<T*>(big + 2 * gb);
+  c.fw.rowV = reinterpret_cast<T*>(big + 2 * gb + tb);
+  unsigned char* big2 = big + 2 * gb + 2 * tb;  // reflected tables (Hirschberg mode, global slab only)
+  c.rf.buf0 = reinterpret_cast<GA<T>*>(big2);
+  c.rf.buf1 = reinterpret_cast<GA<T>*>(big2 + gb);
+  c.rf.rowB = reinterpret_cast<T*>(big2 + 2 * gb);
+  c.rf.rowV = reinterpret_cast<T*>(big2 + 2 * gb + tb);
   __syncthreads();  // cb visible to all threads
 
   const int s_out_stride = a.s_out;
@@ -562,12 +740,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
 
     build_tables(c);
     __syncthreads();
+    if (c.hirschberg) {
+      build_reflected(c);
+      __syncthreads();
+    }
 
     if (a.mode == 0) {
       for (int t = 0; t < a.n_lambda; ++t) {
         const int64_t w = static_cast<int64_t>(r) * a.n_lambda + t;
         const double lam = a.lambda[w];
-        solve(c, lam, &s_out, &s_bestE);
+        solve(c, lam, &s_out, &s_bestE, s_wbest, s_warg);
         for (int q = threadIdx.x; q < s_out_stride; q += blockDim.x)
           a.Q[w * s_out_stride + q] = (q < s_out.m) ? c.sQ[q] : -1;
         if (threadIdx.x == 0) {
@@ -593,14 +775,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
       };
       int32_t status = kStatusOk;
       double theta = 0.0;
-      solve(c, 0.0, &s_out, &s_bestE);
+      solve(c, 0.0, &s_out, &s_bestE, s_wbest, s_warg);
       keep(sQ1, m1, H1, M1);
       if (s_out.H <= a.budget) {
         keep(sQ2, m2, H2, M2);
         hi = 0.0;
       } else {
         __syncthreads();
-        solve(c, hi, &s_out, &s_bestE);
+        solve(c, hi, &s_out, &s_bestE, s_wbest, s_warg);
         keep(sQ2, m2, H2, M2);
         if (s_out.H > a.budget) {
           status = kStatusBudget;
@@ -608,7 +790,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
           for (int it = 0; it < a.steps; ++it) {
             const double mid = 0.5 * (lo + hi);
             __syncthreads();
-            solve(c, mid, &s_out, &s_bestE);
+            solve(c, mid, &s_out, &s_bestE, s_wbest, s_warg);
             if (s_out.H > a.budget) {
               lo = mid;
               keep(sQ1, m1, H1, M1);
@@ -643,36 +825,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
   }
 }
 
-// ---- schedule ----------------------------------------------------------------
-// Group descriptors of layer i >= 3 in row-major order (rows l = i-1 .. p-2,
-// j ascending in groups of kTJ; the last layer has only j = p-1). One CTA per
-// layer, one thread per row; a row's first group index is the sum of the group
-// counts of the rows before it.
-__global__ void k_schedule(int p, int S, int max_groups_, uint32_t* groups, int32_t* ngroups) {
-  const int i = blockIdx.x;
-  if (i < 3) {
-    if (threadIdx.x == 0) ngroups[i] = 0;
-    return;
-  }
-  const bool last = (i == S - 1);
-  auto row_groups = [&](int l) { return last ? 1 : (p - 1 - l + kTJ - 1) / kTJ; };
-  uint32_t* out = groups + static_cast<size_t>(i) * max_groups_;
-  for (int l = i - 1 + threadIdx.x; l <= p - 2; l += blockDim.x) {
-    int o = 0;
-    for (int r = i - 1; r < l; ++r) o += row_groups(r);
-    if (last) {
-      out[o] = pack_group(l, p - 1, 1);
-    } else {
-      for (int j = l + 1; j <= p - 1; j += kTJ) out[o++] = pack_group(l, j, min(kTJ, p - j));
-    }
-  }
-  if (threadIdx.x == 0) {
-    int tot = 0;
-    for (int r = i - 1; r <= p - 2; ++r) tot += row_groups(r);
-    ngroups[i] = tot;
-  }
-}
-
 template <typename T, bool kSmem>
 void* dp_kernel_ptr() {
   return reinterpret_cast<void*>(&k_dp<T, kSmem>);
@@ -680,7 +832,7 @@ void* dp_kernel_ptr() {
 
 size_t small_smem(int p, int S, size_t tsz) {
   auto al = [](size_t b) { return (b + 15) & ~size_t(15); };
-  return al(8 * p) * 4 + al(8 * S) * 2 + al(tsz * p) + al(4 * p) + al(4 * S) * 4 + al(4 * (p + 1));
+  return al(8 * p) * 4 + al(8 * S) * 2 + al(tsz * p) + al(4 * p) + al(4 * S) * 4 + al(8 * S) + al(4 * (p + 1));
 }
 
 size_t table_bytes(int p, size_t tsz) {
@@ -705,13 +857,7 @@ int64_t dp_triples(int p, int s) {
   return t;
 }
 
-size_t dp_schedule_bytes(int p, int s) {
-  const int S = s < p ? s : p;
-  return ((sizeof(uint32_t) * static_cast<size_t>(max_groups(p)) * S + 255) & ~size_t(255)) +
-         ((sizeof(int32_t) * S + 255) & ~size_t(255));
-}
-
-bool dp_plan(int n, int p, int s, bool fp64, DpPlan* plan) {
+bool dp_plan(int n, int p, int s, bool fp64, bool hirschberg, DpPlan* plan) {
   if (p < 2 || p > kMaxP || s < 2 || n < 1) return false;
   const int S = s < p ? s : p;
   int dev = 0;
@@ -723,12 +869,13 @@ bool dp_plan(int n, int p, int s, bool fp64, DpPlan* plan) {
   const size_t small = small_smem(p, S, tsz);
   const size_t big = table_bytes(p, tsz);
   plan->fp64 = fp64;
+  plan->hirschberg = hirschberg;
   plan->threads = kThreads;
-  plan->smem_tables = (small + big + 1024 <= static_cast<size_t>(optin));
+  plan->smem_tables = !hirschberg && (small + big + 1024 <= static_cast<size_t>(optin));
   plan->smem_bytes = small + (plan->smem_tables ? big : 0);
-  const size_t bp = (sizeof(uint16_t) * static_cast<size_t>(S) * tri_size(p) + 255) & ~size_t(255);
-  plan->scratch_per_cta = (bp + (plan->smem_tables ? 0 : big) + 255) & ~size_t(255);
-  plan->max_tasks = max_groups(p);
+  const size_t bp = hirschberg ? 0 : (sizeof(uint16_t) * static_cast<size_t>(S) * tri_size(p) + 255) & ~size_t(255);
+  const size_t slab = plan->smem_tables ? 0 : (hirschberg ? 2 * big : big);
+  plan->scratch_per_cta = (bp + slab + 255) & ~size_t(255);
   void* fn = fp64 ? (plan->smem_tables ? dp_kernel_ptr<double, true>() : dp_kernel_ptr<double, false>())
                   : (plan->smem_tables ? dp_kernel_ptr<float, true>() : dp_kernel_ptr<float, false>());
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(plan->smem_bytes)) !=
@@ -743,13 +890,8 @@ bool dp_plan(int n, int p, int s, bool fp64, DpPlan* plan) {
   return true;
 }
 
-cudaError_t launch_dp(const DpPlan& plan, DpArgs args, uint32_t* tasks, int32_t* ntasks, cudaStream_t st) {
-  const int S = args.s;
-  args.tasks = tasks;
-  args.ntasks = ntasks;
-  args.max_tasks = plan.max_tasks;
-  k_schedule<<<S, 128, 0, st>>>(args.p, S, plan.max_tasks, tasks, ntasks);
-  note_launch();
+cudaError_t launch_dp(const DpPlan& plan, DpArgs args, cudaStream_t st) {
+  args.hirschberg = plan.hirschberg ? 1 : 0;
   void* fn = plan.fp64 ? (plan.smem_tables ? dp_kernel_ptr<double, true>() : dp_kernel_ptr<double, false>())
                        : (plan.smem_tables ? dp_kernel_ptr<float, true>() : dp_kernel_ptr<float, false>());
   void* kargs[] = {&args};

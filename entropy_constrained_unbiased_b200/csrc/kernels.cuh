@@ -63,10 +63,7 @@ struct DpArgs {
   double* mse2;
   int32_t* status;  // [n]
   int s_out;        // row stride of the Q outputs (the caller's s)
-  // schedule of the DP layers (built by the schedule kernel)
-  const uint32_t* tasks;  // [s][max_tasks]
-  const int32_t* ntasks;  // [s]
-  int max_tasks;
+  int hirschberg;   // 1: no back-pointers, divide-and-conquer recovery of the code
   // per-CTA global scratch
   unsigned char* scratch;
   size_t scratch_per_cta;
@@ -74,18 +71,17 @@ struct DpArgs {
 
 struct DpPlan {
   bool fp64;
+  bool hirschberg;
   bool smem_tables;  // pair tables resident in shared memory
   int threads;
   int ctas;
   size_t smem_bytes;
   size_t scratch_per_cta;
-  int max_tasks;
 };
 
 // Plan for the current device; ok = false when the sizes are out of range.
-bool dp_plan(int n, int p, int s, bool fp64, DpPlan* plan);
-size_t dp_schedule_bytes(int p, int s);
-cudaError_t launch_dp(const DpPlan& plan, DpArgs args, uint32_t* tasks, int32_t* ntasks, cudaStream_t st);
+bool dp_plan(int n, int p, int s, bool fp64, bool hirschberg, DpPlan* plan);
+cudaError_t launch_dp(const DpPlan& plan, DpArgs args, cudaStream_t st);
 
 // Exact count of (k, l, j) triples one solve evaluates (host).
 int64_t dp_triples(int p, int s);

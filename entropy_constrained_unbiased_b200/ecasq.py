@@ -179,7 +179,7 @@ def _solve_outputs(n, nl, s, device):
                 status=torch.empty(n, dtype=torch.int32, device=device))
 
 
-def solve(X: torch.Tensor, P: torch.Tensor, s: int, lam, fp64: bool = False):
+def solve(X: torch.Tensor, P: torch.Tensor, s: int, lam, fp64: bool = False, hirschberg: bool = False):
     """Exact Lagrangian solve of each row at each of its lambdas ([n] or [n, L])."""
     L = _need_cuda()
     _dev(X, torch.float32, "X")
@@ -189,7 +189,7 @@ def solve(X: torch.Tensor, P: torch.Tensor, s: int, lam, fp64: bool = False):
     lt = _lam_table(lam, n, X.device)
     nl = lt.shape[1]
     o = _solve_outputs(n, nl, s, X.device)
-    op = opts(fp64)
+    op = opts(fp64, hirschberg=hirschberg)
     ws = workspace(L.ecasq_workspace_size(n, d, p, s, nl, C.byref(op)), X.device)
     _check(L.ecasq_solve(_ptr(X), _ptr(P), n, d, p, s, _ptr(lt), nl, _ptr(o["Q"]), _ptr(o["Q_len"]),
                          _ptr(o["objective"]), _ptr(o["mse"]), _ptr(o["H"]), _ptr(o["status"]), C.byref(op),
@@ -197,13 +197,13 @@ def solve(X: torch.Tensor, P: torch.Tensor, s: int, lam, fp64: bool = False):
     return o
 
 
-def solve_stats(cnt, A, B, P, d: int, s: int, lam, fp64: bool = False):
+def solve_stats(cnt, A, B, P, d: int, s: int, lam, fp64: bool = False, hirschberg: bool = False):
     L = _need_cuda()
     n, p = P.shape
     lt = _lam_table(lam, n, P.device)
     nl = lt.shape[1]
     o = _solve_outputs(n, nl, s, P.device)
-    op = opts(fp64)
+    op = opts(fp64, hirschberg=hirschberg)
     ws = workspace(L.ecasq_workspace_size(n, d, p, s, nl, C.byref(op)), P.device)
     _check(L.ecasq_solve_stats(_ptr(cnt), _ptr(A), _ptr(B), _ptr(P), n, d, p, s, _ptr(lt), nl, _ptr(o["Q"]),
                                _ptr(o["Q_len"]), _ptr(o["objective"]), _ptr(o["mse"]), _ptr(o["H"]),
@@ -227,7 +227,8 @@ _BUDGET_ORDER = ("Q1", "Q1_len", "Q2", "Q2_len", "theta", "lambda_lo", "lambda_h
                  "status")
 
 
-def solve_budget(X: torch.Tensor, P: torch.Tensor, s: int, b: float, steps: int = 30, fp64: bool = False):
+def solve_budget(X: torch.Tensor, P: torch.Tensor, s: int, b: float, steps: int = 30, fp64: bool = False,
+                 hirschberg: bool = False):
     """Entropy budget b: lambda bisection plus two-way time-sharing per row."""
     L = _need_cuda()
     _dev(X, torch.float32, "X")
@@ -235,18 +236,19 @@ def solve_budget(X: torch.Tensor, P: torch.Tensor, s: int, b: float, steps: int 
     n, d = X.shape
     p = P.shape[1]
     o = _budget_outputs(n, s, X.device)
-    op = opts(fp64, steps)
+    op = opts(fp64, steps, hirschberg)
     ws = workspace(L.ecasq_workspace_size(n, d, p, s, 1, C.byref(op)), X.device)
     _check(L.ecasq_solve_budget(_ptr(X), _ptr(P), n, d, p, s, float(b), *[_ptr(o[k]) for k in _BUDGET_ORDER],
                                 C.byref(op), _ptr(ws), ws.numel(), _stream()), "ecasq_solve_budget")
     return o
 
 
-def solve_budget_stats(cnt, A, B, P, d: int, s: int, b: float, steps: int = 30, fp64: bool = False):
+def solve_budget_stats(cnt, A, B, P, d: int, s: int, b: float, steps: int = 30, fp64: bool = False,
+                       hirschberg: bool = False):
     L = _need_cuda()
     n, p = P.shape
     o = _budget_outputs(n, s, P.device)
-    op = opts(fp64, steps)
+    op = opts(fp64, steps, hirschberg)
     ws = workspace(L.ecasq_workspace_size(n, d, p, s, 1, C.byref(op)), P.device)
     _check(L.ecasq_solve_budget_stats(_ptr(cnt), _ptr(A), _ptr(B), _ptr(P), n, d, p, s, float(b),
                                       *[_ptr(o[k]) for k in _BUDGET_ORDER], C.byref(op), _ptr(ws), ws.numel(),

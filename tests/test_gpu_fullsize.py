@@ -48,7 +48,7 @@ def test_fullsize_lambda_workloads(E, O, name, rows):
     w = W.WORKLOADS[name]
     X, Xd, P, cnt, A, B = _full(E, w)
     lam = w.lambdas()
-    g = E.solve_stats(cnt, A, B, P, w.d, w.s, torch.from_numpy(lam).cuda())
+    g = E.solve_stats(cnt, A, B, P, w.d, w.s, torch.from_numpy(lam).cuda(), hirschberg=w.hirschberg)
     assert int(g["status"].abs().sum()) == 0
     Q = g["Q"].cpu().numpy()
     m = g["Q_len"].cpu().numpy()

@@ -270,3 +270,52 @@ def test_encode_flags_out_of_range(E, O):
     m = np.array([3, 3], np.int32)
     _, _, st = E.encode(_cu(X), _cu(P), 4, _cu(Q), _cu(m), seed=3)
     assert list(_np(st)) == [0, -2]
+
+
+# -- Hirschberg mode (O(p^2) DP memory, no back-pointers) ---------------------------
+
+HIRSCH = [  # (seed, n, d, p, s, dist)
+    (40, 2, 1500, 48, 9, "laplace"),
+    (41, 2, 3000, 96, 12, "mixture"),
+    (42, 1, 2000, 200, 16, "normal"),
+    (43, 2, 800, 30, 30, "student_t"),  # s == p
+    (44, 2, 600, 20, 3, "normal"),      # one value between the ends
+    (45, 2, 600, 20, 4, "normal"),
+    (46, 1, 4000, 300, 20, "outlier"),
+]
+
+
+@pytest.mark.parametrize("fp64", [True, False], ids=["fp64", "fp32"])
+@pytest.mark.parametrize("case", HIRSCH, ids=lambda c: f"p{c[3]}s{c[4]}{c[5]}")
+def test_hirschberg_matches_store_mode_and_oracle(E, O, case, fp64):
+    seed, n, d, p, s, dist = case
+    X = _case(seed, n, d, dist)
+    P, _ = O.grid_batch(X, p)
+    lam = _lams(X, 4)
+    h = {k: _np(v) for k, v in E.solve(_cu(X), _cu(P), s, _cu(lam), fp64=fp64, hirschberg=True).items()}
+    st = {k: _np(v) for k, v in E.solve(_cu(X), _cu(P), s, _cu(lam), fp64=fp64).items()}
+    ref = O.solve_batch(X, P, s, lam)
+    tol = RTOL64 if fp64 else RTOL32
+    assert np.all(h["status"] == 0)
+    for r in range(n):
+        for t in range(lam.shape[1]):
+            m = h["Q_len"][r, t]
+            Q = h["Q"][r, t]
+            assert 2 <= m <= min(s, p)
+            assert Q[0] == 0 and Q[m - 1] == p - 1 and np.all(np.diff(Q[:m]) > 0) and np.all(Q[m:] == -1)
+            Jeval, _, _ = _oracle_eval(O, X[r], P[r], Q, m, lam[r, t])
+            assert Jeval <= ref["J"][r, t] * (1 + tol) + 1e-300, (r, t, Jeval, ref["J"][r, t])
+            assert h["objective"][r, t] == pytest.approx(Jeval, rel=RTOL64)
+            assert h["objective"][r, t] == pytest.approx(st["objective"][r, t], rel=tol)
+            if fp64:
+                assert h["objective"][r, t] == pytest.approx(ref["J"][r, t], rel=RTOL64)
+
+
+def test_hirschberg_budget(E, O):
+    X = _case(47, 2, 4000, "student_t")
+    P, _ = O.grid_batch(X, 64)
+    g = {k: _np(v) for k, v in E.solve_budget(_cu(X), _cu(P), 10, 2.5, 30, fp64=True, hirschberg=True).items()}
+    ref = O.solve_budget_batch(X, P, 10, 2.5, 30)
+    for r in range(2):
+        for k_g, k_o in (("theta", "theta"), ("H1", "H1"), ("H2", "H2"), ("mse1", "mse1"), ("mse2", "mse2")):
+            assert g[k_g][r] == pytest.approx(ref[k_o][r], rel=RTOL64, abs=1e-15), k_g
