@@ -35,6 +35,12 @@ from entropy_constrained_unbiased_b200 import workloads as W  # noqa: E402
 MUFU_LG2_PER_CLK_PER_SM = 16  # special-function unit results per clock per SM (sm_100)
 B200_SMS = 148
 
+# DRAM bytes (read + write) per k_dp launch per row, from the ncu capture
+# summarised in profiles/k_dp_weights_296rows_full.md (296 rows: 1.95 MB). The
+# figure belongs to the kernel source it was taken on; it is dropped (null)
+# when that source has changed since.
+DP_TRAFFIC = {"weights": {"bytes_per_row": 1.95e6 / 296, "dp_source_sha1": "a8be1452bba47170"}}
+
 
 def triples_per_solve(p: int, s: int) -> int:
     """(k, l, j) triples one exact solve evaluates: layer 2 has only k = 0
@@ -49,6 +55,19 @@ def triples_per_solve(p: int, s: int) -> int:
             NJ = 1 if last else p - 1 - l
             t += K * NJ
     return t
+
+
+def dp_traffic(w):
+    import hashlib
+
+    rec = DP_TRAFFIC.get(w.name)
+    if rec is None:
+        return None
+    src = os.path.join(ROOT, "entropy_constrained_unbiased_b200", "csrc", "dp.cu")
+    with open(src, "rb") as f:
+        if hashlib.sha1(f.read()).hexdigest()[:16] != rec["dp_source_sha1"]:
+            return None
+    return rec["bytes_per_row"] * w.n
 
 
 def measured_peaks():
@@ -263,7 +282,7 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
                    "entries_per_s": world * n * d / (t_ms * 1e-3 / args.steps),
                    "parallelism": f"dp{world} (rows sharded, no collective)"},
         "roofline": {"bound": "alu", "kernel": "k_dp (DP layers + backtrack + bisection)", "achieved": achieved,
-                     "peak": mufu_peak, "unit": "triples/s", "frac": achieved / mufu_peak, "traffic": None,
+                     "peak": mufu_peak, "unit": "triples/s", "frac": achieved / mufu_peak, "traffic": dp_traffic(w),
                      "peak_basis": f"MUFU lg2 {MUFU_LG2_PER_CLK_PER_SM}/clk/SM x {B200_SMS} SMs x {sm_max:.0f} MHz "
                                    "(1 lg2 per triple)",
                      "measured_lg2_per_s": unit_peaks.get("lg2"),
