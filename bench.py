@@ -152,13 +152,14 @@ class Clocks:
 
 def run_ours(args, w: W.Workload, rank: int, world: int):
     import torch
+    from entropy_constrained_unbiased_b200 import dist as D
     from entropy_constrained_unbiased_b200 import ecasq as E
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     E.load()
     fp64 = args.fp64
-    X_host = W.make_inputs(w)
+    X_host = W.make_inputs(w, rank=rank)
     X = torch.from_numpy(X_host).to(dev)
     n, d, p, s = w.n, w.d, w.p, w.s
     lam = torch.from_numpy(w.lambdas()).to(dev) if w.mode != "budget" else None
@@ -203,9 +204,7 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     dp_ms = []
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    D.barrier()
     torch.cuda.synchronize()
     E.launch_count(reset=True)
     with Clocks(dev.index) as clk:
@@ -221,13 +220,8 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
             stage_ms["encode"].append((ev["e0"] if w.mode != "budget" else ev_dp1).elapsed_time(ev["e1"]))
     launches = E.launch_count(reset=True)
     step_ms = [starts[k].elapsed_time(ends[k]) for k in range(args.steps)]
-    t_ms = float(sum(step_ms))
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([t_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_ms = float(t.item())
-        dist.barrier()
+    t_ms = D.max_over_ranks(float(sum(step_ms)))
+    D.barrier()
 
     # e2e: same step through the C ABI with host buffers, copies inside the timed region
     Xpin = torch.from_numpy(X_host).pin_memory()
@@ -386,16 +380,11 @@ def main():
 
         w = dataclasses.replace(w, n=min(args.rows, w.n))
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
+    from entropy_constrained_unbiased_b200 import dist as D
+
+    rank, world = D.world()
     if world > 1 and args.impl == "ours":
-        import datetime
-
-        import torch
-        import torch.distributed as dist
-
-        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        D.setup("nccl")
     if args.impl == "reference":
         line = run_reference(args, w, rank, world)
     else:
@@ -409,9 +398,7 @@ def main():
     if rank == 0 and line is not None:
         print(json.dumps(line))
     if world > 1 and args.impl == "ours":
-        import torch.distributed as dist
-
-        dist.destroy_process_group()
+        D.teardown()
 
 
 if __name__ == "__main__":

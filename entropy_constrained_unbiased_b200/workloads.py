@@ -95,12 +95,18 @@ def draw(dist: str, rng: np.random.Generator, n: int, d: int, rows: int | None =
     return out
 
 
-def make_inputs(w: Workload | str, rows: int | None = None) -> np.ndarray:
-    """X for a named workload: [n, d] float32, or its first `rows` rows."""
+def make_inputs(w: Workload | str, rows: int | None = None, rank: int = 0) -> np.ndarray:
+    """X for a named workload: [n, d] float32, or its first `rows` rows.
+
+    Rank 0 draws the workload itself; rank r > 0 (multi-GPU weak scaling)
+    draws its own vectors of the same family from the seed [index, r]."""
     if isinstance(w, str):
         w = WORKLOADS[w]
     # The small workload is seeded with 0; the others with [index, 0].
-    rng = np.random.default_rng(0 if w.index == 0 else [w.index, 0])
+    if rank == 0:
+        rng = np.random.default_rng(0 if w.index == 0 else [w.index, 0])
+    else:
+        rng = np.random.default_rng([w.index, rank])
     return draw(w.dist, rng, w.n, w.d, rows)
 
 
