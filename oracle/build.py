@@ -6,15 +6,15 @@ import os
 import subprocess
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-SRC = os.path.join(HERE, "ecasq_oracle.cpp")
+SRCS = [os.path.join(HERE, "ecasq_oracle.cpp"), os.path.join(HERE, "ecasq_approx_oracle.cpp")]
 LIB = os.path.join(HERE, "liboracle.so")
 
 
 def build(force: bool = False) -> str:
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
+    if not force and os.path.exists(LIB) and all(os.path.getmtime(LIB) >= os.path.getmtime(s) for s in SRCS):
         return LIB
     cmd = ["g++", "-O2", "-std=c++17", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
-           "-fPIC", "-shared", "-Wall", "-Wextra", "-o", LIB, SRC]
+           "-fPIC", "-shared", "-Wall", "-Wextra", "-o", LIB] + SRCS
     subprocess.run(cmd, check=True)
     return LIB
 

@@ -51,6 +51,16 @@ def lib():
             "eo_encode_batch": (I, [f32p, I, I64, f64p, I, i32p, i32p, C.c_void_p, C.c_void_p, C.c_void_p,
                                     I, U64, u8p, i64p, i32p]),
             "eo_grid_batch": (I, [f32p, I, I64, I, f64p, i32p]),
+            "eo_hib_tables": (D, [f64p, f64p, f64p, I, I64, i32p, I]),
+            "eo_eval_raw_ib": (I, [f32p, I64, f64p, I, C.POINTER(D)]),
+            "eo_approx_dp": (I, [f64p, f64p, f64p, I, I, I64, D, i32p, C.POINTER(C.c_int32), C.POINTER(D)]),
+            "eo_refine_local": (D, [f64p, f64p, f64p, I, I64, D, i32p, I, I, I]),
+            "eo_refine_point": (I, [f64p, f64p, f64p, I, I64, D, i32p, I, I]),
+            "eo_refine": (I, [f64p, f64p, f64p, I, I64, D, i32p, I, I, C.POINTER(C.c_int32)]),
+            "eo_solve_approx_batch": (I, [f32p, I, I64, f64p, I, I, f64p, I, I, i32p, i32p, f64p, f64p, f64p,
+                                          f64p, i32p]),
+            "eo_solve_approx_budget_batch": (I, [f32p, I, I64, f64p, I, I, D, I, I, i32p, i32p, i32p, i32p,
+                                                 f64p, f64p, f64p, f64p, f64p, f64p, f64p, f64p, f64p, i32p]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -132,6 +142,84 @@ def dp(V, R, L, s, d, lam):
     if st:
         raise ValueError("oracle dp failed")
     return Q[: m.value].copy(), J.value
+
+
+# -- approximation on H(I,B) and iterative refinement (§2.3, §2.4) ------------
+
+def hib_tables(V, R, L, d, Q):
+    Q = np.ascontiguousarray(Q, np.int32)
+    return float(lib().eo_hib_tables(_f64(V), _f64(R), _f64(L), V.shape[0], d, Q, Q.size))
+
+
+def eval_raw_ib(x, qvals):
+    x = _f32(x).ravel()
+    q = _f64(qvals)
+    out = C.c_double()
+    if lib().eo_eval_raw_ib(x, x.size, q, q.size, C.byref(out)):
+        raise ValueError("entry outside the code range")
+    return out.value
+
+
+def approx_dp(V, R, L, s, d, lam):
+    p = V.shape[0]
+    Q = np.full(min(s, p), -1, np.int32)
+    m = C.c_int32()
+    J = C.c_double()
+    if lib().eo_approx_dp(_f64(V), _f64(R), _f64(L), p, s, d, lam, Q, C.byref(m), C.byref(J)):
+        raise ValueError("oracle approx dp failed")
+    return Q[: m.value].copy(), J.value
+
+
+def refine_local(V, R, L, d, lam, Q, t, c):
+    Q = np.ascontiguousarray(Q, np.int32)
+    return float(lib().eo_refine_local(_f64(V), _f64(R), _f64(L), V.shape[0], d, lam, Q, Q.size, t, c))
+
+
+def refine_point(V, R, L, d, lam, Q, t):
+    Q = np.ascontiguousarray(Q, np.int32)
+    return int(lib().eo_refine_point(_f64(V), _f64(R), _f64(L), V.shape[0], d, lam, Q, Q.size, t))
+
+
+def refine(V, R, L, d, lam, Q, iters):
+    """Returns (refined Q, moves, iterations run)."""
+    Q = np.ascontiguousarray(Q, np.int32).copy()
+    done = C.c_int32()
+    moves = lib().eo_refine(_f64(V), _f64(R), _f64(L), V.shape[0], d, lam, Q, Q.size, iters, C.byref(done))
+    return Q, int(moves), int(done.value)
+
+
+def solve_approx_batch(X, P, s, lam, refine=0):
+    """lam: [n] or [n, L]. J is MSE + lam*H(I,B) (refine == 0) or MSE + lam*H (refine > 0)."""
+    X = _f32(X)
+    n, d = X.shape
+    P = _f64(P)
+    p = P.shape[1]
+    lam = _f64(lam).reshape(n, -1)
+    nl = lam.shape[1]
+    out = dict(Q=np.full((n, nl, s), -1, np.int32), m=np.zeros((n, nl), np.int32))
+    for k in ("J", "mse", "H", "HIB"):
+        out[k] = np.zeros((n, nl))
+    out["status"] = np.zeros((n, nl), np.int32)
+    out["threads"] = lib().eo_solve_approx_batch(X, n, d, P, p, s, lam, nl, int(refine), out["Q"], out["m"],
+                                                 out["J"], out["mse"], out["H"], out["HIB"], out["status"])
+    return out
+
+
+def solve_approx_budget_batch(X, P, s, b, steps=30, refine=0):
+    X = _f32(X)
+    n, d = X.shape
+    P = _f64(P)
+    p = P.shape[1]
+    out = dict(Q1=np.full((n, s), -1, np.int32), m1=np.zeros(n, np.int32),
+               Q2=np.full((n, s), -1, np.int32), m2=np.zeros(n, np.int32))
+    for k in ("theta", "lam_lo", "lam_hi", "H1", "H2", "HIB1", "HIB2", "mse1", "mse2"):
+        out[k] = np.zeros(n)
+    out["status"] = np.zeros(n, np.int32)
+    out["threads"] = lib().eo_solve_approx_budget_batch(
+        X, n, d, P, p, s, float(b), steps, int(refine), out["Q1"], out["m1"], out["Q2"], out["m2"],
+        out["theta"], out["lam_lo"], out["lam_hi"], out["H1"], out["H2"], out["HIB1"], out["HIB2"],
+        out["mse1"], out["mse2"], out["status"])
+    return out
 
 
 def philox4x32(ctr, key):
