@@ -57,6 +57,16 @@ def triples_per_solve(p: int, s: int) -> int:
     return t
 
 
+def relaxations_per_solve(p: int, s: int) -> int:
+    """(i, a, x) relaxations G_{i-1}(a) + w(a, x) one solve of the approximation's
+    layered shortest path evaluates: layers i = 2 .. S, x = i-1 .. p-1, a = i-2 .. x-1."""
+    S = min(s, p)
+    return sum(x - i + 2 for i in range(2, S + 1) for x in range(i - 1, p))
+
+
+SMEM_BYTES_PER_CLK_PER_SM = 128  # one 32-lane x 4-byte shared-memory wavefront per clock
+
+
 def dp_traffic(w):
     import hashlib
 
@@ -258,6 +268,7 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
     achieved = n_solves * tps / (dp_avg_ms * 1e-3)
     total_triples = world * n_solves * tps  # one step, all ranks
     value = total_triples * args.steps / (t_ms * 1e-3)
+    approx = approx_timing(args, w, X, stream, flush, dp_avg_ms, sm_max)
     line = {
         "metric": "ECASQ DP (k,l,j) triples/s (whole step: grid + bucketing + DP + bisection + encode + entropy)",
         "value": value,
@@ -285,10 +296,58 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
         "e2e": {"value": total_triples / (float(np.mean(e2e_ms)) * 1e-3), "unit": "triples/s",
                 "h2d_bytes_per_step": n * d * 4, "d2h_bytes_per_step": bo},
         "hbm_kernels": hbm_kernels,
+        "approx": approx,
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
     }
     return line
+
+
+def approx_timing(args, w: W.Workload, X, stream, flush, dp_avg_ms: float, sm_max: float):
+    """The approximation on H(I,B), plain and refined (8 iterations), on the same
+    workload and bucket statistics as the exact solver above; CUDA events around
+    the solver call alone, L2 flushed before each call. Roofline: every
+    relaxation reads one 4-byte cost entry from shared memory (the G value is a
+    broadcast), so at most 32 relaxations per clock per SM."""
+    import torch
+    from entropy_constrained_unbiased_b200 import ecasq as E
+
+    fp64 = args.fp64
+    P, _ = E.uniform_grid(X, w.p)
+    cnt, A, B, _ = E.bucket(X, P)
+    lam = torch.from_numpy(w.lambdas()).to(X.device) if w.mode != "budget" else None
+    rps = relaxations_per_solve(w.p, w.s)
+    peak = SMEM_BYTES_PER_CLK_PER_SM / 4 * B200_SMS * sm_max * 1e6
+    res = {"kernel": "k_approx (layers + recovery + refinement + evaluation + bisection)",
+           "relaxations_per_solve": rps, "bound": "smem", "peak": peak, "unit": "relaxations/s",
+           "peak_basis": f"{SMEM_BYTES_PER_CLK_PER_SM} B/clk/SM shared memory / 4 B per relaxation x {B200_SMS} SMs "
+                         f"x {sm_max:.0f} MHz"}
+
+    def call(refine):
+        if w.mode == "budget":
+            return E.solve_approx_budget_stats(cnt, A, B, P, w.d, w.s, w.b, refine=refine, steps=w.steps, fp64=fp64)
+        return E.solve_approx_stats(cnt, A, B, P, w.d, w.s, lam, refine=refine, fp64=fp64)
+
+    for refine in (0, 8):
+        out = call(refine)  # warm-up
+        torch.cuda.synchronize()
+        ms = []
+        for k in range(max(2, min(args.steps, 3))):
+            flush.fill_(k & 0xFF)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            out = call(refine)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        t = float(np.mean(ms))
+        ns = solves_done(w, out)
+        ach = ns * rps / (t * 1e-3)
+        res[f"refine{refine}"] = {"ms": t, "solves": ns, "achieved": ach, "frac": ach / peak,
+                                  "speedup_vs_exact_dp": dp_avg_ms / t,
+                                  "status_nonzero_rows": int((out["status"] != 0).sum().item())}
+    return res
 
 
 def measure_unit_peaks():

@@ -60,6 +60,21 @@ bool solve_ws(void* ws, int n, int p, const DpPlan& plan, SolveWs* w) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? ECASQ_OK : ECASQ_ERR_CUDA; }
 
+// Workspace of the approximation: the same bucketing buffers, then its slabs.
+size_t approx_ws(void* ws, int n, int p, const ApproxPlan& plan, SolveWs* w) {
+  Carver c{static_cast<unsigned char*>(ws)};
+  const size_t nb = static_cast<size_t>(n) * (p - 1);
+  w->acc = c.take<unsigned long long>(3 * nb);
+  w->flag = c.take<int32_t>(n);
+  w->cnt = c.take<int64_t>(nb);
+  w->A = c.take<double>(nb);
+  w->B = c.take<double>(nb);
+  w->bstatus = c.take<int32_t>(n);
+  w->scratch = c.take<unsigned char>(plan.scratch_per_cta * plan.ctas);
+  w->bytes = c.off;
+  return c.off;
+}
+
 }  // namespace
 
 void note_launch() { ++g_launches; }
@@ -253,6 +268,143 @@ int ecasq_solve_budget_stats(const int64_t* cnt, const double* A, const double* 
                              size_t ws_bytes, void* stream) {
   return solve_budget(nullptr, cnt, A, B, P, n, d, p, s, b, Q1, Q1_len, Q2, Q2_len, theta, lambda_lo, lambda_hi, H1,
                       H2, mse1, mse2, status, opts, ws, ws_bytes, stream);
+}
+
+size_t ecasq_approx_workspace_size(int n, int64_t d, int p, int s, const ecasq_opts* opts) {
+  if (!valid_sizes(n, d, p, s)) return 0;
+  ApproxPlan plan;
+  if (!approx_plan(n, p, s, opts && opts->dp_fp64, &plan)) return 0;
+  SolveWs w;
+  return approx_ws(nullptr, n, p, plan, &w);
+}
+
+static int approx_common(const float* X, const int64_t* cnt, const double* A, const double* B, const double* P, int n,
+                         int64_t d, int p, int s, int refine, const ecasq_opts* opts, void* ws, size_t ws_bytes,
+                         cudaStream_t st, ApproxArgs* args, ApproxPlan* plan) {
+  if (!P || !valid_sizes(n, d, p, s) || refine < 0) return ECASQ_ERR_ARG;
+  if (opts && (opts->reserved != 0 || opts->bisect_steps < 0)) return ECASQ_ERR_ARG;
+  if (!approx_plan(n, p, s, opts && opts->dp_fp64, plan)) return ECASQ_ERR_ARG;
+  SolveWs w;
+  approx_ws(ws, n, p, *plan, &w);
+  if (!ws || ws_bytes < w.bytes) return ECASQ_ERR_WORKSPACE;
+  ApproxArgs& a = *args;
+  a = ApproxArgs{};
+  if (X) {
+    if (launch_bucket(X, P, n, d, p, w.cnt, w.A, w.B, w.bstatus, w.acc, w.flag, st) != cudaSuccess)
+      return ECASQ_ERR_CUDA;
+    a.cnt = w.cnt;
+    a.A = w.A;
+    a.B = w.B;
+    a.in_status = w.bstatus;
+  } else {
+    if (!cnt || !A || !B) return ECASQ_ERR_ARG;
+    a.cnt = cnt;
+    a.A = A;
+    a.B = B;
+  }
+  a.P = P;
+  a.n = n;
+  a.p = p;
+  a.s = s < p ? s : p;
+  a.s_out = s;
+  a.d = d;
+  a.refine = refine;
+  a.steps = (opts && opts->bisect_steps > 0) ? opts->bisect_steps : 30;
+  a.scratch = w.scratch;
+  a.scratch_per_cta = plan->scratch_per_cta;
+  return ECASQ_OK;
+}
+
+static int approx_lambdas(const float* X, const int64_t* cnt, const double* A, const double* B, const double* P,
+                          int n, int64_t d, int p, int s, const double* lambda, int n_lambda, int refine, int32_t* Q,
+                          int32_t* Q_len, double* objective, double* mse, double* H, double* H_IB, int32_t* status,
+                          const ecasq_opts* opts, void* ws, size_t ws_bytes, void* stream) {
+  if (!lambda || n_lambda < 1 || !Q || !Q_len || !objective || !mse || !H || !H_IB || !status) return ECASQ_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ApproxArgs a;
+  ApproxPlan plan;
+  int rc = approx_common(X, cnt, A, B, P, n, d, p, s, refine, opts, ws, ws_bytes, st, &a, &plan);
+  if (rc != ECASQ_OK) return rc;
+  a.mode = 0;
+  a.lambda = lambda;
+  a.n_lambda = n_lambda;
+  a.Q = Q;
+  a.Q_len = Q_len;
+  a.obj = objective;
+  a.mse = mse;
+  a.H = H;
+  a.HIB = H_IB;
+  a.status = status;
+  return cuda_status(launch_approx(plan, a, st));
+}
+
+static int approx_budget(const float* X, const int64_t* cnt, const double* A, const double* B, const double* P, int n,
+                         int64_t d, int p, int s, double b, int refine, int32_t* Q1, int32_t* Q1_len, int32_t* Q2,
+                         int32_t* Q2_len, double* theta, double* lambda_lo, double* lambda_hi, double* H1, double* H2,
+                         double* H_IB1, double* H_IB2, double* mse1, double* mse2, int32_t* status,
+                         const ecasq_opts* opts, void* ws, size_t ws_bytes, void* stream) {
+  if (!Q1 || !Q1_len || !Q2 || !Q2_len || !theta || !lambda_lo || !lambda_hi || !H1 || !H2 || !H_IB1 || !H_IB2 ||
+      !mse1 || !mse2 || !status || !(b >= 0.0))
+    return ECASQ_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ApproxArgs a;
+  ApproxPlan plan;
+  int rc = approx_common(X, cnt, A, B, P, n, d, p, s, refine, opts, ws, ws_bytes, st, &a, &plan);
+  if (rc != ECASQ_OK) return rc;
+  a.mode = 1;
+  a.budget = b;
+  a.Q1 = Q1;
+  a.Q1_len = Q1_len;
+  a.Q2 = Q2;
+  a.Q2_len = Q2_len;
+  a.theta = theta;
+  a.lam_lo = lambda_lo;
+  a.lam_hi = lambda_hi;
+  a.H1 = H1;
+  a.H2 = H2;
+  a.HIB1 = H_IB1;
+  a.HIB2 = H_IB2;
+  a.mse1 = mse1;
+  a.mse2 = mse2;
+  a.status = status;
+  return cuda_status(launch_approx(plan, a, st));
+}
+
+int ecasq_solve_approx(const float* X, const double* P, int n, int64_t d, int p, int s, const double* lambda,
+                       int n_lambda, int refine_iters, int32_t* Q, int32_t* Q_len, double* objective, double* mse,
+                       double* H, double* H_IB, int32_t* status, const ecasq_opts* opts, void* ws, size_t ws_bytes,
+                       void* stream) {
+  if (!X) return ECASQ_ERR_ARG;
+  return approx_lambdas(X, nullptr, nullptr, nullptr, P, n, d, p, s, lambda, n_lambda, refine_iters, Q, Q_len,
+                        objective, mse, H, H_IB, status, opts, ws, ws_bytes, stream);
+}
+
+int ecasq_solve_approx_stats(const int64_t* cnt, const double* A, const double* B, const double* P, int n, int64_t d,
+                             int p, int s, const double* lambda, int n_lambda, int refine_iters, int32_t* Q,
+                             int32_t* Q_len, double* objective, double* mse, double* H, double* H_IB, int32_t* status,
+                             const ecasq_opts* opts, void* ws, size_t ws_bytes, void* stream) {
+  return approx_lambdas(nullptr, cnt, A, B, P, n, d, p, s, lambda, n_lambda, refine_iters, Q, Q_len, objective, mse,
+                        H, H_IB, status, opts, ws, ws_bytes, stream);
+}
+
+int ecasq_solve_approx_budget(const float* X, const double* P, int n, int64_t d, int p, int s, double b,
+                              int refine_iters, int32_t* Q1, int32_t* Q1_len, int32_t* Q2, int32_t* Q2_len,
+                              double* theta, double* lambda_lo, double* lambda_hi, double* H1, double* H2,
+                              double* H_IB1, double* H_IB2, double* mse1, double* mse2, int32_t* status,
+                              const ecasq_opts* opts, void* ws, size_t ws_bytes, void* stream) {
+  if (!X) return ECASQ_ERR_ARG;
+  return approx_budget(X, nullptr, nullptr, nullptr, P, n, d, p, s, b, refine_iters, Q1, Q1_len, Q2, Q2_len, theta,
+                       lambda_lo, lambda_hi, H1, H2, H_IB1, H_IB2, mse1, mse2, status, opts, ws, ws_bytes, stream);
+}
+
+int ecasq_solve_approx_budget_stats(const int64_t* cnt, const double* A, const double* B, const double* P, int n,
+                                    int64_t d, int p, int s, double b, int refine_iters, int32_t* Q1, int32_t* Q1_len,
+                                    int32_t* Q2, int32_t* Q2_len, double* theta, double* lambda_lo,
+                                    double* lambda_hi, double* H1, double* H2, double* H_IB1, double* H_IB2,
+                                    double* mse1, double* mse2, int32_t* status, const ecasq_opts* opts, void* ws,
+                                    size_t ws_bytes, void* stream) {
+  return approx_budget(nullptr, cnt, A, B, P, n, d, p, s, b, refine_iters, Q1, Q1_len, Q2, Q2_len, theta, lambda_lo,
+                       lambda_hi, H1, H2, H_IB1, H_IB2, mse1, mse2, status, opts, ws, ws_bytes, stream);
 }
 
 int ecasq_encode(const float* X, const double* P, int n, int64_t d, int p, int s, const int32_t* Q1,

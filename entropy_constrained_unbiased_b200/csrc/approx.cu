@@ -1,0 +1,659 @@
+// Space-efficient approximation of ECASQ on the surrogate entropy H(I,B), and
+// the iterative refinement ("Entropy-Constrained Adaptive Stochastic
+// Quantization (ECASQ)", gist.science/pt/paper/2608.18147, §2.3 and §2.4).
+//
+// H(I,B) is the entropy of the pair (interval index, rounding bit). An interval
+// [P_a, P_c] of the code contributes h(L(a,c)) + h(R(a,c)) to it, so
+//   MSE + lambda*H(I,B) = sum over intervals of w(a,c),
+//   w(a,c) = V(a,c)/d + lambda*(h(L(a,c)) + h(R(a,c))),
+// a sum of per-interval costs. Its exact minimiser over codes with P_0, P_{p-1}
+// and at most s values is the layered shortest path
+//   G_1(0) = 0,  G_i(c) = min_{a<c} G_{i-1}(a) + w(a,c),  J* = min_{2<=i<=s} G_i(p-1),
+// O(p^2 s) time and O(p s) state per solve: no pair-state, no back-pointers.
+//
+// Refinement works on the exact objective MSE + lambda*H(X^) at the same lambda.
+// The interior values are split by position mod 3 into three classes; moving a
+// value changes only its two intervals and three masses, so a class moves at
+// once. Each value binary-searches its open interval between its neighbours on
+// the sign of the forward difference of its local cost and moves only on a
+// strict decrease; classes run in the order 0, 1, 2, for up to `refine`
+// iterations or until an iteration moves nothing.
+//
+// GPU layout (one CTA per vector, persistent over vectors):
+//   * per vector, fp64 V, R, L of every pair a < c (column-major) and the
+//     layer-precision terms V/d and h(L)+h(R) in a per-CTA global slab
+//     (L2-resident); the latter in padded columns (16-byte aligned, starts
+//     staggered over the banks);
+//   * per solve, the cost table w(a,c) (same padded columns) and the layers
+//     G_1..G_s in shared memory (global slab when they do not fit). One thread
+//     per column c sweeps a upwards with 16-byte loads of its column and of
+//     G_{i-1} (a broadcast): four relaxations per pair of loads, two packed
+//     f32x2 additions and two three-input minima in fp32;
+//   * the argmin is recovered afterwards by recomputing the sums in the same
+//     precision (the minimum is one of them exactly), smallest a first;
+//   * refinement and the fp64 evaluation read the fp64 tables, which are summed
+//     in the order of a direct sum with every operation rounded as written (no
+//     contraction), so every decision is taken on the same values as a plain
+//     fp64 statement of the method.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace ecasq {
+namespace {
+
+// Padded column layout of the cost table, in 16-byte vectors of kvec values:
+// column x (entries a = 0 .. x-1) starts at vector cb[x], 16-byte aligned, and
+// cb[x] = x (mod 8), so the eight columns a quarter-warp reads with one 16-byte
+// load each lie on distinct banks. Returns cb[x+1] from cb[x].
+__host__ __device__ __forceinline__ int next_column(int start, int x, int kvec) {
+  const int end = start + (x + kvec - 1) / kvec;
+  return end + (((x + 1) - end) & 7);
+}
+
+// Two IEEE round-to-nearest additions in one packed f32x2 instruction.
+__device__ __forceinline__ float2 add_f32x2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rc, ra, rb;\n\tmov.b64 {%0, %1}, rc;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
+// Three-input minimum (exact).
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+template <typename T>
+struct AOps;
+
+template <>
+struct AOps<float> {
+  using Vec = float4;
+  __device__ static float4 cost4(float4 v, float4 e, double lam) {
+    const float l = static_cast<float>(lam);
+    return make_float4(__fmaf_rn(l, e.x, v.x), __fmaf_rn(l, e.y, v.y), __fmaf_rn(l, e.z, v.z), __fmaf_rn(l, e.w, v.w));
+  }
+  __device__ static float inf() { return __int_as_float(0x7f800000); }
+  __device__ static float add(float a, float b) { return __fadd_rn(a, b); }
+  __device__ static float cost(float v, float e, double lam) { return __fmaf_rn(static_cast<float>(lam), e, v); }
+  __device__ static float vmin(float a, float b) { return fminf(a, b); }
+  // Four relaxations: two packed additions, two three-input minima.
+  __device__ static void relax(float4 g, float4 w, float& b0, float& b1) {
+    const float2 s01 = add_f32x2(make_float2(g.x, g.y), make_float2(w.x, w.y));
+    const float2 s23 = add_f32x2(make_float2(g.z, g.w), make_float2(w.z, w.w));
+    b0 = min3f(b0, s01.x, s01.y);
+    b1 = min3f(b1, s23.x, s23.y);
+  }
+};
+
+template <>
+struct AOps<double> {
+  using Vec = double2;
+  __device__ static double2 cost4(double2 v, double2 e, double lam) {
+    return make_double2(__dadd_rn(v.x, __dmul_rn(lam, e.x)), __dadd_rn(v.y, __dmul_rn(lam, e.y)));
+  }
+  __device__ static double inf() { return __longlong_as_double(0x7ff0000000000000ll); }
+  __device__ static double add(double a, double b) { return __dadd_rn(a, b); }
+  __device__ static double cost(double v, double e, double lam) { return __dadd_rn(v, __dmul_rn(lam, e)); }
+  __device__ static double vmin(double a, double b) { return fmin(a, b); }
+  __device__ static void relax(double2 g, double2 w, double& b0, double& b1) {
+    b0 = fmin(b0, __dadd_rn(g.x, w.x));
+    b1 = fmin(b1, __dadd_rn(g.y, w.y));
+  }
+};
+
+// -(mu/d) log2(mu/d), 0 for mu <= 0.
+__device__ __forceinline__ double hmass(double mu, double dd) {
+  if (!(mu > 0.0)) return 0.0;
+  const double q = __ddiv_rn(mu, dd);
+  return __dmul_rn(-q, log2(q));
+}
+
+template <typename T>
+struct ACtx {
+  int p, S, tri;
+  double dd;
+  double *sP, *sN, *sA, *sB;
+  int* sQ;
+  double* fbuf;  // [warps][p] local costs of the refinement
+  int* moved;    // refinement move counter (shared)
+  int* msh;      // code size handed from the recovery warp to the block (shared)
+  int pst;       // row stride of the layers (p rounded up to a 16-byte multiple)
+  const int* cb; // [p+1] first 16-byte vector of each padded cost column (shared)
+  T* vt;         // padded columns: V/d in the layer precision
+  T* et;         // padded columns: h(L) + h(R) in the layer precision
+  double* V;     // [tri] fp64 interval tables, pair (a, c) at col_off(c) + a
+  double* R;
+  double* L;
+  T* cost;  // padded columns, w(a, x) at cb[x] * (16 / sizeof(T)) + a
+  T* G;     // [(S+1) * pst]
+  __device__ int at(int a, int e) const { return col_off(e) + a; }
+};
+
+struct AOut {
+  int m;
+  double mse, H, HIB, J;
+};
+
+// Per-vector tables in two passes.
+// Pass 1, column by column (e = 1 .. p-1): thread a (< e) adds bucket e-1 to its
+// running sums N, T1, T2 over a .. e-1 (ascending, the order of a direct sum),
+// every operation rounded as written, and stores V, R, L of (a, e); the threads
+// of one column write adjacent words. Needs blockDim.x >= p - 1.
+// Pass 2, over all pairs evenly: the layer-precision terms V/d and h(L)+h(R).
+template <typename T>
+__device__ void build_pair_terms(const ACtx<T>& c) {
+  const int p = c.p, a = threadIdx.x;
+  double N = 0.0, T1 = 0.0, T2 = 0.0;
+  const double Pa = a < p ? c.sP[a] : 0.0;
+  for (int e = 1; e < p; ++e) {
+    if (a < e) {
+      const int k = e - 1;
+      const double dk = __dsub_rn(c.sP[k], Pa);
+      const double nk = c.sN[k];
+      N = __dadd_rn(N, nk);
+      T1 = __dadd_rn(T1, __dadd_rn(c.sA[k], __dmul_rn(nk, dk)));
+      T2 = __dadd_rn(T2, __dadd_rn(__dadd_rn(c.sB[k], __dmul_rn(__dmul_rn(2.0, dk), c.sA[k])),
+                                   __dmul_rn(__dmul_rn(nk, dk), dk)));
+      const double W = __dsub_rn(c.sP[e], Pa);
+      double V = __dsub_rn(__dmul_rn(W, T1), T2);
+      V = V < 0.0 ? 0.0 : V;
+      const double R = W > 0.0 ? __ddiv_rn(T1, W) : 0.0;
+      const int i = col_off(e) + a;
+      c.V[i] = V;
+      c.R[i] = R;
+      c.L[i] = __dsub_rn(N, R);
+    }
+  }
+  __syncthreads();
+  constexpr int kVec = 16 / sizeof(T);
+  for (int i = threadIdx.x; i < c.tri; i += blockDim.x) {
+    // column e of entry i: col_off(e) <= i < col_off(e + 1)
+    int e = static_cast<int>((1.0f + sqrtf(1.0f + 8.0f * static_cast<float>(i))) * 0.5f);
+    while (col_off(e) > i) --e;
+    while (col_off(e + 1) <= i) ++e;
+    const int aa = i - col_off(e);
+    const int o = c.cb[e] * kVec + aa;
+    c.vt[o] = static_cast<T>(__ddiv_rn(c.V[i], c.dd));
+    c.et[o] = static_cast<T>(__dadd_rn(hmass(c.L[i], c.dd), hmass(c.R[i], c.dd)));
+  }
+}
+
+// Local exact cost of the value at position t placed at index x (fp64): its two
+// intervals and the three masses that depend on it.
+template <typename T>
+__device__ __forceinline__ double local_cost(const ACtx<T>& c, double lam, int a, int e, int x, double r_before,
+                                             double l_after) {
+  const int ia = c.at(a, x), ib = c.at(x, e);
+  const double f = __ddiv_rn(__dadd_rn(c.V[ia], c.V[ib]), c.dd);
+  const double mu_prev = __dadd_rn(r_before, c.L[ia]);
+  const double mu_self = __dadd_rn(c.R[ia], c.L[ib]);
+  const double mu_next = __dadd_rn(c.R[ib], l_after);
+  const double hs = __dadd_rn(__dadd_rn(hmass(mu_prev, c.dd), hmass(mu_self, c.dd)), hmass(mu_next, c.dd));
+  return __dadd_rn(f, __dmul_rn(lam, hs));
+}
+
+// Refinement of c.sQ[0..m-1] in place (all threads). A warp takes one value of
+// the class; its lanes evaluate the local cost at every index of the open
+// interval, then lane 0 runs the binary search over those stored costs (the
+// same decisions a search computing them on demand takes) and the move test.
+template <typename T>
+__device__ void refine_code(const ACtx<T>& c, double lam, int m, int iters) {
+  const int lane = lane_id(), warp = warp_id(), nw = blockDim.x / kWarp;
+  int* Q = c.sQ;
+  double* fb = c.fbuf + static_cast<size_t>(warp) * c.p;
+  for (int it = 0; it < iters; ++it) {
+    if (threadIdx.x == 0) *c.moved = 0;
+    __syncthreads();
+    for (int cls = 0; cls < 3; ++cls) {
+      const int npos = (m - 2 - cls + 2) / 3;  // positions 1 + cls + 3j <= m - 2
+      for (int j = warp; j < npos; j += nw) {
+        const int t = 1 + cls + 3 * j;
+        const int a = Q[t - 1], e = Q[t + 1];
+        const double r_before = (t - 1 > 0) ? c.R[c.at(Q[t - 2], a)] : 0.0;
+        const double l_after = (t + 1 < m - 1) ? c.L[c.at(e, Q[t + 2])] : 0.0;
+        const int lo = a + 1, hi = e - 1;
+        for (int x = lo + lane; x <= hi; x += kWarp) fb[x - lo] = local_cost(c, lam, a, e, x, r_before, l_after);
+        __syncwarp();
+        if (lane == 0) {
+          int l = lo, h = hi;
+          while (l < h) {
+            const int mid = l + (h - l) / 2;
+            if (fb[mid + 1 - lo] < fb[mid - lo])
+              l = mid + 1;
+            else
+              h = mid;
+          }
+          if (l != Q[t] && fb[l - lo] < fb[Q[t] - lo]) {
+            Q[t] = l;  // no other value of the class reads position t
+            atomicAdd(c.moved, 1);
+          }
+        }
+        __syncwarp();
+      }
+      __syncthreads();
+    }
+    if (*c.moved == 0) break;
+    __syncthreads();
+  }
+}
+
+// fp64 evaluation of c.sQ (warp 0). The lanes fetch the intervals' tables and
+// take the logarithms in parallel; lane 0 then adds the terms in ascending
+// order of t, the order of the definitions.
+template <typename T>
+__device__ void evaluate_code(const ACtx<T>& c, double lam, bool refined, int m, AOut* out) {
+  const int lane = lane_id();
+  double* tv = c.fbuf;           // V_t
+  double* th = c.fbuf + c.S;     // h(mu_t)
+  double* tl = c.fbuf + 2 * c.S; // h(L_t)
+  double* tr = c.fbuf + 3 * c.S; // h(R_t)
+  for (int t = lane; t < m; t += kWarp) {
+    double u = 0.0;
+    if (t > 0) u = __dadd_rn(u, c.R[c.at(c.sQ[t - 1], c.sQ[t])]);
+    if (t + 1 < m) {
+      const int i = c.at(c.sQ[t], c.sQ[t + 1]);
+      const double L = c.L[i];
+      u = __dadd_rn(u, L);
+      tv[t] = c.V[i];
+      tl[t] = hmass(L, c.dd);
+      tr[t] = hmass(c.R[i], c.dd);
+    }
+    th[t] = hmass(u, c.dd);
+  }
+  __syncwarp();
+  if (lane == 0) {
+    double sv = 0.0, sh = 0.0, sib = 0.0;
+    for (int t = 0; t < m; ++t) {
+      if (t + 1 < m) sv = __dadd_rn(sv, tv[t]);
+      sh = __dadd_rn(sh, th[t]);
+      if (t + 1 < m) {
+        sib = __dadd_rn(sib, tl[t]);
+        sib = __dadd_rn(sib, tr[t]);
+      }
+    }
+    out->m = m;
+    out->mse = __ddiv_rn(sv, c.dd);
+    out->H = sh;
+    out->HIB = sib;
+    out->J = __dadd_rn(out->mse, __dmul_rn(lam, refined ? sh : sib));
+  }
+  __syncwarp();
+}
+
+// One solve at lambda (all threads): cost table, layers, recovery of the code,
+// refinement, evaluation. Leaves the code in c.sQ and the figures in *out.
+template <typename T>
+__device__ void approx_solve(const ACtx<T>& c, double lam, int refine, AOut* out) {
+  using O = AOps<T>;
+  const int p = c.p, S = c.S, tid = threadIdx.x, bd = blockDim.x;
+  constexpr int kVec = 16 / sizeof(T);
+  using V16 = typename AOps<T>::Vec;
+  // Cost table w = V/d + lambda*(h(L)+h(R)) from the L2-resident pair terms
+  // (same padded layout): 16-byte loads, several in flight per thread, so the
+  // table arrives in about one L2 round trip. Padding words are computed too and
+  // never read.
+  {
+    const int nvec = c.cb[p];
+    const V16* vv = reinterpret_cast<const V16*>(c.vt);
+    const V16* ev = reinterpret_cast<const V16*>(c.et);
+    V16* cv = reinterpret_cast<V16*>(c.cost);
+#pragma unroll 4
+    for (int q = tid; q < nvec; q += bd) cv[q] = AOps<T>::cost4(vv[q], ev[q], lam);
+  }
+  for (int x = tid; x < p; x += bd) c.G[c.pst + x] = (x == 0) ? T(0) : O::inf();
+  __syncthreads();
+  for (int i = 2; i <= S; ++i) {
+    const T* __restrict__ Gp = c.G + (i - 1) * c.pst;
+    T* __restrict__ Gc = c.G + i * c.pst;
+    for (int x = i - 1 + tid; x < p; x += bd) {
+      // min over a = i-2 .. x-1 of G_{i-1}(a) + w(a, x): scalar up to a 16-byte
+      // boundary, then four (fp32) or two (fp64) consecutive a per load of the
+      // column and of the layer (a broadcast), then the scalar tail.
+      const T* __restrict__ col = c.cost + c.cb[x] * kVec;
+      T b0 = O::inf(), b1 = O::inf(), b2 = O::inf(), b3 = O::inf();
+      int a = i - 2;
+      const int ah = min(x, (a + kVec - 1) / kVec * kVec);
+      for (; a < ah; ++a) b0 = O::vmin(b0, O::add(Gp[a], col[a]));
+      const int av = a + (x - a) / (2 * kVec) * (2 * kVec);
+      for (; a < av; a += 2 * kVec) {
+        const V16 g0 = *reinterpret_cast<const V16*>(Gp + a);
+        const V16 g1 = *reinterpret_cast<const V16*>(Gp + a + kVec);
+        const V16 w0 = *reinterpret_cast<const V16*>(col + a);
+        const V16 w1 = *reinterpret_cast<const V16*>(col + a + kVec);
+        AOps<T>::relax(g0, w0, b0, b1);
+        AOps<T>::relax(g1, w1, b2, b3);
+      }
+      for (; a < x; ++a) b1 = O::vmin(b1, O::add(Gp[a], col[a]));
+      Gc[x] = O::vmin(O::vmin(b0, b1), O::vmin(b2, b3));
+    }
+    __syncthreads();
+  }
+  if (warp_id() == 0) {
+    const int lane = lane_id();
+    T bv = O::inf();
+    int bi = 0x7fffffff;
+    for (int i = 2 + lane; i <= S; i += kWarp) {
+      const T g = c.G[i * c.pst + p - 1];
+      if (g < bv) {
+        bv = g;
+        bi = i;
+      }
+    }
+    warp_argmin(bv, bi);
+    int m;
+    if (bi == 0x7fffffff) {  // no finite candidate (non-finite inputs): {P_0, P_{p-1}}
+      m = 2;
+      if (lane == 0) {
+        c.sQ[0] = 0;
+        c.sQ[1] = p - 1;
+      }
+    } else {
+      // Recovery: the smallest a whose sum equals the layer's minimum (it is
+      // one of them exactly); all chunks of the column are tested at once.
+      m = bi;
+      int x = p - 1;
+      if (lane == 0) c.sQ[m - 1] = x;
+      for (int i = m; i >= 2; --i) {
+        const T target = c.G[i * c.pst + x];
+        const T* Gp = c.G + (i - 1) * c.pst;
+        const T* col = c.cost + c.cb[x] * kVec;
+        int found = 0x7fffffff;
+#pragma unroll 4
+        for (int base = i - 2; base < x; base += kWarp) {
+          const int a = base + lane;
+          const bool hit = a < x && O::add(Gp[a], col[a]) == target;
+          const unsigned msk = __ballot_sync(0xffffffffu, hit);
+          if (msk && found == 0x7fffffff) found = base + __ffs(msk) - 1;
+        }
+        if (found == 0x7fffffff) found = i - 2;  // not reached: the minimum is one of the sums
+        x = found;
+        if (lane == 0) c.sQ[i - 2] = x;
+      }
+    }
+    if (lane == 0) *c.msh = m;
+  }
+  __syncthreads();
+  const int m = *c.msh;
+  if (refine > 0) refine_code(c, lam, m, refine);
+  if (warp_id() == 0) evaluate_code(c, lam, refine > 0, m, out);
+  __syncthreads();
+}
+
+template <typename T, bool kSmem>
+__global__ void __launch_bounds__(512, 1) k_approx(ApproxArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ AOut s_out;
+  __shared__ int s_flag;
+  __shared__ int s_misc[2];
+
+  const int p = a.p, S = a.s;
+  ACtx<T> c;
+  c.p = p;
+  c.S = S;
+  c.tri = tri_size(p);
+  c.dd = static_cast<double>(a.d);
+
+  unsigned char* sp = smem;
+  auto carve = [&sp](size_t bytes) {
+    unsigned char* r = sp;
+    sp += (bytes + 15) & ~size_t(15);
+    return r;
+  };
+  c.sP = reinterpret_cast<double*>(carve(sizeof(double) * p));
+  c.sN = reinterpret_cast<double*>(carve(sizeof(double) * p));
+  c.sA = reinterpret_cast<double*>(carve(sizeof(double) * p));
+  c.sB = reinterpret_cast<double*>(carve(sizeof(double) * p));
+  c.sQ = reinterpret_cast<int*>(carve(sizeof(int) * S));
+  int* sQ1 = reinterpret_cast<int*>(carve(sizeof(int) * S));
+  int* sQ2 = reinterpret_cast<int*>(carve(sizeof(int) * S));
+  int* cbs = reinterpret_cast<int*>(carve(sizeof(int) * (p + 1)));
+  c.moved = &s_misc[0];
+  c.msh = &s_misc[1];
+  constexpr int kVec = 16 / sizeof(T);
+  if (threadIdx.x == 0) {
+    cbs[0] = 0;
+    for (int x = 0; x < p; ++x) cbs[x + 1] = next_column(cbs[x], x, kVec);
+  }
+  __syncthreads();
+  c.cb = cbs;
+  c.pst = (p + kVec - 1) / kVec * kVec;
+
+  // Global slab: [V/d][h(L)+h(R)] in T (padded columns), [V][R][L] in fp64,
+  // then the cost table (whose space the refinement and the evaluation reuse)
+  // and the layers when they are not in shared memory.
+  unsigned char* gs = a.scratch + static_cast<size_t>(blockIdx.x) * a.scratch_per_cta;
+  const size_t vb = (16 * static_cast<size_t>(cbs[p]) + 255) & ~size_t(255);
+  const size_t db = (sizeof(double) * static_cast<size_t>(c.tri) + 255) & ~size_t(255);
+  const size_t fb = sizeof(double) * p * (blockDim.x / kWarp);
+  const size_t cbytes = (((vb > fb) ? vb : fb) + 255) & ~size_t(255);
+  c.vt = reinterpret_cast<T*>(gs);
+  c.et = reinterpret_cast<T*>(gs + vb);
+  c.V = reinterpret_cast<double*>(gs + 2 * vb);
+  c.R = reinterpret_cast<double*>(gs + 2 * vb + db);
+  c.L = reinterpret_cast<double*>(gs + 2 * vb + 2 * db);
+  unsigned char* big = kSmem ? sp : gs + 2 * vb + 3 * db;
+  c.cost = reinterpret_cast<T*>(big);
+  c.fbuf = reinterpret_cast<double*>(big);
+  c.G = reinterpret_cast<T*>(big + cbytes);
+
+  for (int r = blockIdx.x; r < a.n; r += gridDim.x) {
+    const double* P = a.P + static_cast<int64_t>(r) * p;
+    const int64_t bo = static_cast<int64_t>(r) * (p - 1);
+    if (threadIdx.x == 0) s_flag = a.in_status ? a.in_status[r] : 0;
+    for (int k = threadIdx.x; k < p; k += blockDim.x) {
+      c.sP[k] = P[k];
+      if (k < p - 1) {
+        c.sN[k] = static_cast<double>(a.cnt[bo + k]);
+        c.sA[k] = a.A[bo + k];
+        c.sB[k] = a.B[bo + k];
+      }
+    }
+    __syncthreads();
+    const bool degenerate = (c.sP[0] == c.sP[p - 1]);
+    int bad = 0;
+    if (!degenerate)
+      for (int k = threadIdx.x; k < p - 1; k += blockDim.x) bad |= !(c.sP[k] < c.sP[k + 1]);
+    bad = __syncthreads_or(bad);
+    const int32_t st = s_flag != 0 ? s_flag : (bad ? kStatusArg : kStatusOk);
+    const int so = a.s_out;
+
+    if (st != kStatusOk || degenerate) {
+      const int qv = (st == kStatusOk) ? 0 : -1;
+      const int ml = (st == kStatusOk) ? 1 : 0;
+      if (a.mode == 0) {
+        for (int t = 0; t < a.n_lambda; ++t) {
+          const int64_t w = static_cast<int64_t>(r) * a.n_lambda + t;
+          for (int q = threadIdx.x; q < so; q += blockDim.x) a.Q[w * so + q] = (q == 0) ? qv : -1;
+          if (threadIdx.x == 0) {
+            a.Q_len[w] = ml;
+            a.obj[w] = a.mse[w] = a.H[w] = a.HIB[w] = 0.0;
+          }
+        }
+      } else {
+        for (int q = threadIdx.x; q < so; q += blockDim.x) {
+          a.Q1[int64_t(r) * so + q] = (q == 0) ? qv : -1;
+          a.Q2[int64_t(r) * so + q] = (q == 0) ? qv : -1;
+        }
+        if (threadIdx.x == 0) {
+          a.Q1_len[r] = a.Q2_len[r] = ml;
+          a.theta[r] = a.lam_lo[r] = a.lam_hi[r] = 0.0;
+          a.H1[r] = a.H2[r] = a.HIB1[r] = a.HIB2[r] = a.mse1[r] = a.mse2[r] = 0.0;
+        }
+      }
+      if (threadIdx.x == 0) a.status[r] = st;
+      __syncthreads();
+      continue;
+    }
+
+    build_pair_terms(c);
+    __syncthreads();
+
+    if (a.mode == 0) {
+      for (int t = 0; t < a.n_lambda; ++t) {
+        const int64_t w = static_cast<int64_t>(r) * a.n_lambda + t;
+        approx_solve(c, a.lambda[w], a.refine, &s_out);
+        for (int q = threadIdx.x; q < so; q += blockDim.x) a.Q[w * so + q] = (q < s_out.m) ? c.sQ[q] : -1;
+        if (threadIdx.x == 0) {
+          a.Q_len[w] = s_out.m;
+          a.obj[w] = s_out.J;
+          a.mse[w] = s_out.mse;
+          a.H[w] = s_out.H;
+          a.HIB[w] = s_out.HIB;
+        }
+        __syncthreads();
+      }
+      if (threadIdx.x == 0) a.status[r] = kStatusOk;
+    } else {
+      // Bisection on lambda with two-way time-sharing; the constrained rate is
+      // H(I,B) for the plain approximation and H(X^) once refined.
+      const bool refined = a.refine > 0;
+      double lo = 0.0;
+      double hi = (c.sP[p - 1] - c.sP[0]) * (c.sP[p - 1] - c.sP[0]);
+      double H1 = 0, H2 = 0, B1 = 0, B2 = 0, M1 = 0, M2 = 0, r1 = 0, r2 = 0;
+      int m1 = 0, m2 = 0;
+      auto keep = [&](int* dst, int& m, double& Hk, double& Bk, double& Mk) {
+        for (int q = threadIdx.x; q < S; q += blockDim.x) dst[q] = c.sQ[q];
+        m = s_out.m;
+        Hk = s_out.H;
+        Bk = s_out.HIB;
+        Mk = s_out.mse;
+      };
+      auto rate = [&]() { return refined ? s_out.H : s_out.HIB; };
+      int32_t status = kStatusOk;
+      double theta = 0.0;
+      approx_solve(c, 0.0, a.refine, &s_out);
+      keep(sQ1, m1, H1, B1, M1);
+      r1 = rate();
+      if (r1 <= a.budget) {
+        keep(sQ2, m2, H2, B2, M2);
+        hi = 0.0;
+      } else {
+        __syncthreads();
+        approx_solve(c, hi, a.refine, &s_out);
+        keep(sQ2, m2, H2, B2, M2);
+        r2 = rate();
+        if (r2 > a.budget) {
+          status = kStatusBudget;
+        } else {
+          for (int it = 0; it < a.steps; ++it) {
+            const double mid = 0.5 * (lo + hi);
+            __syncthreads();
+            approx_solve(c, mid, a.refine, &s_out);
+            const double rr = rate();
+            if (rr > a.budget) {
+              lo = mid;
+              r1 = rr;
+              keep(sQ1, m1, H1, B1, M1);
+            } else {
+              hi = mid;
+              r2 = rr;
+              keep(sQ2, m2, H2, B2, M2);
+            }
+          }
+          const double th = (a.budget - r2) / (r1 - r2);
+          theta = th < 0.0 ? 0.0 : (th > 1.0 ? 1.0 : th);
+        }
+      }
+      __syncthreads();
+      for (int q = threadIdx.x; q < so; q += blockDim.x) {
+        a.Q1[int64_t(r) * so + q] = (q < m1) ? sQ1[q] : -1;
+        a.Q2[int64_t(r) * so + q] = (q < m2) ? sQ2[q] : -1;
+      }
+      if (threadIdx.x == 0) {
+        a.Q1_len[r] = m1;
+        a.Q2_len[r] = m2;
+        a.theta[r] = theta;
+        a.lam_lo[r] = lo;
+        a.lam_hi[r] = hi;
+        a.H1[r] = H1;
+        a.H2[r] = H2;
+        a.HIB1[r] = B1;
+        a.HIB2[r] = B2;
+        a.mse1[r] = M1;
+        a.mse2[r] = M2;
+        a.status[r] = status;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+template <typename T, bool kSmem>
+void* approx_kernel_ptr() {
+  return reinterpret_cast<void*>(&k_approx<T, kSmem>);
+}
+
+void* approx_fn(bool fp64, bool smem) {
+  return fp64 ? (smem ? approx_kernel_ptr<double, true>() : approx_kernel_ptr<double, false>())
+              : (smem ? approx_kernel_ptr<float, true>() : approx_kernel_ptr<float, false>());
+}
+
+size_t al16(size_t b) { return (b + 15) & ~size_t(15); }
+size_t al256(size_t b) { return (b + 255) & ~size_t(255); }
+
+}  // namespace
+
+bool approx_plan(int n, int p, int s, bool fp64, ApproxPlan* plan) {
+  if (p < 2 || p > kMaxP || s < 2 || n < 1) return false;
+  const int S = s < p ? s : p;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  int sms = 0, optin = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  const size_t tsz = fp64 ? 8 : 4;
+  const int kvec = static_cast<int>(16 / tsz);
+  int ncv = 0;
+  for (int x = 0; x < p; ++x) ncv = next_column(ncv, x, kvec);
+  const size_t vb = al256(16 * static_cast<size_t>(ncv));
+  const size_t db = al256(8 * static_cast<size_t>(tri_size(p)));
+  plan->fp64 = fp64;
+  // Table pass 1 gives each thread one a: threads >= p - 1.
+  plan->threads = p <= 128 ? 128 : (p <= 256 ? 256 : 512);
+  const size_t fb = 8 * static_cast<size_t>(p) * (plan->threads / 32);
+  const size_t cbytes = al256(vb > fb ? vb : fb);
+  const int pst = (p + kvec - 1) / kvec * kvec;
+  const size_t small = al16(8 * p) * 4 + al16(4 * S) * 3 + al16(4 * static_cast<size_t>(p + 1));
+  const size_t big = cbytes + al16(tsz * static_cast<size_t>(S + 1) * pst);
+  plan->smem = small + big + 1024 <= static_cast<size_t>(optin);
+  plan->smem_bytes = small + (plan->smem ? big : 0);
+  plan->scratch_per_cta = al256(2 * vb + 3 * db + (plan->smem ? 0 : big));
+  void* fn = approx_fn(fp64, plan->smem);
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(plan->smem_bytes)) !=
+      cudaSuccess)
+    return false;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, plan->threads, plan->smem_bytes) != cudaSuccess ||
+      per_sm < 1)
+    return false;
+  const int ctas = sms * per_sm;
+  plan->ctas = n < ctas ? n : ctas;
+  return true;
+}
+
+cudaError_t launch_approx(const ApproxPlan& plan, ApproxArgs args, cudaStream_t st) {
+  void* kargs[] = {&args};
+  cudaError_t e = cudaLaunchKernel(approx_fn(plan.fp64, plan.smem), dim3(plan.ctas), dim3(plan.threads), kargs,
+                                   plan.smem_bytes, st);
+  note_launch();
+  return e;
+}
+
+int64_t approx_pair_layers(int p, int s) {
+  const int S = s < p ? s : p;
+  int64_t t = 0;
+  for (int i = 2; i <= S; ++i)
+    for (int x = i - 1; x <= p - 1; ++x) t += x - (i - 2);
+  return t;
+}
+
+}  // namespace ecasq

@@ -86,6 +86,60 @@ cudaError_t launch_dp(const DpPlan& plan, DpArgs args, cudaStream_t st);
 // Exact count of (k, l, j) triples one solve evaluates (host).
 int64_t dp_triples(int p, int s);
 
+// ---- approximation on H(I,B) + refinement (approx.cu) ----
+struct ApproxArgs {
+  const int64_t* cnt;
+  const double* A;
+  const double* B;
+  const double* P;
+  const int32_t* in_status;
+  int n, p, s;  // s already clamped to p
+  int64_t d;
+  int refine;  // refinement iterations (0: none)
+  int mode;    // 0: lambda list, 1: entropy budget
+  const double* lambda;
+  int n_lambda;
+  double budget;
+  int steps;
+  int32_t* Q;
+  int32_t* Q_len;
+  double* obj;
+  double* mse;
+  double* H;
+  double* HIB;
+  int32_t* Q1;
+  int32_t* Q1_len;
+  int32_t* Q2;
+  int32_t* Q2_len;
+  double* theta;
+  double* lam_lo;
+  double* lam_hi;
+  double* H1;
+  double* H2;
+  double* HIB1;
+  double* HIB2;
+  double* mse1;
+  double* mse2;
+  int32_t* status;
+  int s_out;
+  unsigned char* scratch;
+  size_t scratch_per_cta;
+};
+
+struct ApproxPlan {
+  bool fp64;
+  bool smem;  // cost table and layers in shared memory
+  int threads;
+  int ctas;
+  size_t smem_bytes;
+  size_t scratch_per_cta;
+};
+
+bool approx_plan(int n, int p, int s, bool fp64, ApproxPlan* plan);
+cudaError_t launch_approx(const ApproxPlan& plan, ApproxArgs args, cudaStream_t st);
+// (i, a, c) relaxations of one solve of the layered shortest path (host).
+int64_t approx_pair_layers(int p, int s);
+
 // ---- encoder (encode.cu) ----
 cudaError_t launch_encode(const float* X, const double* P, int n, int64_t d, int p, int s,
                           const int32_t* Q1, const int32_t* Q1_len, const int32_t* Q2,

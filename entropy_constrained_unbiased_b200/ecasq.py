@@ -19,6 +19,8 @@ OK, ERR_ARG, ERR_RANGE, ERR_WORKSPACE, ERR_CUDA, WARN_BUDGET = 0, -1, -2, -3, -4
 EXPORTS = [
     "ecasq_workspace_size", "ecasq_aux_workspace_size", "ecasq_uniform_grid", "ecasq_bucket", "ecasq_bucket_noalloc",
     "ecasq_solve", "ecasq_solve_stats", "ecasq_solve_budget", "ecasq_solve_budget_stats",
+    "ecasq_approx_workspace_size", "ecasq_solve_approx", "ecasq_solve_approx_stats", "ecasq_solve_approx_budget",
+    "ecasq_solve_approx_budget_stats",
     "ecasq_encode", "ecasq_entropy", "ecasq_status_string", "ecasq_launch_count",
 ]
 
@@ -55,6 +57,11 @@ def load(path: str = LIB_PATH):
         "ecasq_solve_stats": (I, [P, P, P, P, I, I64, I, I, P, I, P, P, P, P, P, P, OP, P, SZ, P]),
         "ecasq_solve_budget": (I, [P, P, I, I64, I, I, D] + [P] * 12 + [OP, P, SZ, P]),
         "ecasq_solve_budget_stats": (I, [P, P, P, P, I, I64, I, I, D] + [P] * 12 + [OP, P, SZ, P]),
+        "ecasq_approx_workspace_size": (SZ, [I, I64, I, I, OP]),
+        "ecasq_solve_approx": (I, [P, P, I, I64, I, I, P, I, I, P, P, P, P, P, P, P, OP, P, SZ, P]),
+        "ecasq_solve_approx_stats": (I, [P, P, P, P, I, I64, I, I, P, I, I, P, P, P, P, P, P, P, OP, P, SZ, P]),
+        "ecasq_solve_approx_budget": (I, [P, P, I, I64, I, I, D, I] + [P] * 14 + [OP, P, SZ, P]),
+        "ecasq_solve_approx_budget_stats": (I, [P, P, P, P, I, I64, I, I, D, I] + [P] * 14 + [OP, P, SZ, P]),
         "ecasq_encode": (I, [P, P, I, I64, I, I, P, P, P, P, P, U64, P, P, P, P]),
         "ecasq_entropy": (I, [P, I, I, P, P]),
         "ecasq_status_string": (C.c_char_p, [I]),
@@ -253,6 +260,87 @@ def solve_budget_stats(cnt, A, B, P, d: int, s: int, b: float, steps: int = 30, 
     _check(L.ecasq_solve_budget_stats(_ptr(cnt), _ptr(A), _ptr(B), _ptr(P), n, d, p, s, float(b),
                                       *[_ptr(o[k]) for k in _BUDGET_ORDER], C.byref(op), _ptr(ws), ws.numel(),
                                       _stream()), "ecasq_solve_budget_stats")
+    return o
+
+
+# -- approximation on H(I,B) and iterative refinement ---------------------------
+
+def solve_approx(X: torch.Tensor, P: torch.Tensor, s: int, lam, refine: int = 0, fp64: bool = False):
+    """Approximate solve of each row at each of its lambdas ([n] or [n, L]); with
+    refine > 0 the code is then refined on the exact objective. Adds H_IB."""
+    L = _need_cuda()
+    _dev(X, torch.float32, "X")
+    _dev(P, torch.float64, "P")
+    n, d = X.shape
+    p = P.shape[1]
+    lt = _lam_table(lam, n, X.device)
+    nl = lt.shape[1]
+    o = _solve_outputs(n, nl, s, X.device)
+    o["H_IB"] = torch.empty((n, nl), dtype=torch.float64, device=X.device)
+    op = opts(fp64)
+    ws = workspace(L.ecasq_approx_workspace_size(n, d, p, s, C.byref(op)), X.device)
+    _check(L.ecasq_solve_approx(_ptr(X), _ptr(P), n, d, p, s, _ptr(lt), nl, int(refine), _ptr(o["Q"]),
+                                _ptr(o["Q_len"]), _ptr(o["objective"]), _ptr(o["mse"]), _ptr(o["H"]),
+                                _ptr(o["H_IB"]), _ptr(o["status"]), C.byref(op), _ptr(ws), ws.numel(), _stream()),
+           "ecasq_solve_approx")
+    return o
+
+
+def solve_approx_stats(cnt, A, B, P, d: int, s: int, lam, refine: int = 0, fp64: bool = False):
+    L = _need_cuda()
+    n, p = P.shape
+    lt = _lam_table(lam, n, P.device)
+    nl = lt.shape[1]
+    o = _solve_outputs(n, nl, s, P.device)
+    o["H_IB"] = torch.empty((n, nl), dtype=torch.float64, device=P.device)
+    op = opts(fp64)
+    ws = workspace(L.ecasq_approx_workspace_size(n, d, p, s, C.byref(op)), P.device)
+    _check(L.ecasq_solve_approx_stats(_ptr(cnt), _ptr(A), _ptr(B), _ptr(P), n, d, p, s, _ptr(lt), nl, int(refine),
+                                      _ptr(o["Q"]), _ptr(o["Q_len"]), _ptr(o["objective"]), _ptr(o["mse"]),
+                                      _ptr(o["H"]), _ptr(o["H_IB"]), _ptr(o["status"]), C.byref(op), _ptr(ws),
+                                      ws.numel(), _stream()), "ecasq_solve_approx_stats")
+    return o
+
+
+_APPROX_BUDGET_ORDER = ("Q1", "Q1_len", "Q2", "Q2_len", "theta", "lambda_lo", "lambda_hi", "H1", "H2", "H_IB1",
+                        "H_IB2", "mse1", "mse2", "status")
+
+
+def _approx_budget_outputs(n, s, device):
+    o = _budget_outputs(n, s, device)
+    for k in ("H_IB1", "H_IB2"):
+        o[k] = torch.empty(n, dtype=torch.float64, device=device)
+    return o
+
+
+def solve_approx_budget(X: torch.Tensor, P: torch.Tensor, s: int, b: float, refine: int = 0, steps: int = 30,
+                        fp64: bool = False):
+    """Entropy budget b for the approximation (rate H(I,B)) or, with refine > 0,
+    for the refined approximation (rate H)."""
+    L = _need_cuda()
+    _dev(X, torch.float32, "X")
+    _dev(P, torch.float64, "P")
+    n, d = X.shape
+    p = P.shape[1]
+    o = _approx_budget_outputs(n, s, X.device)
+    op = opts(fp64, steps)
+    ws = workspace(L.ecasq_approx_workspace_size(n, d, p, s, C.byref(op)), X.device)
+    _check(L.ecasq_solve_approx_budget(_ptr(X), _ptr(P), n, d, p, s, float(b), int(refine),
+                                       *[_ptr(o[k]) for k in _APPROX_BUDGET_ORDER], C.byref(op), _ptr(ws),
+                                       ws.numel(), _stream()), "ecasq_solve_approx_budget")
+    return o
+
+
+def solve_approx_budget_stats(cnt, A, B, P, d: int, s: int, b: float, refine: int = 0, steps: int = 30,
+                              fp64: bool = False):
+    L = _need_cuda()
+    n, p = P.shape
+    o = _approx_budget_outputs(n, s, P.device)
+    op = opts(fp64, steps)
+    ws = workspace(L.ecasq_approx_workspace_size(n, d, p, s, C.byref(op)), P.device)
+    _check(L.ecasq_solve_approx_budget_stats(_ptr(cnt), _ptr(A), _ptr(B), _ptr(P), n, d, p, s, float(b), int(refine),
+                                             *[_ptr(o[k]) for k in _APPROX_BUDGET_ORDER], C.byref(op), _ptr(ws),
+                                             ws.numel(), _stream()), "ecasq_solve_approx_budget_stats")
     return o
 
 

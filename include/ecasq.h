@@ -149,6 +149,69 @@ int ecasq_solve_budget_stats(const int64_t* cnt, const double* A, const double* 
                              double* mse1, double* mse2, int32_t* status,
                              const ecasq_opts* opts, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- Space-efficient approximation (§2.3) and iterative refinement (§2.4) ----
+ *
+ * The approximation replaces H(X^) by H(I,B), the entropy of the pair (index I
+ * of the code interval [q_t, q_{t+1}] holding the entry, rounding bit B). An
+ * entry on an interior code value belongs to the interval that starts there.
+ * With L, R the expected down/up counts of an interval,
+ *   H(I,B) = sum over intervals of h(L) + h(R),  h(mu) = -(mu/d) log2(mu/d),
+ * and H(X^) <= H(I,B) <= H(X^) + 1. MSE + lambda*H(I,B) is a sum of
+ * per-interval costs, so its exact minimiser (P_0, P_{p-1} in Q, |Q| <= s) is a
+ * layered shortest path in O(p^2 s) time with O(p s) state; at budget b its MSE
+ * is no larger than the exact optimum's at b - 1.
+ *
+ * refine_iters > 0 then refines the code on the exact objective MSE +
+ * lambda*H(X^) at the same lambda: the interior values, in three classes by
+ * position mod 3 (a class moves at once, since a value's move changes only its
+ * two intervals and three masses), each search the open interval between their
+ * neighbours by binary search on the sign of the forward difference of their
+ * local cost and move only on a strict decrease; up to refine_iters iterations
+ * (classes 0, 1, 2), stopping early after an iteration with no move. The
+ * refinement never changes |Q|.
+ *
+ * Layers run in fp32 (default) or fp64 (opts->dp_fp64); refinement and the
+ * reported figures are fp64. opts->hirschberg is ignored (no back-pointers are
+ * kept). Workspace: ecasq_approx_workspace_size. Returns as the exact solver. */
+size_t ecasq_approx_workspace_size(int n, int64_t d, int p, int s, const ecasq_opts* opts);
+
+/* Per row and multiplier (lambda [n][n_lambda] >= 0): the code Q [n][n_lambda][s]
+ * and its fp64 mse, H = H(X^), H_IB = H(I,B) [n][n_lambda]; objective = mse +
+ * lambda*H_IB without refinement, mse + lambda*H with it. Buckets X internally. */
+int ecasq_solve_approx(const float* X, const double* P, int n, int64_t d, int p, int s,
+                       const double* lambda, int n_lambda, int refine_iters, int32_t* Q,
+                       int32_t* Q_len, double* objective, double* mse, double* H, double* H_IB,
+                       int32_t* status, const ecasq_opts* opts, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* Same, from bucket statistics (ecasq_bucket). */
+int ecasq_solve_approx_stats(const int64_t* cnt, const double* A, const double* B, const double* P,
+                             int n, int64_t d, int p, int s, const double* lambda, int n_lambda,
+                             int refine_iters, int32_t* Q, int32_t* Q_len, double* objective,
+                             double* mse, double* H, double* H_IB, int32_t* status,
+                             const ecasq_opts* opts, void* ws, size_t ws_bytes, void* stream);
+
+/* Entropy budget b with the bisection and two-way time-sharing of
+ * ecasq_solve_budget. The constrained rate is H(I,B) when refine_iters == 0 and
+ * H(X^) otherwise; theta = (b - rate2)/(rate1 - rate2). H1/H2 are H(X^) and
+ * H_IB1/H_IB2 are H(I,B) of Q1/Q2, whichever rate is constrained. */
+int ecasq_solve_approx_budget(const float* X, const double* P, int n, int64_t d, int p, int s,
+                              double b, int refine_iters, int32_t* Q1, int32_t* Q1_len, int32_t* Q2,
+                              int32_t* Q2_len, double* theta, double* lambda_lo, double* lambda_hi,
+                              double* H1, double* H2, double* H_IB1, double* H_IB2, double* mse1,
+                              double* mse2, int32_t* status, const ecasq_opts* opts, void* ws,
+                              size_t ws_bytes, void* stream);
+
+/* Same, from bucket statistics. */
+int ecasq_solve_approx_budget_stats(const int64_t* cnt, const double* A, const double* B,
+                                    const double* P, int n, int64_t d, int p, int s, double b,
+                                    int refine_iters, int32_t* Q1, int32_t* Q1_len, int32_t* Q2,
+                                    int32_t* Q2_len, double* theta, double* lambda_lo,
+                                    double* lambda_hi, double* H1, double* H2, double* H_IB1,
+                                    double* H_IB2, double* mse1, double* mse2, int32_t* status,
+                                    const ecasq_opts* opts, void* ws, size_t ws_bytes,
+                                    void* stream);
+
 /* Unbiased stochastic rounding (§1, E[X^] = X) with optional two-way
  * time-sharing (§2.1), counter-based randomness Philox4x32-10 (Salmon et al.,
  * SC'11) keyed by seed (low word, high word), counter (j >> 2, r, stream, 0),
