@@ -71,6 +71,13 @@ __device__ __forceinline__ float min3f(float a, float b, float c) {
   return r;
 }
 
+// -(mu/d) log2(mu/d), 0 for mu <= 0.
+__device__ __forceinline__ double hmass(double mu, double dd) {
+  if (!(mu > 0.0)) return 0.0;
+  const double q = __ddiv_rn(mu, dd);
+  return __dmul_rn(-q, log2(q));
+}
+
 template <typename T>
 struct AOps;
 
@@ -82,6 +89,16 @@ struct AOps<float> {
     return make_float4(__fmaf_rn(l, e.x, v.x), __fmaf_rn(l, e.y, v.y), __fmaf_rn(l, e.z, v.z), __fmaf_rn(l, e.w, v.w));
   }
   __device__ static float inf() { return __int_as_float(0x7f800000); }
+  // Layer-precision pair terms: V/d, and h(L) + h(R) with the MUFU log2 (the
+  // fp32 layers resolve no more than that).
+  __device__ static void terms(double V, double R, double L, double dd, double inv_d, float* vt, float* et) {
+    *vt = static_cast<float>(V * inv_d);
+    const float qr = static_cast<float>(R * inv_d), ql = static_cast<float>(L * inv_d);
+    const float hr = qr > 0.0f ? -qr * lg2_approx(qr) : 0.0f;
+    const float hl = ql > 0.0f ? -ql * lg2_approx(ql) : 0.0f;
+    *et = hl + hr;
+    (void)dd;
+  }
   __device__ static float add(float a, float b) { return __fadd_rn(a, b); }
   __device__ static float cost(float v, float e, double lam) { return __fmaf_rn(static_cast<float>(lam), e, v); }
   __device__ static float vmin(float a, float b) { return fminf(a, b); }
@@ -101,6 +118,12 @@ struct AOps<double> {
     return make_double2(__dadd_rn(v.x, __dmul_rn(lam, e.x)), __dadd_rn(v.y, __dmul_rn(lam, e.y)));
   }
   __device__ static double inf() { return __longlong_as_double(0x7ff0000000000000ll); }
+  // fp64 pair terms in the order of the definitions.
+  __device__ static void terms(double V, double R, double L, double dd, double inv_d, double* vt, double* et) {
+    *vt = __ddiv_rn(V, dd);
+    *et = __dadd_rn(hmass(L, dd), hmass(R, dd));
+    (void)inv_d;
+  }
   __device__ static double add(double a, double b) { return __dadd_rn(a, b); }
   __device__ static double cost(double v, double e, double lam) { return __dadd_rn(v, __dmul_rn(lam, e)); }
   __device__ static double vmin(double a, double b) { return fmin(a, b); }
@@ -109,13 +132,6 @@ struct AOps<double> {
     b1 = fmin(b1, __dadd_rn(g.y, w.y));
   }
 };
-
-// -(mu/d) log2(mu/d), 0 for mu <= 0.
-__device__ __forceinline__ double hmass(double mu, double dd) {
-  if (!(mu > 0.0)) return 0.0;
-  const double q = __ddiv_rn(mu, dd);
-  return __dmul_rn(-q, log2(q));
-}
 
 template <typename T>
 struct ACtx {
@@ -148,7 +164,8 @@ struct AOut {
 // running sums N, T1, T2 over a .. e-1 (ascending, the order of a direct sum),
 // every operation rounded as written, and stores V, R, L of (a, e); the threads
 // of one column write adjacent words. Needs blockDim.x >= p - 1.
-// Pass 2, over all pairs evenly: the layer-precision terms V/d and h(L)+h(R).
+// Pass 2, over all pairs evenly: the layer-precision terms V/d and h(L)+h(R)
+// (fp64 as defined for fp64 layers; fp32 with the MUFU log2 for fp32 layers).
 template <typename T>
 __device__ void build_pair_terms(const ACtx<T>& c) {
   const int p = c.p, a = threadIdx.x;
@@ -175,6 +192,7 @@ __device__ void build_pair_terms(const ACtx<T>& c) {
   }
   __syncthreads();
   constexpr int kVec = 16 / sizeof(T);
+  const double inv_d = 1.0 / c.dd;
   for (int i = threadIdx.x; i < c.tri; i += blockDim.x) {
     // column e of entry i: col_off(e) <= i < col_off(e + 1)
     int e = static_cast<int>((1.0f + sqrtf(1.0f + 8.0f * static_cast<float>(i))) * 0.5f);
@@ -182,8 +200,7 @@ __device__ void build_pair_terms(const ACtx<T>& c) {
     while (col_off(e + 1) <= i) ++e;
     const int aa = i - col_off(e);
     const int o = c.cb[e] * kVec + aa;
-    c.vt[o] = static_cast<T>(__ddiv_rn(c.V[i], c.dd));
-    c.et[o] = static_cast<T>(__dadd_rn(hmass(c.L[i], c.dd), hmass(c.R[i], c.dd)));
+    AOps<T>::terms(c.V[i], c.R[i], c.L[i], c.dd, inv_d, c.vt + o, c.et + o);
   }
 }
 

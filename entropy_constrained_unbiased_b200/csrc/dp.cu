@@ -133,7 +133,7 @@ struct Ctx {
   Tables<T> fw;  // the alphabet as given
   Tables<T> rf;  // the reflected alphabet (Hirschberg mode)
   const int* cb;              // [p+1] padded column starts (shared memory)
-  uint16_t* bp;               // [S][tri] back-pointers (store mode)
+  T* fst;                     // [S][tri] layer values F_i(l, j) (store mode; row triangle)
   double *sP, *sN, *sA, *sB;  // [p] alphabet and bucket statistics
   double *sR, *sL;            // [S] evaluation scratch
   T* rmin;                    // [p] row minima (lambda = 0)
@@ -215,7 +215,7 @@ struct Pass {
   int s0, e0, T;
   bool last_only;
   double extra;
-  bool store_bp;
+  bool store_f;  // keep every layer's values for the backtrack
   bool finalize;
 };
 
@@ -252,11 +252,12 @@ __device__ __forceinline__ void finalize_layer(const Ctx<T>& c, const Tables<T>&
 // interleaved streams (each output and stream keeps its own running minimum,
 // so consecutive updates do not wait on one another). The k range common to
 // the warp runs unpredicated; the rest masks the layer value to +inf past the
-// lane's own column.
+// lane's own column. Only the minimum is kept: the backtrack recomputes the
+// argmin of the few states on the optimal path from the stored layers (fsi).
 template <typename T>
 __device__ __forceinline__ void run_task(const Ctx<T>& c, const Tables<T>& tb, int l, int j0, int nv, bool active,
                                          int kmin, const GA<T>* __restrict__ Gp, GA<T>* __restrict__ Gc,
-                                         uint16_t* __restrict__ bpi, T invl) {
+                                         T* __restrict__ fsi, T invl) {
   const int p = c.p;
   if (!active) {
     l = kmin + 1;  // inactive lanes sweep an in-range column and write nothing
@@ -271,14 +272,10 @@ __device__ __forceinline__ void run_task(const Ctx<T>& c, const Tables<T>& tb, i
   const GA<T>* __restrict__ col = Gp + c.cb[l];
 
   T best[kTJ][kNQ];
-  int arg[kTJ][kNQ];
 #pragma unroll
   for (int u = 0; u < kTJ; ++u)
 #pragma unroll
-    for (int s = 0; s < kNQ; ++s) {
-      best[u][s] = Arith<T>::inf();
-      arg[u][s] = kmin;
-    }
+    for (int s = 0; s < kNQ; ++s) best[u][s] = Arith<T>::inf();
   int k = kmin;
 #pragma unroll 2
   for (; k + kNQ <= lmin; k += kNQ) {
@@ -286,13 +283,7 @@ __device__ __forceinline__ void run_task(const Ctx<T>& c, const Tables<T>& tb, i
     for (int s = 0; s < kNQ; ++s) {
       const GA<T> ga = col[k + s];
 #pragma unroll
-      for (int u = 0; u < kTJ; ++u) {
-        const T v = Arith<T>::fold(ga.g, ga.a + b[u]);
-        // The running minimum is one min op per step; the argmin follows it.
-        const bool lt = v < best[u][s];
-        best[u][s] = Arith<T>::vmin(best[u][s], v);
-        arg[u][s] = lt ? k : arg[u][s];
-      }
+      for (int u = 0; u < kTJ; ++u) best[u][s] = Arith<T>::vmin(best[u][s], Arith<T>::fold(ga.g, ga.a + b[u]));
     }
   }
 #pragma unroll 1
@@ -300,32 +291,18 @@ __device__ __forceinline__ void run_task(const Ctx<T>& c, const Tables<T>& tb, i
     GA<T> ga = col[k];
     ga.g = (k < l) ? ga.g : Arith<T>::inf();
 #pragma unroll
-    for (int u = 0; u < kTJ; ++u) {
-      const T v = Arith<T>::fold(ga.g, ga.a + b[u]);
-      const bool lt = v < best[u][0];
-      best[u][0] = Arith<T>::vmin(best[u][0], v);
-      arg[u][0] = lt ? k : arg[u][0];
-    }
-  }
-  // Stream s holds base indices (it saw k = base + s); the tail updated stream
-  // 0 with true indices. Merge with the tie rule (smaller k wins).
-#pragma unroll
-  for (int u = 0; u < kTJ; ++u) {
-#pragma unroll
-    for (int s = 1; s < kNQ; ++s) {
-      const int ks = arg[u][s] + s;
-      if (best[u][s] < best[u][0] || (best[u][s] == best[u][0] && ks < arg[u][0])) {
-        best[u][0] = best[u][s];
-        arg[u][0] = ks;
-      }
-    }
+    for (int u = 0; u < kTJ; ++u) best[u][0] = Arith<T>::vmin(best[u][0], Arith<T>::fold(ga.g, ga.a + b[u]));
   }
 #pragma unroll
   for (int u = 0; u < kTJ; ++u) {
+    T bu = best[u][0];
+#pragma unroll
+    for (int s = 1; s < kNQ; ++s) bu = Arith<T>::vmin(bu, best[u][s]);
     if (u < nv) {
       const int e = ro + j0 + u;
-      Gc[c.cb[j0 + u] + l].g = tb.rowV[e] * invl + best[u][0];
-      if (bpi) bpi[e] = static_cast<uint16_t>(arg[u][0]);
+      const T f = tb.rowV[e] * invl + bu;
+      Gc[c.cb[j0 + u] + l].g = f;
+      if (fsi) fsi[e] = f;
     }
   }
 }
@@ -355,7 +332,7 @@ __device__ __forceinline__ void run_pass(const Ctx<T>& c, const Tables<T>& tb, c
   for (int t = 2; t <= ps.T; ++t) {
     const GA<T>* Gp = tb.layer(t - 1);
     GA<T>* Gc = tb.layer(t);
-    uint16_t* bpi = ps.store_bp ? c.bp + static_cast<size_t>(t) * tri : nullptr;
+    T* fsi = ps.store_f ? c.fst + static_cast<size_t>(t) * tri : nullptr;
     const bool last = ps.last_only && t == ps.T;
     const int r0 = s0 + t - 1;  // first row of the layer
     if (ps.finalize && warp == 0) finalize_layer(c, tb, t - 1, s0, e0, Gp, sep, bestE, &out->bestI, &out->bestK);
@@ -367,8 +344,9 @@ __device__ __forceinline__ void run_pass(const Ctx<T>& c, const Tables<T>& tb, c
         for (int j = (last ? e0 : l + 1) + lane; j <= e0; j += kWarp) {
           const int e = ro + j;
           const T v = sep ? ga.g : Arith<T>::fold(ga.g, ga.a + tb.rowB[e]);
-          Gc[c.cb[j] + l].g = tb.rowV[e] * invl + v;
-          if (bpi) bpi[e] = static_cast<uint16_t>(s0);
+          const T f = tb.rowV[e] * invl + v;
+          Gc[c.cb[j] + l].g = f;
+          if (fsi) fsi[e] = f;
         }
       }
     } else if (sep) {
@@ -393,11 +371,11 @@ __device__ __forceinline__ void run_pass(const Ctx<T>& c, const Tables<T>& tb, c
       for (int l = r0 + warp; l <= e0 - 1; l += kWarps) {
         const int ro = row_off(l, p) - l - 1;
         const T rm = c.rmin[l];
-        const uint16_t ra = static_cast<uint16_t>(c.rarg[l]);
         for (int j = (last ? e0 : l + 1) + lane; j <= e0; j += kWarp) {
           const int e = ro + j;
-          Gc[c.cb[j] + l].g = tb.rowV[e] + rm;
-          if (bpi) bpi[e] = ra;
+          const T f = tb.rowV[e] + rm;
+          Gc[c.cb[j] + l].g = f;
+          if (fsi) fsi[e] = f;
         }
       }
     } else if (r0 <= e0 - 1) {
@@ -425,7 +403,7 @@ __device__ __forceinline__ void run_pass(const Ctx<T>& c, const Tables<T>& tb, c
             decode_group(q, e0, l, j0, nv);
           }
         }
-        run_task(c, tb, l, j0, nv, act, kmin, Gp, Gc, bpi, invl);
+        run_task(c, tb, l, j0, nv, act, kmin, Gp, Gc, fsi, invl);
       }
     }
     __syncthreads();
@@ -544,36 +522,54 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
   Pass full{0, p - 1, S - 1, true, -1.0, !c.hirschberg, true};
   run_pass(c, c.fw, full, sep, invl, out, bestE);
 
+  if (tid == 0 && out->bestI < 1) {  // no finite candidate (non-finite inputs): fall back to {P_0, P_{p-1}}
+    out->bestI = 1;
+    out->bestK = 0;
+  }
+  __syncthreads();
+  const int bi = out->bestI;
   if (tid == 0) {
-    if (out->bestI < 1) {  // no finite candidate (non-finite inputs): fall back to {P_0, P_{p-1}}
-      out->bestI = 1;
-      out->bestK = 0;
-    }
-    const int bi = out->bestI;
     c.sQ[bi] = p - 1;
     c.sQ[bi - 1] = out->bestK;
     c.sQ[0] = 0;
     out->m = bi + 1;
-    if (!c.hirschberg) {
-      // Backtrack: c_{i+1} = p-1, c_i = k, c_{ii-1} = bp_ii(c_ii, c_{ii+1}), c_1 = 0.
-      int l = out->bestK, j = p - 1;
-      for (int ii = bi; ii >= 2; --ii) {
-        const int kk = (ii == 2) ? 0 : static_cast<int>(c.bp[static_cast<size_t>(ii) * tri + row_off(l, p) + j - l - 1]);
-        c.sQ[ii - 2] = kk;
-        j = l;
-        l = kk;
-      }
-      out->nstk = 0;
-    } else {
+    out->nstk = 0;
+    if (c.hirschberg && bi + 1 - 3 >= 1) {
       // Segments (lo, hi): c[lo] (with c[lo-1] when lo >= 1) and the pair
       // (c[hi], c[hi+1]) are known; c[lo+1 .. hi-1] are not.
-      const int m = bi + 1;
-      out->nstk = 0;
-      if (m - 3 >= 1) {
-        c.stk[0] = 0;
-        c.stk[1] = m - 2;
-        out->nstk = 1;
+      c.stk[0] = 0;
+      c.stk[1] = bi - 1;
+      out->nstk = 1;
+    }
+  }
+  if (!c.hirschberg && warp_id() == 0) {
+    // Backtrack from (c_bi, c_{bi+1}) = (bestK, p-1): at layer ii the value
+    // before c_ii is the smallest k reaching min_k fold(F_{ii-1}(k, c_ii),
+    // R(k, c_ii)/d + L(c_ii, c_{ii+1})/d) (sep: min_k F_{ii-1}(k, c_ii)),
+    // recomputed with the operations of the layer sweep; layer 2 has k = 0.
+    const int lane = lane_id();
+    int l = out->bestK, j = p - 1;
+    for (int ii = bi; ii >= 2; --ii) {
+      int kk = 0;
+      if (ii > 2) {
+        const T bb = c.fw.rowB[row_off(l, p) + j - l - 1];
+        const T* Fp = c.fst + static_cast<size_t>(ii - 1) * tri;
+        T best = Arith<T>::inf();
+        int arg = 0x7fffffff;
+        for (int k = ii - 2 + lane; k < l; k += kWarp) {
+          const T g = Fp[row_off(k, p) + l - k - 1];
+          const T v = sep ? g : Arith<T>::fold(g, c.fw.buf0[c.cb[l] + k].a + bb);
+          if (v < best) {
+            best = v;
+            arg = k;
+          }
+        }
+        warp_argmin(best, arg);
+        kk = (arg == 0x7fffffff) ? ii - 2 : arg;  // all +inf only for non-finite inputs
       }
+      if (lane == 0) c.sQ[ii - 2] = kk;
+      j = l;
+      l = kk;
     }
   }
   __syncthreads();
@@ -671,8 +667,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
   c.cb = cbs;
 
   unsigned char* gs = a.scratch + static_cast<size_t>(blockIdx.x) * a.scratch_per_cta;
-  c.bp = reinterpret_cast<uint16_t*>(gs);
-  if (!c.hirschberg) gs += (sizeof(uint16_t) * static_cast<size_t>(S) * tri + 255) & ~size_t(255);
+  c.fst = reinterpret_cast<T*>(gs);
+  if (!c.hirschberg) gs += (sizeof(T) * static_cast<size_t>(S) * tri + 255) & ~size_t(255);
   const size_t tb = (sizeof(T) * static_cast<size_t>(tri) + 15) & ~size_t(15);
   const size_t gb = (2 * sizeof(T) * static_cast<size_t>(layer_elems(p)) + 15) & ~size_t(15);
   unsigned char* big = kSmemTables ? sp : gs;
@@ -873,7 +869,7 @@ bool dp_plan(int n, int p, int s, bool fp64, bool hirschberg, DpPlan* plan) {
   plan->threads = kThreads;
   plan->smem_tables = !hirschberg && (small + big + 1024 <= static_cast<size_t>(optin));
   plan->smem_bytes = small + (plan->smem_tables ? big : 0);
-  const size_t bp = hirschberg ? 0 : (sizeof(uint16_t) * static_cast<size_t>(S) * tri_size(p) + 255) & ~size_t(255);
+  const size_t bp = hirschberg ? 0 : (tsz * static_cast<size_t>(S) * tri_size(p) + 255) & ~size_t(255);
   const size_t slab = plan->smem_tables ? 0 : (hirschberg ? 2 * big : big);
   plan->scratch_per_cta = (bp + slab + 255) & ~size_t(255);
   void* fn = fp64 ? (plan->smem_tables ? dp_kernel_ptr<double, true>() : dp_kernel_ptr<double, false>())
