@@ -36,10 +36,11 @@ MUFU_LG2_PER_CLK_PER_SM = 16  # special-function unit results per clock per SM (
 B200_SMS = 148
 
 # DRAM bytes (read + write) per k_dp launch per row, from the ncu capture
-# summarised in profiles/k_dp_weights_296rows_full.md (296 rows: 1.95 MB). The
-# figure belongs to the kernel source it was taken on; it is dropped (null)
-# when that source has changed since.
-DP_TRAFFIC = {"weights": {"bytes_per_row": 1.95e6 / 296, "dp_source_sha1": "a8be1452bba47170"}}
+# summarised in profiles/k_dp_weights_296rows_full.md (296 rows: 1.41 MB read,
+# 1383 MB written, almost all of it the stored DP layers written back from L2),
+# scaled by the rows of a launch. The figure belongs to the kernel source it was
+# taken on; it is dropped (null) when that source has changed since.
+DP_TRAFFIC = {"weights": {"bytes_per_row": (1.409024e6 + 1383.014e6) / 296, "dp_source_sha1": "15fc3ef0414774be"}}
 
 
 def triples_per_solve(p: int, s: int) -> int:
