@@ -110,3 +110,55 @@ def test_fullsize_budget_workloads(E, O, name, rows):
     # empirical rate tracks the budget
     assert abs(float(np.mean(Hemp)) - w.b) < 0.05
 
+
+
+# -- approximation on H(I,B) and refinement at full size ---------------------------
+
+@pytest.mark.parametrize("refine", [0, 8])
+@pytest.mark.parametrize("name,rows", [("weights", 12), ("gradients", 3)])
+def test_fullsize_approx_budget(E, O, name, rows, refine):
+    """All rows on the device (fp32 layers, as bench.py times them); sampled rows
+    against the oracle: time-shared MSE to 1e-5, the rate identity, and the
+    GPU's fp64 figures of each code against the oracle's raw evaluation."""
+    w = W.WORKLOADS[name]
+    X, Xd, P, cnt, A, B = _full(E, w)
+    g = E.solve_approx_budget_stats(cnt, A, B, P, w.d, w.s, w.b, refine=refine, steps=w.steps)
+    gn = {k: v.cpu().numpy() for k, v in g.items()}
+    assert np.all(gn["status"] == 0)
+    idx = _sample(w.n, rows)
+    Po, _ = O.grid_batch(X[idx], w.p)
+    ref = O.solve_approx_budget_batch(X[idx], Po, w.s, w.b, w.steps, refine=refine)
+    rate = "H" if refine else "H_IB"
+    for a, r in enumerate(idx):
+        th = gn["theta"][r]
+        if 0 < th < 1:
+            assert th * gn[rate + "1"][r] + (1 - th) * gn[rate + "2"][r] == pytest.approx(w.b, rel=1e-12)
+        d_gpu = th * gn["mse1"][r] + (1 - th) * gn["mse2"][r]
+        d_ref = ref["theta"][a] * ref["mse1"][a] + (1 - ref["theta"][a]) * ref["mse2"][a]
+        assert d_gpu == pytest.approx(d_ref, rel=RTOL32), (r, d_gpu, d_ref)
+        for q, m, k in (("Q1", "Q1_len", "1"), ("Q2", "Q2_len", "2")):
+            code = gn[q][r, : gn[m][r]]
+            mse, H, _ = O.eval_raw(X[r], Po[a][code])
+            assert gn["mse" + k][r] == pytest.approx(mse, rel=RTOL64)
+            assert gn["H" + k][r] == pytest.approx(H, rel=RTOL64)
+            assert gn["H_IB" + k][r] == pytest.approx(O.eval_raw_ib(X[r], Po[a][code]), rel=RTOL64)
+
+
+@pytest.mark.parametrize("name,rows", [("sweep", 6), ("mixture", 2), ("small", 1)])
+def test_fullsize_approx_lambda(E, O, name, rows):
+    w = W.WORKLOADS[name]
+    X, Xd, P, cnt, A, B = _full(E, w)
+    lam = w.lambdas()
+    g = E.solve_approx_stats(cnt, A, B, P, w.d, w.s, torch.from_numpy(lam).cuda())
+    assert int(g["status"].abs().sum()) == 0
+    Q, m = g["Q"].cpu().numpy(), g["Q_len"].cpu().numpy()
+    idx = _sample(w.n, rows)
+    Po, _ = O.grid_batch(X[idx], w.p)
+    ref = O.solve_approx_batch(X[idx], Po, w.s, lam[idx])
+    for a, r in enumerate(idx):
+        for t in range(lam.shape[1]):
+            code = Q[r, t, : m[r, t]]
+            mse, _, _ = O.eval_raw(X[r], Po[a][code])
+            J = mse + lam[r, t] * O.eval_raw_ib(X[r], Po[a][code])
+            assert J <= ref["J"][a, t] * (1 + RTOL32), (r, t, J, ref["J"][a, t])
+            assert g["objective"][r, t].item() == pytest.approx(J, rel=RTOL64)
