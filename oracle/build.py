@@ -6,7 +6,8 @@ import os
 import subprocess
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-SRCS = [os.path.join(HERE, "ecasq_oracle.cpp"), os.path.join(HERE, "ecasq_approx_oracle.cpp")]
+SRCS = [os.path.join(HERE, "ecasq_oracle.cpp"), os.path.join(HERE, "ecasq_approx_oracle.cpp"),
+        os.path.join(HERE, "ecasq_rans_oracle.cpp")]
 LIB = os.path.join(HERE, "liboracle.so")
 
 

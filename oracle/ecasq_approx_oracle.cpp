@@ -44,6 +44,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <cstring>
 #include <limits>
 #include <vector>
 
@@ -397,3 +398,36 @@ int eo_solve_approx_budget_batch(const float* X, int n, int64_t d, const double*
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Hardware-aware permissible set (§5 "Generalidade": any permissible alphabet,
+// e.g. the values BF16 can represent). Reading: P is every finite BF16 value
+// from the largest one <= min X to the smallest one >= max X (so that
+// P_0 <= min X and P_{p-1} >= max X, as unbiasedness needs), ascending, with
+// +0 and -0 counted once. Plain enumeration of all 65536 bit patterns.
+extern "C" int eo_bf16_alphabet(const float* x, int64_t d, double* P, int p_max) {
+  float lo = x[0], hi = x[0];
+  for (int64_t t = 0; t < d; ++t) {
+    if (!std::isfinite(x[t])) return -2;
+    lo = std::min(lo, x[t]);
+    hi = std::max(hi, x[t]);
+  }
+  std::vector<double> all;
+  all.reserve(65536);
+  for (uint32_t b = 0; b < 65536u; ++b) {
+    const uint32_t w = b << 16;
+    float f;
+    std::memcpy(&f, &w, 4);
+    if (std::isfinite(f)) all.push_back(double(f));
+  }
+  std::sort(all.begin(), all.end());
+  all.erase(std::unique(all.begin(), all.end()), all.end());  // -0 == +0
+  // largest value <= lo, smallest value >= hi
+  auto it_lo = std::upper_bound(all.begin(), all.end(), double(lo));
+  auto it_hi = std::lower_bound(all.begin(), all.end(), double(hi));
+  if (it_lo == all.begin() || it_hi == all.end()) return -2;
+  --it_lo;
+  const int count = int(it_hi - it_lo) + 1;
+  for (int i = 0; i < count && i < p_max; ++i) P[i] = *(it_lo + i);
+  return count;
+}

@@ -33,6 +33,7 @@ def lib():
         u8p = np.ctypeslib.ndpointer(np.uint8, flags="C_CONTIGUOUS")
         u32p = np.ctypeslib.ndpointer(np.uint32, flags="C_CONTIGUOUS")
         u64p = np.ctypeslib.ndpointer(np.uint64, flags="C_CONTIGUOUS")
+        u16p = np.ctypeslib.ndpointer(np.uint16, flags="C_CONTIGUOUS")
         I, I64, D, U64 = C.c_int, C.c_int64, C.c_double, C.c_uint64
         sig = {
             "eo_uniform_grid": (I, [f32p, I64, I, f64p]),
@@ -52,6 +53,12 @@ def lib():
                                     I, U64, u8p, i64p, i32p]),
             "eo_grid_batch": (I, [f32p, I, I64, I, f64p, i32p]),
             "eo_hib_tables": (D, [f64p, f64p, f64p, I, I64, i32p, I]),
+            "eo_bf16_alphabet": (I, [f32p, I64, f64p, I]),
+            "eo_rans_segment_words": (C.c_int64, []),
+            "eo_rans_segments": (C.c_int64, [I64]),
+            "eo_rans_model": (None, [i64p, I, u32p, u32p]),
+            "eo_rans_encode_batch": (I, [u8p, I, I64, I, i64p, C.c_void_p, I, U64, u16p, i32p, i32p]),
+            "eo_rans_decode_batch": (I, [u16p, i32p, I, I64, I, i64p, C.c_void_p, I, U64, u8p, i32p]),
             "eo_eval_raw_ib": (I, [f32p, I64, f64p, I, C.POINTER(D)]),
             "eo_approx_dp": (I, [f64p, f64p, f64p, I, I, I64, D, i32p, C.POINTER(C.c_int32), C.POINTER(D)]),
             "eo_refine_local": (D, [f64p, f64p, f64p, I, I64, D, i32p, I, I, I]),
@@ -146,6 +153,16 @@ def dp(V, R, L, s, d, lam):
 
 # -- approximation on H(I,B) and iterative refinement (§2.3, §2.4) ------------
 
+def bf16_alphabet(x, p_max=65536):
+    """Every finite BF16 value from the largest <= min x to the smallest >= max x."""
+    x = _f32(x).ravel()
+    P = np.zeros(p_max)
+    n = int(lib().eo_bf16_alphabet(x, x.size, P, p_max))
+    if n < 0:
+        raise ValueError("non-finite entry or range outside BF16")
+    return P[: min(n, p_max)].copy(), n
+
+
 def hib_tables(V, R, L, d, Q):
     Q = np.ascontiguousarray(Q, np.int32)
     return float(lib().eo_hib_tables(_f64(V), _f64(R), _f64(L), V.shape[0], d, Q, Q.size))
@@ -220,6 +237,49 @@ def solve_approx_budget_batch(X, P, s, b, steps=30, refine=0):
         out["theta"], out["lam_lo"], out["lam_hi"], out["H1"], out["H2"], out["HIB1"], out["HIB2"],
         out["mse1"], out["mse2"], out["status"])
     return out
+
+
+# -- entropy coder (rANS) for the emitted indices (§1 "Contexto") ---------------
+
+def rans_model(cnt):
+    cnt = np.ascontiguousarray(cnt, np.int64)
+    s = cnt.size
+    f = np.zeros(s, np.uint32)
+    cum = np.zeros(s + 1, np.uint32)
+    lib().eo_rans_model(cnt, s, f, cum)
+    return f, cum
+
+
+def rans_encode(idx, hist, seed, theta=None, two_codes=False):
+    """idx [n, d] u8, hist [n, 2, s]. Returns words [n, segments, cap] u16,
+    seg_len [n, segments], status [n]."""
+    idx = np.ascontiguousarray(idx, np.uint8)
+    n, d = idx.shape
+    hist = np.ascontiguousarray(hist, np.int64).reshape(n, 2, -1)
+    s = hist.shape[2]
+    nseg = int(lib().eo_rans_segments(d))
+    cap = int(lib().eo_rans_segment_words())
+    words = np.zeros((n, nseg, cap), np.uint16)
+    seg_len = np.zeros((n, nseg), np.int32)
+    st = np.zeros(n, np.int32)
+    th = None if theta is None else np.ascontiguousarray(theta, np.float64).reshape(n)
+    lib().eo_rans_encode_batch(idx, n, d, s, hist, None if th is None else th.ctypes.data_as(C.c_void_p),
+                               int(bool(two_codes)), C.c_uint64(seed), words, seg_len, st)
+    return words, seg_len, st
+
+
+def rans_decode(words, seg_len, d, hist, seed, theta=None, two_codes=False):
+    words = np.ascontiguousarray(words, np.uint16)
+    seg_len = np.ascontiguousarray(seg_len, np.int32)
+    n = words.shape[0]
+    hist = np.ascontiguousarray(hist, np.int64).reshape(n, 2, -1)
+    s = hist.shape[2]
+    idx = np.zeros((n, d), np.uint8)
+    st = np.zeros(n, np.int32)
+    th = None if theta is None else np.ascontiguousarray(theta, np.float64).reshape(n)
+    lib().eo_rans_decode_batch(words, seg_len, n, d, s, hist, None if th is None else th.ctypes.data_as(C.c_void_p),
+                               int(bool(two_codes)), C.c_uint64(seed), idx, st)
+    return idx, st
 
 
 def philox4x32(ctr, key):
