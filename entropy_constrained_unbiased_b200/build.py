@@ -7,7 +7,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libecasq.so")
 PEAKS_LIB = os.path.join(HERE, "libecasq_peaks.so")
-SOURCES = ["api.cu", "dp.cu", "approx.cu", "grid_bucket.cu", "encode.cu"]
+SOURCES = ["api.cu", "dp.cu", "approx.cu", "grid_bucket.cu", "encode.cu", "rans.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -129,6 +129,14 @@ int ecasq_uniform_grid(const float* X, int n, int64_t d, int p, double* P, int32
                                          static_cast<cudaStream_t>(stream)));
 }
 
+int ecasq_bf16_alphabet(const float* X, int n, int64_t d, int p_max, double* P, int32_t* p_len, int32_t* status,
+                        void* ws, size_t ws_bytes, void* stream) {
+  if (!X || !P || !p_len || !status || !valid_sizes(n, d, 2, 2) || p_max < 2 || p_max > 65536) return ECASQ_ERR_ARG;
+  if (!ws || ws_bytes < ecasq_aux_workspace_size(n, d, 2)) return ECASQ_ERR_WORKSPACE;
+  return cuda_status(launch_bf16_alphabet(X, n, d, p_max, P, p_len, status, static_cast<float*>(ws),
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 int ecasq_bucket(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt, double* A, double* B,
                  int32_t* status, void* ws, size_t ws_bytes, void* stream) {
   if (!X || !P || !cnt || !A || !B || !status || !valid_sizes(n, d, p, 2)) return ECASQ_ERR_ARG;
@@ -415,6 +423,26 @@ int ecasq_encode(const float* X, const double* P, int n, int64_t d, int p, int s
   if (Q2 && !Q2_len) return ECASQ_ERR_ARG;
   return cuda_status(launch_encode(X, P, n, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, seed, idx, hist, status,
                                    static_cast<cudaStream_t>(stream)));
+}
+
+int64_t ecasq_rans_segments(int64_t d) { return d >= 1 ? rans_segments(d) : 0; }
+int64_t ecasq_rans_segment_words(void) { return rans_segment_words(); }
+
+int ecasq_rans_encode(const uint8_t* idx, const int64_t* hist, const double* theta, int two_codes, int n, int64_t d,
+                      int s, uint64_t seed, uint16_t* words, int32_t* seg_len, int32_t* status, void* stream) {
+  if (!idx || !hist || !words || !seg_len || !status || !valid_sizes(n, d, 2, 2) || s < 1 || s > 256)
+    return ECASQ_ERR_ARG;
+  return cuda_status(launch_rans_encode(idx, hist, theta, two_codes, n, d, s, seed, words, seg_len, status,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+int ecasq_rans_decode(const uint16_t* words, const int32_t* seg_len, const int64_t* hist, const double* theta,
+                      int two_codes, int n, int64_t d, int s, uint64_t seed, uint8_t* idx, int32_t* status,
+                      void* stream) {
+  if (!idx || !hist || !words || !seg_len || !status || !valid_sizes(n, d, 2, 2) || s < 1 || s > 256)
+    return ECASQ_ERR_ARG;
+  return cuda_status(launch_rans_decode(words, seg_len, hist, theta, two_codes, n, d, s, seed, idx, status,
+                                        static_cast<cudaStream_t>(stream)));
 }
 
 int ecasq_entropy(const int64_t* hist, int n, int s, double* H, void* stream) {

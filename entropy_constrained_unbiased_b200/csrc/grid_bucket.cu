@@ -118,6 +118,73 @@ __global__ void k_grid_finish(const float* __restrict__ part, int n_chunks, int 
   }
 }
 
+// Hardware-aware permissible set ("Entropy-Constrained Adaptive Stochastic
+// Quantization (ECASQ)", §5 "Generalidade": any permissible alphabet, e.g. the
+// values BF16 can represent): every finite BF16 value from the largest one
+// <= min X to the smallest one >= max X, ascending, +0 and -0 once.
+// A BF16 pattern b is the top half of an fp32. Ordered by value, the finite
+// patterns map to 16-bit keys: b | 0x8000 for a clear sign bit, ~b for a set
+// one (-0 -> 0x7FFF, +0 -> 0x8000), so the set is a key range less -0 when +0
+// is in it.
+__device__ __forceinline__ unsigned bf16_key(unsigned b) { return (b & 0x8000u) ? (~b & 0xFFFFu) : (b | 0x8000u); }
+__device__ __forceinline__ unsigned bf16_of_key(unsigned k) { return (k & 0x8000u) ? (k & 0x7FFFu) : (~k & 0xFFFFu); }
+// Largest BF16 pattern with value <= x, and smallest with value >= x.
+__device__ __forceinline__ unsigned bf16_down(float x) {
+  const unsigned u = __float_as_uint(x), b = u >> 16;
+  return ((u & 0xFFFFu) == 0u || !(u & 0x80000000u)) ? b : b + 1u;
+}
+__device__ __forceinline__ unsigned bf16_up(float x) {
+  const unsigned u = __float_as_uint(x), b = u >> 16;
+  return ((u & 0xFFFFu) == 0u || (u & 0x80000000u)) ? b : b + 1u;
+}
+__device__ __forceinline__ bool bf16_finite(unsigned b) { return (b & 0x7F80u) != 0x7F80u; }
+
+__global__ void k_bf16_finish(const float* __restrict__ part, int n_chunks, int p_max, double* __restrict__ P,
+                              int32_t* __restrict__ p_len, int32_t* __restrict__ status) {
+  const int r = blockIdx.x;
+  __shared__ unsigned s_klo, s_khi;
+  __shared__ int s_cnt;
+  if (threadIdx.x == 0) {
+    float lo = INFINITY, hi = -INFINITY;
+    int bad = 0;
+    for (int c = 0; c < n_chunks; ++c) {
+      const float* o = part + (static_cast<int64_t>(r) * n_chunks + c) * 3;
+      lo = fminf(lo, o[0]);
+      hi = fmaxf(hi, o[1]);
+      bad |= __float_as_int(o[2]);
+    }
+    int st = kStatusOk, cnt = 0;
+    unsigned klo = 0, khi = 0;
+    const unsigned blo = bf16_down(lo), bhi = bf16_up(hi);
+    if (bad || !bf16_finite(blo) || !bf16_finite(bhi)) {
+      st = kStatusRange;
+    } else {
+      klo = bf16_key(blo);
+      khi = bf16_key(bhi);
+      cnt = static_cast<int>(khi - klo) + 1 - ((klo <= 0x7FFFu && khi >= 0x8000u) ? 1 : 0);
+      if (cnt > p_max) st = kStatusArg;
+    }
+    s_klo = klo;
+    s_khi = khi;
+    s_cnt = st == kStatusRange ? 0 : cnt;
+    p_len[r] = s_cnt;
+    if (status) status[r] = st;
+  }
+  __syncthreads();
+  const unsigned klo = s_klo, khi = s_khi;
+  const bool skip_neg0 = klo <= 0x7FFFu && khi >= 0x8000u;
+  const int cnt = s_cnt;
+  for (int t = threadIdx.x; t < p_max; t += blockDim.x) {
+    double v = __longlong_as_double(0x7ff8000000000000ll);
+    if (t < cnt) {
+      unsigned k = klo + static_cast<unsigned>(t);
+      if (skip_neg0 && k >= 0x7FFFu) k += 1u;
+      v = static_cast<double>(__uint_as_float(bf16_of_key(k) << 16));
+    }
+    P[static_cast<int64_t>(r) * p_max + t] = v;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Bucketing. Sums are fixed point: an entry of bucket k with u = (x - P_k)/D_k,
 // D_k = P_{k+1} - P_k, adds round(u * 2^36) to the first-moment sum and
@@ -249,6 +316,17 @@ int bucket_fraction_bits(int64_t d) {
 }
 
 int64_t minmax_chunk(int64_t d) { return d < 16384 ? d : 16384; }
+
+cudaError_t launch_bf16_alphabet(const float* X, int n, int64_t d, int p_max, double* P, int32_t* p_len,
+                                 int32_t* status, float* part, cudaStream_t st) {
+  const int64_t chunk = minmax_chunk(d);
+  const int nc = static_cast<int>((d + chunk - 1) / chunk);
+  k_minmax_partial<<<dim3(nc, n), kGridThreads, 0, st>>>(X, d, chunk, nc, part);
+  note_launch();
+  k_bf16_finish<<<n, 256, 0, st>>>(part, nc, p_max, P, p_len, status);
+  note_launch();
+  return cudaGetLastError();
+}
 
 cudaError_t launch_uniform_grid(const float* X, int n, int64_t d, int p, double* P, int32_t* status,
                                 float* part, cudaStream_t st) {

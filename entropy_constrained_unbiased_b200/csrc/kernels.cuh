@@ -22,6 +22,9 @@ cudaError_t launch_bucket(const float* X, const double* P, int n, int64_t d, int
                           double* A, double* B, int32_t* status, unsigned long long* acc,
                           int32_t* flag, cudaStream_t st);
 
+cudaError_t launch_bf16_alphabet(const float* X, int n, int64_t d, int p_max, double* P, int32_t* p_len,
+                                 int32_t* status, float* part, cudaStream_t st);
+
 size_t bucket_noalloc_bytes(int n, int p);
 size_t bucket_noalloc_capacity();
 cudaError_t launch_bucket_noalloc(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt,
@@ -139,6 +142,16 @@ bool approx_plan(int n, int p, int s, bool fp64, ApproxPlan* plan);
 cudaError_t launch_approx(const ApproxPlan& plan, ApproxArgs args, cudaStream_t st);
 // (i, a, c) relaxations of one solve of the layered shortest path (host).
 int64_t approx_pair_layers(int p, int s);
+
+// ---- entropy coder for the indices (rans.cu) ----
+int64_t rans_segments(int64_t d);
+int64_t rans_segment_words();
+cudaError_t launch_rans_encode(const uint8_t* idx, const int64_t* hist, const double* theta, int two_codes, int n,
+                               int64_t d, int s, uint64_t seed, uint16_t* words, int32_t* seg_len, int32_t* status,
+                               cudaStream_t st);
+cudaError_t launch_rans_decode(const uint16_t* words, const int32_t* seg_len, const int64_t* hist, const double* theta,
+                               int two_codes, int n, int64_t d, int s, uint64_t seed, uint8_t* idx, int32_t* status,
+                               cudaStream_t st);
 
 // ---- encoder (encode.cu) ----
 cudaError_t launch_encode(const float* X, const double* P, int n, int64_t d, int p, int s,

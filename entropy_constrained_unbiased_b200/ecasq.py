@@ -17,11 +17,13 @@ LIB_PATH = os.path.join(_HERE, "libecasq.so")
 OK, ERR_ARG, ERR_RANGE, ERR_WORKSPACE, ERR_CUDA, WARN_BUDGET = 0, -1, -2, -3, -4, 1
 
 EXPORTS = [
-    "ecasq_workspace_size", "ecasq_aux_workspace_size", "ecasq_uniform_grid", "ecasq_bucket", "ecasq_bucket_noalloc",
+    "ecasq_workspace_size", "ecasq_aux_workspace_size", "ecasq_uniform_grid", "ecasq_bf16_alphabet", "ecasq_bucket",
+    "ecasq_bucket_noalloc",
     "ecasq_solve", "ecasq_solve_stats", "ecasq_solve_budget", "ecasq_solve_budget_stats",
     "ecasq_approx_workspace_size", "ecasq_solve_approx", "ecasq_solve_approx_stats", "ecasq_solve_approx_budget",
     "ecasq_solve_approx_budget_stats",
-    "ecasq_encode", "ecasq_entropy", "ecasq_status_string", "ecasq_launch_count",
+    "ecasq_encode", "ecasq_entropy", "ecasq_rans_segments", "ecasq_rans_segment_words", "ecasq_rans_encode",
+    "ecasq_rans_decode", "ecasq_status_string", "ecasq_launch_count",
 ]
 
 
@@ -51,6 +53,7 @@ def load(path: str = LIB_PATH):
         "ecasq_workspace_size": (SZ, [I, I64, I, I, I, OP]),
         "ecasq_aux_workspace_size": (SZ, [I, I64, I]),
         "ecasq_uniform_grid": (I, [P, I, I64, I, P, P, P, SZ, P]),
+        "ecasq_bf16_alphabet": (I, [P, I, I64, I, P, P, P, P, SZ, P]),
         "ecasq_bucket": (I, [P, P, I, I64, I, P, P, P, P, P, SZ, P]),
         "ecasq_bucket_noalloc": (I, [P, P, I, I64, I, P, P, P, P, P]),
         "ecasq_solve": (I, [P, P, I, I64, I, I, P, I, P, P, P, P, P, P, OP, P, SZ, P]),
@@ -64,6 +67,10 @@ def load(path: str = LIB_PATH):
         "ecasq_solve_approx_budget_stats": (I, [P, P, P, P, I, I64, I, I, D, I] + [P] * 14 + [OP, P, SZ, P]),
         "ecasq_encode": (I, [P, P, I, I64, I, I, P, P, P, P, P, U64, P, P, P, P]),
         "ecasq_entropy": (I, [P, I, I, P, P]),
+        "ecasq_rans_segments": (I64, [I64]),
+        "ecasq_rans_segment_words": (I64, []),
+        "ecasq_rans_encode": (I, [P, P, P, I, I, I64, I, U64, P, P, P, P]),
+        "ecasq_rans_decode": (I, [P, P, P, P, I, I, I64, I, U64, P, P, P]),
         "ecasq_status_string": (C.c_char_p, [I]),
         "ecasq_launch_count": (C.c_uint64, [I]),
     }
@@ -132,6 +139,21 @@ def uniform_grid(X: torch.Tensor, p: int):
     _check(L.ecasq_uniform_grid(_ptr(X), n, d, p, _ptr(P), _ptr(st), _ptr(ws), ws.numel(), _stream()),
            "ecasq_uniform_grid")
     return P, st
+
+
+def bf16_alphabet(X: torch.Tensor, p_max: int):
+    """Per row, every BF16 value covering [min X, max X]. Returns P [n, p_max]
+    (NaN past each row's count), p_len [n], status [n]."""
+    L = _need_cuda()
+    _dev(X, torch.float32, "X")
+    n, d = X.shape
+    P = torch.empty((n, p_max), dtype=torch.float64, device=X.device)
+    p_len = torch.empty(n, dtype=torch.int32, device=X.device)
+    st = torch.empty(n, dtype=torch.int32, device=X.device)
+    ws = workspace(L.ecasq_aux_workspace_size(n, d, 2), X.device)
+    _check(L.ecasq_bf16_alphabet(_ptr(X), n, d, p_max, _ptr(P), _ptr(p_len), _ptr(st), _ptr(ws), ws.numel(),
+                                 _stream()), "ecasq_bf16_alphabet")
+    return P, p_len, st
 
 
 def bucket(X: torch.Tensor, P: torch.Tensor):
@@ -365,3 +387,38 @@ def entropy(hist: torch.Tensor):
     H = torch.empty(n, dtype=torch.float64, device=hist.device)
     _check(L.ecasq_entropy(_ptr(hist), n, s, _ptr(H), _stream()), "ecasq_entropy")
     return H
+
+
+# -- entropy coder for the indices --------------------------------------------------
+
+def rans_encode(idx: torch.Tensor, hist: torch.Tensor, seed: int, theta=None, two_codes: bool = False):
+    """rANS-code idx [n, d] u8 with per-row models from hist [n, 2, s]. Returns
+    words [n, segments, cap] u16 (stored as int16), seg_len [n, segments], status."""
+    L = _need_cuda()
+    _dev(idx, torch.uint8, "idx")
+    _dev(hist, torch.int64, "hist")
+    n, d = idx.shape
+    s = hist.shape[-1]
+    nseg, cap = int(L.ecasq_rans_segments(d)), int(L.ecasq_rans_segment_words())
+    words = torch.empty((n, nseg, cap), dtype=torch.int16, device=idx.device)
+    seg_len = torch.empty((n, nseg), dtype=torch.int32, device=idx.device)
+    st = torch.empty(n, dtype=torch.int32, device=idx.device)
+    if theta is not None:
+        _dev(theta, torch.float64, "theta")
+    _check(L.ecasq_rans_encode(_ptr(idx), _ptr(hist), _ptr(theta) if theta is not None else None, int(bool(two_codes)),
+                               n, d, s, C.c_uint64(seed), _ptr(words), _ptr(seg_len), _ptr(st), _stream()),
+           "ecasq_rans_encode")
+    return words, seg_len, st
+
+
+def rans_decode(words: torch.Tensor, seg_len: torch.Tensor, hist: torch.Tensor, d: int, seed: int, theta=None,
+                two_codes: bool = False):
+    L = _need_cuda()
+    n = words.shape[0]
+    s = hist.shape[-1]
+    idx = torch.empty((n, d), dtype=torch.uint8, device=words.device)
+    st = torch.empty(n, dtype=torch.int32, device=words.device)
+    _check(L.ecasq_rans_decode(_ptr(words), _ptr(seg_len), _ptr(hist), _ptr(theta) if theta is not None else None,
+                               int(bool(two_codes)), n, d, s, C.c_uint64(seed), _ptr(idx), _ptr(st), _stream()),
+           "ecasq_rans_decode")
+    return idx, st

@@ -82,6 +82,19 @@ size_t ecasq_aux_workspace_size(int n, int64_t d, int p);
 int ecasq_uniform_grid(const float* X, int n, int64_t d, int p, double* P, int32_t* status,
                        void* ws, size_t ws_bytes, void* stream);
 
+/* Hardware-aware permissible set (§5 "Generalidade": any alphabet, e.g. the
+ * values BF16 can represent): per row, every finite BF16 value from the largest
+ * one <= min X to the smallest one >= max X, ascending, with +0 and -0 counted
+ * once; P_0 <= min X and P_{p-1} >= max X as the solver requires.
+ * P [n][p_max] float64 (entries past the row's count are NaN), p_len [n] = the
+ * row's count even when it exceeds p_max. status[r] = ECASQ_ERR_RANGE for a
+ * NaN/Inf entry or a range beyond the finite BF16 values, ECASQ_ERR_ARG when
+ * the count exceeds p_max (P then holds the first p_max values).
+ * 2 <= p_max <= 65536. Rows with different counts need separate solver calls
+ * (the solver takes one p per call). Workspace: ecasq_aux_workspace_size(n, d, 2). */
+int ecasq_bf16_alphabet(const float* X, int n, int64_t d, int p_max, double* P, int32_t* p_len,
+                        int32_t* status, void* ws, size_t ws_bytes, void* stream);
+
 /* Bucketing of each row onto its alphabet (the "+d" term of §2.2
  * "Generalização"): bucket k = max{k <= p-2 : P_k <= x}, so the last bucket is
  * closed; per bucket the count cnt (int64 [n][p-1]) and the shifted moments
@@ -233,6 +246,36 @@ int ecasq_encode(const float* X, const double* P, int n, int64_t d, int p, int s
  * per part H_part = -sum c/d_part log2(c/d_part), combined as
  * (d_0 H_0 + d_1 H_1)/(d_0 + d_1). H [n] float64. */
 int ecasq_entropy(const int64_t* hist, int n, int s, double* H, void* stream);
+
+/* Lossless entropy coding of the emitted indices (§1 "Contexto": the
+ * quantizer's output goes through an entropy coder that gives frequent values
+ * shorter bit strings; H(X^) is what it approaches). Static-model rANS (Duda,
+ * arXiv:1311.2540), one model per row and part from hist [n][2][s] (the
+ * histogram ecasq_encode wrote): probabilities quantised to M = 2^15, f_i =
+ * max(1, floor(c_i M / n_part)) for the symbols that occur, the shortfall to M
+ * added to the most frequent symbol (lowest index on ties), an excess taken from
+ * the largest frequencies first (none below 1). The part of each entry is not
+ * coded: it is recomputed from seed and theta exactly as ecasq_encode drew it
+ * (two_codes = 0: every entry in part 0, as with Q2 == NULL; otherwise the
+ * theta rule of ecasq_encode, theta NULL meaning part 1).
+ * 32-bit states in [2^16, 2^32), 16-bit words; a row is cut into segments of
+ * 16384 entries (ecasq_rans_segments(d) of them), each coded by 32 interleaved
+ * states: the 32 entries of a step go one per state, the renormalisation words
+ * of a step are stacked in state order, the final states follow as (low, high)
+ * pairs. words [n][segments][ecasq_rans_segment_words()] uint16; seg_len
+ * [n][segments] int32 = words used (the coded size of a row is 16 * sum bits).
+ * status[r] = ECASQ_ERR_ARG when an index has no frequency in its part's model
+ * (encode) or the stream is malformed (decode). Asynchronous; device memory. */
+int64_t ecasq_rans_segments(int64_t d);
+int64_t ecasq_rans_segment_words(void);
+int ecasq_rans_encode(const uint8_t* idx, const int64_t* hist, const double* theta, int two_codes, int n,
+                      int64_t d, int s, uint64_t seed, uint16_t* words, int32_t* seg_len, int32_t* status,
+                      void* stream);
+/* Inverse of ecasq_rans_encode: idx [n][d] uint8 from the words, the same hist,
+ * theta, two_codes and seed. */
+int ecasq_rans_decode(const uint16_t* words, const int32_t* seg_len, const int64_t* hist, const double* theta,
+                      int two_codes, int n, int64_t d, int s, uint64_t seed, uint8_t* idx, int32_t* status,
+                      void* stream);
 
 /* Static text for a status code. */
 const char* ecasq_status_string(int code);

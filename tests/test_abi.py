@@ -19,7 +19,7 @@ def lib():
 
 def declared_symbols():
     text = open(os.path.join(ROOT, "include", "ecasq.h")).read()
-    return sorted(set(re.findall(r"\b(ecasq_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(ecasq_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_lists_the_binding_exports():
