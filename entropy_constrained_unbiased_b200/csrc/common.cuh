@@ -80,6 +80,21 @@ __host__ __device__ __forceinline__ int col_off(int l) { return (l * (l - 1)) >>
 __host__ __device__ __forceinline__ int row_off(int l, int p) { return l * (p - 1) - ((l * (l - 1)) >> 1); }
 __host__ __device__ __forceinline__ int tri_size(int p) { return (p * (p - 1)) >> 1; }
 
+// Bucket of x with exact fp32 thresholds: T[k] is the smallest float >= P_k and
+// top the largest float <= P_{p-1}, so for a float x, P_k <= x <=> T[k] <= x
+// and x <= P_{p-1} <=> x <= top; the result is the largest k <= p-2 with
+// P_k <= x, or -1 outside [P_0, P_{p-1}]. The fp32 guess is corrected by the
+// exact comparisons.
+__device__ __forceinline__ int bucket_f32(float x, const float* __restrict__ T, float top, int p, float scale) {
+  if (!(x >= T[0]) || !(x <= top)) return -1;
+  int k = static_cast<int>((x - T[0]) * scale);
+  k = k < 0 ? 0 : (k > p - 2 ? p - 2 : k);
+  while (k > 0 && x < T[k]) --k;
+  while (k < p - 2 && x >= T[k + 1]) ++k;
+  return k;
+}
+
+
 // Bucket of x on an increasing alphabet P (in shared memory): the largest
 // k <= p-2 with P_k <= x. Starts from the uniform-grid guess and walks; -1 when
 // x is outside [P_0, P_{p-1}] or NaN.

@@ -40,7 +40,8 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
   double* sq = sP + p;                             // [2][s] code values
   double* sw = sq + 2 * s;                         // [2][s] interval widths q_{t+1} - q_t
   unsigned int* sh = reinterpret_cast<unsigned int*>(sw + 2 * s);      // [warps][2s] counts
-  unsigned char* imap = reinterpret_cast<unsigned char*>(sh + kEncWarps * 2 * s);  // [2][p]
+  float* sT = reinterpret_cast<float*>(sh + kEncWarps * 2 * s);                     // [p] exact fp32 thresholds
+  unsigned char* imap = reinterpret_cast<unsigned char*>(sT + p);                      // [2][p]
   __shared__ int s_m[2];
   __shared__ int s_bad;
 
@@ -51,7 +52,10 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
   const int fixed_part = (!has2 || th >= 1.0) ? 0 : 1;
   const int nbins = 2 * s;
 
-  for (int k = threadIdx.x; k < p; k += blockDim.x) sP[k] = P[k];
+  for (int k = threadIdx.x; k < p; k += blockDim.x) {
+    sP[k] = P[k];
+    sT[k] = __double2float_ru(P[k]);
+  }
   if (threadIdx.x == 0) {
     s_bad = 0;
     s_m[0] = Q1_len[r];
@@ -98,7 +102,8 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
   }
   __syncthreads();
 
-  const double scale = static_cast<double>(p - 1) / (sP[p - 1] - sP[0]);
+  const float scale = static_cast<float>(static_cast<double>(p - 1) / (sP[p - 1] - sP[0]));
+  const float top = __double2float_rd(sP[p - 1]);
   const int64_t beg = static_cast<int64_t>(blockIdx.x) * kEncChunk;
   const int64_t end = beg + kEncChunk < d ? beg + kEncChunk : d;
   const float* x = X + static_cast<int64_t>(r) * d;
@@ -138,7 +143,7 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
       if (m == 1) {
         if (xd != sq[part * s]) bad = 1;
       } else {
-        const int k = bucket_of(xd, sP, p, scale);
+        const int k = bucket_f32(xv[e], sT, top, p, scale);
         int t = (k >= 0) ? imap[part * p + k] : 255;
         if (t == 255) {
           if (xd == sq[part * s + m - 1])
@@ -197,7 +202,7 @@ __global__ void k_entropy(const int64_t* __restrict__ hist, int n, int s, double
 }
 
 size_t encode_smem(int p, int s) {
-  return sizeof(double) * (p + 4 * s) + sizeof(unsigned int) * kEncWarps * 2 * s + 2 * p;
+  return sizeof(double) * (p + 4 * s) + sizeof(unsigned int) * kEncWarps * 2 * s + sizeof(float) * p + 2 * p;
 }
 
 }  // namespace

@@ -216,6 +216,7 @@ k_bucket(const float* __restrict__ X, int64_t d, int64_t chunk, const double* __
   unsigned int* hc = reinterpret_cast<unsigned int*>(sS + p);     // [p] count
   unsigned int* ha = hc + p;                                       // [2][p] first-moment limbs (lo, hi)
   unsigned int* hb = ha + 2 * p;                                   // [2][p] second-moment limbs
+  float* sT = reinterpret_cast<float*>(hb + 2 * p);                // [p] exact fp32 thresholds
   __shared__ int s_bad;
 
   const double* P = Pall + static_cast<int64_t>(r) * p;
@@ -223,12 +224,14 @@ k_bucket(const float* __restrict__ X, int64_t d, int64_t chunk, const double* __
   for (int k = threadIdx.x; k < p; k += blockDim.x) {
     sP[k] = P[k];
     sS[k] = (k < nb) ? two_f / (P[k + 1] - P[k]) : 0.0;
+    sT[k] = __double2float_ru(P[k]);
   }
   for (int k = threadIdx.x; k < 5 * p; k += blockDim.x) hc[k] = 0u;
   if (threadIdx.x == 0) s_bad = 0;
   __syncthreads();
 
-  const double scale = static_cast<double>(p - 1) / (sP[p - 1] - sP[0]);
+  const float scale = static_cast<float>(static_cast<double>(p - 1) / (sP[p - 1] - sP[0]));
+  const float top = __double2float_rd(sP[p - 1]);
   const double inv_two_f = 0x1p-36;
   const double magic = 0x1p52;  // v + 2^52 keeps round(v) in the low mantissa bits for 0 <= v < 2^52
   const unsigned int lmask = (1u << kLimbBits) - 1u;
@@ -236,7 +239,7 @@ k_bucket(const float* __restrict__ X, int64_t d, int64_t chunk, const double* __
 
   auto one = [&](float xf) {
     const double x = static_cast<double>(xf);
-    const int k = bucket_of(x, sP, p, scale);
+    const int k = bucket_f32(xf, sT, top, p, scale);
     if (k < 0) {
       bad = 1;
       return;
@@ -339,7 +342,7 @@ cudaError_t launch_uniform_grid(const float* X, int n, int64_t d, int p, double*
   return cudaGetLastError();
 }
 
-size_t bucket_smem_bytes(int p) { return static_cast<size_t>(p) * (8 * 2 + 4 * 5); }
+size_t bucket_smem_bytes(int p) { return static_cast<size_t>(p) * (8 * 2 + 4 * 5 + 4); }
 
 int64_t bucket_chunk(int64_t d) { return d < kBucketChunk ? d : kBucketChunk; }
 
