@@ -418,7 +418,9 @@ int ecasq_solve_approx_budget_stats(const int64_t* cnt, const double* A, const d
 int ecasq_encode(const float* X, const double* P, int n, int64_t d, int p, int s, const int32_t* Q1,
                  const int32_t* Q1_len, const int32_t* Q2, const int32_t* Q2_len, const double* theta, uint64_t seed,
                  uint8_t* idx, int64_t* hist, int32_t* status, void* stream) {
-  if (!X || !P || !Q1 || !Q1_len || !idx || !hist || !status || !valid_sizes(n, d, p, s) || s > 256)
+  // s is the row stride of the codes and the histogram (a code of up to 256
+  // values: indices fit in uint8), not bound by the solvers' code size.
+  if (!X || !P || !Q1 || !Q1_len || !idx || !hist || !status || !valid_sizes(n, d, p, 2) || s < 1 || s > 256)
     return ECASQ_ERR_ARG;
   if (Q2 && !Q2_len) return ECASQ_ERR_ARG;
   return cuda_status(launch_encode(X, P, n, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, seed, idx, hist, status,
