@@ -254,7 +254,7 @@ __device__ __forceinline__ void finalize_layer(const Ctx<T>& c, const Tables<T>&
 // the warp runs unpredicated; the rest masks the layer value to +inf past the
 // lane's own column. Only the minimum is kept: the backtrack recomputes the
 // argmin of the few states on the optimal path from the stored layers (fsi).
-template <typename T>
+template <typename T, int kUnroll>
 __device__ __forceinline__ void run_task(const Ctx<T>& c, const Tables<T>& tb, int l, int j0, int nv, bool active,
                                          int kmin, const GA<T>* __restrict__ Gp, GA<T>* __restrict__ Gc,
                                          T* __restrict__ fsi, T invl) {
@@ -277,7 +277,7 @@ __device__ __forceinline__ void run_task(const Ctx<T>& c, const Tables<T>& tb, i
 #pragma unroll
     for (int s = 0; s < kNQ; ++s) best[u][s] = Arith<T>::inf();
   int k = kmin;
-#pragma unroll 2
+#pragma unroll kUnroll
   for (; k + kNQ <= lmin; k += kNQ) {
 #pragma unroll
     for (int s = 0; s < kNQ; ++s) {
@@ -308,7 +308,7 @@ __device__ __forceinline__ void run_task(const Ctx<T>& c, const Tables<T>& tb, i
 }
 
 // Runs the pass; all threads. Leaves layer T in tb.layer(T).
-template <typename T>
+template <typename T, int kUnroll>
 __device__ __forceinline__ void run_pass(const Ctx<T>& c, const Tables<T>& tb, const Pass& ps, bool sep, T invl,
                                          SolveOut* out, T* bestE) {
   const int p = c.p, tri = c.tri;
@@ -403,7 +403,7 @@ __device__ __forceinline__ void run_pass(const Ctx<T>& c, const Tables<T>& tb, c
             decode_group(q, e0, l, j0, nv);
           }
         }
-        run_task(c, tb, l, j0, nv, act, kmin, Gp, Gc, fsi, invl);
+        run_task<T, kUnroll>(c, tb, l, j0, nv, act, kmin, Gp, Gc, fsi, invl);
       }
     }
     __syncthreads();
@@ -501,7 +501,7 @@ __device__ __forceinline__ void evaluate(const Ctx<T>& c, double lam, SolveOut* 
 
 // One full solve at lambda (all threads). Leaves the code in c.sQ and the fp64
 // evaluation in *out (shared).
-template <typename T>
+template <typename T, int kUnroll>
 __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out, T* bestE, T* wbest, int* warg) {
   const int p = c.p, S = c.S, tri = c.tri;
   // Below kMinLambda the entropy terms vanish under the precision of T and
@@ -520,7 +520,7 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
   __syncthreads();
   // The whole alphabet, from c_1 = P_0; the last layer needs only j = p-1.
   Pass full{0, p - 1, S - 1, true, -1.0, !c.hirschberg, true};
-  run_pass(c, c.fw, full, sep, invl, out, bestE);
+  run_pass<T, kUnroll>(c, c.fw, full, sep, invl, out, bestE);
 
   if (tid == 0 && out->bestI < 1) {  // no finite candidate (non-finite inputs): fall back to {P_0, P_{p-1}}
     out->bestI = 1;
@@ -586,12 +586,12 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
     double extra_f = -1.0;
     if (lo >= 1) extra_f = static_cast<double>(c.fw.buf0[c.cb[qlo] + c.sQ[lo - 1]].a);  // R(c[lo-1], c[lo])/d
     Pass fwp{qlo, qhi, mid - lo + 1, mid + 1 == hi, extra_f, false, false};
-    run_pass(c, c.fw, fwp, sep, invl, out, bestE);
+    run_pass<T, kUnroll>(c, c.fw, fwp, sep, invl, out, bestE);
     // Reflected: values c[hi] .. c[mid+1] (reflected), next c[mid]; the mass of
     // c[hi] takes L(c[hi], c[hi+1]) from its right neighbour.
     const double extra_b = static_cast<double>(c.fw.rowB[row_off(qhi, p) + qnext - qhi - 1]);
     Pass bwp{p - 1 - qhi, p - 1 - qlo, hi - mid, false, extra_b, false, false};
-    run_pass(c, c.rf, bwp, sep, invl, out, bestE);
+    run_pass<T, kUnroll>(c, c.rf, bwp, sep, invl, out, bestE);
     const int xlo = qlo + (mid - lo), xhi = qhi - (hi - mid);
     const int yhi = qhi - (hi - mid - 1);
     join(c, c.fw.layer(fwp.T), c.rf.layer(bwp.T), xlo, xhi, yhi, mid + 1 == hi, invl, out, wbest, warg);
@@ -627,6 +627,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
   __shared__ T s_wbest[kWarps];
   __shared__ int s_warg[kWarps];
 
+  // k-loop unroll of the layer tasks: the tables in the global slab (L2) want
+  // more loads in flight; the shared-memory variant has no registers to spare.
+  constexpr int kUnrollK = kSmemTables ? 4 : 8;
   const int p = a.p, S = a.s;
   const int tri = tri_size(p);
   Ctx<T> c;
@@ -745,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
       for (int t = 0; t < a.n_lambda; ++t) {
         const int64_t w = static_cast<int64_t>(r) * a.n_lambda + t;
         const double lam = a.lambda[w];
-        solve(c, lam, &s_out, &s_bestE, s_wbest, s_warg);
+        solve<T, kUnrollK>(c, lam, &s_out, &s_bestE, s_wbest, s_warg);
         for (int q = threadIdx.x; q < s_out_stride; q += blockDim.x)
           a.Q[w * s_out_stride + q] = (q < s_out.m) ? c.sQ[q] : -1;
         if (threadIdx.x == 0) {
@@ -771,14 +774,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
       };
       int32_t status = kStatusOk;
       double theta = 0.0;
-      solve(c, 0.0, &s_out, &s_bestE, s_wbest, s_warg);
+      solve<T, kUnrollK>(c, 0.0, &s_out, &s_bestE, s_wbest, s_warg);
       keep(sQ1, m1, H1, M1);
       if (s_out.H <= a.budget) {
         keep(sQ2, m2, H2, M2);
         hi = 0.0;
       } else {
         __syncthreads();
-        solve(c, hi, &s_out, &s_bestE, s_wbest, s_warg);
+        solve<T, kUnrollK>(c, hi, &s_out, &s_bestE, s_wbest, s_warg);
         keep(sQ2, m2, H2, M2);
         if (s_out.H > a.budget) {
           status = kStatusBudget;
@@ -786,7 +789,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
           for (int it = 0; it < a.steps; ++it) {
             const double mid = 0.5 * (lo + hi);
             __syncthreads();
-            solve(c, mid, &s_out, &s_bestE, s_wbest, s_warg);
+            solve<T, kUnrollK>(c, mid, &s_out, &s_bestE, s_wbest, s_warg);
             if (s_out.H > a.budget) {
               lo = mid;
               keep(sQ1, m1, H1, M1);
