@@ -357,10 +357,14 @@ cudaError_t launch_bucket(const float* X, const double* P, int n, int64_t d, int
   const int64_t chunk = bucket_chunk(d);
   const int nc = static_cast<int>((d + chunk - 1) / chunk);
   const size_t smem = bucket_smem_bytes(p);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaFuncSetAttribute(k_bucket, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
-    attr_set = true;
+  // the attribute is per device: set it once for each device this process uses
+  static bool attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    cudaError_t ea = cudaFuncSetAttribute(k_bucket, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+    if (ea != cudaSuccess) return ea;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   k_bucket<<<dim3(nc, n), kBucketThreads, smem, st>>>(X, d, chunk, P, p, fb, acc, flag);
   note_launch();
