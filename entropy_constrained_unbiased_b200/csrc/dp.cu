@@ -34,6 +34,7 @@
 //     (P'_k = -P_{p-1-k}) for the right part;
 //   * the fp64 evaluation of the chosen code and the bisection run in the same
 //     kernel.
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -71,6 +72,17 @@ struct Arith<double> {
   __device__ static double fold(double g, double m) { return m > 0.0 ? fma(-m, log2(m), g) : g; }
   __device__ static double vmin(double a, double b) { return fmin(a, b); }
 };
+
+// Barrier of the CTAs that share a vector: the block itself, or the whole
+// thread-block cluster (release/acquire at cluster scope, so the layer values
+// the other CTAs wrote to the global slab are visible after it).
+template <int kCL>
+__device__ __forceinline__ void csync() {
+  if constexpr (kCL > 1)
+    cooperative_groups::this_cluster().sync();
+  else
+    __syncthreads();
+}
 
 // One entry of a live DP layer: the layer value G = F(k, l) and a = R(k, l)/d
 // (+ eps) side by side, so one 8- (16-) byte shared load feeds a whole k step.
@@ -138,7 +150,7 @@ struct Ctx {
   double *sR, *sL;            // [S] evaluation scratch
   T* rmin;                    // [p] row minima (lambda = 0)
   int* rarg;                  // [p]
-  int* ctr;                   // [S] task counters
+  int* ctr;                   // [S] task counters (rank 0's, in a cluster)
   int* sQ;                    // [S] code of the last solve
   int* stk;                   // [2S] Hirschberg segment stack
   bool hirschberg;
@@ -308,14 +320,22 @@ __device__ __forceinline__ void run_task(const Ctx<T>& c, const Tables<T>& tb, i
 }
 
 // Runs the pass; all threads. Leaves layer T in tb.layer(T).
-template <typename T, int kUnroll>
+// With a cluster, the CTAs split each layer's tasks (one counter, in rank 0)
+// and compute everything else redundantly from the same data.
+template <typename T, int kUnroll, int kCL>
 __device__ __forceinline__ void run_pass(const Ctx<T>& c, const Tables<T>& tb, const Pass& ps, bool sep, T invl,
                                          SolveOut* out, T* bestE) {
   const int p = c.p, tri = c.tri;
   const int s0 = ps.s0, e0 = ps.e0;
   const int tid = threadIdx.x;
   const int warp = warp_id(), lane = lane_id();
-  for (int t = tid; t < c.S; t += blockDim.x) c.ctr[t] = 0;
+  if constexpr (kCL > 1) {
+    csync<kCL>();  // the other CTAs have finished reading what this pass rewrites
+    if (cooperative_groups::this_cluster().block_rank() == 0)
+      for (int t = tid; t < c.S; t += blockDim.x) c.ctr[t] = 0;
+  } else {
+    for (int t = tid; t < c.S; t += blockDim.x) c.ctr[t] = 0;
+  }
   {  // layer 1: row s0
     GA<T>* G1 = tb.layer(1);
     const T extra = ps.extra > 0.0 ? static_cast<T>(ps.extra) : T(0);
@@ -328,7 +348,7 @@ __device__ __forceinline__ void run_pass(const Ctx<T>& c, const Tables<T>& tb, c
       G1[c.cb[j] + s0].g = f;
     }
   }
-  __syncthreads();
+  csync<kCL>();
   for (int t = 2; t <= ps.T; ++t) {
     const GA<T>* Gp = tb.layer(t - 1);
     GA<T>* Gc = tb.layer(t);
@@ -406,7 +426,7 @@ __device__ __forceinline__ void run_pass(const Ctx<T>& c, const Tables<T>& tb, c
         run_task<T, kUnroll>(c, tb, l, j0, nv, act, kmin, Gp, Gc, fsi, invl);
       }
     }
-    __syncthreads();
+    csync<kCL>();
   }
   if (ps.finalize && warp == 0)
     finalize_layer(c, tb, ps.T, s0, e0, tb.layer(ps.T), sep, bestE, &out->bestI, &out->bestK);
@@ -501,7 +521,7 @@ __device__ __forceinline__ void evaluate(const Ctx<T>& c, double lam, SolveOut* 
 
 // One full solve at lambda (all threads). Leaves the code in c.sQ and the fp64
 // evaluation in *out (shared).
-template <typename T, int kUnroll>
+template <typename T, int kUnroll, int kCL>
 __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out, T* bestE, T* wbest, int* warg) {
   const int p = c.p, S = c.S, tri = c.tri;
   // Below kMinLambda the entropy terms vanish under the precision of T and
@@ -520,7 +540,7 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
   __syncthreads();
   // The whole alphabet, from c_1 = P_0; the last layer needs only j = p-1.
   Pass full{0, p - 1, S - 1, true, -1.0, !c.hirschberg, true};
-  run_pass<T, kUnroll>(c, c.fw, full, sep, invl, out, bestE);
+  run_pass<T, kUnroll, kCL>(c, c.fw, full, sep, invl, out, bestE);
 
   if (tid == 0 && out->bestI < 1) {  // no finite candidate (non-finite inputs): fall back to {P_0, P_{p-1}}
     out->bestI = 1;
@@ -586,12 +606,12 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
     double extra_f = -1.0;
     if (lo >= 1) extra_f = static_cast<double>(c.fw.buf0[c.cb[qlo] + c.sQ[lo - 1]].a);  // R(c[lo-1], c[lo])/d
     Pass fwp{qlo, qhi, mid - lo + 1, mid + 1 == hi, extra_f, false, false};
-    run_pass<T, kUnroll>(c, c.fw, fwp, sep, invl, out, bestE);
+    run_pass<T, kUnroll, kCL>(c, c.fw, fwp, sep, invl, out, bestE);
     // Reflected: values c[hi] .. c[mid+1] (reflected), next c[mid]; the mass of
     // c[hi] takes L(c[hi], c[hi+1]) from its right neighbour.
     const double extra_b = static_cast<double>(c.fw.rowB[row_off(qhi, p) + qnext - qhi - 1]);
     Pass bwp{p - 1 - qhi, p - 1 - qlo, hi - mid, false, extra_b, false, false};
-    run_pass<T, kUnroll>(c, c.rf, bwp, sep, invl, out, bestE);
+    run_pass<T, kUnroll, kCL>(c, c.rf, bwp, sep, invl, out, bestE);
     const int xlo = qlo + (mid - lo), xhi = qhi - (hi - mid);
     const int yhi = qhi - (hi - mid - 1);
     join(c, c.fw.layer(fwp.T), c.rf.layer(bwp.T), xlo, xhi, yhi, mid + 1 == hi, invl, out, wbest, warg);
@@ -618,7 +638,7 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
   __syncthreads();
 }
 
-template <typename T, bool kSmemTables>
+template <typename T, bool kSmemTables, int kCL>
 __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ SolveOut s_out;
@@ -668,8 +688,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
     cbs[p] = cc;
   }
   c.cb = cbs;
+  // CTAs of one cluster share a vector, its slab and rank 0's task counters.
+  if constexpr (kCL > 1) c.ctr = cooperative_groups::this_cluster().map_shared_rank(c.ctr, 0);
 
-  unsigned char* gs = a.scratch + static_cast<size_t>(blockIdx.x) * a.scratch_per_cta;
+  unsigned char* gs = a.scratch + static_cast<size_t>(blockIdx.x / kCL) * a.scratch_per_cta;
   c.fst = reinterpret_cast<T*>(gs);
   if (!c.hirschberg) gs += (sizeof(T) * static_cast<size_t>(S) * tri + 255) & ~size_t(255);
   const size_t tb = (sizeof(T) * static_cast<size_t>(tri) + 15) & ~size_t(15);
@@ -687,7 +709,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
   __syncthreads();  // cb visible to all threads
 
   const int s_out_stride = a.s_out;
-  for (int r = blockIdx.x; r < a.n; r += gridDim.x) {
+  for (int r = blockIdx.x / kCL; r < a.n; r += gridDim.x / kCL) {
     const double* P = a.P + static_cast<int64_t>(r) * p;
     const int64_t bo = static_cast<int64_t>(r) * (p - 1);
     if (threadIdx.x == 0) s_flag = a.in_status ? a.in_status[r] : 0;
@@ -737,6 +759,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
       continue;
     }
 
+    if constexpr (kCL > 1) csync<kCL>();  // the other CTAs are done with the previous vector's tables
     build_tables(c);
     __syncthreads();
     if (c.hirschberg) {
@@ -748,7 +771,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
       for (int t = 0; t < a.n_lambda; ++t) {
         const int64_t w = static_cast<int64_t>(r) * a.n_lambda + t;
         const double lam = a.lambda[w];
-        solve<T, kUnrollK>(c, lam, &s_out, &s_bestE, s_wbest, s_warg);
+        solve<T, kUnrollK, kCL>(c, lam, &s_out, &s_bestE, s_wbest, s_warg);
         for (int q = threadIdx.x; q < s_out_stride; q += blockDim.x)
           a.Q[w * s_out_stride + q] = (q < s_out.m) ? c.sQ[q] : -1;
         if (threadIdx.x == 0) {
@@ -774,14 +797,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
       };
       int32_t status = kStatusOk;
       double theta = 0.0;
-      solve<T, kUnrollK>(c, 0.0, &s_out, &s_bestE, s_wbest, s_warg);
+      solve<T, kUnrollK, kCL>(c, 0.0, &s_out, &s_bestE, s_wbest, s_warg);
       keep(sQ1, m1, H1, M1);
       if (s_out.H <= a.budget) {
         keep(sQ2, m2, H2, M2);
         hi = 0.0;
       } else {
         __syncthreads();
-        solve<T, kUnrollK>(c, hi, &s_out, &s_bestE, s_wbest, s_warg);
+        solve<T, kUnrollK, kCL>(c, hi, &s_out, &s_bestE, s_wbest, s_warg);
         keep(sQ2, m2, H2, M2);
         if (s_out.H > a.budget) {
           status = kStatusBudget;
@@ -789,7 +812,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
           for (int it = 0; it < a.steps; ++it) {
             const double mid = 0.5 * (lo + hi);
             __syncthreads();
-            solve<T, kUnrollK>(c, mid, &s_out, &s_bestE, s_wbest, s_warg);
+            solve<T, kUnrollK, kCL>(c, mid, &s_out, &s_bestE, s_wbest, s_warg);
             if (s_out.H > a.budget) {
               lo = mid;
               keep(sQ1, m1, H1, M1);
@@ -822,11 +845,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
     }
     __syncthreads();
   }
+  // rank 0's task counters stay alive until no CTA of the cluster can reach them
+  if constexpr (kCL > 1) cooperative_groups::this_cluster().sync();
 }
 
-template <typename T, bool kSmem>
+template <typename T, bool kSmem, int kCL>
 void* dp_kernel_ptr() {
-  return reinterpret_cast<void*>(&k_dp<T, kSmem>);
+  return reinterpret_cast<void*>(&k_dp<T, kSmem, kCL>);
+}
+
+// Tables in shared memory run one CTA per vector; tables in the global slab can
+// run a cluster of two CTAs per vector when there are few vectors.
+void* dp_fn(bool fp64, bool smem, int cluster) {
+  if (smem) return fp64 ? dp_kernel_ptr<double, true, 1>() : dp_kernel_ptr<float, true, 1>();
+  if (cluster == 2) return fp64 ? dp_kernel_ptr<double, false, 2>() : dp_kernel_ptr<float, false, 2>();
+  return fp64 ? dp_kernel_ptr<double, false, 1>() : dp_kernel_ptr<float, false, 1>();
 }
 
 size_t small_smem(int p, int S, size_t tsz) {
@@ -875,8 +908,10 @@ bool dp_plan(int n, int p, int s, bool fp64, bool hirschberg, DpPlan* plan) {
   const size_t bp = hirschberg ? 0 : (tsz * static_cast<size_t>(S) * tri_size(p) + 255) & ~size_t(255);
   const size_t slab = plan->smem_tables ? 0 : (hirschberg ? 2 * big : big);
   plan->scratch_per_cta = (bp + slab + 255) & ~size_t(255);
-  void* fn = fp64 ? (plan->smem_tables ? dp_kernel_ptr<double, true>() : dp_kernel_ptr<double, false>())
-                  : (plan->smem_tables ? dp_kernel_ptr<float, true>() : dp_kernel_ptr<float, false>());
+  // Two CTAs per vector when the tables are in the global slab and the
+  // vectors alone would leave more than half of the SMs idle.
+  plan->cluster = (!plan->smem_tables && 2 * n <= sms) ? 2 : 1;
+  void* fn = dp_fn(fp64, plan->smem_tables, plan->cluster);
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(plan->smem_bytes)) !=
       cudaSuccess)
     return false;
@@ -884,17 +919,33 @@ bool dp_plan(int n, int p, int s, bool fp64, bool hirschberg, DpPlan* plan) {
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, plan->smem_bytes) != cudaSuccess ||
       per_sm < 1)
     return false;
-  const int ctas = sms * per_sm;
-  plan->ctas = n < ctas ? n : ctas;
+  const int slots = sms * per_sm / plan->cluster;  // vectors in flight
+  plan->ctas = plan->cluster * (n < slots ? n : slots);
   return true;
 }
 
 cudaError_t launch_dp(const DpPlan& plan, DpArgs args, cudaStream_t st) {
   args.hirschberg = plan.hirschberg ? 1 : 0;
-  void* fn = plan.fp64 ? (plan.smem_tables ? dp_kernel_ptr<double, true>() : dp_kernel_ptr<double, false>())
-                       : (plan.smem_tables ? dp_kernel_ptr<float, true>() : dp_kernel_ptr<float, false>());
+  void* fn = dp_fn(plan.fp64, plan.smem_tables, plan.cluster);
   void* kargs[] = {&args};
-  cudaError_t e = cudaLaunchKernel(fn, dim3(plan.ctas), dim3(plan.threads), kargs, plan.smem_bytes, st);
+  cudaError_t e;
+  if (plan.cluster > 1) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(plan.ctas);
+    cfg.blockDim = dim3(plan.threads);
+    cfg.dynamicSmemBytes = plan.smem_bytes;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = plan.cluster;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelExC(&cfg, fn, kargs);
+  } else {
+    e = cudaLaunchKernel(fn, dim3(plan.ctas), dim3(plan.threads), kargs, plan.smem_bytes, st);
+  }
   note_launch();
   return e;
 }

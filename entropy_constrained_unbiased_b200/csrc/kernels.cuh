@@ -76,6 +76,7 @@ struct DpPlan {
   bool fp64;
   bool hirschberg;
   bool smem_tables;  // pair tables resident in shared memory
+  int cluster;       // CTAs per vector (a thread-block cluster when > 1)
   int threads;
   int ctas;
   size_t smem_bytes;
