@@ -36,11 +36,11 @@ MUFU_LG2_PER_CLK_PER_SM = 16  # special-function unit results per clock per SM (
 B200_SMS = 148
 
 # DRAM bytes (read + write) per k_dp launch per row, from the ncu capture
-# summarised in profiles/k_dp_weights_296rows_full.md (296 rows: 1.41 MB read,
-# 1409 MB written, almost all of it the stored DP layers written back from L2),
+# summarised in profiles/k_dp_weights_296rows_full.md (296 rows: 1.71 MB read,
+# 1411 MB written, almost all of it the stored DP layers written back from L2),
 # scaled by the rows of a launch. The figure belongs to the kernel source it was
 # taken on; it is dropped (null) when that source has changed since.
-DP_TRAFFIC = {"weights": {"bytes_per_row": (1408256 + 1409484544) / 296, "dp_source_sha1": "50ae2e9bad8a815a"}}
+DP_TRAFFIC = {"weights": {"bytes_per_row": (1708544 + 1410748672) / 296, "dp_source_sha1": "a9ffec8785361700"}}
 
 
 def triples_per_solve(p: int, s: int) -> int:
