@@ -25,10 +25,12 @@
 //     (L2-resident); the latter in padded columns (16-byte aligned, starts
 //     staggered over the banks);
 //   * per solve, the cost table w(a,c) (same padded columns) and the layers
-//     G_1..G_s in shared memory (global slab when they do not fit). One thread
-//     per column c sweeps a upwards with 16-byte loads of its column and of
-//     G_{i-1} (a broadcast): four relaxations per pair of loads, two packed
-//     f32x2 additions and two three-input minima in fp32;
+//     G_1..G_s in shared memory (global slab when they do not fit). Each
+//     column's a range is split near its middle; a thread sweeps the lower part
+//     of one column and the upper part of its mirror column (equal work per
+//     thread) with 16-byte loads of the column and of G_{i-1}: four relaxations
+//     per pair of loads, two packed f32x2 additions and two three-input minima
+//     in fp32; the two parts' minima are merged after a barrier;
 //   * the argmin is recovered afterwards by recomputing the sums in the same
 //     precision (the minimum is one of them exactly), smallest a first;
 //   * refinement and the fp64 evaluation read the fp64 tables, which are summed
@@ -306,9 +308,50 @@ __device__ void evaluate_code(const ACtx<T>& c, double lam, bool refined, int m,
   __syncwarp();
 }
 
+// min over a = a0 .. a1-1 of Gp[a] + col[a] (+inf for an empty range): scalar
+// up to a 16-byte boundary, then pairs of 16-byte loads of the column and of
+// the layer (a broadcast within a warp's common range), one more single load,
+// then the scalar tail. Gp and col are 16-byte aligned at a = 0.
+template <typename T>
+__device__ __forceinline__ T sweep_min(const T* __restrict__ Gp, const T* __restrict__ col, int a0, int a1) {
+  using O = AOps<T>;
+  using V16 = typename AOps<T>::Vec;
+  constexpr int kVec = 16 / sizeof(T);
+  T b0 = O::inf(), b1 = O::inf(), b2 = O::inf(), b3 = O::inf();
+  int a = a0;
+  const int ah = min(a1, (a + kVec - 1) / kVec * kVec);
+  for (; a < ah; ++a) b0 = O::vmin(b0, O::add(Gp[a], col[a]));
+  const int av = a + (a1 - a) / (2 * kVec) * (2 * kVec);
+  for (; a < av; a += 2 * kVec) {
+    const V16 g0 = *reinterpret_cast<const V16*>(Gp + a);
+    const V16 g1 = *reinterpret_cast<const V16*>(Gp + a + kVec);
+    const V16 w0 = *reinterpret_cast<const V16*>(col + a);
+    const V16 w1 = *reinterpret_cast<const V16*>(col + a + kVec);
+    O::relax(g0, w0, b0, b1);
+    O::relax(g1, w1, b2, b3);
+  }
+  if (a + kVec <= a1) {
+    O::relax(*reinterpret_cast<const V16*>(Gp + a), *reinterpret_cast<const V16*>(col + a), b2, b3);
+    a += kVec;
+  }
+  for (; a < a1; ++a) b1 = O::vmin(b1, O::add(Gp[a], col[a]));
+  return O::vmin(O::vmin(b0, b1), O::vmin(b2, b3));
+}
+
+// Split point of column x in layer i (a = i-2 .. x-1): the 16-byte boundary at
+// or below the middle, clamped to the column.
+template <typename T>
+__device__ __forceinline__ int column_split(int i, int x) {
+  constexpr int kVec = 16 / sizeof(T);
+  const int mid = ((i - 2 + x) >> 1) / kVec * kVec;
+  return mid < i - 2 ? i - 2 : mid;
+}
+
 // One solve at lambda (all threads): cost table, layers, recovery of the code,
 // refinement, evaluation. Leaves the code in c.sQ and the figures in *out.
-template <typename T>
+// kSplit: each column's a range is shared by two threads (few vectors, one CTA
+// per SM: the longest column is the critical path of a layer).
+template <typename T, bool kSplit>
 __device__ void approx_solve(const ACtx<T>& c, double lam, int refine, AOut* out) {
   using O = AOps<T>;
   const int p = c.p, S = c.S, tid = threadIdx.x, bd = blockDim.x;
@@ -328,31 +371,55 @@ __device__ void approx_solve(const ACtx<T>& c, double lam, int refine, AOut* out
   }
   for (int x = tid; x < p; x += bd) c.G[c.pst + x] = (x == 0) ? T(0) : O::inf();
   __syncthreads();
-  for (int i = 2; i <= S; ++i) {
-    const T* __restrict__ Gp = c.G + (i - 1) * c.pst;
-    T* __restrict__ Gc = c.G + i * c.pst;
-    for (int x = i - 1 + tid; x < p; x += bd) {
-      // min over a = i-2 .. x-1 of G_{i-1}(a) + w(a, x): scalar up to a 16-byte
-      // boundary, then four (fp32) or two (fp64) consecutive a per load of the
-      // column and of the layer (a broadcast), then the scalar tail.
-      const T* __restrict__ col = c.cost + c.cb[x] * kVec;
-      T b0 = O::inf(), b1 = O::inf(), b2 = O::inf(), b3 = O::inf();
-      int a = i - 2;
-      const int ah = min(x, (a + kVec - 1) / kVec * kVec);
-      for (; a < ah; ++a) b0 = O::vmin(b0, O::add(Gp[a], col[a]));
-      const int av = a + (x - a) / (2 * kVec) * (2 * kVec);
-      for (; a < av; a += 2 * kVec) {
-        const V16 g0 = *reinterpret_cast<const V16*>(Gp + a);
-        const V16 g1 = *reinterpret_cast<const V16*>(Gp + a + kVec);
-        const V16 w0 = *reinterpret_cast<const V16*>(col + a);
-        const V16 w1 = *reinterpret_cast<const V16*>(col + a + kVec);
-        AOps<T>::relax(g0, w0, b0, b1);
-        AOps<T>::relax(g1, w1, b2, b3);
+  if constexpr (kSplit) {
+    // Layer i: G_i(x) = min over a = i-2 .. x-1 of G_{i-1}(a) + w(a, x). Column x
+    // is split at a 16-byte boundary near its middle; thread t sweeps the lower
+    // part of column i-1+t and the upper part of column p-1-t, so every thread
+    // does about half of the longest column. The upper parts' minima go to row 0
+    // of G (unused otherwise) and are merged after a barrier. A minimum is exact,
+    // so the split changes no value.
+    T* __restrict__ Gh = c.G;
+    for (int i = 2; i <= S; ++i) {
+      const T* __restrict__ Gp = c.G + (i - 1) * c.pst;
+      T* __restrict__ Gc = c.G + i * c.pst;
+      const int ncol = p - i + 1;
+      for (int t = tid; t < ncol; t += bd) {
+        const int x1 = i - 1 + t, x2 = p - 1 - t;
+        Gc[x1] = sweep_min<T>(Gp, c.cost + c.cb[x1] * kVec, i - 2, column_split<T>(i, x1));
+        Gh[x2] = sweep_min<T>(Gp, c.cost + c.cb[x2] * kVec, column_split<T>(i, x2), x2);
       }
-      for (; a < x; ++a) b1 = O::vmin(b1, O::add(Gp[a], col[a]));
-      Gc[x] = O::vmin(O::vmin(b0, b1), O::vmin(b2, b3));
+      __syncthreads();
+      for (int x = i - 1 + tid; x < p; x += bd) Gc[x] = O::vmin(Gc[x], Gh[x]);
+      __syncthreads();
     }
-    __syncthreads();
+  } else {
+    // One thread per column: the whole a range of column x.
+    for (int i = 2; i <= S; ++i) {
+      const T* __restrict__ Gp = c.G + (i - 1) * c.pst;
+      T* __restrict__ Gc = c.G + i * c.pst;
+      for (int x = i - 1 + tid; x < p; x += bd) {
+        // min over a = i-2 .. x-1 of G_{i-1}(a) + w(a, x): scalar up to a 16-byte
+        // boundary, then four (fp32) or two (fp64) consecutive a per load of the
+        // column and of the layer (a broadcast), then the scalar tail.
+        const T* __restrict__ col = c.cost + c.cb[x] * kVec;
+        T b0 = O::inf(), b1 = O::inf(), b2 = O::inf(), b3 = O::inf();
+        int a = i - 2;
+        const int ah = min(x, (a + kVec - 1) / kVec * kVec);
+        for (; a < ah; ++a) b0 = O::vmin(b0, O::add(Gp[a], col[a]));
+        const int av = a + (x - a) / (2 * kVec) * (2 * kVec);
+        for (; a < av; a += 2 * kVec) {
+          const V16 g0 = *reinterpret_cast<const V16*>(Gp + a);
+          const V16 g1 = *reinterpret_cast<const V16*>(Gp + a + kVec);
+          const V16 w0 = *reinterpret_cast<const V16*>(col + a);
+          const V16 w1 = *reinterpret_cast<const V16*>(col + a + kVec);
+          AOps<T>::relax(g0, w0, b0, b1);
+          AOps<T>::relax(g1, w1, b2, b3);
+        }
+        for (; a < x; ++a) b1 = O::vmin(b1, O::add(Gp[a], col[a]));
+        Gc[x] = O::vmin(O::vmin(b0, b1), O::vmin(b2, b3));
+      }
+      __syncthreads();
+    }
   }
   if (warp_id() == 0) {
     const int lane = lane_id();
@@ -405,7 +472,7 @@ __device__ void approx_solve(const ACtx<T>& c, double lam, int refine, AOut* out
   __syncthreads();
 }
 
-template <typename T, bool kSmem>
+template <typename T, bool kSmem, bool kSplit>
 __global__ void __launch_bounds__(512, 1) k_approx(ApproxArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ AOut s_out;
@@ -517,7 +584,7 @@ __global__ void __launch_bounds__(512, 1) k_approx(ApproxArgs a) {
     if (a.mode == 0) {
       for (int t = 0; t < a.n_lambda; ++t) {
         const int64_t w = static_cast<int64_t>(r) * a.n_lambda + t;
-        approx_solve(c, a.lambda[w], a.refine, &s_out);
+        approx_solve<T, kSplit>(c, a.lambda[w], a.refine, &s_out);
         for (int q = threadIdx.x; q < so; q += blockDim.x) a.Q[w * so + q] = (q < s_out.m) ? c.sQ[q] : -1;
         if (threadIdx.x == 0) {
           a.Q_len[w] = s_out.m;
@@ -547,7 +614,7 @@ __global__ void __launch_bounds__(512, 1) k_approx(ApproxArgs a) {
       auto rate = [&]() { return refined ? s_out.H : s_out.HIB; };
       int32_t status = kStatusOk;
       double theta = 0.0;
-      approx_solve(c, 0.0, a.refine, &s_out);
+      approx_solve<T, kSplit>(c, 0.0, a.refine, &s_out);
       keep(sQ1, m1, H1, B1, M1);
       r1 = rate();
       if (r1 <= a.budget) {
@@ -555,7 +622,7 @@ __global__ void __launch_bounds__(512, 1) k_approx(ApproxArgs a) {
         hi = 0.0;
       } else {
         __syncthreads();
-        approx_solve(c, hi, a.refine, &s_out);
+        approx_solve<T, kSplit>(c, hi, a.refine, &s_out);
         keep(sQ2, m2, H2, B2, M2);
         r2 = rate();
         if (r2 > a.budget) {
@@ -564,7 +631,7 @@ __global__ void __launch_bounds__(512, 1) k_approx(ApproxArgs a) {
           for (int it = 0; it < a.steps; ++it) {
             const double mid = 0.5 * (lo + hi);
             __syncthreads();
-            approx_solve(c, mid, a.refine, &s_out);
+            approx_solve<T, kSplit>(c, mid, a.refine, &s_out);
             const double rr = rate();
             if (rr > a.budget) {
               lo = mid;
@@ -604,14 +671,19 @@ __global__ void __launch_bounds__(512, 1) k_approx(ApproxArgs a) {
   }
 }
 
-template <typename T, bool kSmem>
+template <typename T, bool kSmem, bool kSplit>
 void* approx_kernel_ptr() {
-  return reinterpret_cast<void*>(&k_approx<T, kSmem>);
+  return reinterpret_cast<void*>(&k_approx<T, kSmem, kSplit>);
 }
 
-void* approx_fn(bool fp64, bool smem) {
-  return fp64 ? (smem ? approx_kernel_ptr<double, true>() : approx_kernel_ptr<double, false>())
-              : (smem ? approx_kernel_ptr<float, true>() : approx_kernel_ptr<float, false>());
+template <typename T, bool kSmem>
+void* approx_fn_split(bool split) {
+  return split ? approx_kernel_ptr<T, kSmem, true>() : approx_kernel_ptr<T, kSmem, false>();
+}
+
+void* approx_fn(bool fp64, bool smem, bool split) {
+  return fp64 ? (smem ? approx_fn_split<double, true>(split) : approx_fn_split<double, false>(split))
+              : (smem ? approx_fn_split<float, true>(split) : approx_fn_split<float, false>(split));
 }
 
 size_t al16(size_t b) { return (b + 15) & ~size_t(15); }
@@ -644,7 +716,11 @@ bool approx_plan(int n, int p, int s, bool fp64, ApproxPlan* plan) {
   plan->smem = small + big + 1024 <= static_cast<size_t>(optin);
   plan->smem_bytes = small + (plan->smem ? big : 0);
   plan->scratch_per_cta = al256(2 * vb + 3 * db + (plan->smem ? 0 : big));
-  void* fn = approx_fn(fp64, plan->smem);
+  // Split columns when no SM holds more than one vector: then a layer waits on
+  // its longest column; with several CTAs per SM the others hide that wait and
+  // the split's extra loads and barrier only cost.
+  plan->split = n <= sms;
+  void* fn = approx_fn(fp64, plan->smem, plan->split);
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(plan->smem_bytes)) !=
       cudaSuccess)
     return false;
@@ -659,7 +735,7 @@ bool approx_plan(int n, int p, int s, bool fp64, ApproxPlan* plan) {
 
 cudaError_t launch_approx(const ApproxPlan& plan, ApproxArgs args, cudaStream_t st) {
   void* kargs[] = {&args};
-  cudaError_t e = cudaLaunchKernel(approx_fn(plan.fp64, plan.smem), dim3(plan.ctas), dim3(plan.threads), kargs,
+  cudaError_t e = cudaLaunchKernel(approx_fn(plan.fp64, plan.smem, plan.split), dim3(plan.ctas), dim3(plan.threads), kargs,
                                    plan.smem_bytes, st);
   note_launch();
   return e;

@@ -133,6 +133,7 @@ struct ApproxArgs {
 struct ApproxPlan {
   bool fp64;
   bool smem;  // cost table and layers in shared memory
+  bool split;  // each column's a range shared by two threads (few vectors)
   int threads;
   int ctas;
   size_t smem_bytes;

@@ -95,6 +95,40 @@ def test_approx_fp64_matches_oracle_from_its_statistics(E, O, case, refine):
         np.testing.assert_allclose(g[k_g].cpu().numpy(), ref[k_o], rtol=RTOL_EXACT, atol=1e-300)
 
 
+# More vectors than SMs: the launch runs one thread per column (the small cases
+# above, with fewer vectors than SMs, share each column between two threads).
+MANY = (21, 300, 300, 40, 6, "laplace")
+
+
+@pytest.mark.parametrize("refine", [0, 8])
+def test_approx_many_rows_fp64_matches_oracle_from_its_statistics(E, O, refine):
+    seed, n, d, p, s, dist = MANY
+    X, P = _setup(O, seed, n, d, p, dist)
+    lam = _lams(X, 3)
+    cnt, A, B = _oracle_stats(O, X, P)
+    g = E.solve_approx_stats(cnt, A, B, _cu(P), d, s, _cu(lam), refine=refine, fp64=True)
+    ref = O.solve_approx_batch(X, P, s, lam, refine=refine)
+    assert int(g["status"].abs().sum()) == 0
+    np.testing.assert_array_equal(g["Q_len"].cpu().numpy(), ref["m"])
+    np.testing.assert_array_equal(g["Q"].cpu().numpy(), ref["Q"])
+    np.testing.assert_allclose(g["objective"].cpu().numpy(), ref["J"], rtol=RTOL_EXACT, atol=1e-300)
+
+
+def test_approx_many_rows_fp32_from_X_reaches_the_oracle_optimum(E, O):
+    seed, n, d, p, s, dist = MANY
+    X, P = _setup(O, seed, n, d, p, dist)
+    lam = _lams(X, 3)
+    g = E.solve_approx(_cu(X), _cu(P), s, _cu(lam))
+    ref = O.solve_approx_batch(X, P, s, lam)
+    assert int(g["status"].abs().sum()) == 0
+    Q, m = g["Q"].cpu().numpy(), g["Q_len"].cpu().numpy()
+    for r in range(n):
+        for t in range(lam.shape[1]):
+            q = Q[r, t, : m[r, t]]
+            J = O.eval_raw(X[r], P[r][q])[0] + lam[r, t] * O.eval_raw_ib(X[r], P[r][q])
+            assert J <= ref["J"][r, t] * (1 + RTOL32) + 1e-300, (r, t, J, ref["J"][r, t])
+
+
 @pytest.mark.parametrize("case", CASES, ids=lambda c: f"p{c[3]}s{c[4]}{c[5]}")
 def test_approx_fp32_from_X_reaches_the_oracle_optimum(E, O, case):
     seed, n, d, p, s, dist = case
