@@ -81,6 +81,30 @@ def dp_traffic(w):
     return rec["bytes_per_row"] * w.n
 
 
+SPIN_CYCLES = 4_000_000  # about 2 ms of GPU clock
+
+
+def device_ms(fn, stream, flush, reps=3):
+    """Mean device time (ms) of the launches fn makes, each rep after an L2
+    flush. A spin kernel queued before the first event keeps the stream busy
+    while the host allocates and enqueues fn, so host overhead between the two
+    events is not counted."""
+    import torch
+
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    out = []
+    for k in range(reps):
+        flush.fill_(k & 0xFF)
+        torch.cuda._sleep(SPIN_CYCLES)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        out.append(a.elapsed_time(b))
+    return float(np.mean(out))
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -178,33 +202,25 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
     stream = torch.cuda.current_stream()
 
     def step(X):
-        ev["g0"].record(stream)
         P, st = E.uniform_grid(X, p)
-        ev["g1"].record(stream)
         cnt, A, B, st = E.bucket(X, P)
-        ev["b1"].record(stream)
         ev_dp0.record(stream)
         if w.mode == "budget":
             out = E.solve_budget_stats(cnt, A, B, P, d, s, w.b, w.steps, fp64=fp64)
             ev_dp1.record(stream)
             idx, hist, est = E.encode(X, P, s, out["Q1"], out["Q1_len"], w.seed_encode, out["Q2"], out["Q2_len"],
                                       out["theta"])
-            ev["e1"].record(stream)
         else:
             out = E.solve_stats(cnt, A, B, P, d, s, lam, fp64=fp64, hirschberg=w.hirschberg)
             ev_dp1.record(stream)
             Q = out["Q"][:, 0, :].contiguous()
             Ql = out["Q_len"][:, 0].contiguous()
-            ev["e0"].record(stream)
             idx, hist, est = E.encode(X, P, s, Q, Ql, w.seed_encode)
-            ev["e1"].record(stream)
         Hemp = E.entropy(hist)
         return out, idx, hist, Hemp
 
     ev_dp0 = torch.cuda.Event(enable_timing=True)
     ev_dp1 = torch.cuda.Event(enable_timing=True)
-    ev = {k: torch.cuda.Event(enable_timing=True) for k in ("g0", "g1", "b1", "e0", "e1")}
-    stage_ms = {"grid": [], "bucket": [], "encode": []}
     unit_peaks = measure_unit_peaks()
     for _ in range(args.warmup):
         out, idx, hist, Hemp = step(X)
@@ -226,9 +242,6 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
             ends[k].record(stream)
             torch.cuda.synchronize()
             dp_ms.append(ev_dp0.elapsed_time(ev_dp1))
-            stage_ms["grid"].append(ev["g0"].elapsed_time(ev["g1"]))
-            stage_ms["bucket"].append(ev["g1"].elapsed_time(ev["b1"]))
-            stage_ms["encode"].append((ev["e0"] if w.mode != "budget" else ev_dp1).elapsed_time(ev["e1"]))
     launches = E.launch_count(reset=True)
     step_ms = [starts[k].elapsed_time(ends[k]) for k in range(args.steps)]
     t_ms = D.max_over_ranks(float(sum(step_ms)))
@@ -258,26 +271,24 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
     hbm = float(peaks.get("hbm_gbs", 6650.0))
     entries = n * d
     hbm_kernels = {}
+    # Each stage alone, on the last step's data (device time, see device_ms)
+    P_last, _ = E.uniform_grid(X, p)
+    if w.mode == "budget":
+        enc_args = (out["Q1"], out["Q1_len"], w.seed_encode, out["Q2"], out["Q2_len"], out["theta"])
+    else:
+        enc_args = (out["Q"][:, 0, :].contiguous(), out["Q_len"][:, 0].contiguous(), w.seed_encode)
+    stage_fns = {"grid": lambda: E.uniform_grid(X, p), "bucket": lambda: E.bucket(X, P_last),
+                 "encode": lambda: E.encode(X, P_last, s, *enc_args)}
     for name, bpe in (("grid", 4), ("bucket", 4), ("encode", 5)):
-        ms = float(np.mean(stage_ms[name]))
+        ms = device_ms(stage_fns[name], stream, flush)
         gbs = entries * bpe / (ms * 1e-3) / 1e9
         hbm_kernels[name] = {"ms": ms, "bytes_per_entry": bpe, "achieved_GBps": gbs, "peak_GBps": hbm,
                              "frac": gbs / hbm, "entries_per_s": entries / (ms * 1e-3)}
     # hardware-aware alphabet (BF16 values covering each row), p_max = 512: one
     # read of X plus the alphabet rows written
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
     E.bf16_alphabet(X, 512)
-    bf_ms = []
-    for k in range(3):
-        flush.fill_(k & 0xFF)
-        e0.record(stream)
-        E.bf16_alphabet(X, 512)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        bf_ms.append(e0.elapsed_time(e1))
     bf_bytes = entries * 4 + n * 512 * 8
-    bf_t = float(np.mean(bf_ms))
+    bf_t = device_ms(lambda: E.bf16_alphabet(X, 512), stream, flush)
     hbm_kernels["bf16_alphabet"] = {"ms": bf_t, "bytes": bf_bytes, "achieved_GBps": bf_bytes / (bf_t * 1e-3) / 1e9,
                                     "peak_GBps": hbm, "frac": bf_bytes / (bf_t * 1e-3) / 1e9 / hbm}
     # entropy coder on the last step's indices (rANS, per-row models from the
@@ -299,15 +310,7 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
         assert rc == 0, rc
 
     coder()
-    rc_ms = []
-    for k in range(3):
-        flush.fill_(k & 0xFF)
-        e0.record(stream)
-        coder()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        rc_ms.append(e0.elapsed_time(e1))
-    rc_t = float(np.mean(rc_ms))
+    rc_t = device_ms(coder, stream, flush)
     coded_bits = 16.0 * float(seg_len.sum().item())
     hbm_kernels["rans_encode"] = {"ms": rc_t, "entries_per_s": entries / (rc_t * 1e-3),
                                   "bits_per_entry": coded_bits / entries,
@@ -386,17 +389,7 @@ def approx_timing(args, w: W.Workload, X, stream, flush, dp_avg_ms: float, sm_ma
     for refine in (0, 8):
         out = call(refine)  # warm-up
         torch.cuda.synchronize()
-        ms = []
-        for k in range(max(2, min(args.steps, 3))):
-            flush.fill_(k & 0xFF)
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            out = call(refine)
-            e1.record(stream)
-            torch.cuda.synchronize()
-            ms.append(e0.elapsed_time(e1))
-        t = float(np.mean(ms))
+        t = device_ms(lambda: call(refine), stream, flush, reps=max(2, min(args.steps, 3)))
         ns = solves_done(w, out)
         ach = ns * rps / (t * 1e-3)
         res[f"refine{refine}"] = {"ms": t, "solves": ns, "achieved": ach, "frac": ach / peak,
