@@ -40,7 +40,7 @@ B200_SMS = 148
 # 1411 MB written, almost all of it the stored DP layers written back from L2),
 # scaled by the rows of a launch. The figure belongs to the kernel source it was
 # taken on; it is dropped (null) when that source has changed since.
-DP_TRAFFIC = {"weights": {"bytes_per_row": (1708544 + 1410748672) / 296, "dp_source_sha1": "a9ffec8785361700"}}
+DP_TRAFFIC = {"weights": {"bytes_per_row": (1708544 + 1410748672) / 296, "dp_source_sha1": "ba90d42feb4558bf"}}
 
 
 def triples_per_solve(p: int, s: int) -> int:

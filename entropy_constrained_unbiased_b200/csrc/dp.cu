@@ -15,19 +15,25 @@
 //   F_i(l, j) = V(l,j)/(lambda d) + min_{k} [ F_{i-1}(k,l) + h((R(k,l) + L(l,j))/d) ]
 //   J*/lambda = min_{i,k} F_i(k, p-1) + h(R(k,p-1)/d),   h(m) = -m log2 m.
 // The whole programme is scaled by 1/lambda, so one (k,l,j) triple is one add,
-// one MUFU log2 and one FMA plus the running argmin. lambda = 0 is the
+// one MUFU log2 and one FMA plus the running minimum. lambda = 0 is the
 // separable MSE-only programme (the minimum over k no longer depends on j).
 //
 // Design (this file):
 //   * one CTA per vector, persistent over every solve of that vector (all
 //     lambdas, or the whole bisection), so the pair tables are built once;
+//     with the tables in the global slab and at most one vector per two SMs,
+//     a cluster of two CTAs shares each vector: they split every layer's tasks
+//     through one counter in rank 0's shared memory and synchronise at cluster
+//     barriers;
 //   * the tables and the two live DP layers sit in shared memory when they fit
 //     (fp32, p <= 128) and in a per-CTA global (L2-resident) slab otherwise;
 //   * a DP layer is split into tasks of 32 lanes; a lane owns 4 outputs
 //     (l, j0..j0+3) of one row and sweeps k down the column of l in two
 //     interleaved streams; tasks are decoded in closed form from their index,
 //     longest rows first, and taken by warps from a shared counter;
-//   * store mode keeps back-pointers in a per-CTA global slab and backtracks;
+//   * store mode keeps every layer's values in a per-CTA global slab (no
+//     back-pointers); the backtrack recomputes the argmin of the few states on
+//     the optimal path;
 //     Hirschberg mode keeps none: a forward pass finds the optimum and its last
 //     pair, then the code is recovered by divide and conquer, joining a forward
 //     pass over the left part with a pass over the reflected alphabet
