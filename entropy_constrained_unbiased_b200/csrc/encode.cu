@@ -102,6 +102,9 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
   }
   __syncthreads();
 
+  // Part test u < theta with u = sel * 2^-32: theta * 2^32 is exact in fp64 and
+  // sel is an integer, so it is sel < ceil(theta * 2^32) (at most 2^32).
+  const uint64_t th_cut = mix ? static_cast<uint64_t>(ceil(th * 0x1p32)) : 0;
   const float scale = static_cast<float>(static_cast<double>(p - 1) / (sP[p - 1] - sP[0]));
   const float top = __double2float_rd(sP[p - 1]);
   const int64_t beg = static_cast<int64_t>(blockIdx.x) * kEncChunk;
@@ -137,7 +140,7 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
       if (e >= cnt) break;
       const double xd = static_cast<double>(xv[e]);
       int part = fixed_part;
-      if (mix) part = (static_cast<double>(sel[e]) * 0x1p-32 < th) ? 0 : 1;
+      if (mix) part = (static_cast<uint64_t>(sel[e]) < th_cut) ? 0 : 1;
       const int m = s_m[part];
       int out = 0;
       if (m == 1) {

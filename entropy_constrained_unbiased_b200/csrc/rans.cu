@@ -173,13 +173,16 @@ __device__ void stage_chunk(const uint8_t* __restrict__ xrow, int64_t d, int64_t
     uint32_t bits = mode == 1 ? 0xffffffffu : 0u;
     if (mode == 2) {
       const int64_t e0 = e_lo + static_cast<int64_t>(lane) * kWarp;
+      // u < theta with u = word * 2^-32 is word < ceil(theta * 2^32): theta * 2^32
+      // is exact in fp64 and the word is an integer.
+      const uint64_t cut = static_cast<uint64_t>(ceil(th * 0x1p32));
 #pragma unroll
       for (int b = 0; b < 8; ++b) {
         const uint4 w = Philox4x32::block(make_uint4(static_cast<uint32_t>((e0 >> 2) + b), row, 1u, 0u), k0, k1);
-        bits |= (static_cast<double>(w.x) * 0x1p-32 < th ? 0u : 1u) << (4 * b);
-        bits |= (static_cast<double>(w.y) * 0x1p-32 < th ? 0u : 1u) << (4 * b + 1);
-        bits |= (static_cast<double>(w.z) * 0x1p-32 < th ? 0u : 1u) << (4 * b + 2);
-        bits |= (static_cast<double>(w.w) * 0x1p-32 < th ? 0u : 1u) << (4 * b + 3);
+        bits |= (static_cast<uint64_t>(w.x) < cut ? 0u : 1u) << (4 * b);
+        bits |= (static_cast<uint64_t>(w.y) < cut ? 0u : 1u) << (4 * b + 1);
+        bits |= (static_cast<uint64_t>(w.z) < cut ? 0u : 1u) << (4 * b + 2);
+        bits |= (static_cast<uint64_t>(w.w) < cut ? 0u : 1u) << (4 * b + 3);
       }
     }
     st.part[lane] = bits;
