@@ -14,7 +14,7 @@
 //        Q0, Q1, Q2 of the values in turn, each in parallel, by binary search
 //        inside its local interval; unbiasedness is kept.
 //
-// Readings (each is listed in the design doc):
+// Readings where the page leaves a step open:
 //   * (I, B) of an entry in [q_t, q_{t+1}] is (t, 0) with probability
 //     1 - u and (t, 1) with probability u, u = (x - q_t)/(q_{t+1} - q_t); an
 //     entry on an interior value q_t belongs to the interval that starts there

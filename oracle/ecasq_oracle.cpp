@@ -16,7 +16,7 @@
 //                              l, plus the MSE of [x_l, x_j] with l, j consecutive
 //   §2.2 "Generalização"       arbitrary permissible set P, O(p^2 s + d)
 //
-// Readings where the page is silent (each one is listed in the design doc):
+// Readings where the page is silent:
 //   * MSE is the per-entry mean; H is in bits per entry and is the entropy of the
 //     EXPECTED output distribution mu/d of the stochastic quantizer.
 //   * Q always holds P_0 and P_{p-1} (unbiasedness needs q_1 <= min X and

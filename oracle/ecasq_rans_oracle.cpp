@@ -10,7 +10,7 @@
 // names no coder; this is range-variant asymmetric numeral systems (rANS, Duda,
 // "Asymmetric numeral systems", arXiv:1311.2540) with a static model.
 //
-// Readings (each is listed in the design doc):
+// Readings where the page leaves a step open:
 //   * one model per vector and time-sharing part (the codes Q1, Q2), from the
 //     encoder's histogram; the part of an entry is not coded: the decoder
 //     recomputes it from the seed exactly as the encoder drew it;
