@@ -113,7 +113,7 @@ int ecasq_bucket(const float* X, const double* P, int n, int64_t d, int p, int64
  * Outputs, layout and status are those of ecasq_bucket.
  * Scratch: a fixed 8 MiB array in the library's device memory, held by every
  * GPU that loads the library until the process exits. It must hold
- * 24*n*(p-1) + 4*n bytes (each term rounded up to 256), e.g. n <= 2750 rows at
+ * 24*n*(p-1) + 4*n bytes (each term rounded up to 256), e.g. n <= 2748 rows at
  * p = 128 or n <= 1369 at p = 256; larger sizes return ECASQ_ERR_WORKSPACE
  * and launch nothing. The call allocates nothing: the first call on a device
  * resolves the array's device address (with that device current), so make
@@ -232,8 +232,14 @@ int ecasq_solve_approx_budget_stats(const int64_t* cnt, const double* A, const d
  *   - Q2 == NULL: every entry uses Q1 (part 0).
  *   - Q2 != NULL, 0 < theta[r] < 1: entry uses Q1 iff u(stream 1) < theta[r],
  *     else Q2 (part 1); theta >= 1: Q1 only; theta <= 0 (or theta NULL): Q2 only.
- *   - x in [q_i, q_{i+1}] of its code rounds up iff u(stream 0) <
- *     (x - q_i)/(q_{i+1} - q_i) in IEEE fp64 (two subtractions, one division).
+ *   - x in [q_i, q_{i+1}] of its code rounds up with probability
+ *     (x - q_i)/(q_{i+1} - q_i); the test, with the division moved across, is
+ *     u(stream 0) * (q_{i+1} - q_i) < x - q_i, each side one IEEE fp64
+ *     operation with round-to-nearest (the width q_{i+1} - q_i is one
+ *     subtraction, the product one multiplication, x - q_i one subtraction;
+ *     no fused multiply-add), so x = q_i never rounds up and x = q_{i+1}
+ *     always does. The time-sharing test u(stream 1) < theta[r] is the exact
+ *     integer test word < ceil(theta[r] * 2^32).
  * idx [n][d] uint8 = position of the emitted value in the code used (so s <= 256);
  * hist [n][2][s] int64 counts per part and position (overwritten).
  * status[r] = ECASQ_ERR_RANGE for an entry outside its code's range. */

@@ -318,6 +318,28 @@ def test_philox_round_structure_matches_numpy(O, ctr, key):
     np.testing.assert_array_equal(ours, got)
 
 
+def _philox_kat():
+    rows = []
+    with open(os.path.join(GOLD, "philox4x32_kat.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            w = [int(t, 16) for t in line.split()]
+            assert len(w) == 10
+            rows.append((tuple(w[0:4]), tuple(w[4:6]), tuple(w[6:10])))
+    return rows
+
+
+@pytest.mark.parametrize("ctr,key,want", _philox_kat())
+def test_philox4x32_known_answers(O, ctr, key, want):
+    """The published Philox4x32-10 known-answer vectors (Random123, Salmon et
+    al. SC'11): a wrong multiplier, Weyl increment, word order or round count
+    changes every output word."""
+    got = O.philox4x32(ctr, key)
+    assert [int(v) for v in got] == list(want), [f"{int(v):08x}" for v in got]
+
+
 def test_philox4x32_uniformity(O):
     """Chi-square over 2^14 blocks (65536 words) in 64 cells."""
     words = []
@@ -385,6 +407,43 @@ def test_entropy_of_histogram(O):
     hist[0, :3] = [1, 1, 2]          # H = 1.5 bits over 4 entries
     hist[1, :2] = [2, 2]             # H = 1 bit over 4 entries
     assert O.entropy(hist, 4) == pytest.approx((4 * 1.5 + 4 * 1.0) / 8, rel=1e-15)
+
+
+def _grid_cases():
+    rng = np.random.default_rng([41, 0])
+    cases = []
+    for p in (2, 3, 7, 17, 64, 128, 256, 512):
+        for lo, hi in ((-1.0, 1.0), (0.0, 3.0), (-2.5e-3, 7.0e-2), (1000.0, 1000.5), (-3.0e5, -2.0e5)):
+            cases.append((p, lo, hi))
+    for _ in range(6):
+        a, b = np.sort(rng.standard_normal(2) * 10.0 ** rng.integers(-3, 4, 2))
+        cases.append((int(rng.integers(2, 513)), float(a), float(b)))
+    return cases
+
+
+@pytest.mark.parametrize("p,lo,hi", _grid_cases())
+def test_grid_interior_is_uniform(O, p, lo, hi):
+    """A uniform grid spanning [min X, max X]: P_k equals the exact rational
+    lo + (hi - lo) k / (p - 1) to within the rounding of a few fp64 operations,
+    and every spacing P_{k+1} - P_k equals (hi - lo)/(p - 1) likewise. A grid
+    built with k/p (or any other slip in the spacing) is off by span/p at the
+    interior points, far beyond these bounds."""
+    rng = np.random.default_rng([43, p])
+    x = rng.uniform(lo, hi, size=257).astype(np.float32)
+    x[0], x[-1] = np.float32(lo), np.float32(hi)
+    flo, fhi = float(x.min()), float(x.max())
+    P, st = O.uniform_grid(x, p)
+    Pb, stb = O.grid_batch(x[None, :], p)
+    assert st == 0 and stb[0] == 0
+    np.testing.assert_array_equal(P, Pb[0])
+    span = Fraction(fhi) - Fraction(flo)
+    tol = 4 * np.spacing(max(abs(flo), abs(fhi), float(span)))
+    for k in range(p):
+        exact = Fraction(flo) + span * k / (p - 1)
+        assert abs(Fraction(float(P[k])) - exact) <= Fraction(tol), (k, float(P[k]), float(exact))
+    assert P[0] == flo and P[-1] == fhi
+    step = float(span / (p - 1))
+    assert np.all(np.abs(np.diff(P) - step) <= 2 * tol)
 
 
 def test_grid_is_exact_endpoints(O):
