@@ -50,6 +50,31 @@ struct Philox4x32 {
     }
     return c;
   }
+
+  // The same generator with the ten round keys (k0 + r W_A, k1 + r W_B)
+  // precomputed by the host and passed as kernel parameters, so that a round
+  // is two 32x32->64 multiplications and two three-input XORs.
+  struct RoundKeys {
+    uint32_t k0[10], k1[10];
+  };
+  __host__ static RoundKeys round_keys(uint32_t k0, uint32_t k1) {
+    RoundKeys K;
+    for (int r = 0; r < 10; ++r) {
+      K.k0[r] = k0 + static_cast<uint32_t>(r) * kWeylA;
+      K.k1[r] = k1 + static_cast<uint32_t>(r) * kWeylB;
+    }
+    return K;
+  }
+  __device__ __forceinline__ static uint4 block(uint4 c, const RoundKeys& K) {
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+      const uint64_t p0 = static_cast<uint64_t>(kMulA) * c.x;
+      const uint64_t p1 = static_cast<uint64_t>(kMulB) * c.z;
+      c = make_uint4(static_cast<uint32_t>(p1 >> 32) ^ c.y ^ K.k0[r], static_cast<uint32_t>(p1),
+                     static_cast<uint32_t>(p0 >> 32) ^ c.w ^ K.k1[r], static_cast<uint32_t>(p0));
+    }
+    return c;
+  }
 };
 
 template <typename T>
@@ -106,5 +131,45 @@ __device__ __forceinline__ int bucket_of(double x, const double* __restrict__ P,
   while (k < p - 2 && P[k + 1] <= x) ++k;
   return k;
 }
+
+
+// Uniform-grid description of an alphabet row: P_k = P_0 + (k + eta_k) D with
+// D = (P_{p-1} - P_0)/(p-1). A row counts as uniform when every |eta_k| is at
+// most 2^-36 bucket widths; then the bucket of x follows from (x - P_0)/D
+// computed directly, with an exact search only for entries very close to a
+// grid point (bucketing and encoding use this).
+constexpr double kEtaMax = 0x1p-36;
+
+// eta_k = (P_k - P_0)/D - k with every operation rounded as written (the bucket
+// kernel and the finish kernel must agree bit for bit).
+__device__ __forceinline__ double grid_eta(double Pk, double P0, double invD, int k) {
+  return __dsub_rn(__dmul_rn(__dsub_rn(Pk, P0), invD), static_cast<double>(k));
+}
+
+struct RowGrid {
+  double P0, D, invD;
+};
+
+__device__ __forceinline__ RowGrid row_grid(const double* __restrict__ P, int p) {
+  RowGrid g;
+  g.P0 = P[0];
+  const double span = __dsub_rn(P[p - 1], g.P0);
+  g.D = __ddiv_rn(span, static_cast<double>(p - 1));
+  g.invD = __ddiv_rn(1.0, g.D);
+  return g;
+}
+
+// Whether the row takes the uniform fast path; called by every thread of the
+// block (block-wide OR). eta_out (optional, shared) receives eta_k.
+__device__ __forceinline__ bool row_is_uniform(const double* __restrict__ P, int p, const RowGrid& g, double* eta_out) {
+  int bad = !(g.D > 0.0) || !isfinite(g.invD);
+  for (int k = threadIdx.x; k < p; k += blockDim.x) {
+    const double e = grid_eta(P[k], g.P0, g.invD, k);
+    if (eta_out) eta_out[k] = e;
+    if (!(fabs(e) <= kEtaMax)) bad = 1;
+  }
+  return !__syncthreads_or(bad);
+}
+
 
 }  // namespace ecasq

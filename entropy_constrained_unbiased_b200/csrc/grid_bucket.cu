@@ -186,137 +186,395 @@ __global__ void k_bf16_finish(const float* __restrict__ part, int n_chunks, int 
 }
 
 // ---------------------------------------------------------------------------
-// Bucketing. Sums are fixed point: an entry of bucket k with u = (x - P_k)/D_k,
-// D_k = P_{k+1} - P_k, adds round(u * 2^36) to the first-moment sum and
-// round(u^2 * 2^36) to the second. Integer sums make the result independent
-// of the order in which entries are added.
+// Bucketing (the "+d" pass of §2.2 "Generalização"). An entry x of bucket k
+// (P_k <= x < P_{k+1}; the last bucket closed) contributes a normalised offset
+// v in [0, 1], kept as fixed point: round(v 2^F) and round(v^2 2^F) with F = 36
+// fraction bits (32 for rows of 2^27 entries or more, so that the 64-bit row
+// sums cannot overflow). Integer sums make the result independent of the order
+// of addition. The finish kernel turns them back into A_k = sum (x - P_k) and
+// B_k = sum (x - P_k)^2.
 //
-// Only 32-bit shared-memory atomics are native on this GPU (64-bit and
-// floating-point ones are emulated and collapse when lanes collide, which
-// heavy-tailed inputs make the rule). So each 36-bit value is added as two
-// 18-bit limbs to 32-bit counters. A limb is below 2^18 except the high limb
-// of an entry exactly at the top of its bucket (2^18), so 2^13 entries per CTA
-// keep every counter below 2^31. Per entry: one count and four limb additions,
-// all return-less 32-bit atomics.
+// Two ways to find k and v:
+//  * uniform rows: P_k = P_0 + (k + eta_k) D with D = (P_{p-1} - P_0)/(p-1)
+//    and |eta_k| <= 2^-36 for every k (an fp64 uniform grid qualifies unless
+//    |P_0| is very large against the span). G = (x - P_0)/D in fp64 is within
+//    2^-41 bucket widths of its exact value (p <= 512), so when
+//    v = G - floor(G) lies more than 2^-20 from 0 and from 1, k = floor(G) is
+//    the entry's bucket for certain and v = (x - P_k)/D + eta_k up to that
+//    error: no shared-memory lookup at all. The few entries within 2^-20 of a
+//    grid point take the exact search and v = clamp((x - P_k)/D + eta_k, 0, 1),
+//    the clamp moving v by at most |eta_k|. Then A_k = D (S1 - n_k eta_k) and
+//    B_k = D^2 (S2 - 2 eta_k S1 + n_k eta_k^2) with S1 = sum v, S2 = sum v^2.
+//  * other rows: k by the exact search on P, v = (x - P_k)/D_k, A_k = D_k S1,
+//    B_k = D_k^2 S2.
+//
+// Accumulation: 32-bit shared-memory counters, added by return-less atomics:
+// per entry the count (an increment, which the hardware combines across lanes
+// that hit the same counter) and two limbs of each moment (bits 0..17 and
+// 18..F). Additions of different values to one address by lanes of a warp are
+// serialised, and real data concentrates in a few buckets, so the limbs of
+// the kHotW busiest consecutive buckets (chosen from the counts of the CTA's
+// first 8192 entries) get one counter per lane, laid out [bucket][lane] so
+// that the 32 lanes of a warp always fall on 32 distinct banks; the other
+// buckets share one counter per bucket. Shared counters are folded into 64-bit
+// registers of the bucket's owner thread every 8192 entries (8192 limbs of at
+// most 2^18 stay below 2^32); a lane counter receives at most 2048 entries per
+// CTA and is summed once at the end. Each CTA adds its totals to the row's
+// 64-bit sums in global memory.
 
 constexpr int kBucketThreads = 256;
-constexpr int kFixBits = 36;
+constexpr int kBucketSub = 8192;          // entries between two folds of the shared counters
+constexpr int kBucketSubsPerCta = 8;      // 65536 entries per CTA
+constexpr int kBucketOwn = 2;             // buckets owned per thread (p - 1 <= 511)
+constexpr int kHotW = 48;                 // buckets with one counter per lane
+constexpr int kLimbBlock = kHotW * kWarp + kMaxP;  // words per limb: [kHotW][32] lane counters, then [kMaxP]
 constexpr int kLimbBits = 18;
-constexpr int64_t kBucketChunk = 8192;  // entries per CTA (see above)
+constexpr double kFastEps = 0x1p-20;      // distance of v from a grid point on the fast path
 
-__global__ void __launch_bounds__(kBucketThreads)
-k_bucket(const float* __restrict__ X, int64_t d, int64_t chunk, const double* __restrict__ Pall, int p, int fb,
+// Per-CTA state of the bucketing kernel in shared memory.
+struct BucketRow {
+  const double* P;   // [p]
+  const double* E;   // [p] eta_k (uniform rows) or 1/D_k (other rows)
+  const float* T;    // [p] smallest float >= P_k
+  unsigned int* cnt;   // [kMaxP] counts
+  unsigned int* limb;  // [4][kLimbBlock]
+  double invD, twoF, twoH;
+  float top, scale;
+  int p, hot0, uni, bad;
+};
+
+// Fixed point: a = v 2^(F+14) + 2^52 + 2^13 keeps round(v 2^F) in bits 14.. of
+// the integer part, so the low limb is the low word >> 14 and the high limb the
+// low bits of the high word.
+__device__ __forceinline__ void bucket_add(unsigned int* cnt, unsigned int* limb, int k, double v, int hot0,
+                                           int lane, double twoF, double twoH) {
+  const double magic = 0x1p52 + 0x1p13;
+  atomicAdd(cnt + k, 1u);
+  const double a = fma(v, twoF, magic);
+  const double t = v * twoH;
+  const double b = fma(t, t, magic);
+  const int hk = k - hot0;
+  const int off = (static_cast<unsigned>(hk) < static_cast<unsigned>(kHotW)) ? hk * kWarp + lane : kHotW * kWarp + k;
+  unsigned int* c = limb + off;
+  atomicAdd(c, static_cast<unsigned>(__double2loint(a)) >> 14);
+  atomicAdd(c + kLimbBlock, static_cast<unsigned>(__double2hiint(a)) & 0x7FFFFu);
+  atomicAdd(c + 2 * kLimbBlock, static_cast<unsigned>(__double2loint(b)) >> 14);
+  atomicAdd(c + 3 * kLimbBlock, static_cast<unsigned>(__double2hiint(b)) & 0x7FFFFu);
+}
+
+// Exact bucket k = max{k <= p-2 : P_k <= x} (fp32-threshold search) and offset
+// v of up to four entries, then their counters; entries outside
+// [P_0, P_{p-1}] or NaN set the bad flag. Uniform rows: v = clamp((x - P_k)/D
+// + eta_k, 0, 1); other rows: v = min((x - P_k)/D_k, 1). Kept out of line: on
+// uniform rows it runs only for groups holding an entry within 2^-20 bucket
+// widths of a grid point.
+__device__ __noinline__ void bucket_exact(BucketRow* S, const float* xv, int cnt) {
+  const int lane = lane_id();
+  for (int e = 0; e < cnt; ++e) {
+    const float xf = xv[e];
+    const int k = bucket_f32(xf, S->T, S->top, S->p, S->scale);
+    if (k < 0) {
+      S->bad = 1;
+      continue;
+    }
+    const double y = __dsub_rn(static_cast<double>(xf), S->P[k]);
+    const double w = S->uni ? __dadd_rn(__dmul_rn(y, S->invD), S->E[k]) : __dmul_rn(y, S->E[k]);
+    bucket_add(S->cnt, S->limb, k, fmin(fmax(w, 0.0), 1.0), S->hot0, lane, S->twoF, S->twoH);
+  }
+}
+
+// Bucketing (the "+d" pass of §2.2 "Generalização"). An entry x of bucket k
+// (P_k <= x < P_{k+1}; the last bucket closed) contributes a normalised offset
+// v in [0, 1], kept as fixed point: round(v 2^F) and round(v^2 2^F) with F = 36
+// fraction bits (32 for rows of 2^27 entries or more, so that the 64-bit row
+// sums cannot overflow). Integer sums make the result independent of the order
+// of addition. The finish kernel turns them back into A_k = sum (x - P_k) and
+// B_k = sum (x - P_k)^2.
+//
+// Two ways to find k and v:
+//  * uniform rows: P_k = P_0 + (k + eta_k) D with D = (P_{p-1} - P_0)/(p-1)
+//    and |eta_k| <= 2^-36 for every k (an fp64 uniform grid qualifies unless
+//    |P_0| is very large against the span). G = (x - P_0)/D in fp64 is within
+//    2^-41 bucket widths of its exact value (p <= 512), so when
+//    v = G - floor(G) lies more than 2^-20 from 0 and from 1, k = floor(G) is
+//    the entry's bucket for certain and v = (x - P_k)/D + eta_k up to that
+//    error: no shared-memory lookup at all. Groups of four entries holding one
+//    within 2^-20 of a grid point take the exact search, with
+//    v = clamp((x - P_k)/D + eta_k, 0, 1), the clamp moving v by at most |eta_k|.
+//    Then A_k = D (S1 - n_k eta_k) and B_k = D^2 (S2 - 2 eta_k S1 + n_k eta_k^2)
+//    with S1 = sum v, S2 = sum v^2.
+//  * other rows: k by the exact search on P, v = (x - P_k)/D_k, A_k = D_k S1,
+//    B_k = D_k^2 S2.
+//
+// Accumulation: 32-bit shared-memory counters, added by return-less atomics:
+// per entry the count (an increment, which the hardware combines across lanes
+// that hit the same counter) and two limbs (bits 0..17 and 18..F) of each
+// moment. Additions of different values to one address by lanes of a warp are
+// serialised, and real data concentrates in a few buckets, so the limbs of the
+// kHotW busiest consecutive buckets (chosen from a sample of the CTA's entries)
+// get one counter per lane, laid out [bucket][lane] so that the 32 lanes of a
+// warp always fall on 32 distinct banks; the other buckets share one counter
+// per bucket. Shared counters are folded into 64-bit registers of the bucket's
+// owner thread every 8192 entries (8192 limbs of at most 2^18 stay below 2^32);
+// a lane counter receives at most 2048 entries per CTA and is summed once at
+// the end. Each CTA adds its totals to the row's 64-bit sums in global memory.
+__global__ void __launch_bounds__(kBucketThreads, 3)
+k_bucket(const float* __restrict__ X, int64_t d, const double* __restrict__ Pall, int p, int fb,
          unsigned long long* __restrict__ acc, int32_t* __restrict__ flag) {
+  __shared__ unsigned int sc[kMaxP];                 // counts (every bucket)
+  __shared__ unsigned int sl[4 * kLimbBlock];       // limbs: [4][kLimbBlock]
+  __shared__ unsigned int spre[kMaxP + 1];           // sample counts, then their prefix sums
+  __shared__ BucketRow S;
   extern __shared__ __align__(16) unsigned char smem[];
-  (void)fb;
   const int r = blockIdx.y;
   const int nb = p - 1;
-  double* sP = reinterpret_cast<double*>(smem);                    // [p]
-  double* sS = sP + p;                                             // [p] 2^36 / D_k
-  unsigned int* hc = reinterpret_cast<unsigned int*>(sS + p);     // [p] count
-  unsigned int* ha = hc + p;                                       // [2][p] first-moment limbs (lo, hi)
-  unsigned int* hb = ha + 2 * p;                                   // [2][p] second-moment limbs
-  float* sT = reinterpret_cast<float*>(hb + 2 * p);                // [p] exact fp32 thresholds
-  __shared__ int s_bad;
+  double* sP = reinterpret_cast<double*>(smem);      // [p] P
+  double* sE = sP + p;                               // [p] eta_k (uniform rows) or 1/D_k (other rows)
+  float* sT = reinterpret_cast<float*>(sE + p);      // [p] smallest float >= P_k
 
   const double* P = Pall + static_cast<int64_t>(r) * p;
-  const double two_f = 0x1p36;
   for (int k = threadIdx.x; k < p; k += blockDim.x) {
     sP[k] = P[k];
-    sS[k] = (k < nb) ? two_f / (P[k + 1] - P[k]) : 0.0;
     sT[k] = __double2float_ru(P[k]);
   }
-  for (int k = threadIdx.x; k < 5 * p; k += blockDim.x) hc[k] = 0u;
-  if (threadIdx.x == 0) s_bad = 0;
+  for (int k = threadIdx.x; k < kMaxP; k += blockDim.x) sc[k] = 0u;
+  for (int k = threadIdx.x; k <= kMaxP; k += blockDim.x) spre[k] = 0u;
+  for (int k = threadIdx.x; k < 4 * kLimbBlock; k += blockDim.x) sl[k] = 0u;
   __syncthreads();
-
-  const float scale = static_cast<float>(static_cast<double>(p - 1) / (sP[p - 1] - sP[0]));
-  const float top = __double2float_rd(sP[p - 1]);
-  const double inv_two_f = 0x1p-36;
-  const double magic = 0x1p52;  // v + 2^52 keeps round(v) in the low mantissa bits for 0 <= v < 2^52
-  const unsigned int lmask = (1u << kLimbBits) - 1u;
-  int bad = 0;
-
-  auto one = [&](float xf) {
-    const double x = static_cast<double>(xf);
-    const int k = bucket_f32(xf, sT, top, p, scale);
-    if (k < 0) {
-      bad = 1;
-      return;
+  const RowGrid g = row_grid(sP, p);
+  const bool uni = row_is_uniform(sP, p, g, sE);  // includes a barrier
+  if (!uni) {
+    for (int k = threadIdx.x; k < nb; k += blockDim.x) {
+      const double w = __dsub_rn(sP[k + 1], sP[k]);
+      sE[k] = w > 0.0 ? __ddiv_rn(1.0, w) : 0.0;
     }
-    const double u = (x - sP[k]) * sS[k];  // in [0, 2^36]
-    const unsigned long long a = static_cast<unsigned long long>(__double_as_longlong(u + magic));
-    const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(fma(u, u * inv_two_f, magic)));
-    atomicAdd(hc + k, 1u);
-    atomicAdd(ha + k, static_cast<unsigned int>(a) & lmask);
-    atomicAdd(ha + p + k, static_cast<unsigned int>(a >> kLimbBits) & ((1u << (kFixBits + 1 - kLimbBits)) - 1u));
-    atomicAdd(hb + k, static_cast<unsigned int>(b) & lmask);
-    atomicAdd(hb + p + k, static_cast<unsigned int>(b >> kLimbBits) & ((1u << (kFixBits + 1 - kLimbBits)) - 1u));
-  };
+  }
+  const double twoF = ldexp(1.0, fb + 14), twoH = ldexp(1.0, (fb + 14) / 2);
+  if (threadIdx.x == 0) {
+    S.P = sP;
+    S.E = sE;
+    S.T = sT;
+    S.cnt = sc;
+    S.limb = sl;
+    S.invD = g.invD;
+    S.twoF = twoF;
+    S.twoH = twoH;
+    S.top = __double2float_rd(sP[p - 1]);
+    S.scale = static_cast<float>(static_cast<double>(p - 1) / (sP[p - 1] - sP[0]));
+    S.p = p;
+    S.hot0 = 0;
+    S.uni = uni;
+    S.bad = 0;
+  }
+  __syncthreads();
+  const int lane = lane_id();
+  const unsigned pm2 = static_cast<unsigned>(p - 2);
+  const double lim = 0.5 - kFastEps;
 
   const float* x = X + static_cast<int64_t>(r) * d;
+  const int64_t chunk = static_cast<int64_t>(kBucketSub) * kBucketSubsPerCta;
   const int64_t beg = static_cast<int64_t>(blockIdx.x) * chunk;
   const int len = static_cast<int>((beg + chunk < d ? beg + chunk : d) - beg);
   const float* xc = x + beg;
-  const bool vec = ((reinterpret_cast<uintptr_t>(xc) & 15u) == 0);
-  int t = 0;
-  if (vec) {
-    const int nv = len >> 2;
-    const float4* x4 = reinterpret_cast<const float4*>(xc);
-    for (int i = threadIdx.x; i < nv; i += blockDim.x) {
-      const float4 v = __ldcs(x4 + i);
-      one(v.x);
-      one(v.y);
-      one(v.z);
-      one(v.w);
-    }
-    t = nv << 2;
-  }
-  for (int i = t + threadIdx.x; i < len; i += blockDim.x) one(__ldcs(xc + i));
-  if (bad) s_bad = 1;
-  __syncthreads();
 
-  unsigned long long* gacc = acc + static_cast<int64_t>(r) * nb * 3;
-  for (int k = threadIdx.x; k < nb; k += blockDim.x) {
-    const unsigned int c = hc[k];
-    if (c) {
-      const unsigned long long sa = static_cast<unsigned long long>(ha[k]) +
-                                    (static_cast<unsigned long long>(ha[p + k]) << kLimbBits);
-      const unsigned long long sb = static_cast<unsigned long long>(hb[k]) +
-                                    (static_cast<unsigned long long>(hb[p + k]) << kLimbBits);
-      atomicAdd(gacc + 3 * k + 0, static_cast<unsigned long long>(c));
-      atomicAdd(gacc + 3 * k + 1, sa);
-      atomicAdd(gacc + 3 * k + 2, sb);
+  // Hot window: bucket counts of a sample of blockDim entries spread over the
+  // chunk, then the kHotW consecutive buckets with the most sampled entries.
+  {
+    const int i = threadIdx.x * (len > kBucketThreads ? len / kBucketThreads : 1);
+    if (i < len) {
+      const float xf = __ldg(xc + i);
+      int k = -1;
+      if (uni) {
+        const double G = __dmul_rn(__dsub_rn(static_cast<double>(xf), g.P0), g.invD);
+        const double kf = floor(G);
+        if (kf >= 0.0 && kf <= static_cast<double>(p - 2)) k = static_cast<int>(kf);
+      } else {
+        k = bucket_f32(xf, sT, S.top, p, S.scale);
+      }
+      if (k >= 0) atomicAdd(spre + k, 1u);
+    }
+    __syncthreads();
+    if (warp_id() == 0) {
+      unsigned run = 0;
+      for (int j = 0; j < 16; ++j) run += spre[lane * 16 + j];
+      unsigned excl = run;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned t = __shfl_up_sync(0xffffffffu, excl, o);
+        if (lane >= o) excl += t;
+      }
+      excl -= run;
+      unsigned cnts[16];
+      for (int j = 0; j < 16; ++j) cnts[j] = spre[lane * 16 + j];
+      __syncwarp();
+      for (int j = 0; j < 16; ++j) {
+        spre[lane * 16 + j] = excl;  // exclusive prefix; spre[kMaxP] = total
+        excl += cnts[j];
+      }
+      if (lane == 31) spre[kMaxP] = excl;
+      __syncwarp();
+      const int last = nb > kHotW ? nb - kHotW : 0;
+      unsigned best = 0;
+      int bs = 0x7fffffff;
+      for (int s0 = lane; s0 <= last; s0 += kWarp) {
+        const unsigned sum = spre[s0 + kHotW < kMaxP ? s0 + kHotW : kMaxP] - spre[s0];
+        if (bs == 0x7fffffff || sum > best) {
+          best = sum;
+          bs = s0;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int os = __shfl_xor_sync(0xffffffffu, bs, o);
+        if (os != 0x7fffffff && (bs == 0x7fffffff || ob > best || (ob == best && os < bs))) {
+          best = ob;
+          bs = os;
+        }
+      }
+      if (lane == 0) S.hot0 = bs == 0x7fffffff ? 0 : bs;
+    }
+    __syncthreads();
+  }
+  const int hot0 = S.hot0;
+
+  // Main pass: the float4 groups from the first 16-byte boundary, kB per
+  // thread per step with the next kB loads in flight, the counters folded every
+  // kBucketSub entries; then the head and tail entries.
+  const int head = (reinterpret_cast<uintptr_t>(x) & 3u) ? len
+                   : static_cast<int>(((16u - (reinterpret_cast<uintptr_t>(xc) & 15u)) & 15u) >> 2);
+  const int h = head < len ? head : len;
+  const int nv = (len - h) >> 2;
+  const float4* x4 = reinterpret_cast<const float4*>(xc + h);
+  constexpr int kB = 2;
+  constexpr int kStepsPerFold = kBucketSub / (4 * kBucketThreads * kB);  // steps between two folds
+  const int steps = (nv + kBucketThreads * kB - 1) / (kBucketThreads * kB);
+  unsigned long long tc[kBucketOwn] = {}, ta[kBucketOwn] = {}, tb[kBucketOwn] = {};
+  auto fold = [&]() {
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kBucketOwn; ++j) {
+      const int k = threadIdx.x + j * kBucketThreads;
+      if (k < nb) {
+        const int o = kHotW * kWarp + k;
+        tc[j] += sc[k];
+        ta[j] += static_cast<unsigned long long>(sl[o]) +
+                 (static_cast<unsigned long long>(sl[kLimbBlock + o]) << kLimbBits);
+        tb[j] += static_cast<unsigned long long>(sl[2 * kLimbBlock + o]) +
+                 (static_cast<unsigned long long>(sl[3 * kLimbBlock + o]) << kLimbBits);
+        sc[k] = sl[o] = sl[kLimbBlock + o] = sl[2 * kLimbBlock + o] = sl[3 * kLimbBlock + o] = 0u;
+      }
+    }
+    __syncthreads();
+  };
+  float4 nxt[kB];
+#pragma unroll
+  for (int u = 0; u < kB; ++u) {
+    const int i = threadIdx.x + u * kBucketThreads;
+    nxt[u] = (i < nv) ? __ldcs(x4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int st = 0; st < steps; ++st) {
+    float4 cur[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      cur[u] = nxt[u];
+      const int i = threadIdx.x + ((st + 1) * kB + u) * kBucketThreads;
+      nxt[u] = (i < nv) ? __ldcs(x4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int i = threadIdx.x + (st * kB + u) * kBucketThreads;
+      if (i < nv) {
+        const float xv[4] = {cur[u].x, cur[u].y, cur[u].z, cur[u].w};
+        int k[4];
+        double v[4];
+        unsigned okm = 0;
+        if (uni) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const double G = __dmul_rn(__dsub_rn(static_cast<double>(xv[e]), g.P0), g.invD);
+            const double kf = floor(G);
+            v[e] = __dsub_rn(G, kf);
+            k[e] = static_cast<int>(kf);
+            okm |= (fabs(v[e] - 0.5) < lim && static_cast<unsigned>(k[e]) <= pm2) ? (1u << e) : 0u;
+          }
+        }
+        if (okm == 0xFu) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) bucket_add(sc, sl, k[e], v[e], hot0, lane, twoF, twoH);
+        } else {
+          bucket_exact(&S, xv, 4);
+        }
+      }
+    }
+    if ((st + 1) % kStepsPerFold == 0) fold();
+  }
+  // head and tail entries (fewer than 4 + 4), one per thread
+  {
+    const int tail0 = h + 4 * nv;
+    if (threadIdx.x < h || (threadIdx.x >= 4 && threadIdx.x - 4 + tail0 < len)) {
+      const int i = threadIdx.x < h ? threadIdx.x : tail0 + threadIdx.x - 4;
+      const float xv[1] = {__ldcs(xc + i)};
+      bucket_exact(&S, xv, 1);
     }
   }
-  if (threadIdx.x == 0 && s_bad) atomicOr(flag + r, 1);
+  fold();
+  unsigned long long* gacc = acc + static_cast<int64_t>(r) * nb * 3;
+#pragma unroll
+  for (int j = 0; j < kBucketOwn; ++j) {
+    const int k = threadIdx.x + j * kBucketThreads;
+    if (k < nb) {
+      if (tc[j]) atomicAdd(gacc + 3 * k + 0, tc[j]);
+      if (ta[j]) atomicAdd(gacc + 3 * k + 1, ta[j]);
+      if (tb[j]) atomicAdd(gacc + 3 * k + 2, tb[j]);
+    }
+  }
+  // lane counters of the hot buckets: one (limb, bucket) sum over the lanes per thread
+  for (int q = threadIdx.x; q < 4 * kHotW; q += blockDim.x) {
+    const int li = q / kHotW, j = q - li * kHotW, k = hot0 + j;
+    if (k >= nb) continue;
+    const unsigned int* c = sl + li * kLimbBlock + j * kWarp;
+    unsigned long long sum = 0;
+#pragma unroll 8
+    for (int l = 0; l < kWarp; ++l) sum += c[(l + lane) & (kWarp - 1)];
+    if (sum) atomicAdd(gacc + 3 * k + 1 + (li >> 1), sum << ((li & 1) ? kLimbBits : 0));
+  }
+  if (threadIdx.x == 0 && S.bad) atomicOr(flag + r, 1);
 }
 
-// Fixed-point accumulators -> cnt (int64), A = sum y, B = sum y^2 (fp64).
+// Fixed-point row sums -> cnt (int64), A = sum (x - P_k), B = sum (x - P_k)^2 (fp64).
 __global__ void k_bucket_finish(const unsigned long long* __restrict__ acc, const double* __restrict__ Pall,
                                 int p, int fb, const int32_t* __restrict__ flag, int64_t* __restrict__ cnt,
                                 double* __restrict__ A, double* __restrict__ B, int32_t* __restrict__ status) {
   const int r = blockIdx.x;
   const int nb = p - 1;
   const double* P = Pall + static_cast<int64_t>(r) * p;
-  const unsigned long long* g = acc + static_cast<int64_t>(r) * nb * 3;
+  const unsigned long long* gs = acc + static_cast<int64_t>(r) * nb * 3;
   const double inv_two_fb = ldexp(1.0, -fb);
+  const RowGrid g = row_grid(P, p);
+  const bool uni = row_is_uniform(P, p, g, nullptr);
   for (int k = threadIdx.x; k < nb; k += blockDim.x) {
-    const double D = P[k + 1] - P[k];
     const int64_t o = static_cast<int64_t>(r) * nb + k;
-    cnt[o] = static_cast<int64_t>(g[3 * k + 0]);
-    A[o] = static_cast<double>(g[3 * k + 1]) * inv_two_fb * D;
-    B[o] = static_cast<double>(g[3 * k + 2]) * inv_two_fb * D * D;
+    const double c = static_cast<double>(gs[3 * k + 0]);
+    const double S1 = static_cast<double>(gs[3 * k + 1]) * inv_two_fb;
+    const double S2 = static_cast<double>(gs[3 * k + 2]) * inv_two_fb;
+    cnt[o] = static_cast<int64_t>(gs[3 * k + 0]);
+    if (uni) {
+      const double e = grid_eta(P[k], g.P0, g.invD, k);
+      A[o] = g.D * (S1 - c * e);
+      B[o] = g.D * g.D * (S2 - 2.0 * e * S1 + c * e * e);
+    } else {
+      const double w = P[k + 1] - P[k];
+      A[o] = S1 * w;
+      B[o] = S2 * w * w;
+    }
   }
   if (threadIdx.x == 0 && status) status[r] = flag[r] ? kStatusRange : kStatusOk;
 }
 
 }  // namespace
 
-int bucket_fraction_bits(int64_t d) {
-  (void)d;
-  return kFixBits;
-}
+int bucket_fraction_bits(int64_t d) { return d < (int64_t(1) << 27) ? 36 : 32; }
 
 int64_t minmax_chunk(int64_t d) { return d < 16384 ? d : 16384; }
 
@@ -342,9 +600,12 @@ cudaError_t launch_uniform_grid(const float* X, int n, int64_t d, int p, double*
   return cudaGetLastError();
 }
 
-size_t bucket_smem_bytes(int p) { return static_cast<size_t>(p) * (8 * 2 + 4 * 5 + 4); }
+size_t bucket_smem_bytes(int p) { return static_cast<size_t>(p) * (8 * 2 + 4); }
 
-int64_t bucket_chunk(int64_t d) { return d < kBucketChunk ? d : kBucketChunk; }
+int64_t bucket_chunk(int64_t d) {
+  const int64_t c = static_cast<int64_t>(kBucketSub) * kBucketSubsPerCta;
+  return d < c ? d : c;
+}
 
 cudaError_t launch_bucket(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt,
                           double* A, double* B, int32_t* status, unsigned long long* acc,
@@ -354,19 +615,10 @@ cudaError_t launch_bucket(const float* X, const double* P, int n, int64_t d, int
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(flag, 0, sizeof(int32_t) * n, st);
   if (e != cudaSuccess) return e;
-  const int64_t chunk = bucket_chunk(d);
+  const int64_t chunk = static_cast<int64_t>(kBucketSub) * kBucketSubsPerCta;
   const int nc = static_cast<int>((d + chunk - 1) / chunk);
-  const size_t smem = bucket_smem_bytes(p);
-  // the attribute is per device: set it once for each device this process uses
-  static bool attr_set[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    cudaError_t ea = cudaFuncSetAttribute(k_bucket, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
-    if (ea != cudaSuccess) return ea;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
-  }
-  k_bucket<<<dim3(nc, n), kBucketThreads, smem, st>>>(X, d, chunk, P, p, fb, acc, flag);
+  // 37 KB of static and at most 10 KB of dynamic shared memory (p = 512): no attribute needed
+  k_bucket<<<dim3(nc, n), kBucketThreads, bucket_smem_bytes(p), st>>>(X, d, P, p, fb, acc, flag);
   note_launch();
   k_bucket_finish<<<n, 256, 0, st>>>(acc, P, p, fb, flag, cnt, A, B, status);
   note_launch();
