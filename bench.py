@@ -33,13 +33,14 @@ sys.path.insert(0, ROOT)
 from entropy_constrained_unbiased_b200 import workloads as W  # noqa: E402
 
 MUFU_LG2_PER_CLK_PER_SM = 16  # special-function unit results per clock per SM (sm_100)
+METRIC = "ECASQ DP (k,l,j) triples/s"  # the same string in both arms
 B200_SMS = 148
 
-# DRAM bytes (read + write) per k_dp launch per row, from the ncu capture
-# summarised in profiles/k_dp_weights_296rows_full.md (296 rows: 1.71 MB read,
-# 1411 MB written, almost all of it the stored DP layers written back from L2),
-# scaled by the rows of a launch. The figure belongs to the kernel source it was
-# taken on; it is dropped (null) when that source has changed since.
+# DRAM bytes (read + write) per k_dp launch per row, from one ncu capture of
+# k_dp on the first 296 rows of the weights workload (1.71 MB read, 1411 MB
+# written, almost all of it the stored DP layers written back from L2), scaled
+# by the rows of a launch. The figure belongs to the kernel source it was taken
+# on; it is dropped (null) when that source has changed since.
 DP_TRAFFIC = {"weights": {"bytes_per_row": (1708544 + 1410748672) / 296, "dp_source_sha1": "ba90d42feb4558bf"}}
 
 
@@ -277,13 +278,12 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
         enc_args = (out["Q1"], out["Q1_len"], w.seed_encode, out["Q2"], out["Q2_len"], out["theta"])
     else:
         enc_args = (out["Q"][:, 0, :].contiguous(), out["Q_len"][:, 0].contiguous(), w.seed_encode)
-    stage_fns = {"grid": lambda: E.uniform_grid(X, p), "bucket": lambda: E.bucket(X, P_last),
-                 "encode": lambda: E.encode(X, P_last, s, *enc_args)}
-    for name, bpe in (("grid", 4), ("bucket", 4), ("encode", 5)):
-        ms = device_ms(stage_fns[name], stream, flush)
-        gbs = entries * bpe / (ms * 1e-3) / 1e9
-        hbm_kernels[name] = {"ms": ms, "bytes_per_entry": bpe, "achieved_GBps": gbs, "peak_GBps": hbm,
-                             "frac": gbs / hbm, "entries_per_s": entries / (ms * 1e-3)}
+    hbm_kernels.update(stage_figures(E, X, P_last, p, s, enc_args, stream, flush, hbm))
+    hbm_kernels["input"] = f"this workload ({n} x {d})"
+    # The HBM-bound stages on the gradients input (256 x 2^20 fp32 = 1 GiB,
+    # larger than L2), with codes from the exact budget solver on it.
+    if w.name != "gradients" and not args.no_gradients_stages:
+        hbm_kernels["gradients_input"] = gradients_stage_figures(E, dev, stream, flush, hbm, rank)
     # hardware-aware alphabet (BF16 values covering each row), p_max = 512: one
     # read of X plus the alphabet rows written
     E.bf16_alphabet(X, 512)
@@ -326,9 +326,10 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
     achieved = n_solves * tps / (dp_avg_ms * 1e-3)
     total_triples = world * n_solves * tps  # one step, all ranks
     value = total_triples * args.steps / (t_ms * 1e-3)
-    approx = approx_timing(args, w, X, stream, flush, dp_avg_ms, sm_max)
+    approx, approx_outs = approx_timing(args, w, X, stream, flush, dp_avg_ms, sm_max)
+    approx["vnmse"] = vnmse_report(w, X, out, approx_outs)
     line = {
-        "metric": "ECASQ DP (k,l,j) triples/s (whole step: grid + bucketing + DP + bisection + encode + entropy)",
+        "metric": METRIC,
         "value": value,
         "unit": "triples/s",
         "n_gpus": world,
@@ -341,6 +342,7 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
         "dtype": "f64" if fp64 else "f32",
         "data": "synthetic",
         "config": {"workload": describe(w), "n": n, "d": d, "p": p, "s": s, "l2": "flushed between steps",
+                   "step": "uniform grid + bucketing + DP solves (bisection + time-sharing) + encode + entropy",
                    "dp_solves_per_step": n_solves, "triples_per_solve": tps,
                    "entries_per_s": world * n * d / (t_ms * 1e-3 / args.steps),
                    "parallelism": f"dp{world} (rows sharded, no collective)"},
@@ -359,6 +361,80 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
         "clocks": clk.summary(),
     }
     return line
+
+
+def stage_figures(E, X, P, p, s, enc_args, stream, flush, hbm):
+    """Device time of the uniform grid (min/max pass + grid), bucketing and
+    encoding, each call alone after an L2 flush; algorithmic bytes: 4 B/entry
+    read for the grid and for bucketing, 4 B read + 1 B written for encoding
+    (the histograms are fused)."""
+    entries = X.numel()
+    fns = {"grid": lambda: E.uniform_grid(X, p), "bucket": lambda: E.bucket(X, P),
+           "encode": lambda: E.encode(X, P, s, *enc_args)}
+    out = {}
+    for name, bpe in (("grid", 4), ("bucket", 4), ("encode", 5)):
+        fns[name]()
+        ms = device_ms(fns[name], stream, flush)
+        gbs = entries * bpe / (ms * 1e-3) / 1e9
+        out[name] = {"ms": ms, "bytes_per_entry": bpe, "achieved_GBps": gbs, "peak_GBps": hbm,
+                     "frac": gbs / hbm, "entries_per_s": entries / (ms * 1e-3)}
+    return out
+
+
+def gradients_stage_figures(E, dev, stream, flush, hbm, rank):
+    import torch
+
+    g = W.WORKLOADS["gradients"]
+    X = torch.from_numpy(W.make_inputs(g, rank=rank)).to(dev)
+    P, _ = E.uniform_grid(X, g.p)
+    cnt, A, B, _ = E.bucket(X, P)
+    o = E.solve_budget_stats(cnt, A, B, P, g.d, g.s, g.b, g.steps)
+    del cnt, A, B
+    enc = (o["Q1"], o["Q1_len"], g.seed_encode, o["Q2"], o["Q2_len"], o["theta"])
+    res = stage_figures(E, X, P, g.p, g.s, enc, stream, flush, hbm)
+    res["input"] = f"gradients: {g.n} x {g.d} fp32, p={g.p}, s={g.s}, codes of the b={g.b} budget solve"
+    del X, P, o
+    torch.cuda.empty_cache()
+    return res
+
+
+def vnmse_report(w: W.Workload, X, exact, approx_out):
+    """vNMSE = E||X^ - X||^2 / ||X||^2 per row (§4 "Precisão" reports the mean
+    excess of the approximation and of its refinement over the optimum). Budget
+    workloads compare the time-shared MSE at the same budget b; the exact and
+    refined solvers constrain H(X^), the plain approximation H(I,B)."""
+    import torch
+
+    nx = X.double().pow(2).sum(dim=1)
+    d = X.shape[1]
+
+    def ts(o):
+        if w.mode == "budget":
+            th = o["theta"]
+            return (th * o["mse1"] + (1.0 - th) * o["mse2"]) * d / nx
+        return o["mse"][:, 0] * d / nx
+
+    def rate(o):  # time-shared H(X^), bits per entry
+        if w.mode == "budget":
+            th = o["theta"]
+            return th * o["H1"] + (1.0 - th) * o["H2"]
+        return o["H"][:, 0]
+
+    ve = ts(exact)
+    ok = torch.isfinite(ve) & (ve > 0)
+    res = {"definition": "d * MSE / ||x||^2 per row, mean over rows; rate_H = time-shared H(X^) in bits/entry",
+           "exact": float(ve[ok].mean().item()), "exact_rate_H": float(rate(exact)[ok].mean().item())}
+    for key, o in approx_out.items():
+        va = ts(o)
+        res[key] = float(va[ok].mean().item())
+        res[f"{key}_rate_H"] = float(rate(o)[ok].mean().item())
+        if w.mode == "budget":
+            res[f"excess_{key}_over_exact"] = float((va[ok] / ve[ok] - 1.0).mean().item())
+    if w.mode == "budget":
+        res["note"] = ("at the same budget b the plain approximation constrains H(I,B) <= b, which leaves "
+                       "H(X^) lower (H(I,B) <= H(X^) + 1); the refined one constrains H(X^) like the exact solver")
+    res["pages_context"] = "mean excess 4.97% (approximation) and 1.37% (refined) on the pages' own inputs"
+    return res
 
 
 def approx_timing(args, w: W.Workload, X, stream, flush, dp_avg_ms: float, sm_max: float):
@@ -386,8 +462,10 @@ def approx_timing(args, w: W.Workload, X, stream, flush, dp_avg_ms: float, sm_ma
             return E.solve_approx_budget_stats(cnt, A, B, P, w.d, w.s, w.b, refine=refine, steps=w.steps, fp64=fp64)
         return E.solve_approx_stats(cnt, A, B, P, w.d, w.s, lam, refine=refine, fp64=fp64)
 
+    outs = {}
     for refine in (0, 8):
         out = call(refine)  # warm-up
+        outs["approx" if refine == 0 else "refined8"] = out
         torch.cuda.synchronize()
         t = device_ms(lambda: call(refine), stream, flush, reps=max(2, min(args.steps, 3)))
         ns = solves_done(w, out)
@@ -395,7 +473,7 @@ def approx_timing(args, w: W.Workload, X, stream, flush, dp_avg_ms: float, sm_ma
         res[f"refine{refine}"] = {"ms": t, "solves": ns, "achieved": ach, "frac": ach / peak,
                                   "speedup_vs_exact_dp": dp_avg_ms / t,
                                   "status_nonzero_rows": int((out["status"] != 0).sum().item())}
-    return res
+    return res, outs
 
 
 def measure_unit_peaks():
@@ -460,11 +538,12 @@ def run_reference(args, w: W.Workload, rank: int, world: int):
     v = float(np.mean([x["value"] for x in vals]))
     cb = dict(vals[-1])
     cb["value"] = v
-    return {"impl": "reference", "metric": "ECASQ DP (k,l,j) triples/s (fp64 CPU oracle, row sample)",
+    return {"impl": "reference", "metric": METRIC,
             "value": v, "unit": "triples/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": wall * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": describe(w), "n": w.n, "d": w.d, "p": w.p, "s": w.s},
+            "config": {"workload": describe(w), "n": w.n, "d": w.d, "p": w.p, "s": w.s,
+                       "step": "fp64 CPU oracle on a row sample: grid + bucketing + DP solves"},
             "cpu_baseline": cb,
             "e2e": {"value": v, "unit": "triples/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -479,6 +558,8 @@ def main():
     ap.add_argument("--fp64", action="store_true", help="fp64 DP layers (parity mode)")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-gradients-stages", action="store_true",
+                    help="skip the grid/bucketing/encoding figures on the 1 GiB gradients input")
     ap.add_argument("--rows", type=int, default=0, help="first rows only (profiling runs; not a bench line)")
     args = ap.parse_args()
     w = W.WORKLOADS[args.workload]

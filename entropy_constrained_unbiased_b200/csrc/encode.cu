@@ -89,14 +89,14 @@ __device__ __noinline__ uint32_t enc_fix(EncRow* S, const float* xv, const uint3
 // interval and w' = (q_{t+1} - q_t) 2^-32; with u = word 2^-32 (both scalings
 // exact) u (q_{t+1} - q_t) = word w' as real numbers, so the product is
 // taken as word * w' in one rounding.
-__global__ void __launch_bounds__(kEncThreads)
-k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d, int p, int s,
-         const int32_t* __restrict__ Q1, const int32_t* __restrict__ Q1_len, const int32_t* __restrict__ Q2,
-         const int32_t* __restrict__ Q2_len, const double* __restrict__ theta, const Philox4x32::RoundKeys K,
-         uint8_t* __restrict__ idx, unsigned long long* __restrict__ hist, int32_t* __restrict__ status) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ EncRow S;
-  __shared__ int s_wexact;
+template <bool kMix>
+__device__ __forceinline__ void encode_row(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d,
+                                           int p, int s, const int32_t* __restrict__ Q1,
+                                           const int32_t* __restrict__ Q1_len, const int32_t* __restrict__ Q2,
+                                           const int32_t* __restrict__ Q2_len, const double* __restrict__ theta,
+                                           const Philox4x32::RoundKeys& K, uint8_t* __restrict__ idx,
+                                           unsigned long long* __restrict__ hist, int32_t* __restrict__ status,
+                                           unsigned char* smem, EncRow& S, int& s_wexact) {
   const int r = blockIdx.y;
   const int nbins = 2 * s + 1;
   double2* sR = reinterpret_cast<double2*>(smem);                          // [2][p] (q_t, w') per bucket
@@ -230,7 +230,7 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
       const uint32_t blk = blk0 + static_cast<uint32_t>(f);
       const uint4 ru = Philox4x32::block(make_uint4(blk, static_cast<uint32_t>(r), 0u, 0u), rk);
       uint4 su = make_uint4(0u, 0u, 0u, 0u);
-      if (mix) su = Philox4x32::block(make_uint4(blk, static_cast<uint32_t>(r), 1u, 0u), rk);
+      if (kMix) su = Philox4x32::block(make_uint4(blk, static_cast<uint32_t>(r), 1u, 0u), rk);
       const uint32_t rw[4] = {ru.x, ru.y, ru.z, ru.w};
       const uint32_t sel[4] = {su.x, su.y, su.z, su.w};
       int part[4];
@@ -238,7 +238,7 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
       unsigned okm = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        part[e] = mix ? (sel[e] <= th_last ? 0 : 1) : fixed_part;
+        part[e] = kMix ? (sel[e] <= th_last ? 0 : 1) : fixed_part;
         const float gf = fmaf(xv[e], s_f, c_f);
         const float kf = floorf(gf);
         const int k = static_cast<int>(kf);
@@ -285,6 +285,23 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
     if (tot) atomicAdd(gh + b, tot);
   }
   if (threadIdx.x == 0 && S.bad) status[r] = kStatusRange;
+}
+
+// One CTA per (row, chunk of kEncChunk entries); rows coded with two codes
+// (0 < theta < 1) and rows coded with one take separate specialisations.
+__global__ void __launch_bounds__(kEncThreads)
+k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d, int p, int s,
+         const int32_t* __restrict__ Q1, const int32_t* __restrict__ Q1_len, const int32_t* __restrict__ Q2,
+         const int32_t* __restrict__ Q2_len, const double* __restrict__ theta, const Philox4x32::RoundKeys K,
+         uint8_t* __restrict__ idx, unsigned long long* __restrict__ hist, int32_t* __restrict__ status) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ EncRow S;
+  __shared__ int s_wexact;
+  const double th = (Q2 != nullptr && theta) ? theta[blockIdx.y] : 0.0;
+  if (Q2 != nullptr && th > 0.0 && th < 1.0)
+    encode_row<true>(X, Pall, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, idx, hist, status, smem, S, s_wexact);
+  else
+    encode_row<false>(X, Pall, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, idx, hist, status, smem, S, s_wexact);
 }
 
 // H = (d0 H0 + d1 H1)/(d0 + d1), H_part = -sum c/d_part log2(c/d_part). One warp per row.

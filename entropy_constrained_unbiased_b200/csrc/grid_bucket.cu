@@ -186,41 +186,7 @@ __global__ void k_bf16_finish(const float* __restrict__ part, int n_chunks, int 
 }
 
 // ---------------------------------------------------------------------------
-// Bucketing (the "+d" pass of §2.2 "Generalização"). An entry x of bucket k
-// (P_k <= x < P_{k+1}; the last bucket closed) contributes a normalised offset
-// v in [0, 1], kept as fixed point: round(v 2^F) and round(v^2 2^F) with F = 36
-// fraction bits (32 for rows of 2^27 entries or more, so that the 64-bit row
-// sums cannot overflow). Integer sums make the result independent of the order
-// of addition. The finish kernel turns them back into A_k = sum (x - P_k) and
-// B_k = sum (x - P_k)^2.
-//
-// Two ways to find k and v:
-//  * uniform rows: P_k = P_0 + (k + eta_k) D with D = (P_{p-1} - P_0)/(p-1)
-//    and |eta_k| <= 2^-36 for every k (an fp64 uniform grid qualifies unless
-//    |P_0| is very large against the span). G = (x - P_0)/D in fp64 is within
-//    2^-41 bucket widths of its exact value (p <= 512), so when
-//    v = G - floor(G) lies more than 2^-20 from 0 and from 1, k = floor(G) is
-//    the entry's bucket for certain and v = (x - P_k)/D + eta_k up to that
-//    error: no shared-memory lookup at all. The few entries within 2^-20 of a
-//    grid point take the exact search and v = clamp((x - P_k)/D + eta_k, 0, 1),
-//    the clamp moving v by at most |eta_k|. Then A_k = D (S1 - n_k eta_k) and
-//    B_k = D^2 (S2 - 2 eta_k S1 + n_k eta_k^2) with S1 = sum v, S2 = sum v^2.
-//  * other rows: k by the exact search on P, v = (x - P_k)/D_k, A_k = D_k S1,
-//    B_k = D_k^2 S2.
-//
-// Accumulation: 32-bit shared-memory counters, added by return-less atomics:
-// per entry the count (an increment, which the hardware combines across lanes
-// that hit the same counter) and two limbs of each moment (bits 0..17 and
-// 18..F). Additions of different values to one address by lanes of a warp are
-// serialised, and real data concentrates in a few buckets, so the limbs of
-// the kHotW busiest consecutive buckets (chosen from the counts of the CTA's
-// first 8192 entries) get one counter per lane, laid out [bucket][lane] so
-// that the 32 lanes of a warp always fall on 32 distinct banks; the other
-// buckets share one counter per bucket. Shared counters are folded into 64-bit
-// registers of the bucket's owner thread every 8192 entries (8192 limbs of at
-// most 2^18 stay below 2^32); a lane counter receives at most 2048 entries per
-// CTA and is summed once at the end. Each CTA adds its totals to the row's
-// 64-bit sums in global memory.
+// Bucketing: constants and the per-CTA state shared by the kernels below.
 
 constexpr int kBucketThreads = 256;
 constexpr int kBucketSub = 8192;          // entries between two folds of the shared counters
@@ -230,6 +196,11 @@ constexpr int kHotW = 48;                 // buckets with one counter per lane
 constexpr int kLimbBlock = kHotW * kWarp + kMaxP;  // words per limb: [kHotW][32] lane counters, then [kMaxP]
 constexpr int kLimbBits = 18;
 constexpr double kFastEps = 0x1p-20;      // distance of v from a grid point on the fast path
+// The fast path evaluates G = (x - P_0)/D as fma(x, 1/D, -P_0/D); the rounding
+// of -P_0/D and of 1/D then move G by at most (2|P_0/D| + p) 2^-53, below 2^-37
+// bucket widths for |P_0/D| <= 2^15 (rows straddling zero have |P_0/D| <= p). Rows beyond
+// that take the exact search for every entry.
+constexpr double kFmaOffsetMax = 0x1p15;
 
 // Per-CTA state of the bucketing kernel in shared memory.
 struct BucketRow {
@@ -294,8 +265,9 @@ __device__ __noinline__ void bucket_exact(BucketRow* S, const float* xv, int cnt
 // Two ways to find k and v:
 //  * uniform rows: P_k = P_0 + (k + eta_k) D with D = (P_{p-1} - P_0)/(p-1)
 //    and |eta_k| <= 2^-36 for every k (an fp64 uniform grid qualifies unless
-//    |P_0| is very large against the span). G = (x - P_0)/D in fp64 is within
-//    2^-41 bucket widths of its exact value (p <= 512), so when
+//    |P_0| is very large against the span). G = (x - P_0)/D, evaluated in fp64
+//    as fma(x, 1/D, -P_0/D), is within 2^-37 bucket widths of its exact value
+//    (p <= 512, |P_0/D| <= 2^15), so when
 //    v = G - floor(G) lies more than 2^-20 from 0 and from 1, k = floor(G) is
 //    the entry's bucket for certain and v = (x - P_k)/D + eta_k up to that
 //    error: no shared-memory lookup at all. Groups of four entries holding one
@@ -370,6 +342,8 @@ k_bucket(const float* __restrict__ X, int64_t d, const double* __restrict__ Pall
   const int lane = lane_id();
   const unsigned pm2 = static_cast<unsigned>(p - 2);
   const double lim = 0.5 - kFastEps;
+  const double c0 = -(g.P0 * g.invD);
+  const bool fastg = uni && fabs(c0) <= kFmaOffsetMax;
 
   const float* x = X + static_cast<int64_t>(r) * d;
   const int64_t chunk = static_cast<int64_t>(kBucketSub) * kBucketSubsPerCta;
@@ -488,18 +462,16 @@ k_bucket(const float* __restrict__ X, int64_t d, const double* __restrict__ Pall
         const float xv[4] = {cur[u].x, cur[u].y, cur[u].z, cur[u].w};
         int k[4];
         double v[4];
-        unsigned okm = 0;
-        if (uni) {
+        bool all = fastg;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const double G = __dmul_rn(__dsub_rn(static_cast<double>(xv[e]), g.P0), g.invD);
-            const double kf = floor(G);
-            v[e] = __dsub_rn(G, kf);
-            k[e] = static_cast<int>(kf);
-            okm |= (fabs(v[e] - 0.5) < lim && static_cast<unsigned>(k[e]) <= pm2) ? (1u << e) : 0u;
-          }
+        for (int e = 0; e < 4; ++e) {
+          const double G = fma(static_cast<double>(xv[e]), g.invD, c0);
+          const double kf = floor(G);
+          v[e] = __dsub_rn(G, kf);
+          k[e] = static_cast<int>(kf);
+          all = all && fabs(v[e] - 0.5) < lim && static_cast<unsigned>(k[e]) <= pm2;
         }
-        if (okm == 0xFu) {
+        if (all) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) bucket_add(sc, sl, k[e], v[e], hot0, lane, twoF, twoH);
         } else {
@@ -540,6 +512,240 @@ k_bucket(const float* __restrict__ X, int64_t d, const double* __restrict__ Pall
     if (sum) atomicAdd(gacc + 3 * k + 1 + (li >> 1), sum << ((li & 1) ? kLimbBits : 0));
   }
   if (threadIdx.x == 0 && S.bad) atomicOr(flag + r, 1);
+}
+
+// ---------------------------------------------------------------------------
+// Bucketing of long rows with small alphabets (p <= 257, d >= 2^16): the same
+// fixed point, fast path and exact fallback as k_bucket, with every bucket's
+// limbs in per-lane counters (4 limbs x 256 buckets x 32 lanes x 4 bytes = 128
+// KB of shared memory, one bank per lane), so a limb atomic never serialises
+// and its address is k * 32 + lane. One persistent CTA of 1024 threads per SM
+// walks a contiguous range of (row, 64K-entry chunk) pairs. Lane counters
+// receive at most 32 * 256 entries per 256K entries of the CTA; every 256K
+// entries, and when the row changes, each thread folds one (limb, bucket) row
+// of 32 lane counters into a 64-bit register, and at a row change the CTA
+// adds its totals to the row's sums in global memory.
+
+constexpr int kWideThreads = 1024;
+constexpr int kWideChunk = 65536;           // entries per (row, chunk) work item
+constexpr int kWideChunksPerFold = 4;       // 2^18 entries between two folds
+constexpr int kWideBuckets = 256;           // p - 1 <= 256
+constexpr int kWideLimbBlock = kWideBuckets * kWarp;
+constexpr size_t kWideSmem = sizeof(unsigned int) * (4 * kWideLimbBlock + kWideBuckets) +
+                             (sizeof(double) * 2 + sizeof(float)) * (kWideBuckets + 1);
+
+struct WideRow {
+  const double* P;
+  const double* E;
+  const float* T;
+  unsigned int* cnt;
+  unsigned int* limb;
+  double invD, twoF, twoH;
+  float top, scale;
+  int p, uni, bad;
+};
+
+__device__ __forceinline__ void wide_add(unsigned int* cnt, unsigned int* limb_lane, int k, double v, double twoF,
+                                         double twoH) {
+  const double magic = 0x1p52 + 0x1p13;
+  atomicAdd(cnt + k, 1u);
+  const double a = fma(v, twoF, magic);
+  const double t = v * twoH;
+  const double b = fma(t, t, magic);
+  unsigned int* c = limb_lane + k * kWarp;
+  atomicAdd(c, static_cast<unsigned>(__double2loint(a)) >> 14);
+  atomicAdd(c + kWideLimbBlock, static_cast<unsigned>(__double2hiint(a)) & 0x7FFFFu);
+  atomicAdd(c + 2 * kWideLimbBlock, static_cast<unsigned>(__double2loint(b)) >> 14);
+  atomicAdd(c + 3 * kWideLimbBlock, static_cast<unsigned>(__double2hiint(b)) & 0x7FFFFu);
+}
+
+__device__ __noinline__ void wide_exact(WideRow* S, const float* xv, int cnt) {
+  unsigned int* limb_lane = S->limb + lane_id();
+  for (int e = 0; e < cnt; ++e) {
+    const float xf = xv[e];
+    const int k = bucket_f32(xf, S->T, S->top, S->p, S->scale);
+    if (k < 0) {
+      S->bad = 1;
+      continue;
+    }
+    const double y = __dsub_rn(static_cast<double>(xf), S->P[k]);
+    const double w = S->uni ? __dadd_rn(__dmul_rn(y, S->invD), S->E[k]) : __dmul_rn(y, S->E[k]);
+    wide_add(S->cnt, limb_lane, k, fmin(fmax(w, 0.0), 1.0), S->twoF, S->twoH);
+  }
+}
+
+__global__ void __launch_bounds__(kWideThreads, 1)
+k_bucket_wide(const float* __restrict__ X, int n, int64_t d, const double* __restrict__ Pall, int p, int fb,
+              unsigned long long* __restrict__ acc, int32_t* __restrict__ flag) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ WideRow S;
+  unsigned int* sl = reinterpret_cast<unsigned int*>(smem);          // [4][256][32] lane counters
+  unsigned int* sc = sl + 4 * kWideLimbBlock;                        // [256] counts
+  double* sP = reinterpret_cast<double*>(sc + kWideBuckets);         // [p]
+  double* sE = sP + (kWideBuckets + 1);                              // [p]
+  float* sT = reinterpret_cast<float*>(sE + (kWideBuckets + 1));     // [p]
+  const int nb = p - 1;
+  const int lane = lane_id();
+  const int tid = threadIdx.x;
+  const double twoF = ldexp(1.0, fb + 14), twoH = ldexp(1.0, (fb + 14) / 2);
+  const unsigned pm2 = static_cast<unsigned>(p - 2);
+  const double lim = 0.5 - kFastEps;
+  // the (limb, bucket) row of 32 lane counters this thread folds
+  const int fl = tid / kWideBuckets, fk = tid % kWideBuckets;
+  unsigned long long facc = 0, fcnt = 0;
+
+  for (int k = tid; k < 4 * kWideLimbBlock; k += kWideThreads) sl[k] = 0u;
+  for (int k = tid; k < kWideBuckets; k += kWideThreads) sc[k] = 0u;
+
+  const int64_t cpr = (d + kWideChunk - 1) / kWideChunk;  // chunks per row
+  const int64_t Q = static_cast<int64_t>(n) * cpr;
+  const int64_t q0 = Q * blockIdx.x / gridDim.x, q1 = Q * (blockIdx.x + 1) / gridDim.x;
+  int row = -1;
+  RowGrid g{};
+  bool uni = false, fastg = false;
+  double c0 = 0.0;
+  int since_fold = 0;
+
+  // fold the lane counters and counts into registers (all threads)
+  auto fold = [&]() {
+    __syncthreads();
+    uint4* c4 = reinterpret_cast<uint4*>(sl + fl * kWideLimbBlock + fk * kWarp);
+    unsigned long long sum = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int jj = (j + tid) & 7;  // rotate the 16-byte column: threads of a quarter-warp on distinct banks
+      const uint4 v = c4[jj];
+      sum += static_cast<unsigned long long>(v.x) + v.y + v.z + v.w;
+      c4[jj] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    facc += sum;
+    if (fl == 0) {
+      fcnt += sc[fk];
+      sc[fk] = 0u;
+    }
+    __syncthreads();
+  };
+  // add the folded totals of `row` to its global sums
+  auto flush = [&]() {
+    if (fk < nb) {
+      unsigned long long* gacc = acc + (static_cast<int64_t>(row) * nb + fk) * 3;
+      if (facc) atomicAdd(gacc + 1 + (fl >> 1), facc << ((fl & 1) ? kLimbBits : 0));
+      if (fl == 0 && fcnt) atomicAdd(gacc, fcnt);
+    }
+    facc = 0;
+    fcnt = 0;
+    if (tid == 0 && S.bad) atomicOr(flag + row, 1);
+  };
+
+  for (int64_t q = q0; q < q1; ++q) {
+    const int r = static_cast<int>(q / cpr);
+    const int64_t ci = q - static_cast<int64_t>(r) * cpr;
+    if (r != row) {
+      if (row >= 0) {
+        fold();
+        flush();
+        since_fold = 0;
+      }
+      __syncthreads();
+      row = r;
+      const double* P = Pall + static_cast<int64_t>(r) * p;
+      for (int k = tid; k < p; k += kWideThreads) {
+        sP[k] = P[k];
+        sT[k] = __double2float_ru(P[k]);
+      }
+      __syncthreads();
+      g = row_grid(sP, p);
+      uni = row_is_uniform(sP, p, g, sE);  // includes a barrier
+      c0 = -(g.P0 * g.invD);
+      fastg = uni && fabs(c0) <= kFmaOffsetMax;
+      if (!uni) {
+        for (int k = tid; k < nb; k += kWideThreads) {
+          const double w = __dsub_rn(sP[k + 1], sP[k]);
+          sE[k] = w > 0.0 ? __ddiv_rn(1.0, w) : 0.0;
+        }
+      }
+      if (tid == 0) {
+        S.P = sP;
+        S.E = sE;
+        S.T = sT;
+        S.cnt = sc;
+        S.limb = sl;
+        S.invD = g.invD;
+        S.twoF = twoF;
+        S.twoH = twoH;
+        S.top = __double2float_rd(sP[p - 1]);
+        S.scale = static_cast<float>(static_cast<double>(p - 1) / (sP[p - 1] - sP[0]));
+        S.p = p;
+        S.uni = uni;
+        S.bad = 0;
+      }
+      __syncthreads();
+    }
+    const float* xc = X + static_cast<int64_t>(r) * d + ci * kWideChunk;
+    const int len = static_cast<int>((ci + 1) * kWideChunk < d ? kWideChunk : d - ci * kWideChunk);
+    const int head = (reinterpret_cast<uintptr_t>(X + static_cast<int64_t>(r) * d) & 3u)
+                         ? len
+                         : static_cast<int>(((16u - (reinterpret_cast<uintptr_t>(xc) & 15u)) & 15u) >> 2);
+    const int h = head < len ? head : len;
+    const int nv = (len - h) >> 2;
+    const float4* x4 = reinterpret_cast<const float4*>(xc + h);
+    unsigned int* limb_lane = sl + lane;
+    constexpr int kB = 2;
+    float4 nxt[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int i = tid + u * kWideThreads;
+      nxt[u] = (i < nv) ? __ldcs(x4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int i0 = 0; i0 < nv; i0 += kB * kWideThreads) {
+      float4 cur[kB];
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        cur[u] = nxt[u];
+        const int i = i0 + tid + (kB + u) * kWideThreads;
+        nxt[u] = (i < nv) ? __ldcs(x4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        if (i0 + tid + u * kWideThreads < nv) {
+          const float xv[4] = {cur[u].x, cur[u].y, cur[u].z, cur[u].w};
+          int k[4];
+          double v[4];
+          bool all = fastg;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const double G = fma(static_cast<double>(xv[e]), g.invD, c0);
+            const double kf = floor(G);
+            v[e] = __dsub_rn(G, kf);
+            k[e] = static_cast<int>(kf);
+            all = all && fabs(v[e] - 0.5) < lim && static_cast<unsigned>(k[e]) <= pm2;
+          }
+          if (all) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) wide_add(sc, limb_lane, k[e], v[e], twoF, twoH);
+          } else {
+            wide_exact(&S, xv, 4);
+          }
+        }
+      }
+    }
+    {
+      const int tail0 = h + 4 * nv;
+      if (tid < h || (tid >= 4 && tid - 4 + tail0 < len)) {
+        const int i = tid < h ? tid : tail0 + tid - 4;
+        const float xv[1] = {__ldcs(xc + i)};
+        wide_exact(&S, xv, 1);
+      }
+    }
+    if (++since_fold == kWideChunksPerFold) {
+      fold();
+      since_fold = 0;
+    }
+  }
+  if (row >= 0) {
+    fold();
+    flush();
+  }
 }
 
 // Fixed-point row sums -> cnt (int64), A = sum (x - P_k), B = sum (x - P_k)^2 (fp64).
@@ -607,6 +813,19 @@ int64_t bucket_chunk(int64_t d) {
   return d < c ? d : c;
 }
 
+// The wide kernel needs more than the default 48 KB of dynamic shared memory;
+// the attribute is per device and is set once for each (thread-safe).
+cudaError_t wide_smem_attribute(int dev) {
+  static std::once_flag once[64];
+  static cudaError_t result[64];
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::call_once(once[dev], [dev]() {
+    result[dev] = cudaFuncSetAttribute(k_bucket_wide, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kWideSmem));
+  });
+  return result[dev];
+}
+
 cudaError_t launch_bucket(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt,
                           double* A, double* B, int32_t* status, unsigned long long* acc,
                           int32_t* flag, cudaStream_t st) {
@@ -615,10 +834,22 @@ cudaError_t launch_bucket(const float* X, const double* P, int n, int64_t d, int
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(flag, 0, sizeof(int32_t) * n, st);
   if (e != cudaSuccess) return e;
-  const int64_t chunk = static_cast<int64_t>(kBucketSub) * kBucketSubsPerCta;
-  const int nc = static_cast<int>((d + chunk - 1) / chunk);
-  // 37 KB of static and at most 10 KB of dynamic shared memory (p = 512): no attribute needed
-  k_bucket<<<dim3(nc, n), kBucketThreads, bucket_smem_bytes(p), st>>>(X, d, P, p, fb, acc, flag);
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int64_t wide_items = static_cast<int64_t>(n) * ((d + kWideChunk - 1) / kWideChunk);
+  if (p - 1 <= kWideBuckets && d >= kWideChunk && wide_items >= sms) {
+    e = wide_smem_attribute(dev);
+    if (e != cudaSuccess) return e;
+    k_bucket_wide<<<sms, kWideThreads, kWideSmem, st>>>(X, n, d, P, p, fb, acc, flag);
+  } else {
+    const int64_t chunk = static_cast<int64_t>(kBucketSub) * kBucketSubsPerCta;
+    const int nc = static_cast<int>((d + chunk - 1) / chunk);
+    // 37 KB of static and at most 10 KB of dynamic shared memory (p = 512): no attribute needed
+    k_bucket<<<dim3(nc, n), kBucketThreads, bucket_smem_bytes(p), st>>>(X, d, P, p, fb, acc, flag);
+  }
   note_launch();
   k_bucket_finish<<<n, 256, 0, st>>>(acc, P, p, fb, flag, cnt, A, B, status);
   note_launch();
