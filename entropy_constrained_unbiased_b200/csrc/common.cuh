@@ -98,6 +98,21 @@ __device__ __forceinline__ void warp_argmin(T& v, int& i) {
   }
 }
 
+// Return-less 32-bit additions to shared memory through 32-bit shared-window
+// addresses (red.shared.add.u32), with a compile-time byte offset.
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+template <int kOff = 0>
+__device__ __forceinline__ void red_shared_add(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared.add.u32 [%0+%2], %1;" ::"r"(addr), "r"(v), "n"(kOff) : "memory");
+}
+// +1: the hardware combines the lanes of a warp that hit the same counter.
+template <int kOff = 0>
+__device__ __forceinline__ void red_shared_inc(uint32_t addr) {
+  asm volatile("red.shared.add.u32 [%0+%1], 1;" ::"r"(addr), "n"(kOff) : "memory");
+}
+
 // Triangle addressing of the pair tables (0 <= k < l < p):
 //   column l holds the entries (k, l), k = 0 .. l-1, at col_off(l) + k;
 //   row l holds the entries (l, j), j = l+1 .. p-1, at row_off(l, p) + (j - l - 1).

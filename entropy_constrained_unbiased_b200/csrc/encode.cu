@@ -23,7 +23,7 @@ namespace {
 
 constexpr int kEncThreads = 256;
 constexpr int kEncWarps = kEncThreads / kWarp;
-constexpr int64_t kEncChunk = 16384;  // entries per CTA (multiple of 4)
+constexpr int64_t kEncChunk = 32768;  // entries per CTA (multiple of 4)
 
 // Per-CTA state of the encoder in shared memory: the row's alphabet, both
 // codes, and the per-bucket records of the fast path.
@@ -31,7 +31,7 @@ struct EncRow {
   const double* P;       // [p]
   const float* T;        // [p] smallest float >= P_k
   const double* q;       // [2][s] code values
-  const double* w;       // [2][s] widths q_{t+1} - q_t
+  const int32_t* qi;     // [2][s] code indices into P
   const unsigned char* tmap;  // [2][p] bucket -> interval (255: none)
   unsigned int* hist;    // [warps][2s + 1] (bin 2s: entries the fast path left to the exact one)
   int p, s, m[2];
@@ -62,23 +62,18 @@ __device__ __forceinline__ int enc_exact(EncRow& S, float xf, int part, uint32_t
     return 0;
   }
   const double y = __dsub_rn(xd, S.q[part * s + t]);
-  const double prod = __dmul_rn(__dmul_rn(static_cast<double>(word), 0x1p-32), S.w[part * s + t]);
+  const double w = __dsub_rn(S.P[S.qi[part * s + t + 1]], S.P[S.qi[part * s + t]]);
+  const double prod = __dmul_rn(__dmul_rn(static_cast<double>(word), 0x1p-32), w);
   return t + ((prod < y) ? 1 : 0);
 }
 
-// The entries of a group of up to four that the fast path did not decide (bit
-// e of okm clear): exact code, histogram, byte in `packed`. Kept out of line so
-// that the fast loop carries none of it.
-__device__ __noinline__ uint32_t enc_fix(EncRow* S, const float* xv, const uint32_t* rw, const int* part, int cnt,
-                                         unsigned okm, uint32_t packed) {
-  unsigned int* wh = S->hist + warp_id() * (2 * S->s + 1);
-  for (int e = 0; e < cnt; ++e) {
-    if (okm & (1u << e)) continue;
-    const int out = enc_exact(*S, xv[e], part[e], rw[e]);
-    atomicAdd(wh + part[e] * S->s + out, 1u);
-    packed = (packed & ~(0xFFu << (8 * e))) | (static_cast<uint32_t>(out) << (8 * e));
-  }
-  return packed;
+// Exact code of one entry that the fast path did not decide, with its
+// histogram count; kept out of line (scalar arguments, so that the fast loop
+// keeps its values in registers) so that the fast loop carries none of it.
+__device__ __noinline__ int enc_fix1(EncRow* S, float x, uint32_t word, int part) {
+  const int out = enc_exact(*S, x, part, word);
+  red_shared_inc(smem_addr(S->hist + warp_id() * (2 * S->s + 1) + part * S->s + out));
+  return out;
 }
 
 // Bucket of an entry on the fast path: on rows whose alphabet is a uniform
@@ -102,10 +97,10 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
   double2* sR = reinterpret_cast<double2*>(smem);                          // [2][p] (q_t, w') per bucket
   double* sP = reinterpret_cast<double*>(sR + 2 * p);                       // [p]
   double* sq = sP + p;                                                      // [2][s] code values
-  double* sw = sq + 2 * s;                                                  // [2][s] widths
-  unsigned int* sh = reinterpret_cast<unsigned int*>(sw + 2 * s);           // [warps][2s + 1] counts
+  unsigned int* sh = reinterpret_cast<unsigned int*>(sq + 2 * s);           // [warps][2s + 1] counts
   float* sT = reinterpret_cast<float*>(sh + kEncWarps * nbins);             // [p] exact fp32 thresholds
-  unsigned char* tmap = reinterpret_cast<unsigned char*>(sT + p);           // [2][p] bucket -> interval
+  int32_t* sqi = reinterpret_cast<int32_t*>(sT + p);                      // [2][s] code indices
+  unsigned char* tmap = reinterpret_cast<unsigned char*>(sqi + 2 * s);      // [2][p] bucket -> interval
 
   const double* P = Pall + static_cast<int64_t>(r) * p;
   const bool has2 = (Q2 != nullptr);
@@ -121,7 +116,7 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
     S.P = sP;
     S.T = sT;
     S.q = sq;
-    S.w = sw;
+    S.qi = sqi;
     S.tmap = tmap;
     S.hist = sh;
     S.p = p;
@@ -173,13 +168,31 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
       if (t + 1 < m) {
         const double w = __dsub_rn(sP[q[t + 1]], sP[q[t]]);
         const double ws = __dmul_rn(w, 0x1p-32);
-        sw[part * s + t] = w;
         if (!(__dmul_rn(ws, 0x1p32) == w) || !(ws >= 0x1p-1022)) s_wexact = 0;  // scaling not exact
-        for (int k = q[t]; k < q[t + 1]; ++k) {
-          tmap[part * p + k] = static_cast<unsigned char>(t);
-          sR[part * p + k] = make_double2(sP[q[t]], ws);
-        }
       }
+    }
+    for (int t = threadIdx.x; t < m; t += blockDim.x) sqi[part * s + t] = q[t];
+  }
+  __syncthreads();
+  // bucket k lies in interval t = max{t <= m-2 : q_t <= k} when q_0 <= k < q_{m-1}
+  for (int part = 0; part < 2; ++part) {
+    const int m = S.m[part];
+    const bool used = (part == 0) ? (fixed_part == 0 || mix) : (fixed_part == 1 || mix);
+    if (!used || m < 2) continue;
+    const int32_t* qi = sqi + part * s;
+    for (int k = threadIdx.x; k < p; k += blockDim.x) {
+      if (k < qi[0] || k >= qi[m - 1]) continue;
+      int lo = 0, hi = m - 2;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (qi[mid] <= k)
+          lo = mid;
+        else
+          hi = mid - 1;
+      }
+      tmap[part * p + k] = static_cast<unsigned char>(lo);
+      const double w = __dsub_rn(sP[qi[lo + 1]], sP[qi[lo]]);
+      sR[part * p + k] = make_double2(sq[part * s + lo], __dmul_rn(w, 0x1p-32));
     }
   }
   const RowGrid g = row_grid(sP, p);
@@ -209,7 +222,7 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
   uint8_t* o = idx + static_cast<int64_t>(r) * d + beg;
   const bool vec = ((reinterpret_cast<uintptr_t>(x) & 15u) == 0) && ((reinterpret_cast<uintptr_t>(o) & 3u) == 0);
   const int nf = vec ? (len >> 2) : 0;  // full float4 groups on the vector path
-  unsigned int* wh = sh + warp_id() * nbins;
+  const uint32_t wh_base = smem_addr(sh + warp_id() * nbins);
   const int trash = 2 * s;
   const uint32_t blk0 = static_cast<uint32_t>(static_cast<uint64_t>(beg) >> 2);
   Philox4x32::RoundKeys rk;
@@ -224,8 +237,10 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
     uint32_t* o4 = reinterpret_cast<uint32_t*>(o);
     const unsigned pm2 = static_cast<unsigned>(p - 2);
     const float lim = 0.5f - eps_f;
+    float4 nxt = (threadIdx.x < nf) ? __ldcs(x4 + threadIdx.x) : make_float4(0.f, 0.f, 0.f, 0.f);
     for (int f = threadIdx.x; f < nf; f += kEncThreads) {
-      const float4 v = __ldcs(x4 + f);
+      const float4 v = nxt;
+      if (f + kEncThreads < nf) nxt = __ldcs(x4 + f + kEncThreads);
       const float xv[4] = {v.x, v.y, v.z, v.w};
       const uint32_t blk = blk0 + static_cast<uint32_t>(f);
       const uint4 ru = Philox4x32::block(make_uint4(blk, static_cast<uint32_t>(r), 0u, 0u), rk);
@@ -239,9 +254,12 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         part[e] = kMix ? (sel[e] <= th_last ? 0 : 1) : fixed_part;
+        // floor(g) by rounding (g - 0.5) to an integer with 1.5 * 2^23 (exact for
+        // 0 <= g < 2^22; at integer g the fractional test below fails)
         const float gf = fmaf(xv[e], s_f, c_f);
-        const float kf = floorf(gf);
-        const int k = static_cast<int>(kf);
+        const float tf = __fadd_rn(__fadd_rn(gf, -0.5f), 12582912.0f);
+        const float kf = __fsub_rn(tf, 12582912.0f);
+        const int k = __float_as_int(tf) - 0x4B400000;
         const bool kin = static_cast<unsigned>(k) <= pm2;
         const int pk = part[e] * p + (kin ? k : 0);
         const double2 rec = sR[pk];
@@ -250,11 +268,19 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
         const double y = __dsub_rn(static_cast<double>(xv[e]), rec.x);
         const double prod = __dmul_rn(static_cast<double>(rw[e]), rec.y);
         const int out = t + ((prod < y) ? 1 : 0);
-        atomicAdd(wh + (ok ? part[e] * s + out : trash), 1u);
+        red_shared_inc(wh_base + 4u * static_cast<uint32_t>(ok ? part[e] * s + out : trash));
         packed |= static_cast<uint32_t>(out & 0xFF) << (8 * e);
         okm |= ok ? (1u << e) : 0u;
       }
-      if (okm != 0xFu) packed = enc_fix(&S, xv, rw, part, 4, okm, packed);
+      if (okm != 0xFu) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (!(okm & (1u << e))) {
+            const int out = enc_fix1(&S, xv[e], rw[e], part[e]);
+            packed = (packed & ~(0xFFu << (8 * e))) | (static_cast<uint32_t>(out) << (8 * e));
+          }
+        }
+      }
       o4[f] = packed;
     }
   }
@@ -263,7 +289,9 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
   for (int j = 4 * nf + 4 * threadIdx.x; j < len; j += 4 * kEncThreads) {
     const int cnt = len - j < 4 ? len - j : 4;
     float xv[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int e = 0; e < cnt; ++e) xv[e] = __ldcs(x + j + e);
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (e < cnt) xv[e] = __ldcs(x + j + e);
     // the Philox counter block of entry j is its index in the row >> 2
     const uint32_t blk = blk0 + static_cast<uint32_t>(j >> 2);
     const uint4 ru = Philox4x32::block(make_uint4(blk, static_cast<uint32_t>(r), 0u, 0u), rk);
@@ -271,10 +299,13 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
     if (mix) su = Philox4x32::block(make_uint4(blk, static_cast<uint32_t>(r), 1u, 0u), rk);
     const uint32_t rw[4] = {ru.x, ru.y, ru.z, ru.w};
     const uint32_t sel[4] = {su.x, su.y, su.z, su.w};
-    int part[4];
-    for (int e = 0; e < 4; ++e) part[e] = mix ? (sel[e] <= th_last ? 0 : 1) : fixed_part;
-    const uint32_t packed = enc_fix(&S, xv, rw, part, cnt, 0u, 0u);
-    for (int e = 0; e < cnt; ++e) o[j + e] = static_cast<uint8_t>(packed >> (8 * e));
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (e < cnt) {
+        const int part = mix ? (sel[e] <= th_last ? 0 : 1) : fixed_part;
+        o[j + e] = static_cast<uint8_t>(enc_fix1(&S, xv[e], rw[e], part));
+      }
+    }
   }
   __syncthreads();
   unsigned long long* gh = hist + static_cast<int64_t>(r) * 2 * s;
@@ -289,7 +320,7 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
 
 // One CTA per (row, chunk of kEncChunk entries); rows coded with two codes
 // (0 < theta < 1) and rows coded with one take separate specialisations.
-__global__ void __launch_bounds__(kEncThreads)
+__global__ void __launch_bounds__(kEncThreads, 5)
 k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d, int p, int s,
          const int32_t* __restrict__ Q1, const int32_t* __restrict__ Q1_len, const int32_t* __restrict__ Q2,
          const int32_t* __restrict__ Q2_len, const double* __restrict__ theta, const Philox4x32::RoundKeys K,
@@ -328,8 +359,8 @@ __global__ void k_entropy(const int64_t* __restrict__ hist, int n, int s, double
 }
 
 size_t encode_smem(int p, int s) {
-  return sizeof(double2) * 2 * p + sizeof(double) * (p + 4 * s) + sizeof(unsigned int) * kEncWarps * (2 * s + 1) +
-         sizeof(float) * p + 2 * p;
+  return sizeof(double2) * 2 * p + sizeof(double) * (p + 2 * s) + sizeof(unsigned int) * kEncWarps * (2 * s + 1) +
+         sizeof(float) * p + sizeof(int32_t) * 2 * s + 2 * p;
 }
 
 }  // namespace

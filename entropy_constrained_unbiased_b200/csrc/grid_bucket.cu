@@ -202,6 +202,18 @@ constexpr double kFastEps = 0x1p-20;      // distance of v from a grid point on 
 // that take the exact search for every entry.
 constexpr double kFmaOffsetMax = 0x1p15;
 
+// k = floor(G) and v = G - k for 0 <= G < 2^31 away from the integers, with
+// fp64 additions instead of conversions: (G - 0.5) is exact, and adding
+// 1.5 * 2^52 rounds it to the nearest integer, which is floor(G) unless G is an
+// integer (then v = 0 or 1 and the caller's fast-path test fails); the integer
+// sits in the low word. Outside that range k and v are meaningless and the
+// test fails as well (k out of [0, p-2], or v not finite).
+__device__ __forceinline__ void floor_split(double G, int& k, double& v) {
+  const double t = __dadd_rn(__dadd_rn(G, -0.5), 0x1.8p52);
+  k = __double2loint(t);
+  v = __dsub_rn(G, __dsub_rn(t, 0x1.8p52));
+}
+
 // Per-CTA state of the bucketing kernel in shared memory.
 struct BucketRow {
   const double* P;   // [p]
@@ -217,20 +229,22 @@ struct BucketRow {
 // Fixed point: a = v 2^(F+14) + 2^52 + 2^13 keeps round(v 2^F) in bits 14.. of
 // the integer part, so the low limb is the low word >> 14 and the high limb the
 // low bits of the high word.
-__device__ __forceinline__ void bucket_add(unsigned int* cnt, unsigned int* limb, int k, double v, int hot0,
+// cnt_base, limb_base: shared-window byte addresses of the counts and limbs.
+__device__ __forceinline__ void bucket_add(uint32_t cnt_base, uint32_t limb_base, int k, double v, int hot0,
                                            int lane, double twoF, double twoH) {
   const double magic = 0x1p52 + 0x1p13;
-  atomicAdd(cnt + k, 1u);
+  red_shared_inc(cnt_base + 4u * static_cast<uint32_t>(k));
   const double a = fma(v, twoF, magic);
   const double t = v * twoH;
   const double b = fma(t, t, magic);
   const int hk = k - hot0;
   const int off = (static_cast<unsigned>(hk) < static_cast<unsigned>(kHotW)) ? hk * kWarp + lane : kHotW * kWarp + k;
-  unsigned int* c = limb + off;
-  atomicAdd(c, static_cast<unsigned>(__double2loint(a)) >> 14);
-  atomicAdd(c + kLimbBlock, static_cast<unsigned>(__double2hiint(a)) & 0x7FFFFu);
-  atomicAdd(c + 2 * kLimbBlock, static_cast<unsigned>(__double2loint(b)) >> 14);
-  atomicAdd(c + 3 * kLimbBlock, static_cast<unsigned>(__double2hiint(b)) & 0x7FFFFu);
+  const uint32_t c = limb_base + 4u * static_cast<uint32_t>(off);
+  constexpr int kL = 4 * kLimbBlock;  // bytes between limbs
+  red_shared_add<0>(c, static_cast<unsigned>(__double2loint(a)) >> 14);
+  red_shared_add<kL>(c, static_cast<unsigned>(__double2hiint(a)) & 0x7FFFFu);
+  red_shared_add<2 * kL>(c, static_cast<unsigned>(__double2loint(b)) >> 14);
+  red_shared_add<3 * kL>(c, static_cast<unsigned>(__double2hiint(b)) & 0x7FFFFu);
 }
 
 // Exact bucket k = max{k <= p-2 : P_k <= x} (fp32-threshold search) and offset
@@ -250,7 +264,8 @@ __device__ __noinline__ void bucket_exact(BucketRow* S, const float* xv, int cnt
     }
     const double y = __dsub_rn(static_cast<double>(xf), S->P[k]);
     const double w = S->uni ? __dadd_rn(__dmul_rn(y, S->invD), S->E[k]) : __dmul_rn(y, S->E[k]);
-    bucket_add(S->cnt, S->limb, k, fmin(fmax(w, 0.0), 1.0), S->hot0, lane, S->twoF, S->twoH);
+    bucket_add(smem_addr(S->cnt), smem_addr(S->limb), k, fmin(fmax(w, 0.0), 1.0), S->hot0, lane, S->twoF,
+               S->twoH);
   }
 }
 
@@ -411,6 +426,7 @@ k_bucket(const float* __restrict__ X, int64_t d, const double* __restrict__ Pall
     __syncthreads();
   }
   const int hot0 = S.hot0;
+  const uint32_t sc_base = smem_addr(sc), sl_base = smem_addr(sl);
 
   // Main pass: the float4 groups from the first 16-byte boundary, kB per
   // thread per step with the next kB loads in flight, the counters folded every
@@ -466,14 +482,12 @@ k_bucket(const float* __restrict__ X, int64_t d, const double* __restrict__ Pall
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const double G = fma(static_cast<double>(xv[e]), g.invD, c0);
-          const double kf = floor(G);
-          v[e] = __dsub_rn(G, kf);
-          k[e] = static_cast<int>(kf);
+          floor_split(G, k[e], v[e]);
           all = all && fabs(v[e] - 0.5) < lim && static_cast<unsigned>(k[e]) <= pm2;
         }
         if (all) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) bucket_add(sc, sl, k[e], v[e], hot0, lane, twoF, twoH);
+          for (int e = 0; e < 4; ++e) bucket_add(sc_base, sl_base, k[e], v[e], hot0, lane, twoF, twoH);
         } else {
           bucket_exact(&S, xv, 4);
         }
@@ -545,22 +559,25 @@ struct WideRow {
   int p, uni, bad;
 };
 
-__device__ __forceinline__ void wide_add(unsigned int* cnt, unsigned int* limb_lane, int k, double v, double twoF,
+// cnt_base, lane_base: shared-window byte addresses of the counts and of this
+// lane's column of limb counters.
+__device__ __forceinline__ void wide_add(uint32_t cnt_base, uint32_t lane_base, int k, double v, double twoF,
                                          double twoH) {
   const double magic = 0x1p52 + 0x1p13;
-  atomicAdd(cnt + k, 1u);
+  red_shared_inc(cnt_base + 4u * static_cast<uint32_t>(k));
   const double a = fma(v, twoF, magic);
   const double t = v * twoH;
   const double b = fma(t, t, magic);
-  unsigned int* c = limb_lane + k * kWarp;
-  atomicAdd(c, static_cast<unsigned>(__double2loint(a)) >> 14);
-  atomicAdd(c + kWideLimbBlock, static_cast<unsigned>(__double2hiint(a)) & 0x7FFFFu);
-  atomicAdd(c + 2 * kWideLimbBlock, static_cast<unsigned>(__double2loint(b)) >> 14);
-  atomicAdd(c + 3 * kWideLimbBlock, static_cast<unsigned>(__double2hiint(b)) & 0x7FFFFu);
+  const uint32_t c = lane_base + static_cast<uint32_t>(k) * (4u * kWarp);
+  constexpr int kL = 4 * kWideLimbBlock;  // bytes between limbs
+  red_shared_add<0>(c, static_cast<unsigned>(__double2loint(a)) >> 14);
+  red_shared_add<kL>(c, static_cast<unsigned>(__double2hiint(a)) & 0x7FFFFu);
+  red_shared_add<2 * kL>(c, static_cast<unsigned>(__double2loint(b)) >> 14);
+  red_shared_add<3 * kL>(c, static_cast<unsigned>(__double2hiint(b)) & 0x7FFFFu);
 }
 
 __device__ __noinline__ void wide_exact(WideRow* S, const float* xv, int cnt) {
-  unsigned int* limb_lane = S->limb + lane_id();
+  const uint32_t lane_base = smem_addr(S->limb + lane_id()), cnt_base = smem_addr(S->cnt);
   for (int e = 0; e < cnt; ++e) {
     const float xf = xv[e];
     const int k = bucket_f32(xf, S->T, S->top, S->p, S->scale);
@@ -570,7 +587,7 @@ __device__ __noinline__ void wide_exact(WideRow* S, const float* xv, int cnt) {
     }
     const double y = __dsub_rn(static_cast<double>(xf), S->P[k]);
     const double w = S->uni ? __dadd_rn(__dmul_rn(y, S->invD), S->E[k]) : __dmul_rn(y, S->E[k]);
-    wide_add(S->cnt, limb_lane, k, fmin(fmax(w, 0.0), 1.0), S->twoF, S->twoH);
+    wide_add(cnt_base, lane_base, k, fmin(fmax(w, 0.0), 1.0), S->twoF, S->twoH);
   }
 }
 
@@ -689,7 +706,7 @@ k_bucket_wide(const float* __restrict__ X, int n, int64_t d, const double* __res
     const int h = head < len ? head : len;
     const int nv = (len - h) >> 2;
     const float4* x4 = reinterpret_cast<const float4*>(xc + h);
-    unsigned int* limb_lane = sl + lane;
+    const uint32_t lane_base = smem_addr(sl + lane), cnt_base = smem_addr(sc);
     constexpr int kB = 2;
     float4 nxt[kB];
 #pragma unroll
@@ -715,14 +732,12 @@ k_bucket_wide(const float* __restrict__ X, int n, int64_t d, const double* __res
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const double G = fma(static_cast<double>(xv[e]), g.invD, c0);
-            const double kf = floor(G);
-            v[e] = __dsub_rn(G, kf);
-            k[e] = static_cast<int>(kf);
+            floor_split(G, k[e], v[e]);
             all = all && fabs(v[e] - 0.5) < lim && static_cast<unsigned>(k[e]) <= pm2;
           }
           if (all) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) wide_add(sc, limb_lane, k[e], v[e], twoF, twoH);
+            for (int e = 0; e < 4; ++e) wide_add(cnt_base, lane_base, k[e], v[e], twoF, twoH);
           } else {
             wide_exact(&S, xv, 4);
           }
