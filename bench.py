@@ -1,7 +1,7 @@
 """Benchmark of the ECASQ solver hot path on B200.
 
 One step = the whole path on one batch of synthetic vectors already in HBM:
-uniform grid -> bucketing -> DP solves (lambda bisection + time-sharing, or
+uniform grid + bucketing -> DP solves (lambda bisection + time-sharing, or
 fixed lambdas) -> stochastic-rounding encode -> empirical entropy.
 
 Default workload: 4096 x 4096 weight-like rows (0.02 * Student-t, nu = 4),
@@ -203,8 +203,7 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
     stream = torch.cuda.current_stream()
 
     def step(X):
-        P, st = E.uniform_grid(X, p)
-        cnt, A, B, st = E.bucket(X, P)
+        P, cnt, A, B, st = E.grid_bucket(X, p)
         ev_dp0.record(stream)
         if w.mode == "budget":
             out = E.solve_budget_stats(cnt, A, B, P, d, s, w.b, w.steps, fp64=fp64)
@@ -364,15 +363,17 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
 
 
 def stage_figures(E, X, P, p, s, enc_args, stream, flush, hbm):
-    """Device time of the uniform grid (min/max pass + grid), bucketing and
-    encoding, each call alone after an L2 flush; algorithmic bytes: 4 B/entry
-    read for the grid and for bucketing, 4 B read + 1 B written for encoding
-    (the histograms are fused)."""
+    """Device time of the uniform grid (min/max pass + grid), bucketing, the two
+    in one call, and encoding, each call alone after an L2 flush; algorithmic
+    bytes: 4 B/entry read for the grid, for bucketing and for the combined call,
+    4 B read + 1 B written for encoding (the histograms are fused)."""
     entries = X.numel()
     fns = {"grid": lambda: E.uniform_grid(X, p), "bucket": lambda: E.bucket(X, P),
-           "encode": lambda: E.encode(X, P, s, *enc_args)}
+           "grid_bucket": lambda: E.grid_bucket(X, p), "encode": lambda: E.encode(X, P, s, *enc_args)}
     out = {}
-    for name, bpe in (("grid", 4), ("bucket", 4), ("encode", 5)):
+    # grid_bucket: the grid and bucketing in one call, one read of X (4 B/entry)
+    # when rows fit in shared memory, else the two passes above (8 B/entry)
+    for name, bpe in (("grid", 4), ("bucket", 4), ("grid_bucket", 4), ("encode", 5)):
         fns[name]()
         ms = device_ms(fns[name], stream, flush)
         gbs = entries * bpe / (ms * 1e-3) / 1e9

@@ -147,6 +147,22 @@ int ecasq_bucket(const float* X, const double* P, int n, int64_t d, int p, int64
   return cuda_status(launch_bucket(X, P, n, d, p, cnt, A, B, status, acc, flag, static_cast<cudaStream_t>(stream)));
 }
 
+int ecasq_grid_bucket(const float* X, int n, int64_t d, int p, double* P, int64_t* cnt, double* A, double* B,
+                      int32_t* status, void* ws, size_t ws_bytes, void* stream) {
+  if (!X || !P || !cnt || !A || !B || !status || !valid_sizes(n, d, p, 2)) return ECASQ_ERR_ARG;
+  if (!ws || ws_bytes < ecasq_aux_workspace_size(n, d, p)) return ECASQ_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (grid_bucket_fused_ok(d, p)) return cuda_status(launch_grid_bucket_fused(X, n, d, p, P, cnt, A, B, status, st));
+  // two passes: the grid (its partials), then bucketing (its accumulators), in
+  // the same workspace one after the other on the stream
+  cudaError_t e = launch_uniform_grid(X, n, d, p, P, status, static_cast<float*>(ws), st);
+  if (e != cudaSuccess) return ECASQ_ERR_CUDA;
+  Carver c{static_cast<unsigned char*>(ws)};
+  auto* acc = c.take<unsigned long long>(3 * static_cast<size_t>(n) * (p - 1));
+  auto* flag = c.take<int32_t>(n);
+  return cuda_status(launch_bucket(X, P, n, d, p, cnt, A, B, status, acc, flag, st));
+}
+
 int ecasq_bucket_noalloc(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt, double* A,
                          double* B, int32_t* status, void* stream) {
   if (!X || !P || !cnt || !A || !B || !status || !valid_sizes(n, d, p, 2)) return ECASQ_ERR_ARG;

@@ -15,6 +15,7 @@ constexpr int32_t kStatusOk = 0;
 constexpr int32_t kStatusArg = -1;
 constexpr int32_t kStatusRange = -2;
 constexpr int32_t kStatusBudget = 1;
+constexpr int32_t kStatusStall = -4;  // a bounded device wait gave up (mirrors ECASQ_ERR_CUDA)
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & (kWarp - 1); }
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
@@ -111,6 +112,40 @@ __device__ __forceinline__ void red_shared_add(uint32_t addr, uint32_t v) {
 template <int kOff = 0>
 __device__ __forceinline__ void red_shared_inc(uint32_t addr) {
   asm volatile("red.shared.add.u32 [%0+%1], 1;" ::"r"(addr), "n"(kOff) : "memory");
+}
+
+// Untiled bulk copies global -> shared (cp.async.bulk, completion counted in
+// bytes on an mbarrier; addresses 16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(mbar)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t mbar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(mbar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Waits for the phase of the given parity, giving up after `limit` attempts
+// (each attempt may suspend the thread for a bounded time); true on success.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t mbar, uint32_t parity, int limit) {
+  for (int i = 0; i < limit; ++i)
+    if (mbar_try_wait(mbar, parity)) return true;
+  return false;
 }
 
 // Triangle addressing of the pair tables (0 <= k < l < p):

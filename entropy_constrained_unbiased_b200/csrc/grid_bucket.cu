@@ -7,6 +7,7 @@
 // again. Both kernels here are HBM-bound streams over X (4 bytes per entry).
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <mutex>
 
@@ -560,7 +561,8 @@ struct WideRow {
 };
 
 // cnt_base, lane_base: shared-window byte addresses of the counts and of this
-// lane's column of limb counters.
+// lane's column of limb counters ([4][buckets][32], kLB words per limb).
+template <int kLB = kWideLimbBlock>
 __device__ __forceinline__ void wide_add(uint32_t cnt_base, uint32_t lane_base, int k, double v, double twoF,
                                          double twoH) {
   const double magic = 0x1p52 + 0x1p13;
@@ -569,13 +571,14 @@ __device__ __forceinline__ void wide_add(uint32_t cnt_base, uint32_t lane_base, 
   const double t = v * twoH;
   const double b = fma(t, t, magic);
   const uint32_t c = lane_base + static_cast<uint32_t>(k) * (4u * kWarp);
-  constexpr int kL = 4 * kWideLimbBlock;  // bytes between limbs
+  constexpr int kL = 4 * kLB;  // bytes between limbs
   red_shared_add<0>(c, static_cast<unsigned>(__double2loint(a)) >> 14);
   red_shared_add<kL>(c, static_cast<unsigned>(__double2hiint(a)) & 0x7FFFFu);
   red_shared_add<2 * kL>(c, static_cast<unsigned>(__double2loint(b)) >> 14);
   red_shared_add<3 * kL>(c, static_cast<unsigned>(__double2hiint(b)) & 0x7FFFFu);
 }
 
+template <int kLB = kWideLimbBlock>
 __device__ __noinline__ void wide_exact(WideRow* S, const float* xv, int cnt) {
   const uint32_t lane_base = smem_addr(S->limb + lane_id()), cnt_base = smem_addr(S->cnt);
   for (int e = 0; e < cnt; ++e) {
@@ -587,7 +590,7 @@ __device__ __noinline__ void wide_exact(WideRow* S, const float* xv, int cnt) {
     }
     const double y = __dsub_rn(static_cast<double>(xf), S->P[k]);
     const double w = S->uni ? __dadd_rn(__dmul_rn(y, S->invD), S->E[k]) : __dmul_rn(y, S->E[k]);
-    wide_add(cnt_base, lane_base, k, fmin(fmax(w, 0.0), 1.0), S->twoF, S->twoH);
+    wide_add<kLB>(cnt_base, lane_base, k, fmin(fmax(w, 0.0), 1.0), S->twoF, S->twoH);
   }
 }
 
@@ -763,6 +766,275 @@ k_bucket_wide(const float* __restrict__ X, int n, int64_t d, const double* __res
   }
 }
 
+// ---------------------------------------------------------------------------
+// Uniform grid and bucketing in one read of X, for rows that fit in shared
+// memory (d <= 16384) and alphabets of at most 129 values. One persistent CTA
+// walks rows blockIdx.x, blockIdx.x + gridDim.x, ...; each row is staged in
+// shared memory by an untiled bulk copy (the next row's copy is issued before
+// the current row is processed, into the other of two buffers), then:
+//   min / max / finiteness -> the uniform grid, computed exactly as
+//   k_grid_finish does (P_k = lo + (hi - lo) k / (p - 1) in IEEE fp64, no
+//   contraction, P_{p-1} = hi) and written out; the bucketing of k_bucket_wide
+//   from shared memory into per-lane counters (4 limbs x 128 buckets x 32
+//   lanes, 64 KB); and the finish of k_bucket_finish for the row's buckets, so
+//   that cnt, A, B are written directly (no global atomics, no finish kernel).
+// Rows that hold a NaN or an infinity get a NaN grid, zero statistics and
+// status ECASQ_ERR_RANGE. A bounded wait for a staging copy that gives up
+// marks the row with status kStatusStall and ends the CTA after waiting (also
+// bounded) for its other copy in flight.
+
+constexpr int kFuseThreads = 512;
+constexpr int kFuseMaxD = 16384;                    // entries of a staged row
+constexpr int kFuseBuckets = 128;                   // p - 1 <= 128
+constexpr int kFuseLimbBlock = kFuseBuckets * kWarp;
+constexpr int kFuseWaitLimit = 1 << 22;
+
+size_t fuse_smem_bytes(int64_t d) {
+  const size_t dpad = static_cast<size_t>((d + 3) & ~int64_t(3));
+  return 16 + 2 * 4 * dpad + 4 * (4 * kFuseLimbBlock + kFuseBuckets) + 8 * 4 * kFuseBuckets +
+         (8 * 2 + 4) * (kFuseBuckets + 1) + 4 * 3 * (kFuseThreads / kWarp);
+}
+
+__global__ void __launch_bounds__(kFuseThreads, 2)
+k_grid_bucket_rows(const float* __restrict__ X, int n, int64_t d, int p, int fb, double* __restrict__ Pout,
+                   int64_t* __restrict__ cnt_out, double* __restrict__ A_out, double* __restrict__ B_out,
+                   int32_t* __restrict__ status) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ WideRow S;
+  __shared__ float s_lo, s_hi;
+  __shared__ int s_bad;
+  const int dpad = static_cast<int>((d + 3) & ~int64_t(3));
+  unsigned long long* mbar = reinterpret_cast<unsigned long long*>(smem);  // [2]
+  float* buf0 = reinterpret_cast<float*>(smem + 16);
+  float* buf1 = buf0 + dpad;
+  unsigned int* sl = reinterpret_cast<unsigned int*>(buf1 + dpad);         // [4][128][32] lane counters
+  unsigned int* sc = sl + 4 * kFuseLimbBlock;                              // [128] counts
+  unsigned long long* ssum = reinterpret_cast<unsigned long long*>(sc + kFuseBuckets);  // [4][128] limb sums
+  double* sP = reinterpret_cast<double*>(ssum + 4 * kFuseBuckets);         // [129]
+  double* sE = sP + (kFuseBuckets + 1);                                     // [129]
+  float* sT = reinterpret_cast<float*>(sE + (kFuseBuckets + 1));          // [129]
+  float* sred = sT + (kFuseBuckets + 1);                                   // [warps][3]
+  const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
+  const int nb = p - 1;
+  const double twoF = ldexp(1.0, fb + 14), twoH = ldexp(1.0, (fb + 14) / 2);
+  const unsigned pm2 = static_cast<unsigned>(p - 2);
+  const double lim = 0.5 - kFastEps;
+  // bulk staging needs 16-byte aligned rows of a multiple of 16 bytes
+  const bool bulk = ((d & 3) == 0) && ((reinterpret_cast<uintptr_t>(X) & 15u) == 0);
+  const uint32_t bytes = static_cast<uint32_t>(d * 4);
+  const uint32_t mb0 = smem_addr(mbar), mb1 = smem_addr(mbar + 1);
+  const uint32_t bb0 = smem_addr(buf0), bb1 = smem_addr(buf1);
+
+  for (int k = tid; k < 4 * kFuseLimbBlock; k += kFuseThreads) sl[k] = 0u;
+  for (int k = tid; k < kFuseBuckets; k += kFuseThreads) sc[k] = 0u;
+  if (tid == 0) {
+    if (bulk) {
+      mbar_init(mb0, 1);
+      mbar_init(mb1, 1);
+      fence_mbar_init();
+    }
+  }
+  __syncthreads();
+  if (tid == 0 && bulk && blockIdx.x < n) {
+    mbar_expect_tx(mb0, bytes);
+    bulk_copy_g2s(bb0, X + static_cast<int64_t>(blockIdx.x) * d, bytes, mb0);
+  }
+
+  int it = 0;
+  for (int r = blockIdx.x; r < n; r += gridDim.x, ++it) {
+    const int b = it & 1;
+    const float* xs = b ? buf1 : buf0;
+    // the next row's copy into the other buffer (free since the previous
+    // iteration's last barrier)
+    if (tid == 0 && bulk && r + static_cast<int>(gridDim.x) < n) {
+      fence_proxy_async_shared();
+      mbar_expect_tx(b ? mb0 : mb1, bytes);
+      bulk_copy_g2s(b ? bb0 : bb1, X + static_cast<int64_t>(r + gridDim.x) * d, bytes, b ? mb0 : mb1);
+    }
+    if (bulk) {
+      const bool ok = mbar_wait_bounded(b ? mb1 : mb0, static_cast<uint32_t>((it >> 1) & 1), kFuseWaitLimit);
+      if (__syncthreads_or(!ok)) {
+        if (tid == 0) {
+          status[r] = kStatusStall;
+          // the other buffer's copy, if one was issued, before the CTA ends
+          if (r + static_cast<int>(gridDim.x) < n)
+            mbar_wait_bounded(b ? mb0 : mb1, static_cast<uint32_t>(((it + 1) >> 1) & 1), kFuseWaitLimit);
+        }
+        return;
+      }
+    } else {
+      float* xw = b ? buf1 : buf0;
+      const float* xg = X + static_cast<int64_t>(r) * d;
+      for (int i = tid; i < d; i += kFuseThreads) xw[i] = xg[i];
+      __syncthreads();
+    }
+
+    // min / max / finiteness of the row
+    {
+      float lo = INFINITY, hi = -INFINITY;
+      int bad = 0;
+      const int nf = static_cast<int>(d >> 2);
+      const float4* x4 = reinterpret_cast<const float4*>(xs);
+      for (int i = tid; i < nf; i += kFuseThreads) {
+        const float4 v = x4[i];
+        mm_update(v.x, lo, hi, bad);
+        mm_update(v.y, lo, hi, bad);
+        mm_update(v.z, lo, hi, bad);
+        mm_update(v.w, lo, hi, bad);
+      }
+      for (int i = 4 * nf + tid; i < d; i += kFuseThreads) mm_update(xs[i], lo, hi, bad);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+        bad |= __shfl_xor_sync(0xffffffffu, bad, o);
+      }
+      if (lane == 0) {
+        sred[3 * warp] = lo;
+        sred[3 * warp + 1] = hi;
+        sred[3 * warp + 2] = __int_as_float(bad);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        for (int w = 1; w < kFuseThreads / kWarp; ++w) {
+          lo = fminf(lo, sred[3 * w]);
+          hi = fmaxf(hi, sred[3 * w + 1]);
+          bad |= __float_as_int(sred[3 * w + 2]);
+        }
+        s_lo = lo;
+        s_hi = hi;
+        s_bad = bad;
+      }
+      __syncthreads();
+    }
+    const bool row_bad = s_bad != 0;
+    {
+      // the uniform grid, as k_grid_finish computes it
+      const double lo = s_lo, hi = s_hi;
+      const double span = __dsub_rn(hi, lo);
+      const double den = static_cast<double>(p - 1);
+      for (int k = tid; k < p; k += kFuseThreads) {
+        const double v = (k == p - 1) ? hi : __dadd_rn(lo, __ddiv_rn(__dmul_rn(span, static_cast<double>(k)), den));
+        Pout[static_cast<int64_t>(r) * p + k] = row_bad ? __longlong_as_double(0x7ff8000000000000ll) : v;
+        sP[k] = v;
+        sT[k] = __double2float_ru(v);
+      }
+    }
+    int64_t* cr = cnt_out + static_cast<int64_t>(r) * nb;
+    double* Ar = A_out + static_cast<int64_t>(r) * nb;
+    double* Br = B_out + static_cast<int64_t>(r) * nb;
+    if (row_bad) {
+      for (int k = tid; k < nb; k += kFuseThreads) {
+        cr[k] = 0;
+        Ar[k] = 0.0;
+        Br[k] = 0.0;
+      }
+      if (tid == 0) status[r] = kStatusRange;
+      __syncthreads();
+      continue;
+    }
+    __syncthreads();
+    const RowGrid g = row_grid(sP, p);
+    const bool uni = row_is_uniform(sP, p, g, sE);  // includes a barrier
+    if (!uni) {
+      for (int k = tid; k < nb; k += kFuseThreads) {
+        const double w = __dsub_rn(sP[k + 1], sP[k]);
+        sE[k] = w > 0.0 ? __ddiv_rn(1.0, w) : 0.0;
+      }
+    }
+    const double c0 = -(g.P0 * g.invD);
+    const bool fastg = uni && fabs(c0) <= kFmaOffsetMax;
+    if (tid == 0) {
+      S.P = sP;
+      S.E = sE;
+      S.T = sT;
+      S.cnt = sc;
+      S.limb = sl;
+      S.invD = g.invD;
+      S.twoF = twoF;
+      S.twoH = twoH;
+      S.top = __double2float_rd(sP[p - 1]);
+      S.scale = static_cast<float>(static_cast<double>(p - 1) / (sP[p - 1] - sP[0]));
+      S.p = p;
+      S.uni = uni;
+      S.bad = 0;
+    }
+    __syncthreads();
+
+    // bucketing from shared memory
+    {
+      const uint32_t lane_base = smem_addr(sl + lane), cnt_base = smem_addr(sc);
+      const int nf = static_cast<int>(d >> 2);
+      const float4* x4 = reinterpret_cast<const float4*>(xs);
+      for (int i = tid; i < nf; i += kFuseThreads) {
+        const float4 c4 = x4[i];
+        const float xv[4] = {c4.x, c4.y, c4.z, c4.w};
+        int k[4];
+        double v[4];
+        bool all = fastg;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const double G = fma(static_cast<double>(xv[e]), g.invD, c0);
+          floor_split(G, k[e], v[e]);
+          all = all && fabs(v[e] - 0.5) < lim && static_cast<unsigned>(k[e]) <= pm2;
+        }
+        if (all) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) wide_add<kFuseLimbBlock>(cnt_base, lane_base, k[e], v[e], twoF, twoH);
+        } else {
+          wide_exact<kFuseLimbBlock>(&S, xv, 4);
+        }
+      }
+      for (int i = 4 * nf + tid; i < d; i += kFuseThreads) {
+        const float xv[1] = {xs[i]};
+        wide_exact<kFuseLimbBlock>(&S, xv, 1);
+      }
+    }
+    __syncthreads();
+    // the row's limb sums (thread: one limb of one bucket), then its statistics
+    {
+      const int li = tid / kFuseBuckets, k = tid % kFuseBuckets;
+      unsigned long long sum = 0;
+      if (k < nb && sc[k] != 0u) {
+        uint4* c4 = reinterpret_cast<uint4*>(sl + li * kFuseLimbBlock + k * kWarp);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int jj = (j + tid) & 7;
+          const uint4 v = c4[jj];
+          sum += static_cast<unsigned long long>(v.x) + v.y + v.z + v.w;
+          c4[jj] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      ssum[li * kFuseBuckets + k] = sum;
+    }
+    __syncthreads();
+    {
+      const double inv_two_fb = ldexp(1.0, -fb);
+      for (int k = tid; k < nb; k += kFuseThreads) {
+        const unsigned long long cn = sc[k];
+        const unsigned long long s1 = ssum[k] + (ssum[kFuseBuckets + k] << kLimbBits);
+        const unsigned long long s2 = ssum[2 * kFuseBuckets + k] + (ssum[3 * kFuseBuckets + k] << kLimbBits);
+        const double c = static_cast<double>(cn);
+        const double S1 = static_cast<double>(s1) * inv_two_fb;
+        const double S2 = static_cast<double>(s2) * inv_two_fb;
+        cr[k] = static_cast<int64_t>(cn);
+        if (uni) {
+          const double e = sE[k];
+          Ar[k] = g.D * (S1 - c * e);
+          Br[k] = g.D * g.D * (S2 - 2.0 * e * S1 + c * e * e);
+        } else {
+          const double w = sP[k + 1] - sP[k];
+          Ar[k] = S1 * w;
+          Br[k] = S2 * w * w;
+        }
+        sc[k] = 0u;
+      }
+      if (tid == 0) status[r] = S.bad ? kStatusRange : kStatusOk;
+    }
+    __syncthreads();
+  }
+}
+
 // Fixed-point row sums -> cnt (int64), A = sum (x - P_k), B = sum (x - P_k)^2 (fp64).
 __global__ void k_bucket_finish(const unsigned long long* __restrict__ acc, const double* __restrict__ Pall,
                                 int p, int fb, const int32_t* __restrict__ flag, int64_t* __restrict__ cnt,
@@ -867,6 +1139,32 @@ cudaError_t launch_bucket(const float* X, const double* P, int n, int64_t d, int
   }
   note_launch();
   k_bucket_finish<<<n, 256, 0, st>>>(acc, P, p, fb, flag, cnt, A, B, status);
+  note_launch();
+  return cudaGetLastError();
+}
+
+bool grid_bucket_fused_ok(int64_t d, int p) { return d >= 1 && d <= kFuseMaxD && p - 1 <= kFuseBuckets; }
+
+cudaError_t launch_grid_bucket_fused(const float* X, int n, int64_t d, int p, double* P, int64_t* cnt, double* A,
+                                     double* B, int32_t* status, cudaStream_t st) {
+  static std::once_flag once[64];
+  static cudaError_t result[64];
+  int dev = 0, sms = 0, per_sm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::call_once(once[dev], [dev]() {
+    result[dev] = cudaFuncSetAttribute(k_grid_bucket_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(fuse_smem_bytes(kFuseMaxD)));
+  });
+  if (result[dev] != cudaSuccess) return result[dev];
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const size_t smem = fuse_smem_bytes(d);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_grid_bucket_rows, kFuseThreads, smem);
+  if (e != cudaSuccess) return e;
+  const int grid = std::min(n, sms * std::max(per_sm, 1));
+  k_grid_bucket_rows<<<grid, kFuseThreads, smem, st>>>(X, n, d, p, bucket_fraction_bits(d), P, cnt, A, B, status);
   note_launch();
   return cudaGetLastError();
 }

@@ -22,6 +22,11 @@ cudaError_t launch_bucket(const float* X, const double* P, int n, int64_t d, int
                           double* A, double* B, int32_t* status, unsigned long long* acc,
                           int32_t* flag, cudaStream_t st);
 
+// Uniform grid + bucketing in one read of X (rows that fit in shared memory).
+bool grid_bucket_fused_ok(int64_t d, int p);
+cudaError_t launch_grid_bucket_fused(const float* X, int n, int64_t d, int p, double* P, int64_t* cnt, double* A,
+                                     double* B, int32_t* status, cudaStream_t st);
+
 cudaError_t launch_bf16_alphabet(const float* X, int n, int64_t d, int p_max, double* P, int32_t* p_len,
                                  int32_t* status, float* part, cudaStream_t st);
 

@@ -18,7 +18,7 @@ OK, ERR_ARG, ERR_RANGE, ERR_WORKSPACE, ERR_CUDA, WARN_BUDGET = 0, -1, -2, -3, -4
 
 EXPORTS = [
     "ecasq_workspace_size", "ecasq_aux_workspace_size", "ecasq_uniform_grid", "ecasq_bf16_alphabet", "ecasq_bucket",
-    "ecasq_bucket_noalloc",
+    "ecasq_bucket_noalloc", "ecasq_grid_bucket",
     "ecasq_solve", "ecasq_solve_stats", "ecasq_solve_budget", "ecasq_solve_budget_stats",
     "ecasq_approx_workspace_size", "ecasq_solve_approx", "ecasq_solve_approx_stats", "ecasq_solve_approx_budget",
     "ecasq_solve_approx_budget_stats",
@@ -55,6 +55,7 @@ def load(path: str = LIB_PATH):
         "ecasq_uniform_grid": (I, [P, I, I64, I, P, P, P, SZ, P]),
         "ecasq_bf16_alphabet": (I, [P, I, I64, I, P, P, P, P, SZ, P]),
         "ecasq_bucket": (I, [P, P, I, I64, I, P, P, P, P, P, SZ, P]),
+        "ecasq_grid_bucket": (I, [P, I, I64, I, P, P, P, P, P, P, SZ, P]),
         "ecasq_bucket_noalloc": (I, [P, P, I, I64, I, P, P, P, P, P]),
         "ecasq_solve": (I, [P, P, I, I64, I, I, P, I, P, P, P, P, P, P, OP, P, SZ, P]),
         "ecasq_solve_stats": (I, [P, P, P, P, I, I64, I, I, P, I, P, P, P, P, P, P, OP, P, SZ, P]),
@@ -170,6 +171,23 @@ def bucket(X: torch.Tensor, P: torch.Tensor):
     _check(L.ecasq_bucket(_ptr(X), _ptr(P), n, d, p, _ptr(cnt), _ptr(A), _ptr(B), _ptr(st), _ptr(ws), ws.numel(),
                           _stream()), "ecasq_bucket")
     return cnt, A, B, st
+
+
+def grid_bucket(X: torch.Tensor, p: int):
+    """Uniform grid and bucketing in one call (one read of X when rows fit in
+    shared memory). Returns P [n,p] f64, cnt [n,p-1] i64, A, B [n,p-1] f64, status."""
+    L = _need_cuda()
+    _dev(X, torch.float32, "X")
+    n, d = X.shape
+    P = torch.empty((n, p), dtype=torch.float64, device=X.device)
+    cnt = torch.empty((n, p - 1), dtype=torch.int64, device=X.device)
+    A = torch.empty((n, p - 1), dtype=torch.float64, device=X.device)
+    B = torch.empty((n, p - 1), dtype=torch.float64, device=X.device)
+    st = torch.empty(n, dtype=torch.int32, device=X.device)
+    ws = workspace(L.ecasq_aux_workspace_size(n, d, p), X.device)
+    _check(L.ecasq_grid_bucket(_ptr(X), n, d, p, _ptr(P), _ptr(cnt), _ptr(A), _ptr(B), _ptr(st), _ptr(ws),
+                               ws.numel(), _stream()), "ecasq_grid_bucket")
+    return P, cnt, A, B, st
 
 
 def bucket_noalloc(X: torch.Tensor, P: torch.Tensor):

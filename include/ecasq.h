@@ -104,6 +104,17 @@ int ecasq_bf16_alphabet(const float* X, int n, int64_t d, int p_max, double* P, 
 int ecasq_bucket(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt,
                  double* A, double* B, int32_t* status, void* ws, size_t ws_bytes, void* stream);
 
+/* ecasq_uniform_grid followed by ecasq_bucket, in one call: P, cnt, A, B and
+ * status as those two calls give them (the grid bit for bit). Rows of at most
+ * 16384 entries with p <= 129 are read from HBM once (each row is staged in
+ * shared memory, its grid and its statistics computed from there); other sizes
+ * run the two passes. A row holding a NaN or an infinity gets a NaN grid,
+ * status ECASQ_ERR_RANGE and (on the one-read path) zero statistics. On the
+ * one-read path, status ECASQ_ERR_CUDA marks a row whose staging copy the
+ * device stopped waiting for. Workspace: ecasq_aux_workspace_size(n, d, p). */
+int ecasq_grid_bucket(const float* X, int n, int64_t d, int p, double* P, int64_t* cnt, double* A,
+                      double* B, int32_t* status, void* ws, size_t ws_bytes, void* stream);
+
 /* ecasq_bucket without a workspace, for callers that cannot allocate device
  * memory where they bucket: plugins inside a framework whose own caching
  * allocator owns all device memory, and fixed-budget real-time or embedded

@@ -100,6 +100,76 @@ def test_bucket_flags_out_of_range(E, O):
     assert list(_np(st)) == [0, -2]
 
 
+# -- grid and bucketing in one call ------------------------------------------------
+
+GRID_BUCKET_CASES = [  # (dist, n, d, p): one-read path (aligned, d <= 16384, p <= 129), its unaligned
+    ("normal", 5, 1024, 64),  # fallback (odd d), and the two-pass path (larger d or p)
+    ("student_t", 7, 4096, 128),
+    ("laplace", 3, 16384, 129),
+    ("grad", 4, 4099, 128),
+    ("outlier", 3, 777, 33),
+    ("lognormal", 2, 3, 2),
+    ("normal", 2, 1, 16),
+    ("grad", 3, 20000, 128),
+    ("mixture", 3, 5000, 256),
+]
+
+
+def _check_grid_bucket(O, X, P, cnt, A, B, st, p):
+    Po, sto = O.grid_batch(X, p)
+    assert np.all(sto == 0) and np.all(_np(st) == 0)
+    np.testing.assert_array_equal(_np(P), Po)
+    for r in range(X.shape[0]):
+        co, Ao, Bo, so = O.bucket(X[r], Po[r])
+        assert so == 0
+        np.testing.assert_array_equal(_np(cnt[r]), co)
+        span = Po[r, -1] - Po[r, 0]
+        np.testing.assert_allclose(_np(A[r]), Ao, rtol=1e-9, atol=1e-12 * span)
+        np.testing.assert_allclose(_np(B[r]), Bo, rtol=1e-9, atol=1e-12 * span ** 2)
+
+
+@pytest.mark.parametrize("dist,n,d,p", GRID_BUCKET_CASES)
+def test_grid_bucket_matches_oracle(E, O, dist, n, d, p):
+    X = _case(13, n, d, dist)
+    P, cnt, A, B, st = E.grid_bucket(_cu(X), p)
+    _check_grid_bucket(O, X, P, cnt, A, B, st, p)
+    # the same statistics as the two separate calls
+    P2, _ = E.uniform_grid(_cu(X), p)
+    c2, A2, B2, _ = E.bucket(_cu(X), P2)
+    assert torch.equal(P, P2) and torch.equal(cnt, c2)
+    np.testing.assert_allclose(_np(A), _np(A2), rtol=1e-12, atol=1e-15 * float((P2[:, -1] - P2[:, 0]).max()))
+
+
+def test_grid_bucket_unaligned_rows(E, O):
+    """Rows whose start is not 16-byte aligned (d a multiple of 4, the base
+    pointer 4 bytes past an aligned one): the staging falls back to plain loads."""
+    X = _case(14, 6, 4096, "student_t")
+    flat = torch.empty(X.size + 1, dtype=torch.float32, device="cuda")
+    Xd = flat[1:].view(X.shape)
+    Xd.copy_(torch.from_numpy(X))
+    assert Xd.data_ptr() % 16 != 0
+    P, cnt, A, B, st = E.grid_bucket(Xd, 128)
+    _check_grid_bucket(O, X, P, cnt, A, B, st, 128)
+
+
+def test_grid_bucket_flags_and_constant_rows(E, O):
+    X = _case(15, 4, 4096, "normal")
+    X[1, 100] = np.nan
+    X[2, :] = 0.5
+    X[3, 7] = np.inf
+    P, cnt, A, B, st = E.grid_bucket(_cu(X), 64)
+    assert list(_np(st)) == [0, -2, 0, -2]
+    Pn = _np(P)
+    assert np.all(np.isnan(Pn[1])) and np.all(np.isnan(Pn[3]))
+    for r in (0, 2):
+        Po, _ = O.uniform_grid(X[r], 64)
+        np.testing.assert_array_equal(Pn[r], Po)
+        co, Ao, Bo, _ = O.bucket(X[r], Po)
+        np.testing.assert_array_equal(_np(cnt[r]), co)
+        np.testing.assert_allclose(_np(A[r]), Ao, rtol=1e-9, atol=1e-12 * max(Po[-1] - Po[0], 1e-30))
+    assert int(_np(cnt[2])[-1]) == 4096 and float(_np(A[2]).max()) == 0.0
+
+
 # -- the DP ------------------------------------------------------------------------
 
 SMALL = [  # (seed, n, d, p, s, dist)
