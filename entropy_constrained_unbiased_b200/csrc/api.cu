@@ -28,8 +28,10 @@ struct Carver {
   }
 };
 
-bool valid_sizes(int n, int64_t d, int p, int s) {
-  return n >= 1 && d >= 1 && d <= INT32_MAX && p >= 2 && p <= kMaxP && s >= 2 && s <= kMaxS;
+// pmax: kMaxP for the exact solver, kMaxPWide for the alphabet-sized passes
+// (grid, bucketing, encoding) and the approximation.
+bool valid_sizes(int n, int64_t d, int p, int s, int pmax = kMaxP) {
+  return n >= 1 && d >= 1 && d <= INT32_MAX && p >= 2 && p <= pmax && s >= 2 && s <= kMaxS;
 }
 
 // Workspace layout of the solver calls (ws == null measures it).
@@ -104,7 +106,7 @@ uint64_t ecasq_launch_count(int reset) {
 }
 
 size_t ecasq_aux_workspace_size(int n, int64_t d, int p) {
-  if (!valid_sizes(n, d, p, 2)) return 0;
+  if (!valid_sizes(n, d, p, 2, kMaxPWide)) return 0;
   const int64_t nc = (d + minmax_chunk(d) - 1) / minmax_chunk(d);
   const size_t grid = al256(sizeof(float) * 3 * static_cast<size_t>(n) * nc);
   const size_t bucket = al256(sizeof(unsigned long long) * 3 * static_cast<size_t>(n) * (p - 1)) +
@@ -123,7 +125,7 @@ size_t ecasq_workspace_size(int n, int64_t d, int p, int s, int n_lambda, const 
 
 int ecasq_uniform_grid(const float* X, int n, int64_t d, int p, double* P, int32_t* status, void* ws,
                        size_t ws_bytes, void* stream) {
-  if (!X || !P || !status || !valid_sizes(n, d, p, 2)) return ECASQ_ERR_ARG;
+  if (!X || !P || !status || !valid_sizes(n, d, p, 2, kMaxPWide)) return ECASQ_ERR_ARG;
   if (!ws || ws_bytes < ecasq_aux_workspace_size(n, d, p)) return ECASQ_ERR_WORKSPACE;
   return cuda_status(launch_uniform_grid(X, n, d, p, P, status, static_cast<float*>(ws),
                                          static_cast<cudaStream_t>(stream)));
@@ -139,7 +141,7 @@ int ecasq_bf16_alphabet(const float* X, int n, int64_t d, int p_max, double* P, 
 
 int ecasq_bucket(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt, double* A, double* B,
                  int32_t* status, void* ws, size_t ws_bytes, void* stream) {
-  if (!X || !P || !cnt || !A || !B || !status || !valid_sizes(n, d, p, 2)) return ECASQ_ERR_ARG;
+  if (!X || !P || !cnt || !A || !B || !status || !valid_sizes(n, d, p, 2, kMaxPWide)) return ECASQ_ERR_ARG;
   if (!ws || ws_bytes < ecasq_aux_workspace_size(n, d, p)) return ECASQ_ERR_WORKSPACE;
   Carver c{static_cast<unsigned char*>(ws)};
   auto* acc = c.take<unsigned long long>(3 * static_cast<size_t>(n) * (p - 1));
@@ -149,7 +151,7 @@ int ecasq_bucket(const float* X, const double* P, int n, int64_t d, int p, int64
 
 int ecasq_grid_bucket(const float* X, int n, int64_t d, int p, double* P, int64_t* cnt, double* A, double* B,
                       int32_t* status, void* ws, size_t ws_bytes, void* stream) {
-  if (!X || !P || !cnt || !A || !B || !status || !valid_sizes(n, d, p, 2)) return ECASQ_ERR_ARG;
+  if (!X || !P || !cnt || !A || !B || !status || !valid_sizes(n, d, p, 2, kMaxPWide)) return ECASQ_ERR_ARG;
   if (!ws || ws_bytes < ecasq_aux_workspace_size(n, d, p)) return ECASQ_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (grid_bucket_fused_ok(d, p)) return cuda_status(launch_grid_bucket_fused(X, n, d, p, P, cnt, A, B, status, st));
@@ -295,7 +297,7 @@ int ecasq_solve_budget_stats(const int64_t* cnt, const double* A, const double* 
 }
 
 size_t ecasq_approx_workspace_size(int n, int64_t d, int p, int s, const ecasq_opts* opts) {
-  if (!valid_sizes(n, d, p, s)) return 0;
+  if (!valid_sizes(n, d, p, s, kMaxPWide)) return 0;
   ApproxPlan plan;
   if (!approx_plan(n, p, s, opts && opts->dp_fp64, &plan)) return 0;
   SolveWs w;
@@ -305,7 +307,7 @@ size_t ecasq_approx_workspace_size(int n, int64_t d, int p, int s, const ecasq_o
 static int approx_common(const float* X, const int64_t* cnt, const double* A, const double* B, const double* P, int n,
                          int64_t d, int p, int s, int refine, const ecasq_opts* opts, void* ws, size_t ws_bytes,
                          cudaStream_t st, ApproxArgs* args, ApproxPlan* plan) {
-  if (!P || !valid_sizes(n, d, p, s) || refine < 0) return ECASQ_ERR_ARG;
+  if (!P || !valid_sizes(n, d, p, s, kMaxPWide) || refine < 0) return ECASQ_ERR_ARG;
   if (opts && (opts->reserved != 0 || opts->bisect_steps < 0)) return ECASQ_ERR_ARG;
   if (!approx_plan(n, p, s, opts && opts->dp_fp64, plan)) return ECASQ_ERR_ARG;
   SolveWs w;
@@ -436,7 +438,8 @@ int ecasq_encode(const float* X, const double* P, int n, int64_t d, int p, int s
                  uint8_t* idx, int64_t* hist, int32_t* status, void* stream) {
   // s is the row stride of the codes and the histogram (a code of up to 256
   // values: indices fit in uint8), not bound by the solvers' code size.
-  if (!X || !P || !Q1 || !Q1_len || !idx || !hist || !status || !valid_sizes(n, d, p, 2) || s < 1 || s > 256)
+  if (!X || !P || !Q1 || !Q1_len || !idx || !hist || !status || !valid_sizes(n, d, p, 2, kMaxPWide) || s < 1 ||
+      s > 256)
     return ECASQ_ERR_ARG;
   if (Q2 && !Q2_len) return ECASQ_ERR_ARG;
   return cuda_status(launch_encode(X, P, n, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, seed, idx, hist, status,

@@ -472,6 +472,132 @@ __device__ void approx_solve(const ACtx<T>& c, double lam, int refine, AOut* out
   __syncthreads();
 }
 
+// Outputs of a row that needs no solve: a degenerate row (one value, status
+// ok) or a rejected one (status st, empty codes).
+__device__ void approx_fill_trivial(const ApproxArgs& a, int r, int32_t st) {
+  const int so = a.s_out;
+  const int qv = (st == kStatusOk) ? 0 : -1;
+  const int ml = (st == kStatusOk) ? 1 : 0;
+  if (a.mode == 0) {
+    for (int t = 0; t < a.n_lambda; ++t) {
+      const int64_t w = static_cast<int64_t>(r) * a.n_lambda + t;
+      for (int q = threadIdx.x; q < so; q += blockDim.x) a.Q[w * so + q] = (q == 0) ? qv : -1;
+      if (threadIdx.x == 0) {
+        a.Q_len[w] = ml;
+        a.obj[w] = a.mse[w] = a.H[w] = a.HIB[w] = 0.0;
+      }
+    }
+  } else {
+    for (int q = threadIdx.x; q < so; q += blockDim.x) {
+      a.Q1[int64_t(r) * so + q] = (q == 0) ? qv : -1;
+      a.Q2[int64_t(r) * so + q] = (q == 0) ? qv : -1;
+    }
+    if (threadIdx.x == 0) {
+      a.Q1_len[r] = a.Q2_len[r] = ml;
+      a.theta[r] = a.lam_lo[r] = a.lam_hi[r] = 0.0;
+      a.H1[r] = a.H2[r] = a.HIB1[r] = a.HIB2[r] = a.mse1[r] = a.mse2[r] = 0.0;
+    }
+  }
+  if (threadIdx.x == 0) a.status[r] = st;
+}
+
+// The per-row driver shared by the approximation kernels: each lambda of the
+// row's list (mode 0), or the bisection on lambda with two-way time-sharing
+// (mode 1, the constrained rate H(I,B) for the plain approximation and H(X^)
+// once refined), writing the row's outputs. solve(lambda) leaves the code in
+// sQ and its figures in s_out (all threads); bracket = (P_{p-1} - P_0)^2.
+template <class Solve>
+__device__ void approx_drive(const ApproxArgs& a, int r, const int* sQ, int* sQ1, int* sQ2, int S, double bracket,
+                             AOut& s_out, Solve solve) {
+  const int so = a.s_out;
+  if (a.mode == 0) {
+    for (int t = 0; t < a.n_lambda; ++t) {
+      const int64_t w = static_cast<int64_t>(r) * a.n_lambda + t;
+      solve(a.lambda[w]);
+      for (int q = threadIdx.x; q < so; q += blockDim.x) a.Q[w * so + q] = (q < s_out.m) ? sQ[q] : -1;
+      if (threadIdx.x == 0) {
+        a.Q_len[w] = s_out.m;
+        a.obj[w] = s_out.J;
+        a.mse[w] = s_out.mse;
+        a.H[w] = s_out.H;
+        a.HIB[w] = s_out.HIB;
+      }
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) a.status[r] = kStatusOk;
+  } else {
+    // Bisection on lambda with two-way time-sharing; the constrained rate is
+    // H(I,B) for the plain approximation and H(X^) once refined.
+    const bool refined = a.refine > 0;
+    double lo = 0.0;
+    double hi = bracket;
+    double H1 = 0, H2 = 0, B1 = 0, B2 = 0, M1 = 0, M2 = 0, r1 = 0, r2 = 0;
+    int m1 = 0, m2 = 0;
+    auto keep = [&](int* dst, int& m, double& Hk, double& Bk, double& Mk) {
+      for (int q = threadIdx.x; q < S; q += blockDim.x) dst[q] = sQ[q];
+      m = s_out.m;
+      Hk = s_out.H;
+      Bk = s_out.HIB;
+      Mk = s_out.mse;
+    };
+    auto rate = [&]() { return refined ? s_out.H : s_out.HIB; };
+    int32_t status = kStatusOk;
+    double theta = 0.0;
+    solve(0.0);
+    keep(sQ1, m1, H1, B1, M1);
+    r1 = rate();
+    if (r1 <= a.budget) {
+      keep(sQ2, m2, H2, B2, M2);
+      hi = 0.0;
+    } else {
+      __syncthreads();
+      solve(hi);
+      keep(sQ2, m2, H2, B2, M2);
+      r2 = rate();
+      if (r2 > a.budget) {
+        status = kStatusBudget;
+      } else {
+        for (int it = 0; it < a.steps; ++it) {
+          const double mid = 0.5 * (lo + hi);
+          __syncthreads();
+          solve(mid);
+          const double rr = rate();
+          if (rr > a.budget) {
+            lo = mid;
+            r1 = rr;
+            keep(sQ1, m1, H1, B1, M1);
+          } else {
+            hi = mid;
+            r2 = rr;
+            keep(sQ2, m2, H2, B2, M2);
+          }
+        }
+        const double th = (a.budget - r2) / (r1 - r2);
+        theta = th < 0.0 ? 0.0 : (th > 1.0 ? 1.0 : th);
+      }
+    }
+    __syncthreads();
+    for (int q = threadIdx.x; q < so; q += blockDim.x) {
+      a.Q1[int64_t(r) * so + q] = (q < m1) ? sQ1[q] : -1;
+      a.Q2[int64_t(r) * so + q] = (q < m2) ? sQ2[q] : -1;
+    }
+    if (threadIdx.x == 0) {
+      a.Q1_len[r] = m1;
+      a.Q2_len[r] = m2;
+      a.theta[r] = theta;
+      a.lam_lo[r] = lo;
+      a.lam_hi[r] = hi;
+      a.H1[r] = H1;
+      a.H2[r] = H2;
+      a.HIB1[r] = B1;
+      a.HIB2[r] = B2;
+      a.mse1[r] = M1;
+      a.mse2[r] = M2;
+      a.status[r] = status;
+    }
+  }
+}
+
 template <typename T, bool kSmem, bool kSplit>
 __global__ void __launch_bounds__(512, 1) k_approx(ApproxArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -548,32 +674,9 @@ __global__ void __launch_bounds__(512, 1) k_approx(ApproxArgs a) {
       for (int k = threadIdx.x; k < p - 1; k += blockDim.x) bad |= !(c.sP[k] < c.sP[k + 1]);
     bad = __syncthreads_or(bad);
     const int32_t st = s_flag != 0 ? s_flag : (bad ? kStatusArg : kStatusOk);
-    const int so = a.s_out;
 
     if (st != kStatusOk || degenerate) {
-      const int qv = (st == kStatusOk) ? 0 : -1;
-      const int ml = (st == kStatusOk) ? 1 : 0;
-      if (a.mode == 0) {
-        for (int t = 0; t < a.n_lambda; ++t) {
-          const int64_t w = static_cast<int64_t>(r) * a.n_lambda + t;
-          for (int q = threadIdx.x; q < so; q += blockDim.x) a.Q[w * so + q] = (q == 0) ? qv : -1;
-          if (threadIdx.x == 0) {
-            a.Q_len[w] = ml;
-            a.obj[w] = a.mse[w] = a.H[w] = a.HIB[w] = 0.0;
-          }
-        }
-      } else {
-        for (int q = threadIdx.x; q < so; q += blockDim.x) {
-          a.Q1[int64_t(r) * so + q] = (q == 0) ? qv : -1;
-          a.Q2[int64_t(r) * so + q] = (q == 0) ? qv : -1;
-        }
-        if (threadIdx.x == 0) {
-          a.Q1_len[r] = a.Q2_len[r] = ml;
-          a.theta[r] = a.lam_lo[r] = a.lam_hi[r] = 0.0;
-          a.H1[r] = a.H2[r] = a.HIB1[r] = a.HIB2[r] = a.mse1[r] = a.mse2[r] = 0.0;
-        }
-      }
-      if (threadIdx.x == 0) a.status[r] = st;
+      approx_fill_trivial(a, r, st);
       __syncthreads();
       continue;
     }
@@ -581,92 +684,384 @@ __global__ void __launch_bounds__(512, 1) k_approx(ApproxArgs a) {
     build_pair_terms(c);
     __syncthreads();
 
-    if (a.mode == 0) {
-      for (int t = 0; t < a.n_lambda; ++t) {
-        const int64_t w = static_cast<int64_t>(r) * a.n_lambda + t;
-        approx_solve<T, kSplit>(c, a.lambda[w], a.refine, &s_out);
-        for (int q = threadIdx.x; q < so; q += blockDim.x) a.Q[w * so + q] = (q < s_out.m) ? c.sQ[q] : -1;
-        if (threadIdx.x == 0) {
-          a.Q_len[w] = s_out.m;
-          a.obj[w] = s_out.J;
-          a.mse[w] = s_out.mse;
-          a.H[w] = s_out.H;
-          a.HIB[w] = s_out.HIB;
+    approx_drive(a, r, c.sQ, sQ1, sQ2, S, (c.sP[p - 1] - c.sP[0]) * (c.sP[p - 1] - c.sP[0]), s_out,
+                 [&](double lam) { approx_solve<T, kSplit>(c, lam, a.refine, &s_out); });
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The approximation for large alphabets (p > 512, up to 65536 values: e.g.
+// every BF16 value of a range, §5 "Generalidade"), in O(p) memory per vector
+// besides the layers. The pair terms V, R, L of an interval [P_a, P_e] come
+// from six prefix sums over the buckets, with u_k = P_k - P_0:
+//   N  = sum n_k,
+//   T1 = sum (x - P_a)   = SA + SNU - u_a N,
+//   T2 = sum (x - P_a)^2 = SB + 2 SAU - 2 u_a SA + SNUU - 2 u_a SNU + u_a^2 N,
+// over k = a .. e-1 (SA = sum A_k, SB = sum B_k, SNU = sum n_k u_k,
+// SAU = sum A_k u_k, SNUU = sum n_k u_k^2; each a difference of two prefix
+// sums), then V = W T1 - T2 (clamped at 0), R = T1 / W, L = N - R with
+// W = P_e - P_a. The differences cancel: the relative error of T2 grows like
+// (u_e / W)^2 times the fp64 unit, below 1e-7 for the alphabets this path
+// serves, so the layers run in fp32 (their own resolution) with the cost
+// w(a,e) = V/d + lambda (h(L) + h(R)) computed on the fly for every
+// relaxation, and the recovery recomputes the same fp32 values. The
+// refinement compares local costs from the same prefix terms in fp64; the
+// reported figures of the final code (mse, H, H(I,B), objective) are direct
+// fp64 sums over each interval's buckets in the order of the definitions.
+
+struct WCtx {
+  int p, S, pst;
+  double dd, inv_d;
+  const double* P;  // [p] the row of the alphabet
+  double* pre;      // [6][p] prefix sums N, SA, SB, SNU, SAU, SNUU (index k: buckets 0 .. k-1)
+  double* nb;       // [p] bucket counts, A, B (for the direct sums)
+  double* ab;
+  double* bb;
+  float* G;         // [(S+1) * pst] layers
+  double* fbuf;     // [warps][p] local costs of the refinement
+  int* sQ;
+  int* moved;
+  int* msh;
+};
+
+__device__ __forceinline__ void wpair(const WCtx& c, int a, int e, double& V, double& R, double& L) {
+  const double* pr = c.pre;
+  const int p = c.p;
+  const double N = __dsub_rn(pr[e], pr[a]);
+  const double SA = __dsub_rn(pr[p + e], pr[p + a]);
+  const double SB = __dsub_rn(pr[2 * p + e], pr[2 * p + a]);
+  const double SNU = __dsub_rn(pr[3 * p + e], pr[3 * p + a]);
+  const double SAU = __dsub_rn(pr[4 * p + e], pr[4 * p + a]);
+  const double SNUU = __dsub_rn(pr[5 * p + e], pr[5 * p + a]);
+  const double ua = __dsub_rn(c.P[a], c.P[0]);
+  const double W = __dsub_rn(c.P[e], c.P[a]);
+  const double T1 = SA + SNU - ua * N;
+  const double T2 = SB + 2.0 * SAU - 2.0 * ua * SA + SNUU - 2.0 * ua * SNU + ua * ua * N;
+  V = fmax(W * T1 - T2, 0.0);
+  R = W > 0.0 ? T1 / W : 0.0;
+  L = N - R;
+}
+
+// The layers' cost w(a, e) in fp32 (as the fp32 table path forms it).
+__device__ __forceinline__ float wcost(const WCtx& c, int a, int e, float lamf) {
+  double V, R, L;
+  wpair(c, a, e, V, R, L);
+  const float vt = static_cast<float>(V * c.inv_d);
+  const float qr = static_cast<float>(R * c.inv_d), ql = static_cast<float>(L * c.inv_d);
+  const float hr = qr > 0.0f ? -qr * lg2_approx(qr) : 0.0f;
+  const float hl = ql > 0.0f ? -ql * lg2_approx(ql) : 0.0f;
+  return __fmaf_rn(lamf, hl + hr, vt);
+}
+
+// Direct fp64 sums over buckets a .. e-1, every operation rounded as written,
+// in the order of build_pair_terms (the oracle's tables).
+__device__ void wpair_direct(const WCtx& c, int a, int e, double& V, double& R, double& L) {
+  double N = 0.0, T1 = 0.0, T2 = 0.0;
+  const double Pa = c.P[a];
+  for (int k = a; k < e; ++k) {
+    const double dk = __dsub_rn(c.P[k], Pa);
+    const double nk = c.nb[k];
+    N = __dadd_rn(N, nk);
+    T1 = __dadd_rn(T1, __dadd_rn(c.ab[k], __dmul_rn(nk, dk)));
+    T2 = __dadd_rn(T2, __dadd_rn(__dadd_rn(c.bb[k], __dmul_rn(__dmul_rn(2.0, dk), c.ab[k])), __dmul_rn(__dmul_rn(nk, dk), dk)));
+  }
+  const double W = __dsub_rn(c.P[e], Pa);
+  V = __dsub_rn(__dmul_rn(W, T1), T2);
+  V = V < 0.0 ? 0.0 : V;
+  R = W > 0.0 ? __ddiv_rn(T1, W) : 0.0;
+  L = __dsub_rn(N, R);
+}
+
+__device__ __forceinline__ double wlocal_cost(const WCtx& c, double lam, int a, int e, int x, double r_before,
+                                              double l_after) {
+  double Va, Ra, La, Vb, Rb, Lb;
+  wpair(c, a, x, Va, Ra, La);
+  wpair(c, x, e, Vb, Rb, Lb);
+  const double f = __ddiv_rn(__dadd_rn(Va, Vb), c.dd);
+  const double mu_prev = __dadd_rn(r_before, La);
+  const double mu_self = __dadd_rn(Ra, Lb);
+  const double mu_next = __dadd_rn(Rb, l_after);
+  const double hs = __dadd_rn(__dadd_rn(hmass(mu_prev, c.dd), hmass(mu_self, c.dd)), hmass(mu_next, c.dd));
+  return __dadd_rn(f, __dmul_rn(lam, hs));
+}
+
+// Refinement as refine_code, on the prefix terms.
+__device__ void wrefine(const WCtx& c, double lam, int m, int iters) {
+  const int lane = lane_id(), warp = warp_id(), nw = blockDim.x / kWarp;
+  int* Q = c.sQ;
+  double* fb = c.fbuf + static_cast<size_t>(warp) * c.p;
+  for (int it = 0; it < iters; ++it) {
+    if (threadIdx.x == 0) *c.moved = 0;
+    __syncthreads();
+    for (int cls = 0; cls < 3; ++cls) {
+      const int npos = (m - 2 - cls + 2) / 3;
+      for (int j = warp; j < npos; j += nw) {
+        const int t = 1 + cls + 3 * j;
+        const int a = Q[t - 1], e = Q[t + 1];
+        double Vx, Rx, Lx;
+        double r_before = 0.0, l_after = 0.0;
+        if (t - 1 > 0) {
+          wpair(c, Q[t - 2], a, Vx, Rx, Lx);
+          r_before = Rx;
         }
-        __syncthreads();
-      }
-      if (threadIdx.x == 0) a.status[r] = kStatusOk;
-    } else {
-      // Bisection on lambda with two-way time-sharing; the constrained rate is
-      // H(I,B) for the plain approximation and H(X^) once refined.
-      const bool refined = a.refine > 0;
-      double lo = 0.0;
-      double hi = (c.sP[p - 1] - c.sP[0]) * (c.sP[p - 1] - c.sP[0]);
-      double H1 = 0, H2 = 0, B1 = 0, B2 = 0, M1 = 0, M2 = 0, r1 = 0, r2 = 0;
-      int m1 = 0, m2 = 0;
-      auto keep = [&](int* dst, int& m, double& Hk, double& Bk, double& Mk) {
-        for (int q = threadIdx.x; q < S; q += blockDim.x) dst[q] = c.sQ[q];
-        m = s_out.m;
-        Hk = s_out.H;
-        Bk = s_out.HIB;
-        Mk = s_out.mse;
-      };
-      auto rate = [&]() { return refined ? s_out.H : s_out.HIB; };
-      int32_t status = kStatusOk;
-      double theta = 0.0;
-      approx_solve<T, kSplit>(c, 0.0, a.refine, &s_out);
-      keep(sQ1, m1, H1, B1, M1);
-      r1 = rate();
-      if (r1 <= a.budget) {
-        keep(sQ2, m2, H2, B2, M2);
-        hi = 0.0;
-      } else {
-        __syncthreads();
-        approx_solve<T, kSplit>(c, hi, a.refine, &s_out);
-        keep(sQ2, m2, H2, B2, M2);
-        r2 = rate();
-        if (r2 > a.budget) {
-          status = kStatusBudget;
-        } else {
-          for (int it = 0; it < a.steps; ++it) {
-            const double mid = 0.5 * (lo + hi);
-            __syncthreads();
-            approx_solve<T, kSplit>(c, mid, a.refine, &s_out);
-            const double rr = rate();
-            if (rr > a.budget) {
-              lo = mid;
-              r1 = rr;
-              keep(sQ1, m1, H1, B1, M1);
-            } else {
-              hi = mid;
-              r2 = rr;
-              keep(sQ2, m2, H2, B2, M2);
-            }
+        if (t + 1 < m - 1) {
+          wpair(c, e, Q[t + 2], Vx, Rx, Lx);
+          l_after = Lx;
+        }
+        const int lo = a + 1, hi = e - 1;
+        for (int x = lo + lane; x <= hi; x += kWarp) fb[x - lo] = wlocal_cost(c, lam, a, e, x, r_before, l_after);
+        __syncwarp();
+        if (lane == 0) {
+          int l = lo, h = hi;
+          while (l < h) {
+            const int mid = l + (h - l) / 2;
+            if (fb[mid + 1 - lo] < fb[mid - lo])
+              l = mid + 1;
+            else
+              h = mid;
           }
-          const double th = (a.budget - r2) / (r1 - r2);
-          theta = th < 0.0 ? 0.0 : (th > 1.0 ? 1.0 : th);
+          if (l != Q[t] && fb[l - lo] < fb[Q[t] - lo]) {
+            Q[t] = l;
+            atomicAdd(c.moved, 1);
+          }
+        }
+        __syncwarp();
+      }
+      __syncthreads();
+    }
+    if (*c.moved == 0) break;
+    __syncthreads();
+  }
+}
+
+// fp64 figures of c.sQ (warp 0), as evaluate_code, from direct sums.
+__device__ void wevaluate(const WCtx& c, double lam, bool refined, int m, AOut* out) {
+  const int lane = lane_id();
+  double* tv = c.fbuf;
+  double* th = c.fbuf + c.S;
+  double* tl = c.fbuf + 2 * c.S;
+  double* tr = c.fbuf + 3 * c.S;
+  double* tR = c.fbuf + 4 * c.S;
+  double* tL = c.fbuf + 5 * c.S;
+  for (int t = lane; t + 1 < m; t += kWarp) {
+    double V, R, L;
+    wpair_direct(c, c.sQ[t], c.sQ[t + 1], V, R, L);
+    tv[t] = V;
+    tR[t] = R;
+    tL[t] = L;
+    tl[t] = hmass(L, c.dd);
+    tr[t] = hmass(R, c.dd);
+  }
+  __syncwarp();
+  for (int t = lane; t < m; t += kWarp) {
+    double u = 0.0;
+    if (t > 0) u = __dadd_rn(u, tR[t - 1]);
+    if (t + 1 < m) u = __dadd_rn(u, tL[t]);
+    th[t] = hmass(u, c.dd);
+  }
+  __syncwarp();
+  if (lane == 0) {
+    double sv = 0.0, sh = 0.0, sib = 0.0;
+    for (int t = 0; t < m; ++t) {
+      if (t + 1 < m) sv = __dadd_rn(sv, tv[t]);
+      sh = __dadd_rn(sh, th[t]);
+      if (t + 1 < m) {
+        sib = __dadd_rn(sib, tl[t]);
+        sib = __dadd_rn(sib, tr[t]);
+      }
+    }
+    out->m = m;
+    out->mse = __ddiv_rn(sv, c.dd);
+    out->H = sh;
+    out->HIB = sib;
+    out->J = __dadd_rn(out->mse, __dmul_rn(lam, refined ? sh : sib));
+  }
+  __syncwarp();
+}
+
+__device__ void approx_solve_wide(const WCtx& c, double lam, int refine, AOut* out) {
+  const int p = c.p, S = c.S, tid = threadIdx.x, bd = blockDim.x;
+  const float inf = __int_as_float(0x7f800000);
+  const float lamf = static_cast<float>(lam);
+  for (int x = tid; x < p; x += bd) c.G[c.pst + x] = (x == 0) ? 0.0f : inf;
+  __syncthreads();
+  for (int i = 2; i <= S; ++i) {
+    const float* __restrict__ Gp = c.G + (i - 1) * c.pst;
+    float* __restrict__ Gc = c.G + i * c.pst;
+    for (int x = i - 1 + tid; x < p; x += bd) {
+      float best = inf;
+      for (int a = i - 2; a < x; ++a) best = fminf(best, __fadd_rn(Gp[a], wcost(c, a, x, lamf)));
+      Gc[x] = best;
+    }
+    __syncthreads();
+  }
+  if (warp_id() == 0) {
+    const int lane = lane_id();
+    float bv = inf;
+    int bi = 0x7fffffff;
+    for (int i = 2 + lane; i <= S; i += kWarp) {
+      const float g = c.G[i * c.pst + p - 1];
+      if (g < bv) {
+        bv = g;
+        bi = i;
+      }
+    }
+    warp_argmin(bv, bi);
+    int m;
+    if (bi == 0x7fffffff) {
+      m = 2;
+      if (lane == 0) {
+        c.sQ[0] = 0;
+        c.sQ[1] = p - 1;
+      }
+    } else {
+      m = bi;
+      int x = p - 1;
+      if (lane == 0) c.sQ[m - 1] = x;
+      for (int i = m; i >= 2; --i) {
+        const float target = c.G[i * c.pst + x];
+        const float* Gp = c.G + (i - 1) * c.pst;
+        int found = 0x7fffffff;
+        for (int base = i - 2; base < x && found == 0x7fffffff; base += kWarp) {
+          const int a = base + lane;
+          const bool hit = a < x && __fadd_rn(Gp[a], wcost(c, a, x, lamf)) == target;
+          const unsigned msk = __ballot_sync(0xffffffffu, hit);
+          if (msk) found = base + __ffs(msk) - 1;
+        }
+        if (found == 0x7fffffff) found = i - 2;  // not reached: the minimum is one of the sums
+        x = found;
+        if (lane == 0) c.sQ[i - 2] = x;
+      }
+    }
+    if (lane == 0) *c.msh = m;
+  }
+  __syncthreads();
+  const int m = *c.msh;
+  if (refine > 0) wrefine(c, lam, m, refine);
+  if (warp_id() == 0) wevaluate(c, lam, refine > 0, m, out);
+  __syncthreads();
+}
+
+constexpr int kWideApproxThreads = 512;
+
+__global__ void __launch_bounds__(kWideApproxThreads, 1) k_approx_wide(ApproxArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ AOut s_out;
+  __shared__ int s_flag;
+  __shared__ int s_misc[2];
+  __shared__ double s_tot[6][kWideApproxThreads / kWarp];
+  const int p = a.p, S = a.s, tid = threadIdx.x, lane = lane_id(), warp = warp_id();
+  constexpr int kNW = kWideApproxThreads / kWarp;
+  WCtx c;
+  c.p = p;
+  c.S = S;
+  c.pst = (p + 3) & ~3;
+  c.dd = static_cast<double>(a.d);
+  c.inv_d = 1.0 / c.dd;
+  c.sQ = reinterpret_cast<int*>(smem);
+  int* sQ1 = c.sQ + S;
+  int* sQ2 = sQ1 + S;
+  c.moved = &s_misc[0];
+  c.msh = &s_misc[1];
+  unsigned char* gs = a.scratch + static_cast<size_t>(blockIdx.x) * a.scratch_per_cta;
+  auto take = [&gs](size_t bytes) {
+    unsigned char* r = gs;
+    gs += (bytes + 255) & ~size_t(255);
+    return r;
+  };
+  c.pre = reinterpret_cast<double*>(take(sizeof(double) * 6 * static_cast<size_t>(p)));
+  c.nb = reinterpret_cast<double*>(take(sizeof(double) * p));
+  c.ab = reinterpret_cast<double*>(take(sizeof(double) * p));
+  c.bb = reinterpret_cast<double*>(take(sizeof(double) * p));
+  c.G = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(S + 1) * c.pst));
+  c.fbuf = reinterpret_cast<double*>(take(sizeof(double) * static_cast<size_t>(kNW) * p));
+
+  for (int r = blockIdx.x; r < a.n; r += gridDim.x) {
+    const double* P = a.P + static_cast<int64_t>(r) * p;
+    const int64_t bo = static_cast<int64_t>(r) * (p - 1);
+    c.P = P;
+    if (tid == 0) s_flag = a.in_status ? a.in_status[r] : 0;
+    for (int k = tid; k < p - 1; k += kWideApproxThreads) {
+      c.nb[k] = static_cast<double>(a.cnt[bo + k]);
+      c.ab[k] = a.A[bo + k];
+      c.bb[k] = a.B[bo + k];
+    }
+    __syncthreads();
+    const bool degenerate = (P[0] == P[p - 1]);
+    int bad = 0;
+    if (!degenerate)
+      for (int k = tid; k < p - 1; k += kWideApproxThreads) bad |= !(P[k] < P[k + 1]);
+    bad = __syncthreads_or(bad);
+    const int32_t st = s_flag != 0 ? s_flag : (bad ? kStatusArg : kStatusOk);
+    if (st != kStatusOk || degenerate) {
+      approx_fill_trivial(a, r, st);
+      __syncthreads();
+      continue;
+    }
+    // prefix sums: each thread scans a contiguous chunk of buckets, then the
+    // chunk totals are scanned across the block
+    {
+      const int nbk = p - 1;
+      const int chunk = (nbk + kWideApproxThreads - 1) / kWideApproxThreads;
+      const int k0 = tid * chunk, k1 = min(k0 + chunk, nbk);
+      const double P0 = P[0];
+      double t[6] = {0, 0, 0, 0, 0, 0};
+      for (int k = k0; k < k1; ++k) {
+        const double u = P[k] - P0, n = c.nb[k], A = c.ab[k];
+        t[0] += n;
+        t[1] += A;
+        t[2] += c.bb[k];
+        t[3] += n * u;
+        t[4] += A * u;
+        t[5] += n * u * u;
+      }
+      double inc[6];
+#pragma unroll
+      for (int j = 0; j < 6; ++j) {
+        double v = t[j];
+#pragma unroll
+        for (int o = 1; o < kWarp; o <<= 1) {
+          const double y = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= o) v += y;
+        }
+        inc[j] = v;
+        if (lane == kWarp - 1) s_tot[j][warp] = v;
+      }
+      __syncthreads();
+      if (warp == 0) {
+#pragma unroll
+        for (int j = 0; j < 6; ++j) {
+          double v = lane < kNW ? s_tot[j][lane] : 0.0;
+#pragma unroll
+          for (int o = 1; o < kWarp; o <<= 1) {
+            const double y = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += y;
+          }
+          if (lane < kNW) s_tot[j][lane] = v;  // inclusive over warps
         }
       }
       __syncthreads();
-      for (int q = threadIdx.x; q < so; q += blockDim.x) {
-        a.Q1[int64_t(r) * so + q] = (q < m1) ? sQ1[q] : -1;
-        a.Q2[int64_t(r) * so + q] = (q < m2) ? sQ2[q] : -1;
-      }
-      if (threadIdx.x == 0) {
-        a.Q1_len[r] = m1;
-        a.Q2_len[r] = m2;
-        a.theta[r] = theta;
-        a.lam_lo[r] = lo;
-        a.lam_hi[r] = hi;
-        a.H1[r] = H1;
-        a.H2[r] = H2;
-        a.HIB1[r] = B1;
-        a.HIB2[r] = B2;
-        a.mse1[r] = M1;
-        a.mse2[r] = M2;
-        a.status[r] = status;
+      double run[6];
+#pragma unroll
+      for (int j = 0; j < 6; ++j) run[j] = (inc[j] - t[j]) + (warp > 0 ? s_tot[j][warp - 1] : 0.0);
+      if (tid == 0)
+        for (int j = 0; j < 6; ++j) c.pre[j * p] = 0.0;
+      for (int k = k0; k < k1; ++k) {
+        const double u = P[k] - P0, n = c.nb[k], A = c.ab[k];
+        run[0] += n;
+        run[1] += A;
+        run[2] += c.bb[k];
+        run[3] += n * u;
+        run[4] += A * u;
+        run[5] += n * u * u;
+#pragma unroll
+        for (int j = 0; j < 6; ++j) c.pre[j * p + k + 1] = run[j];
       }
     }
+    __syncthreads();
+    approx_drive(a, r, c.sQ, sQ1, sQ2, S, (P[p - 1] - P[0]) * (P[p - 1] - P[0]), s_out,
+                 [&](double lam) { approx_solve_wide(c, lam, a.refine, &s_out); });
     __syncthreads();
   }
 }
@@ -692,13 +1087,29 @@ size_t al256(size_t b) { return (b + 255) & ~size_t(255); }
 }  // namespace
 
 bool approx_plan(int n, int p, int s, bool fp64, ApproxPlan* plan) {
-  if (p < 2 || p > kMaxP || s < 2 || n < 1) return false;
+  if (p < 2 || p > kMaxPWide || s < 2 || n < 1) return false;
   const int S = s < p ? s : p;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   int sms = 0, optin = 0;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  plan->wide = p > kMaxP;
+  if (plan->wide) {
+    // large alphabets: fp32 layers only, one CTA per SM, O(p) slab per CTA
+    if (fp64) return false;
+    const size_t pst = static_cast<size_t>((p + 3) & ~3);
+    plan->fp64 = false;
+    plan->smem = false;
+    plan->split = false;
+    plan->threads = kWideApproxThreads;
+    plan->smem_bytes = al16(sizeof(int) * 3 * static_cast<size_t>(S));
+    plan->scratch_per_cta = al256(8 * 6 * static_cast<size_t>(p)) + 3 * al256(8 * static_cast<size_t>(p)) +
+                            al256(4 * static_cast<size_t>(S + 1) * pst) +
+                            al256(8 * static_cast<size_t>(kWideApproxThreads / kWarp) * p);
+    plan->ctas = n < sms ? n : sms;
+    return true;
+  }
   const size_t tsz = fp64 ? 8 : 4;
   const int kvec = static_cast<int>(16 / tsz);
   int ncv = 0;
@@ -735,8 +1146,8 @@ bool approx_plan(int n, int p, int s, bool fp64, ApproxPlan* plan) {
 
 cudaError_t launch_approx(const ApproxPlan& plan, ApproxArgs args, cudaStream_t st) {
   void* kargs[] = {&args};
-  cudaError_t e = cudaLaunchKernel(approx_fn(plan.fp64, plan.smem, plan.split), dim3(plan.ctas), dim3(plan.threads), kargs,
-                                   plan.smem_bytes, st);
+  void* fn = plan.wide ? reinterpret_cast<void*>(&k_approx_wide) : approx_fn(plan.fp64, plan.smem, plan.split);
+  cudaError_t e = cudaLaunchKernel(fn, dim3(plan.ctas), dim3(plan.threads), kargs, plan.smem_bytes, st);
   note_launch();
   return e;
 }

@@ -7,7 +7,8 @@
 namespace ecasq {
 
 constexpr int kWarp = 32;
-constexpr int kMaxP = 512;    // largest alphabet the kernels accept
+constexpr int kMaxP = 512;    // largest alphabet of the exact solver and of the shared-memory kernels
+constexpr int kMaxPWide = 65536;  // largest alphabet of bucketing, encoding and the approximation
 constexpr int kMaxS = 255;    // largest code size
 
 // Per-vector status codes written by the device (mirrors include/ecasq.h).

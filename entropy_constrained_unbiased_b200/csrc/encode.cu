@@ -335,6 +335,114 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
     encode_row<false>(X, Pall, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, idx, hist, status, smem, S, s_wexact);
 }
 
+// Encoder for large alphabets (p > 512): no per-bucket tables; the interval of
+// an entry is found by bisection over the code's values (at most 256), the
+// largest t <= m-2 with q_t <= x, exactly as the rounding rule reads. Same
+// randomness, tests and outputs as k_encode.
+__global__ void __launch_bounds__(kEncThreads)
+k_encode_code(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d, int p, int s,
+              const int32_t* __restrict__ Q1, const int32_t* __restrict__ Q1_len, const int32_t* __restrict__ Q2,
+              const int32_t* __restrict__ Q2_len, const double* __restrict__ theta, const Philox4x32::RoundKeys K,
+              uint8_t* __restrict__ idx, unsigned long long* __restrict__ hist, int32_t* __restrict__ status) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ int s_m[2];
+  __shared__ int s_bad;
+  const int r = blockIdx.y;
+  double* sq = reinterpret_cast<double*>(smem);                      // [2][s] code values
+  unsigned int* sh = reinterpret_cast<unsigned int*>(sq + 2 * s);   // [warps][2s] counts
+  const int nbins = 2 * s;
+  const double* P = Pall + static_cast<int64_t>(r) * p;
+  const bool has2 = (Q2 != nullptr);
+  const double th = (has2 && theta) ? theta[r] : 0.0;
+  const bool mix = has2 && th > 0.0 && th < 1.0;
+  const int fixed_part = (!has2 || th >= 1.0) ? 0 : 1;
+  if (threadIdx.x == 0) {
+    s_bad = 0;
+    s_m[0] = Q1_len[r];
+    s_m[1] = has2 ? Q2_len[r] : 0;
+  }
+  for (int k = threadIdx.x; k < kEncWarps * nbins; k += blockDim.x) sh[k] = 0u;
+  __syncthreads();
+  int bad_code = 0;
+  for (int part = 0; part < 2; ++part) {
+    const int m = s_m[part];
+    const int32_t* Q = (part == 0 ? Q1 : Q2);
+    const bool used = (part == 0) ? (fixed_part == 0 || mix) : (fixed_part == 1 || mix);
+    if (!used) continue;
+    if (Q == nullptr || m < 1 || m > s) {
+      bad_code = 1;
+      continue;
+    }
+    const int32_t* q = Q + static_cast<int64_t>(r) * s;
+    for (int t = threadIdx.x; t < m; t += blockDim.x) {
+      if (q[t] < 0 || q[t] >= p || (t > 0 && q[t] <= q[t - 1]))
+        bad_code = 1;
+      else
+        sq[part * s + t] = P[q[t]];
+    }
+  }
+  if (__syncthreads_or(bad_code)) {
+    if (threadIdx.x == 0) status[r] = kStatusArg;
+    return;
+  }
+  const uint32_t th_last = mix ? static_cast<uint32_t>(static_cast<uint64_t>(ceil(th * 0x1p32)) - 1u) : 0u;
+  const int64_t beg = static_cast<int64_t>(blockIdx.x) * kEncChunk;
+  const int len = static_cast<int>((beg + kEncChunk < d ? beg + kEncChunk : d) - beg);
+  const float* x = X + static_cast<int64_t>(r) * d + beg;
+  uint8_t* o = idx + static_cast<int64_t>(r) * d + beg;
+  const uint32_t blk0 = static_cast<uint32_t>(static_cast<uint64_t>(beg) >> 2);
+  const uint32_t wh_base = smem_addr(sh + warp_id() * nbins);
+  int bad = 0;
+  for (int j = 4 * threadIdx.x; j < len; j += 4 * kEncThreads) {
+    const int cnt = len - j < 4 ? len - j : 4;
+    const uint32_t blk = blk0 + static_cast<uint32_t>(j >> 2);
+    const uint4 ru = Philox4x32::block(make_uint4(blk, static_cast<uint32_t>(r), 0u, 0u), K);
+    uint4 su = make_uint4(0u, 0u, 0u, 0u);
+    if (mix) su = Philox4x32::block(make_uint4(blk, static_cast<uint32_t>(r), 1u, 0u), K);
+    const uint32_t rw[4] = {ru.x, ru.y, ru.z, ru.w};
+    const uint32_t sel[4] = {su.x, su.y, su.z, su.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (e >= cnt) continue;
+      const int part = mix ? (sel[e] <= th_last ? 0 : 1) : fixed_part;
+      const int m = s_m[part];
+      const double* qv = sq + part * s;
+      const double xd = static_cast<double>(__ldcs(x + j + e));
+      int out = 0;
+      if (m == 1) {
+        if (xd != qv[0]) bad = 1;
+      } else if (!(xd >= qv[0]) || !(xd <= qv[m - 1])) {
+        bad = 1;
+      } else {
+        int lo = 0, hi = m - 2;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (qv[mid] <= xd)
+            lo = mid;
+          else
+            hi = mid - 1;
+        }
+        const double y = __dsub_rn(xd, qv[lo]);
+        const double w = __dsub_rn(qv[lo + 1], qv[lo]);
+        const double u = __dmul_rn(static_cast<double>(rw[e]), 0x1p-32);
+        out = lo + ((__dmul_rn(u, w) < y) ? 1 : 0);
+      }
+      o[j + e] = static_cast<uint8_t>(out);
+      red_shared_inc(wh_base + 4u * static_cast<uint32_t>(part * s + out));
+    }
+  }
+  if (bad) s_bad = 1;
+  __syncthreads();
+  unsigned long long* gh = hist + static_cast<int64_t>(r) * nbins;
+  for (int b = threadIdx.x; b < nbins; b += blockDim.x) {
+    unsigned long long tot = 0;
+#pragma unroll
+    for (int w = 0; w < kEncWarps; ++w) tot += sh[w * nbins + b];
+    if (tot) atomicAdd(gh + b, tot);
+  }
+  if (threadIdx.x == 0 && s_bad) status[r] = kStatusRange;
+}
+
 // H = (d0 H0 + d1 H1)/(d0 + d1), H_part = -sum c/d_part log2(c/d_part). One warp per row.
 __global__ void k_entropy(const int64_t* __restrict__ hist, int n, int s, double* __restrict__ H) {
   const int r = blockIdx.x * (blockDim.x / kWarp) + warp_id();
@@ -377,8 +485,14 @@ cudaError_t launch_encode(const float* X, const double* P, int n, int64_t d, int
   const size_t smem = encode_smem(p, s);
   const Philox4x32::RoundKeys K =
       Philox4x32::round_keys(static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
-  k_encode<<<dim3(nc, n), kEncThreads, smem, st>>>(X, P, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, idx,
-                                                    reinterpret_cast<unsigned long long*>(hist), status);
+  if (p > kMaxP) {
+    const size_t sm2 = sizeof(double) * 2 * s + sizeof(unsigned int) * kEncWarps * 2 * s;
+    k_encode_code<<<dim3(nc, n), kEncThreads, sm2, st>>>(X, P, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, idx,
+                                                         reinterpret_cast<unsigned long long*>(hist), status);
+  } else {
+    k_encode<<<dim3(nc, n), kEncThreads, smem, st>>>(X, P, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, idx,
+                                                      reinterpret_cast<unsigned long long*>(hist), status);
+  }
   note_launch();
   return cudaGetLastError();
 }

@@ -1035,6 +1035,68 @@ k_grid_bucket_rows(const float* __restrict__ X, int n, int64_t d, int p, int fb,
   }
 }
 
+// ---------------------------------------------------------------------------
+// Bucketing for alphabets beyond the shared-memory counters (p > 512, up to
+// 65536 values, e.g. every BF16 value of a range): the bucket by bisection on
+// the row of P, the offset v as in k_bucket (uniform rows: (x - P_k)/D + eta_k;
+// other rows: (x - P_k)/D_k), and 64-bit global additions of the count and the
+// two fixed-point moments. A large alphabet spreads the entries over many
+// buckets, so few additions contend.
+
+constexpr int kGenThreads = 256;
+constexpr int64_t kGenChunk = 16384;
+
+__global__ void __launch_bounds__(kGenThreads)
+k_bucket_general(const float* __restrict__ X, int64_t d, const double* __restrict__ Pall, int p, int fb,
+                 unsigned long long* __restrict__ acc, int32_t* __restrict__ flag) {
+  __shared__ int s_bad;
+  const int r = blockIdx.y;
+  const int nb = p - 1;
+  const double* P = Pall + static_cast<int64_t>(r) * p;
+  if (threadIdx.x == 0) s_bad = 0;
+  const RowGrid g = row_grid(P, p);
+  const bool uni = row_is_uniform(P, p, g, nullptr);  // includes a barrier
+  const double twoF = ldexp(1.0, fb);
+  const double P0 = P[0], Pl = P[p - 1];
+  const int64_t beg = static_cast<int64_t>(blockIdx.x) * kGenChunk;
+  const int64_t end = beg + kGenChunk < d ? beg + kGenChunk : d;
+  const float* x = X + static_cast<int64_t>(r) * d;
+  unsigned long long* ga = acc + static_cast<int64_t>(r) * nb * 3;
+  int bad = 0;
+  for (int64_t i = beg + threadIdx.x; i < end; i += kGenThreads) {
+    const double xd = static_cast<double>(__ldcs(x + i));
+    if (!(xd >= P0) || !(xd <= Pl)) {
+      bad = 1;
+      continue;
+    }
+    int lo = 0, hi = p - 2;  // the largest k <= p-2 with P_k <= x
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (P[mid] <= xd)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    const int k = lo;
+    const double y = __dsub_rn(xd, P[k]);
+    double v;
+    if (uni) {
+      v = __dadd_rn(__dmul_rn(y, g.invD), grid_eta(P[k], g.P0, g.invD, k));
+    } else {
+      const double w = __dsub_rn(P[k + 1], P[k]);
+      v = w > 0.0 ? __ddiv_rn(y, w) : 0.0;
+    }
+    v = fmin(fmax(v, 0.0), 1.0);
+    unsigned long long* c = ga + 3 * static_cast<int64_t>(k);
+    atomicAdd(c, 1ull);
+    atomicAdd(c + 1, __double2ull_rn(v * twoF));
+    atomicAdd(c + 2, __double2ull_rn(__dmul_rn(v, v) * twoF));
+  }
+  if (bad) s_bad = 1;
+  __syncthreads();
+  if (threadIdx.x == 0 && s_bad) atomicOr(flag + r, 1);
+}
+
 // Fixed-point row sums -> cnt (int64), A = sum (x - P_k), B = sum (x - P_k)^2 (fp64).
 __global__ void k_bucket_finish(const unsigned long long* __restrict__ acc, const double* __restrict__ Pall,
                                 int p, int fb, const int32_t* __restrict__ flag, int64_t* __restrict__ cnt,
@@ -1127,7 +1189,10 @@ cudaError_t launch_bucket(const float* X, const double* P, int n, int64_t d, int
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   const int64_t wide_items = static_cast<int64_t>(n) * ((d + kWideChunk - 1) / kWideChunk);
-  if (p - 1 <= kWideBuckets && d >= kWideChunk && wide_items >= sms) {
+  if (p > kMaxP) {
+    const int nc = static_cast<int>((d + kGenChunk - 1) / kGenChunk);
+    k_bucket_general<<<dim3(nc, n), kGenThreads, 0, st>>>(X, d, P, p, fb, acc, flag);
+  } else if (p - 1 <= kWideBuckets && d >= kWideChunk && wide_items >= sms) {
     e = wide_smem_attribute(dev);
     if (e != cudaSuccess) return e;
     k_bucket_wide<<<sms, kWideThreads, kWideSmem, st>>>(X, n, d, P, p, fb, acc, flag);

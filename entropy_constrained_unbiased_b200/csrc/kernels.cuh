@@ -136,6 +136,7 @@ struct ApproxArgs {
 };
 
 struct ApproxPlan {
+  bool wide;  // alphabet beyond 512 values: pair terms from prefix sums (fp32 layers only)
   bool fp64;
   bool smem;  // cost table and layers in shared memory
   bool split;  // each column's a range shared by two threads (few vectors)

@@ -32,8 +32,11 @@
  *     [min X, max X], so both ends are forced by unbiasedness there).
  *   - A code Q is returned as ascending indices into the vector's row of P,
  *     padded with -1 up to s; Q_len holds |Q|.
- *   - Limits: 2 <= p <= 512, 2 <= s <= 255 (s > p is treated as s = p),
- *     1 <= d <= 2^31 - 1, n >= 1.
+ *   - Limits: 2 <= s <= 255 (s > p is treated as s = p), 1 <= d <= 2^31 - 1,
+ *     n >= 1; 2 <= p <= 512 for the exact solver (ecasq_solve*,
+ *     ecasq_workspace_size), 2 <= p <= 65536 for the grid, bucketing,
+ *     encoding and the approximation (large alphabets, e.g. every BF16 value of
+ *     a range; above 512 values the approximation runs fp32 layers only).
  *   - Entropies are in bits per entry; the MSE is the per-entry mean
  *     (1/d) * sum (q_hi - x)(x - q_lo); the objective is MSE + lambda * H.
  */
@@ -196,7 +199,14 @@ int ecasq_solve_budget_stats(const int64_t* cnt, const double* A, const double* 
  *
  * Layers run in fp32 (default) or fp64 (opts->dp_fp64); refinement and the
  * reported figures are fp64. opts->hirschberg is ignored (no back-pointers are
- * kept). Workspace: ecasq_approx_workspace_size. Returns as the exact solver. */
+ * kept). Workspace: ecasq_approx_workspace_size. Returns as the exact solver.
+ *
+ * Alphabets of more than 512 values (up to 65536): the pair terms are computed
+ * for every relaxation from six O(p) prefix sums over the buckets instead of
+ * O(p^2) tables (memory O(p s) per vector), the layers run in fp32 (dp_fp64 = 1
+ * returns ECASQ_ERR_ARG), the refinement compares local costs from the same
+ * prefix sums in fp64, and the reported figures are direct fp64 sums over each
+ * interval's buckets. Time O(p^2 s) per solve. */
 size_t ecasq_approx_workspace_size(int n, int64_t d, int p, int s, const ecasq_opts* opts);
 
 /* Per row and multiplier (lambda [n][n_lambda] >= 0): the code Q [n][n_lambda][s]

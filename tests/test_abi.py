@@ -44,14 +44,18 @@ def test_argument_errors_return_before_cuda(lib):
     assert lib.ecasq_uniform_grid(null, 1, 16, 8, null, null, null, 0, null) == -1
     assert lib.ecasq_bucket(null, null, 1, 16, 1, null, null, null, null, null, 0, null) == -1
     assert lib.ecasq_aux_workspace_size(0, 16, 8) == 0
-    assert lib.ecasq_aux_workspace_size(4, 16, 600) == 0
+    # alphabet-sized passes (grid, bucketing, encoding, approximation) take up to
+    # 65536 values, the exact solver up to 512
+    assert lib.ecasq_aux_workspace_size(4, 16, 65537) == 0
+    assert lib.ecasq_aux_workspace_size(4, 16, 600) > 0
     assert lib.ecasq_aux_workspace_size(4, 1024, 64) > 0
+    assert lib.ecasq_workspace_size(4, 16, 600, 4, 1, None) == 0
     assert lib.ecasq_entropy(null, 1, 4, null, null) == -1
     assert lib.ecasq_encode(null, null, 1, 16, 8, 4, null, null, null, null, null, 1, null, null, null, null) == -1
     # approximation: null X, negative refinement count, bad sizes
     dummy = C.c_void_p(16)  # never dereferenced: the checks fail first
     assert lib.ecasq_approx_workspace_size(0, 16, 8, 4, None) == 0
-    assert lib.ecasq_approx_workspace_size(4, 16, 600, 4, None) == 0
+    assert lib.ecasq_approx_workspace_size(4, 16, 65537, 4, None) == 0
     assert lib.ecasq_solve_approx(null, dummy, 1, 16, 8, 4, dummy, 1, 0, *[dummy] * 7, None, dummy, 64, null) == -1
     assert lib.ecasq_solve_approx_stats(dummy, dummy, dummy, dummy, 1, 16, 8, 4, dummy, 1, -1, *[dummy] * 7, None,
                                         dummy, 64, null) == -1

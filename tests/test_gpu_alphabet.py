@@ -80,3 +80,100 @@ def test_solver_on_a_bf16_alphabet(E, O, fp64, tol):
             assert np.all((vals.astype(np.float32).view(np.uint32) & 0xFFFF) == 0)
             mse, H, _ = O.eval_raw(X[r], vals)
             assert mse + lam[r, t] * H <= ref["J"][r, t] * (1 + tol) + 1e-300
+
+
+# -- large alphabets (p > 512): bucketing, the approximation, encoding -------------
+
+def _wide_rows(seed, n, d):
+    """Rows whose BF16 alphabet is the same 1237 values (0.0498 .. 40): each row
+    holds 0.05 and 40, the rest lognormal in between."""
+    rng = np.random.default_rng([59, seed])
+    X = np.exp(rng.uniform(np.log(0.05), np.log(40.0), size=(n, d)) + 0.3 * rng.standard_normal((n, d)))
+    X = np.clip(X, 0.05, 40.0).astype(np.float32)
+    X[:, 0], X[:, 1] = np.float32(0.05), np.float32(40.0)
+    return X
+
+
+@pytest.fixture(scope="module")
+def wide(E):
+    X = _wide_rows(0, 3, 20000)
+    Pd, p_len, st = E.bf16_alphabet(torch.from_numpy(X).cuda(), 2048)
+    p = int(p_len[0].item())
+    assert int(st.abs().sum()) == 0 and np.all(p_len.cpu().numpy() == p) and p > 512
+    P = Pd[:, :p].contiguous()
+    return X, P, p
+
+
+def test_bucket_large_alphabet(E, O, wide):
+    X, P, p = wide
+    cnt, A, B, st = E.bucket(torch.from_numpy(X).cuda(), P)
+    assert int(st.abs().sum()) == 0
+    Pn = P.cpu().numpy()
+    for r in range(X.shape[0]):
+        co, Ao, Bo, so = O.bucket(X[r], Pn[r])
+        assert so == 0
+        np.testing.assert_array_equal(cnt[r].cpu().numpy(), co)
+        span = Pn[r, -1] - Pn[r, 0]
+        np.testing.assert_allclose(A[r].cpu().numpy(), Ao, rtol=1e-9, atol=1e-12 * span)
+        np.testing.assert_allclose(B[r].cpu().numpy(), Bo, rtol=1e-9, atol=1e-12 * span ** 2)
+
+
+@pytest.mark.parametrize("refine", [0, 4])
+def test_approx_large_alphabet(E, O, wide, refine):
+    """The approximation on a 1237-value BF16 alphabet (fp32 layers, pair terms
+    from prefix sums): the code's objective within 1e-5 of the oracle's optimum
+    (plain), the GPU's fp64 figures of its code equal to the oracle's raw
+    evaluation, every code value a BF16 number; refined codes never worse
+    than the plain ones on the exact objective."""
+    X, P, p = wide
+    Xd = torch.from_numpy(X).cuda()
+    lam = np.var(X.astype(np.float64), axis=1)[:, None] * np.array([[0.0, 0.003, 0.03]])
+    s = 12
+    g = E.solve_approx(Xd, P, s, torch.from_numpy(lam).cuda(), refine=refine)
+    assert int(g["status"].abs().sum()) == 0
+    Pn = P.cpu().numpy()
+    Q, m = g["Q"].cpu().numpy(), g["Q_len"].cpu().numpy()
+    ref = O.solve_approx_batch(X, Pn, s, lam, refine=0)
+    for r in range(X.shape[0]):
+        for t in range(lam.shape[1]):
+            vals = Pn[r][Q[r, t, : m[r, t]]]
+            assert np.all((vals.astype(np.float32).view(np.uint32) & 0xFFFF) == 0)
+            mse, H, _ = O.eval_raw(X[r], vals)
+            hib = O.eval_raw_ib(X[r], vals)
+            assert g["mse"][r, t].item() == pytest.approx(mse, rel=1e-9)
+            assert g["H"][r, t].item() == pytest.approx(H, rel=1e-9, abs=1e-12)
+            assert g["H_IB"][r, t].item() == pytest.approx(hib, rel=1e-9, abs=1e-12)
+            J_ib = mse + lam[r, t] * hib
+            if refine == 0:
+                assert J_ib <= ref["J"][r, t] * (1 + 1e-5), (r, t, J_ib, ref["J"][r, t])
+                assert g["objective"][r, t].item() == pytest.approx(J_ib, rel=1e-9)
+            else:
+                assert g["objective"][r, t].item() == pytest.approx(mse + lam[r, t] * H, rel=1e-9)
+                # refinement starts from the plain code and only moves on a decrease
+                mse0, H0, _ = O.eval_raw(X[r], Pn[r][ref["Q"][r, t, : ref["m"][r, t]]])
+                assert mse + lam[r, t] * H <= (mse0 + lam[r, t] * H0) * (1 + 1e-5) + 1e-300
+
+
+def test_approx_budget_and_encode_large_alphabet(E, O, wide):
+    X, P, p = wide
+    Xd = torch.from_numpy(X).cuda()
+    s, b = 12, 2.5
+    g = E.solve_approx_budget(Xd, P, s, b, refine=0, steps=30)
+    gn = {k: v.cpu().numpy() for k, v in g.items()}
+    assert np.all(gn["status"] == 0)
+    Pn = P.cpu().numpy()
+    ref = O.solve_approx_budget_batch(X, Pn, s, b, 30, refine=0)
+    for r in range(X.shape[0]):
+        th = gn["theta"][r]
+        if 0 < th < 1:
+            assert th * gn["H_IB1"][r] + (1 - th) * gn["H_IB2"][r] == pytest.approx(b, rel=1e-12)
+        d_gpu = th * gn["mse1"][r] + (1 - th) * gn["mse2"][r]
+        d_ref = ref["theta"][r] * ref["mse1"][r] + (1 - ref["theta"][r]) * ref["mse2"][r]
+        assert d_gpu == pytest.approx(d_ref, rel=1e-5), (r, d_gpu, d_ref)
+    # time-shared encoding on the large alphabet: bit-exact against the oracle
+    idx, hist, est = E.encode(Xd, P, s, g["Q1"], g["Q1_len"], 7, g["Q2"], g["Q2_len"], g["theta"])
+    assert int(est.abs().sum()) == 0
+    io, ho, so = O.encode_batch(X, Pn, gn["Q1"], gn["Q1_len"], s, 7, gn["Q2"], gn["Q2_len"], gn["theta"])
+    assert np.all(so == 0)
+    np.testing.assert_array_equal(idx.cpu().numpy(), io)
+    np.testing.assert_array_equal(hist.cpu().numpy(), ho)
