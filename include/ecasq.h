@@ -131,9 +131,12 @@ int ecasq_grid_bucket(const float* X, int n, int64_t d, int p, double* P, int64_
  * p = 128 or n <= 1369 at p = 256; larger sizes return ECASQ_ERR_WORKSPACE
  * and launch nothing. The call allocates nothing: the first call on a device
  * resolves the array's device address (with that device current), so make
- * that first call before any stream capture. Every call on a device shares
- * the array (the call clears it on the stream before use): calls that overlap
- * on the same GPU race, so serialise them (one stream, or events). */
+ * that first call before any stream capture. The address is kept for the
+ * life of the process: a cudaDeviceReset (or any other teardown of the
+ * device's primary context) invalidates it, so do not call this entry point on
+ * a device after resetting it. Every call on a device shares the array (the
+ * call clears it on the stream before use): calls that overlap on the same
+ * GPU race, so serialise them (one stream, or events). */
 int ecasq_bucket_noalloc(const float* X, const double* P, int n, int64_t d, int p, int64_t* cnt,
                          double* A, double* B, int32_t* status, void* stream);
 

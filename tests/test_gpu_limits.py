@@ -87,3 +87,23 @@ def test_sizes_out_of_range_are_rejected(E):
     assert L.ecasq_approx_workspace_size(1, 0, 64, 8, None) == 0
     assert L.ecasq_encode(dummy, dummy, 1, 100, 64, 257, dummy, dummy, null, null, null, 1, dummy, dummy, dummy,
                           null) == -1
+
+
+def test_bucket_sums_do_not_overflow_on_long_rows(E, O):
+    """One row of 2^27 + 5 entries with p = 2, every entry in the one bucket
+    (the worst case for the 64-bit fixed-point sums): rows of 2^27 entries or
+    more keep 32 fraction bits, so the sums stay below 2^63. Counts exact and
+    moments to 1e-9 against the oracle's compensated sums."""
+    d = (1 << 27) + 5
+    rng = np.random.default_rng(61)
+    X = rng.random((1, d), dtype=np.float32)
+    X[0, 0], X[0, 1] = 0.0, 1.0
+    Xd = torch.from_numpy(X).cuda()
+    P, cnt, A, B, st = E.grid_bucket(Xd, 2)
+    assert int(st.abs().sum()) == 0 and int(cnt[0, 0]) == d
+    Po, _ = O.grid_batch(X, 2)
+    np.testing.assert_array_equal(P.cpu().numpy(), Po)
+    co, Ao, Bo, so = O.bucket(X[0], Po[0])
+    assert so == 0 and int(co[0]) == d
+    assert float(A[0, 0]) == pytest.approx(Ao[0], rel=1e-9)
+    assert float(B[0, 0]) == pytest.approx(Bo[0], rel=1e-9)
