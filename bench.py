@@ -59,6 +59,61 @@ def triples_per_solve(p: int, s: int) -> int:
     return t
 
 
+def _su(n: int) -> int:  # 1 + 2 + ... + n (0 for n <= 0)
+    return n * (n + 1) // 2 if n > 0 else 0
+
+
+def _sq(n: int) -> int:  # 1 + 4 + ... + n^2 (0 for n <= 0)
+    return n * (n + 1) * (2 * n + 1) // 6 if n > 0 else 0
+
+
+def pass_triples(s0: int, e0: int, T: int, last_only: bool) -> int:
+    """(k, l, j) triples of one forward pass over the alphabet range s0..e0
+    with T values from c_1 = P_s0: layer 2 has only k = s0; layer t >= 3 every
+    s0 + t - 2 <= k < l < j <= e0 with l >= s0 + t - 1; the last layer only
+    j = e0 when last_only. The whole-alphabet pass (0, p-1, S-1, True) is
+    triples_per_solve(p, s)."""
+    tot = 0
+    for t in range(2, T + 1):
+        last = last_only and t == T
+        a, b = s0 + t - 1, e0 - 1  # rows l
+        if a > b:
+            continue
+        if t == 2:
+            tot += (b - a + 1) if last else _su(e0 - a) - _su(e0 - b - 1)
+            continue
+        kmin = s0 + t - 2
+        ua, ub = a - kmin, b - kmin  # u = l - kmin >= 1: the k values of row l
+        su = _su(ub) - _su(ua - 1)
+        tot += su if last else (e0 - kmin) * su - (_sq(ub) - _sq(ua - 1))
+    return tot
+
+
+def hirschberg_triples(code, p: int, s: int) -> int:
+    """Triples one Hirschberg-mode solve evaluates, given the code it found
+    (indices into P, c_0 = 0 .. c_{m-1} = p-1): the whole-alphabet forward
+    pass, then per segment (lo, hi) of unknown values c[lo+1 .. hi-1] with
+    mid = lo + ceil((hi - lo - 1) / 2) a forward pass from c[lo] over
+    c[lo] .. c[hi] with mid - lo + 1 values (only the last value c[hi] in its
+    last layer when mid + 1 = hi) and a pass over the reflected range with
+    hi - mid values; segments split at (c[mid], c[mid+1])."""
+    S = min(s, p)
+    tot = pass_triples(0, p - 1, S - 1, True)
+    m = len(code)
+    stack = [(0, m - 2)] if m >= 4 else []
+    while stack:
+        lo, hi = stack.pop()
+        mid = lo + (hi - lo) // 2  # lo + ceil((hi - lo - 1) / 2)
+        qlo, qhi = int(code[lo]), int(code[hi])
+        tot += pass_triples(qlo, qhi, mid - lo + 1, mid + 1 == hi)
+        tot += pass_triples(p - 1 - qhi, p - 1 - qlo, hi - mid, False)
+        if mid - lo - 1 >= 1:
+            stack.append((lo, mid))
+        if hi - mid - 2 >= 1:
+            stack.append((mid + 1, hi))
+    return tot
+
+
 def relaxations_per_solve(p: int, s: int) -> int:
     """(i, a, x) relaxations G_{i-1}(a) + w(a, x) one solve of the approximation's
     layered shortest path evaluates: layers i = 2 .. S, x = i-1 .. p-1, a = i-2 .. x-1."""
@@ -279,10 +334,16 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
         enc_args = (out["Q"][:, 0, :].contiguous(), out["Q_len"][:, 0].contiguous(), w.seed_encode)
     hbm_kernels.update(stage_figures(E, X, P_last, p, s, enc_args, stream, flush, hbm))
     hbm_kernels["input"] = f"this workload ({n} x {d})"
-    # The HBM-bound stages on the gradients input (256 x 2^20 fp32 = 1 GiB,
-    # larger than L2), with codes from the exact budget solver on it.
-    if w.name != "gradients" and not args.no_gradients_stages:
-        hbm_kernels["gradients_input"] = gradients_stage_figures(E, dev, stream, flush, hbm, rank)
+    sm_max = float(peaks.get("sm_max_mhz", 1965.0))
+    mufu_peak = MUFU_LG2_PER_CLK_PER_SM * B200_SMS * sm_max * 1e6
+    # The other workloads' exact solves, and the HBM-bound stages on the
+    # gradients input (256 x 2^20 fp32 = 1 GiB, larger than L2) with codes from
+    # the exact budget solver on it.
+    dp_workloads = {}
+    if w.name == "weights" and not args.no_other_workloads:
+        hbm_kernels["gradients_input"], dp_workloads["gradients"] = gradients_figures(
+            E, dev, stream, flush, hbm, mufu_peak, rank)
+        dp_workloads.update(small_dp_figures(E, dev, stream, flush, mufu_peak, rank))
     # hardware-aware alphabet (BF16 values covering each row), p_max = 512: one
     # read of X plus the alphabet rows written
     E.bf16_alphabet(X, 512)
@@ -319,8 +380,6 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
                                   "frac": (entries + coded_bits / 8) / (rc_t * 1e-3) / 1e9 / hbm,
                                   "status_nonzero_rows": int((rst != 0).sum().item())}
     del words
-    sm_max = float(peaks.get("sm_max_mhz", 1965.0))
-    mufu_peak = MUFU_LG2_PER_CLK_PER_SM * B200_SMS * sm_max * 1e6
     dp_avg_ms = float(np.mean(dp_ms))
     achieved = n_solves * tps / (dp_avg_ms * 1e-3)
     total_triples = world * n_solves * tps  # one step, all ranks
@@ -355,10 +414,17 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
         "e2e": {"value": total_triples / (float(np.mean(e2e_ms)) * 1e-3), "unit": "triples/s",
                 "h2d_bytes_per_step": n * d * 4, "d2h_bytes_per_step": bo},
         "hbm_kernels": hbm_kernels,
+        "dp_workloads": dp_workloads,
         "approx": approx,
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
     }
+    if w.hirschberg:
+        ev = evaluated_triples(w, out)
+        line["roofline"]["evaluated_triples_per_step"] = ev
+        line["roofline"]["evaluated_frac"] = ev / (dp_avg_ms * 1e-3) / mufu_peak
+        line["roofline"]["note"] = ("achieved/frac count the whole-alphabet pass; evaluated_* adds the divide and "
+                                    "conquer's recovery passes")
     return line
 
 
@@ -382,19 +448,87 @@ def stage_figures(E, X, P, p, s, enc_args, stream, flush, hbm):
     return out
 
 
-def gradients_stage_figures(E, dev, stream, flush, hbm, rank):
+def dp_figure(E, w: W.Workload, cnt, A, B, P, stream, flush, mufu_peak, reps=2):
+    """Device time of one exact-solver call on a workload's bucket statistics
+    (L2 flushed before each call) and its triples/s against the MUFU peak.
+    Hirschberg's recovery passes are work the triple count leaves out."""
+    import torch
+
+    if w.mode == "budget":
+        def call():
+            return E.solve_budget_stats(cnt, A, B, P, w.d, w.s, w.b, w.steps)
+    else:
+        lam = torch.from_numpy(w.lambdas()).to(P.device)
+
+        def call():
+            return E.solve_stats(cnt, A, B, P, w.d, w.s, lam, hirschberg=w.hirschberg)
+    out = call()
+    torch.cuda.synchronize()
+    ms = device_ms(call, stream, flush, reps=reps)
+    ns = solves_done(w, out)
+    tps = triples_per_solve(w.p, w.s)
+    ach = ns * tps / (ms * 1e-3)
+    res = {"workload": describe(w), "ms": ms, "solves": ns, "triples_per_solve": tps, "achieved": ach,
+           "frac": ach / mufu_peak, "status_nonzero_rows": int((out["status"] != 0).sum().item())}
+    if w.hirschberg:
+        ev = evaluated_triples(w, out)
+        res["note"] = ("achieved/frac count the whole-alphabet pass only (the metric's triples); the "
+                       "evaluated_* figures add the recovery passes of the divide and conquer")
+        res["evaluated_triples"] = ev
+        res["evaluated_achieved"] = ev / (ms * 1e-3)
+        res["evaluated_frac"] = ev / (ms * 1e-3) / mufu_peak
+    return res, out
+
+
+def evaluated_triples(w: W.Workload, out) -> int:
+    """Triples the Hirschberg-mode solves of a fixed-lambda call evaluated,
+    from the codes they returned (rows with a nonzero status, lambda = 0 and
+    constant rows are left out)."""
+    Q = out["Q"].cpu().numpy()
+    m = out["Q_len"].cpu().numpy()
+    st = out["status"].cpu().numpy()
+    lam = w.lambdas()
+    tot = 0
+    for r in range(Q.shape[0]):
+        if st[r] != 0:
+            continue
+        for t in range(Q.shape[1]):
+            if lam[r, t] > 0 and m[r, t] >= 2:
+                tot += hirschberg_triples(Q[r, t, : m[r, t]], w.p, w.s)
+    return tot
+
+
+def gradients_figures(E, dev, stream, flush, hbm, mufu_peak, rank):
+    """On the gradients input (256 x 2^20 fp32 = 1 GiB, larger than L2): the
+    exact budget solve (k_dp) and the HBM-bound stages, with the codes of that
+    solve for the encoder."""
     import torch
 
     g = W.WORKLOADS["gradients"]
     X = torch.from_numpy(W.make_inputs(g, rank=rank)).to(dev)
     P, _ = E.uniform_grid(X, g.p)
     cnt, A, B, _ = E.bucket(X, P)
-    o = E.solve_budget_stats(cnt, A, B, P, g.d, g.s, g.b, g.steps)
+    dp, o = dp_figure(E, g, cnt, A, B, P, stream, flush, mufu_peak)
     del cnt, A, B
     enc = (o["Q1"], o["Q1_len"], g.seed_encode, o["Q2"], o["Q2_len"], o["theta"])
     res = stage_figures(E, X, P, g.p, g.s, enc, stream, flush, hbm)
     res["input"] = f"gradients: {g.n} x {g.d} fp32, p={g.p}, s={g.s}, codes of the b={g.b} budget solve"
     del X, P, o
+    torch.cuda.empty_cache()
+    return res, dp
+
+
+def small_dp_figures(E, dev, stream, flush, mufu_peak, rank, names=("sweep", "mixture")):
+    """k_dp on the lambda-sweep and Hirschberg workloads, each on its own input."""
+    import torch
+
+    res = {}
+    for name in names:
+        w = W.WORKLOADS[name]
+        X = torch.from_numpy(W.make_inputs(w, rank=rank)).to(dev)
+        P, cnt, A, B, _ = E.grid_bucket(X, w.p)
+        res[name], _ = dp_figure(E, w, cnt, A, B, P, stream, flush, mufu_peak)
+        del X, P, cnt, A, B
     torch.cuda.empty_cache()
     return res
 
@@ -559,8 +693,9 @@ def main():
     ap.add_argument("--fp64", action="store_true", help="fp64 DP layers (parity mode)")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-gradients-stages", action="store_true",
-                    help="skip the grid/bucketing/encoding figures on the 1 GiB gradients input")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the exact-solver figures of the gradients, sweep and mixture workloads and the "
+                         "grid/bucketing/encoding figures on the 1 GiB gradients input")
     ap.add_argument("--rows", type=int, default=0, help="first rows only (profiling runs; not a bench line)")
     args = ap.parse_args()
     w = W.WORKLOADS[args.workload]

@@ -5,6 +5,7 @@ import ctypes as C
 import os
 import re
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -99,3 +100,36 @@ def test_triple_count_matches_enumeration():
         assert triples_per_solve(p, s) == t
     assert triples_per_solve(64, 8) == 151347
     assert triples_per_solve(128, 16) == 3522197
+
+
+def _pass_enum(s0, e0, T, last_only):
+    t_ = 0
+    for t in range(2, T + 1):
+        last = last_only and t == T
+        for l in range(s0 + t - 1, e0):
+            ks = [s0] if t == 2 else range(s0 + t - 2, l)
+            js = [e0] if last else range(l + 1, e0 + 1)
+            t_ += len(list(ks)) * len(list(js))
+    return t_
+
+
+def test_hirschberg_triple_count_matches_enumeration():
+    """Triples of a Hirschberg-mode solve: the whole-alphabet pass plus, per
+    segment, a forward and a reflected pass, each enumerated directly; the
+    segments follow the split rule on random codes."""
+    from bench import hirschberg_triples, pass_triples, triples_per_solve
+    rng = np.random.default_rng(3)
+    for p, s in [(12, 5), (30, 8), (40, 12), (9, 9)]:
+        assert pass_triples(0, p - 1, min(s, p) - 1, True) == triples_per_solve(p, s)
+        for _ in range(5):
+            m = int(rng.integers(2, min(s, p) + 1))
+            code = np.concatenate([[0], np.sort(rng.choice(np.arange(1, p - 1), m - 2, replace=False)), [p - 1]])
+            want = _pass_enum(0, p - 1, min(s, p) - 1, True)
+            segs = [(0, m - 2)] if m >= 4 else []
+            while segs:
+                lo, hi = segs.pop()
+                mid = lo + (hi - lo - 1 + 1) // 2
+                want += _pass_enum(code[lo], code[hi], mid - lo + 1, mid + 1 == hi)
+                want += _pass_enum(p - 1 - code[hi], p - 1 - code[lo], hi - mid, False)
+                segs += [sg for sg in ((lo, mid), (mid + 1, hi)) if sg[1] - sg[0] - 1 >= 1]
+            assert hirschberg_triples(code, p, s) == want, (p, s, code)
