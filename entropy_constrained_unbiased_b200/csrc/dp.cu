@@ -30,7 +30,9 @@
 //   * a DP layer is split into tasks of 32 lanes; a lane owns 4 outputs
 //     (l, j0..j0+3) of one row and sweeps k down the column of l in two
 //     interleaved streams; tasks are decoded in closed form from their index,
-//     longest rows first, and taken by warps from a shared counter;
+//     longest rows first, and taken by warps from a shared counter; with the
+//     tables in the global slab a warp prefetches its next task's column and
+//     rows into L2 while it runs the current one;
 //   * store mode keeps every layer's values in a per-CTA global slab (no
 //     back-pointers); the backtrack recomputes the argmin of the few states on
 //     the optimal path;
@@ -325,10 +327,25 @@ __device__ __forceinline__ void run_task(const Ctx<T>& c, const Tables<T>& tb, i
   }
 }
 
+// Prefetch of a task's column of the previous layer (128-byte lines) and of
+// the b and V/d rows its outputs read (tables in the global slab).
+template <typename T>
+__device__ __forceinline__ void prefetch_task(const Ctx<T>& c, const Tables<T>& tb, int l, int j0, int kmin,
+                                              const GA<T>* Gp) {
+  const uintptr_t beg = reinterpret_cast<uintptr_t>(Gp + c.cb[l] + kmin) & ~uintptr_t(127);
+  const uintptr_t end = reinterpret_cast<uintptr_t>(Gp + c.cb[l] + l);
+  for (uintptr_t a = beg; a < end; a += 128) asm volatile("prefetch.L2 [%0];" ::"l"(a));
+  const int ro = row_off(l, c.p) - l - 1;
+  asm volatile("prefetch.L2 [%0];" ::"l"(tb.rowB + ro + j0));
+  asm volatile("prefetch.L2 [%0];" ::"l"(tb.rowV + ro + j0));
+}
+
 // Runs the pass; all threads. Leaves layer T in tb.layer(T).
 // With a cluster, the CTAs split each layer's tasks (one counter, in rank 0)
-// and compute everything else redundantly from the same data.
-template <typename T, int kUnroll, int kCL>
+// and compute everything else redundantly from the same data. With the tables
+// in the global slab (kSlab), a warp decodes its next task before running the
+// current one and prefetches that task's column and rows into L2.
+template <typename T, int kUnroll, int kCL, bool kSlab>
 __device__ __forceinline__ void run_pass(const Ctx<T>& c, const Tables<T>& tb, const Pass& ps, bool sep, T invl,
                                          SolveOut* out, T* bestE) {
   const int p = c.p, tri = c.tri;
@@ -410,26 +427,62 @@ __device__ __forceinline__ void run_pass(const Ctx<T>& c, const Tables<T>& tb, c
       const int nt = (ng + kWarp - 1) / kWarp;
       // Tasks in index order are the longest rows first. The next task index
       // is fetched before the current task runs.
-      int tn = 0;
-      if (lane == 0) tn = atomicAdd(c.ctr + t, 1);
-      tn = __shfl_sync(0xffffffffu, tn, 0);
-      while (tn < nt) {
-        const int tk = tn;
+      if constexpr (kSlab) {
+        auto decode = [&](int tk, int& l, int& j0, int& nv) {
+          const int q = tk * kWarp + lane;
+          l = 0;
+          j0 = 0;
+          nv = 0;
+          if (q < ng) {
+            if (last) {
+              l = e0 - 1 - q;
+              j0 = e0;
+              nv = 1;
+            } else {
+              decode_group(q, e0, l, j0, nv);
+            }
+          }
+        };
+        int tn = 0;
         if (lane == 0) tn = atomicAdd(c.ctr + t, 1);
         tn = __shfl_sync(0xffffffffu, tn, 0);
-        const int q = tk * kWarp + lane;
-        const bool act = q < ng;
-        int l = 0, j0 = 0, nv = 0;
-        if (act) {
-          if (last) {
-            l = e0 - 1 - q;
-            j0 = e0;
-            nv = 1;
-          } else {
-            decode_group(q, e0, l, j0, nv);
-          }
+        int nl = 0, nj0 = 0, nnv = 0;
+        if (tn < nt) {
+          decode(tn, nl, nj0, nnv);
+          if (nnv > 0) prefetch_task(c, tb, nl, nj0, kmin, Gp);
         }
-        run_task<T, kUnroll>(c, tb, l, j0, nv, act, kmin, Gp, Gc, fsi, invl);
+        while (tn < nt) {
+          const int l = nl, j0 = nj0, nv = nnv;
+          if (lane == 0) tn = atomicAdd(c.ctr + t, 1);
+          tn = __shfl_sync(0xffffffffu, tn, 0);
+          if (tn < nt) {
+            decode(tn, nl, nj0, nnv);
+            if (nnv > 0) prefetch_task(c, tb, nl, nj0, kmin, Gp);
+          }
+          run_task<T, kUnroll>(c, tb, l, j0, nv, nv > 0, kmin, Gp, Gc, fsi, invl);
+        }
+      } else {
+        int tn = 0;
+        if (lane == 0) tn = atomicAdd(c.ctr + t, 1);
+        tn = __shfl_sync(0xffffffffu, tn, 0);
+        while (tn < nt) {
+          const int tk = tn;
+          if (lane == 0) tn = atomicAdd(c.ctr + t, 1);
+          tn = __shfl_sync(0xffffffffu, tn, 0);
+          const int q = tk * kWarp + lane;
+          const bool act = q < ng;
+          int l = 0, j0 = 0, nv = 0;
+          if (act) {
+            if (last) {
+              l = e0 - 1 - q;
+              j0 = e0;
+              nv = 1;
+            } else {
+              decode_group(q, e0, l, j0, nv);
+            }
+          }
+          run_task<T, kUnroll>(c, tb, l, j0, nv, act, kmin, Gp, Gc, fsi, invl);
+        }
       }
     }
     csync<kCL>();
@@ -527,7 +580,7 @@ __device__ __forceinline__ void evaluate(const Ctx<T>& c, double lam, SolveOut* 
 
 // One full solve at lambda (all threads). Leaves the code in c.sQ and the fp64
 // evaluation in *out (shared).
-template <typename T, int kUnroll, int kCL>
+template <typename T, int kUnroll, int kCL, bool kSlab>
 __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out, T* bestE, T* wbest, int* warg) {
   const int p = c.p, S = c.S, tri = c.tri;
   // Below kMinLambda the entropy terms vanish under the precision of T and
@@ -546,7 +599,7 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
   __syncthreads();
   // The whole alphabet, from c_1 = P_0; the last layer needs only j = p-1.
   Pass full{0, p - 1, S - 1, true, -1.0, !c.hirschberg, true};
-  run_pass<T, kUnroll, kCL>(c, c.fw, full, sep, invl, out, bestE);
+  run_pass<T, kUnroll, kCL, kSlab>(c, c.fw, full, sep, invl, out, bestE);
 
   if (tid == 0 && out->bestI < 1) {  // no finite candidate (non-finite inputs): fall back to {P_0, P_{p-1}}
     out->bestI = 1;
@@ -612,12 +665,12 @@ __device__ __forceinline__ void solve(const Ctx<T>& c, double lam, SolveOut* out
     double extra_f = -1.0;
     if (lo >= 1) extra_f = static_cast<double>(c.fw.buf0[c.cb[qlo] + c.sQ[lo - 1]].a);  // R(c[lo-1], c[lo])/d
     Pass fwp{qlo, qhi, mid - lo + 1, mid + 1 == hi, extra_f, false, false};
-    run_pass<T, kUnroll, kCL>(c, c.fw, fwp, sep, invl, out, bestE);
+    run_pass<T, kUnroll, kCL, kSlab>(c, c.fw, fwp, sep, invl, out, bestE);
     // Reflected: values c[hi] .. c[mid+1] (reflected), next c[mid]; the mass of
     // c[hi] takes L(c[hi], c[hi+1]) from its right neighbour.
     const double extra_b = static_cast<double>(c.fw.rowB[row_off(qhi, p) + qnext - qhi - 1]);
     Pass bwp{p - 1 - qhi, p - 1 - qlo, hi - mid, false, extra_b, false, false};
-    run_pass<T, kUnroll, kCL>(c, c.rf, bwp, sep, invl, out, bestE);
+    run_pass<T, kUnroll, kCL, kSlab>(c, c.rf, bwp, sep, invl, out, bestE);
     const int xlo = qlo + (mid - lo), xhi = qhi - (hi - mid);
     const int yhi = qhi - (hi - mid - 1);
     join(c, c.fw.layer(fwp.T), c.rf.layer(bwp.T), xlo, xhi, yhi, mid + 1 == hi, invl, out, wbest, warg);
@@ -777,7 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
       for (int t = 0; t < a.n_lambda; ++t) {
         const int64_t w = static_cast<int64_t>(r) * a.n_lambda + t;
         const double lam = a.lambda[w];
-        solve<T, kUnrollK, kCL>(c, lam, &s_out, &s_bestE, s_wbest, s_warg);
+        solve<T, kUnrollK, kCL, !kSmemTables>(c, lam, &s_out, &s_bestE, s_wbest, s_warg);
         for (int q = threadIdx.x; q < s_out_stride; q += blockDim.x)
           a.Q[w * s_out_stride + q] = (q < s_out.m) ? c.sQ[q] : -1;
         if (threadIdx.x == 0) {
@@ -803,14 +856,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
       };
       int32_t status = kStatusOk;
       double theta = 0.0;
-      solve<T, kUnrollK, kCL>(c, 0.0, &s_out, &s_bestE, s_wbest, s_warg);
+      solve<T, kUnrollK, kCL, !kSmemTables>(c, 0.0, &s_out, &s_bestE, s_wbest, s_warg);
       keep(sQ1, m1, H1, M1);
       if (s_out.H <= a.budget) {
         keep(sQ2, m2, H2, M2);
         hi = 0.0;
       } else {
         __syncthreads();
-        solve<T, kUnrollK, kCL>(c, hi, &s_out, &s_bestE, s_wbest, s_warg);
+        solve<T, kUnrollK, kCL, !kSmemTables>(c, hi, &s_out, &s_bestE, s_wbest, s_warg);
         keep(sQ2, m2, H2, M2);
         if (s_out.H > a.budget) {
           status = kStatusBudget;
@@ -818,7 +871,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dp(DpArgs a) {
           for (int it = 0; it < a.steps; ++it) {
             const double mid = 0.5 * (lo + hi);
             __syncthreads();
-            solve<T, kUnrollK, kCL>(c, mid, &s_out, &s_bestE, s_wbest, s_warg);
+            solve<T, kUnrollK, kCL, !kSmemTables>(c, mid, &s_out, &s_bestE, s_wbest, s_warg);
             if (s_out.H > a.budget) {
               lo = mid;
               keep(sQ1, m1, H1, M1);
