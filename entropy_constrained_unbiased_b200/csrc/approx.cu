@@ -719,6 +719,10 @@ struct WCtx {
   double* ab;
   double* bb;
   float* G;         // [(S+1) * pst] layers
+  float* tG;        // tiled layers: [warps][kWT][kS] staged layer values of an A-tile
+  float* tpart;     // [warps][kS][kWT] per-warp partial minima of an X-tile
+  float* tw;        // [warps][kWT][kWT] pair costs of a block
+  float* tdiag;     // [kWT][kWT] costs of the diagonal block
   double* fbuf;     // [warps][p] local costs of the refinement
   int* sQ;
   int* moved;
@@ -880,21 +884,116 @@ __device__ void wevaluate(const WCtx& c, double lam, bool refined, int m, AOut* 
   __syncwarp();
 }
 
+// Tiled layers (S - 1 <= kS layers after the first). Every pair cost w(a, x)
+// is computed once per solve and relaxes all layers: G_i(x) depends only on
+// G_{i-1}(a), a < x, so once the columns left of an X-tile of kWT columns are
+// final in every layer, the pairs (a, x) with a in an earlier A-tile of kWT
+// rows relax layers 2 .. S together. The warps share the earlier A-tiles (lane =
+// column x; the A-tile's layer values staged in shared memory and read as
+// broadcasts), their partial minima are merged, and warp 0 finishes the
+// diagonal block (a, x in the same tile, a < x) layer by layer. A minimum
+// does not depend on the order of its terms, so every G_i(x) equals the one
+// the layer-by-layer sweep gives; below the first reachable column
+// (x < i - 1) the layer holds +inf.
+constexpr int kWT = 32;
+
+// Layers kept per lane by the tiled sweep for a code of S values (0: the
+// layer-by-layer sweep, S > 33).
+__host__ __device__ inline int wide_tile_layers(int S) {
+  return S - 1 <= 8 ? 8 : (S - 1 <= 16 ? 16 : (S - 1 <= 32 ? 32 : 0));
+}
+
+template <int kS>
+__device__ __noinline__ void wide_layers_tiled(const WCtx& c, float lamf) {
+  const int p = c.p, S = c.S, pst = c.pst, tid = threadIdx.x, bd = blockDim.x;
+  const int lane = lane_id(), warp = warp_id(), nw = bd / kWarp;
+  const float inf = __int_as_float(0x7f800000);
+  for (int i = 1; i <= S; ++i)
+    for (int x = tid; x < p; x += bd) c.G[i * pst + x] = (i == 1 && x == 0) ? 0.0f : inf;
+  __syncthreads();
+  float* gs = c.tG + static_cast<size_t>(warp) * kWT * kS;
+  float* ws = c.tw + static_cast<size_t>(warp) * kWT * kWT;
+  float* part = c.tpart + static_cast<size_t>(warp) * kS * kWT;
+  const int ntile = (p + kWT - 1) / kWT;
+  for (int xt = 0; xt < ntile; ++xt) {
+    const int x0 = xt * kWT, x = x0 + lane;
+    const bool xin = x < p;
+#pragma unroll
+    for (int q = 0; q < kS; ++q) part[q * kWT + lane] = inf;
+    for (int at = warp; at < xt; at += nw) {
+      const int a0 = at * kWT;
+      // the block's costs ws[j][lane] = w(a0 + j, x), then gs[j][q] = G_{q+1}(a0 + j)
+      // (layers past S - 1 are not read); the partial minima stay in shared
+      // memory between blocks so that the cost evaluation has the registers
+      for (int j = 0; j < kWT; ++j) ws[j * kWT + lane] = xin ? wcost(c, a0 + j, x, lamf) : 0.0f;
+#pragma unroll
+      for (int q = 0; q < kS; ++q) gs[lane * kS + q] = (q + 1 <= S - 1) ? c.G[(q + 1) * pst + a0 + lane] : inf;
+      __syncwarp();
+      float best[kS];
+#pragma unroll
+      for (int q = 0; q < kS; ++q) best[q] = part[q * kWT + lane];
+#pragma unroll 1
+      for (int j = 0; j < kWT; ++j) {
+        const float w = ws[j * kWT + lane];
+        const float4* g4 = reinterpret_cast<const float4*>(gs + j * kS);
+#pragma unroll
+        for (int q4 = 0; q4 < kS / 4; ++q4) {
+          const float4 g = g4[q4];
+          best[4 * q4 + 0] = fminf(best[4 * q4 + 0], __fadd_rn(g.x, w));
+          best[4 * q4 + 1] = fminf(best[4 * q4 + 1], __fadd_rn(g.y, w));
+          best[4 * q4 + 2] = fminf(best[4 * q4 + 2], __fadd_rn(g.z, w));
+          best[4 * q4 + 3] = fminf(best[4 * q4 + 3], __fadd_rn(g.w, w));
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < kS; ++q) part[q * kWT + lane] = best[q];
+      __syncwarp();
+    }
+    __syncthreads();
+    if (warp == 0) {
+      float* wd = c.tdiag;  // wd[j][lane] = w(x0 + j, x), +inf unless j < lane
+      for (int j = 0; j < kWT; ++j) wd[j * kWT + lane] = (xin && j < lane) ? wcost(c, x0 + j, x, lamf) : inf;
+      __syncwarp();
+      float prev = xin ? c.G[pst + x] : inf;  // layer i - 1 at this column
+      for (int i = 2; i <= S; ++i) {
+        float b = inf;
+        for (int w = 0; w < nw; ++w) b = fminf(b, c.tpart[(static_cast<size_t>(w) * kS + (i - 2)) * kWT + lane]);
+        for (int j = 0; j < kWT; ++j) {
+          const float gj = __shfl_sync(0xffffffffu, prev, j);
+          b = fminf(b, __fadd_rn(gj, wd[j * kWT + lane]));
+        }
+        if (xin) c.G[i * pst + x] = b;
+        prev = b;
+      }
+    }
+    __syncthreads();
+  }
+}
+
 __device__ void approx_solve_wide(const WCtx& c, double lam, int refine, AOut* out) {
   const int p = c.p, S = c.S, tid = threadIdx.x, bd = blockDim.x;
   const float inf = __int_as_float(0x7f800000);
   const float lamf = static_cast<float>(lam);
-  for (int x = tid; x < p; x += bd) c.G[c.pst + x] = (x == 0) ? 0.0f : inf;
-  __syncthreads();
-  for (int i = 2; i <= S; ++i) {
-    const float* __restrict__ Gp = c.G + (i - 1) * c.pst;
-    float* __restrict__ Gc = c.G + i * c.pst;
-    for (int x = i - 1 + tid; x < p; x += bd) {
-      float best = inf;
-      for (int a = i - 2; a < x; ++a) best = fminf(best, __fadd_rn(Gp[a], wcost(c, a, x, lamf)));
-      Gc[x] = best;
-    }
+  const int kS = wide_tile_layers(S);
+  if (kS == 8) {
+    wide_layers_tiled<8>(c, lamf);
+  } else if (kS == 16) {
+    wide_layers_tiled<16>(c, lamf);
+  } else if (kS == 32) {
+    wide_layers_tiled<32>(c, lamf);
+  } else {
+    for (int x = tid; x < p; x += bd) c.G[c.pst + x] = (x == 0) ? 0.0f : inf;
     __syncthreads();
+    for (int i = 2; i <= S; ++i) {
+      const float* __restrict__ Gp = c.G + (i - 1) * c.pst;
+      float* __restrict__ Gc = c.G + i * c.pst;
+      for (int x = i - 1 + tid; x < p; x += bd) {
+        float best = inf;
+        for (int a = i - 2; a < x; ++a) best = fminf(best, __fadd_rn(Gp[a], wcost(c, a, x, lamf)));
+        Gc[x] = best;
+      }
+      __syncthreads();
+    }
   }
   if (warp_id() == 0) {
     const int lane = lane_id();
@@ -945,6 +1044,15 @@ __device__ void approx_solve_wide(const WCtx& c, double lam, int refine, AOut* o
 
 constexpr int kWideApproxThreads = 512;
 
+// Dynamic shared memory of k_approx_wide: the three codes, then the tiled
+// sweep's staging, partial minima, block costs and diagonal block.
+__host__ __device__ inline size_t wide_smem_head(int S) { return (sizeof(int) * 3 * static_cast<size_t>(S) + 15) & ~size_t(15); }
+__host__ __device__ inline size_t wide_smem_bytes(int S) {
+  const size_t kS = static_cast<size_t>(wide_tile_layers(S));
+  const size_t nw = kWideApproxThreads / kWarp;
+  return wide_smem_head(S) + (kS ? sizeof(float) * (2 * nw * kWT * kS + nw * kWT * kWT + kWT * kWT) : 0);
+}
+
 __global__ void __launch_bounds__(kWideApproxThreads, 1) k_approx_wide(ApproxArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ AOut s_out;
@@ -962,6 +1070,14 @@ __global__ void __launch_bounds__(kWideApproxThreads, 1) k_approx_wide(ApproxArg
   c.sQ = reinterpret_cast<int*>(smem);
   int* sQ1 = c.sQ + S;
   int* sQ2 = sQ1 + S;
+  {
+    const int kS = wide_tile_layers(S);
+    unsigned char* ts = smem + wide_smem_head(S);
+    c.tG = reinterpret_cast<float*>(ts);
+    c.tpart = c.tG + static_cast<size_t>(kNW) * kWT * kS;
+    c.tw = c.tpart + static_cast<size_t>(kNW) * kS * kWT;
+    c.tdiag = c.tw + static_cast<size_t>(kNW) * kWT * kWT;
+  }
   c.moved = &s_misc[0];
   c.msh = &s_misc[1];
   unsigned char* gs = a.scratch + static_cast<size_t>(blockIdx.x) * a.scratch_per_cta;
@@ -1103,7 +1219,11 @@ bool approx_plan(int n, int p, int s, bool fp64, ApproxPlan* plan) {
     plan->smem = false;
     plan->split = false;
     plan->threads = kWideApproxThreads;
-    plan->smem_bytes = al16(sizeof(int) * 3 * static_cast<size_t>(S));
+    plan->smem_bytes = wide_smem_bytes(S);
+    if (cudaFuncSetAttribute(reinterpret_cast<const void*>(&k_approx_wide),
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(plan->smem_bytes)) !=
+        cudaSuccess)
+      return false;
     plan->scratch_per_cta = al256(8 * 6 * static_cast<size_t>(p)) + 3 * al256(8 * static_cast<size_t>(p)) +
                             al256(4 * static_cast<size_t>(S + 1) * pst) +
                             al256(8 * static_cast<size_t>(kWideApproxThreads / kWarp) * p);

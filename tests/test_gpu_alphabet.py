@@ -177,3 +177,27 @@ def test_approx_budget_and_encode_large_alphabet(E, O, wide):
     assert np.all(so == 0)
     np.testing.assert_array_equal(idx.cpu().numpy(), io)
     np.testing.assert_array_equal(hist.cpu().numpy(), ho)
+
+
+@pytest.mark.parametrize("s", [6, 24, 40])
+def test_approx_large_alphabet_code_sizes(E, O, wide, s):
+    """Code sizes on each side of the tiled layer sweep's register blocks (up to
+    8, 16 and 32 layers after the first) and past them (the layer-by-layer
+    sweep): the objective within 1e-5 of the oracle's optimum and the fp64
+    figures equal to the oracle's raw evaluation."""
+    X, P, p = wide
+    Xd = torch.from_numpy(X).cuda()
+    lam = np.var(X.astype(np.float64), axis=1)[:, None] * np.array([[0.001, 0.01]])
+    g = E.solve_approx(Xd, P, s, torch.from_numpy(lam).cuda())
+    assert int(g["status"].abs().sum()) == 0
+    Pn = P.cpu().numpy()
+    Q, m = g["Q"].cpu().numpy(), g["Q_len"].cpu().numpy()
+    ref = O.solve_approx_batch(X, Pn, s, lam, refine=0)
+    for r in range(X.shape[0]):
+        for t in range(lam.shape[1]):
+            assert 2 <= m[r, t] <= s
+            vals = Pn[r][Q[r, t, : m[r, t]]]
+            mse, _, _ = O.eval_raw(X[r], vals)
+            J_ib = mse + lam[r, t] * O.eval_raw_ib(X[r], vals)
+            assert J_ib <= ref["J"][r, t] * (1 + 1e-5), (r, t, J_ib, ref["J"][r, t])
+            assert g["objective"][r, t].item() == pytest.approx(J_ib, rel=1e-9)
