@@ -710,6 +710,13 @@ __global__ void __launch_bounds__(512, 1) k_approx(ApproxArgs a) {
 // reported figures of the final code (mse, H, H(I,B), objective) are direct
 // fp64 sums over each interval's buckets in the order of the definitions.
 
+// One end of an interval: the six prefix sums up to index k (buckets
+// 0 .. k-1), P_k and u_k = P_k - P_0. A pair's terms are differences of its
+// two ends' sums, so a column's end can be loaded once and reused.
+struct WSide {
+  double N, SA, SB, SNU, SAU, SNUU, P, u;
+};
+
 struct WCtx {
   int p, S, pst;
   double dd, inv_d;
@@ -721,7 +728,8 @@ struct WCtx {
   float* G;         // [(S+1) * pst] layers
   float* tG;        // tiled layers: [warps][kWT][kS] staged layer values of an A-tile
   float* tpart;     // [warps][kS][kWT] per-warp partial minima of an X-tile
-  float* tw;        // [warps][kWT][kWT] pair costs of a block
+  float* tw;        // [warps][kWA][kWT] pair costs of a block
+  WSide* tside;     // [warps][kWA] the A-tile's ends of the pair terms
   float* tdiag;     // [kWT][kWT] costs of the diagonal block
   double* fbuf;     // [warps][p] local costs of the refinement
   int* sQ;
@@ -729,17 +737,30 @@ struct WCtx {
   int* msh;
 };
 
-__device__ __forceinline__ void wpair(const WCtx& c, int a, int e, double& V, double& R, double& L) {
+__device__ __forceinline__ WSide wside(const WCtx& c, int k) {
   const double* pr = c.pre;
   const int p = c.p;
-  const double N = __dsub_rn(pr[e], pr[a]);
-  const double SA = __dsub_rn(pr[p + e], pr[p + a]);
-  const double SB = __dsub_rn(pr[2 * p + e], pr[2 * p + a]);
-  const double SNU = __dsub_rn(pr[3 * p + e], pr[3 * p + a]);
-  const double SAU = __dsub_rn(pr[4 * p + e], pr[4 * p + a]);
-  const double SNUU = __dsub_rn(pr[5 * p + e], pr[5 * p + a]);
-  const double ua = __dsub_rn(c.P[a], c.P[0]);
-  const double W = __dsub_rn(c.P[e], c.P[a]);
+  WSide w;
+  w.N = pr[k];
+  w.SA = pr[p + k];
+  w.SB = pr[2 * p + k];
+  w.SNU = pr[3 * p + k];
+  w.SAU = pr[4 * p + k];
+  w.SNUU = pr[5 * p + k];
+  w.P = c.P[k];
+  w.u = __dsub_rn(c.P[k], c.P[0]);
+  return w;
+}
+
+__device__ __forceinline__ void wpair_sides(const WSide& sa, const WSide& se, double& V, double& R, double& L) {
+  const double N = __dsub_rn(se.N, sa.N);
+  const double SA = __dsub_rn(se.SA, sa.SA);
+  const double SB = __dsub_rn(se.SB, sa.SB);
+  const double SNU = __dsub_rn(se.SNU, sa.SNU);
+  const double SAU = __dsub_rn(se.SAU, sa.SAU);
+  const double SNUU = __dsub_rn(se.SNUU, sa.SNUU);
+  const double ua = sa.u;
+  const double W = __dsub_rn(se.P, sa.P);
   const double T1 = SA + SNU - ua * N;
   const double T2 = SB + 2.0 * SAU - 2.0 * ua * SA + SNUU - 2.0 * ua * SNU + ua * ua * N;
   V = fmax(W * T1 - T2, 0.0);
@@ -747,15 +768,23 @@ __device__ __forceinline__ void wpair(const WCtx& c, int a, int e, double& V, do
   L = N - R;
 }
 
+__device__ __forceinline__ void wpair(const WCtx& c, int a, int e, double& V, double& R, double& L) {
+  wpair_sides(wside(c, a), wside(c, e), V, R, L);
+}
+
 // The layers' cost w(a, e) in fp32 (as the fp32 table path forms it).
-__device__ __forceinline__ float wcost(const WCtx& c, int a, int e, float lamf) {
+__device__ __forceinline__ float wcost_sides(const WCtx& c, const WSide& sa, const WSide& se, float lamf) {
   double V, R, L;
-  wpair(c, a, e, V, R, L);
+  wpair_sides(sa, se, V, R, L);
   const float vt = static_cast<float>(V * c.inv_d);
   const float qr = static_cast<float>(R * c.inv_d), ql = static_cast<float>(L * c.inv_d);
   const float hr = qr > 0.0f ? -qr * lg2_approx(qr) : 0.0f;
   const float hl = ql > 0.0f ? -ql * lg2_approx(ql) : 0.0f;
   return __fmaf_rn(lamf, hl + hr, vt);
+}
+
+__device__ __forceinline__ float wcost(const WCtx& c, int a, int e, float lamf) {
+  return wcost_sides(c, wside(c, a), wside(c, e), lamf);
 }
 
 // Direct fp64 sums over buckets a .. e-1, every operation rounded as written,
@@ -887,15 +916,17 @@ __device__ void wevaluate(const WCtx& c, double lam, bool refined, int m, AOut* 
 // Tiled layers (S - 1 <= kS layers after the first). Every pair cost w(a, x)
 // is computed once per solve and relaxes all layers: G_i(x) depends only on
 // G_{i-1}(a), a < x, so once the columns left of an X-tile of kWT columns are
-// final in every layer, the pairs (a, x) with a in an earlier A-tile of kWT
+// final in every layer, the pairs (a, x) with a in an earlier A-tile of kWA
 // rows relax layers 2 .. S together. The warps share the earlier A-tiles (lane =
-// column x; the A-tile's layer values staged in shared memory and read as
-// broadcasts), their partial minima are merged, and warp 0 finishes the
-// diagonal block (a, x in the same tile, a < x) layer by layer. A minimum
-// does not depend on the order of its terms, so every G_i(x) equals the one
-// the layer-by-layer sweep gives; below the first reachable column
-// (x < i - 1) the layer holds +inf.
-constexpr int kWT = 32;
+// column x, whose end of the pair terms stays in registers for the whole
+// X-tile; the A-tile's ends and layer values staged in shared memory and read
+// as broadcasts), their partial minima are merged, and warp 0 runs the
+// diagonal block (a, x in the same tile, a < x; its pair costs computed by all
+// warps) layer by layer. A minimum does not depend on the order of its terms,
+// so every G_i(x) equals the one the layer-by-layer sweep gives; below the
+// first reachable column (x < i - 1) the layer holds +inf.
+constexpr int kWT = 32;  // columns of an X-tile (one per lane)
+constexpr int kWA = 16;  // rows of an A-tile
 
 // Layers kept per lane by the tiled sweep for a code of S values (0: the
 // layer-by-layer sweep, S > 33).
@@ -911,29 +942,36 @@ __device__ __noinline__ void wide_layers_tiled(const WCtx& c, float lamf) {
   for (int i = 1; i <= S; ++i)
     for (int x = tid; x < p; x += bd) c.G[i * pst + x] = (i == 1 && x == 0) ? 0.0f : inf;
   __syncthreads();
-  float* gs = c.tG + static_cast<size_t>(warp) * kWT * kS;
-  float* ws = c.tw + static_cast<size_t>(warp) * kWT * kWT;
-  float* part = c.tpart + static_cast<size_t>(warp) * kS * kWT;
+  float* gs = c.tG + static_cast<size_t>(warp) * kWA * kS;      // [kWA][kS]
+  float* ws = c.tw + static_cast<size_t>(warp) * kWA * kWT;      // [kWA][kWT]
+  float* part = c.tpart + static_cast<size_t>(warp) * kS * kWT;  // [kS][kWT]
+  WSide* as = c.tside + static_cast<size_t>(warp) * kWA;         // [kWA]
   const int ntile = (p + kWT - 1) / kWT;
   for (int xt = 0; xt < ntile; ++xt) {
     const int x0 = xt * kWT, x = x0 + lane;
     const bool xin = x < p;
+    const WSide xs = wside(c, xin ? x : p - 1);
 #pragma unroll
     for (int q = 0; q < kS; ++q) part[q * kWT + lane] = inf;
-    for (int at = warp; at < xt; at += nw) {
-      const int a0 = at * kWT;
-      // the block's costs ws[j][lane] = w(a0 + j, x), then gs[j][q] = G_{q+1}(a0 + j)
-      // (layers past S - 1 are not read); the partial minima stay in shared
-      // memory between blocks so that the cost evaluation has the registers
-      for (int j = 0; j < kWT; ++j) ws[j * kWT + lane] = xin ? wcost(c, a0 + j, x, lamf) : 0.0f;
+    for (int at = warp; at < xt * (kWT / kWA); at += nw) {
+      const int a0 = at * kWA;
+      // the A-tile's ends and gs[j][q] = G_{q+1}(a0 + j) (layers past S - 1
+      // are not read), then the block's costs ws[j][lane] = w(a0 + j, x); the
+      // partial minima stay in shared memory between blocks so that the cost
+      // evaluation has the registers
+      if (lane < kWA) {
+        as[lane] = wside(c, a0 + lane);
 #pragma unroll
-      for (int q = 0; q < kS; ++q) gs[lane * kS + q] = (q + 1 <= S - 1) ? c.G[(q + 1) * pst + a0 + lane] : inf;
+        for (int q = 0; q < kS; ++q) gs[lane * kS + q] = (q + 1 <= S - 1) ? c.G[(q + 1) * pst + a0 + lane] : inf;
+      }
+      __syncwarp();
+      for (int j = 0; j < kWA; ++j) ws[j * kWT + lane] = xin ? wcost_sides(c, as[j], xs, lamf) : 0.0f;
       __syncwarp();
       float best[kS];
 #pragma unroll
       for (int q = 0; q < kS; ++q) best[q] = part[q * kWT + lane];
 #pragma unroll 1
-      for (int j = 0; j < kWT; ++j) {
+      for (int j = 0; j < kWA; ++j) {
         const float w = ws[j * kWT + lane];
         const float4* g4 = reinterpret_cast<const float4*>(gs + j * kS);
 #pragma unroll
@@ -949,11 +987,12 @@ __device__ __noinline__ void wide_layers_tiled(const WCtx& c, float lamf) {
       for (int q = 0; q < kS; ++q) part[q * kWT + lane] = best[q];
       __syncwarp();
     }
+    // the diagonal block's costs wd[j][lane] = w(x0 + j, x), +inf unless j < lane
+    for (int j = warp; j < kWT; j += nw)
+      c.tdiag[j * kWT + lane] = (xin && j < lane) ? wcost_sides(c, wside(c, x0 + j), xs, lamf) : inf;
     __syncthreads();
     if (warp == 0) {
-      float* wd = c.tdiag;  // wd[j][lane] = w(x0 + j, x), +inf unless j < lane
-      for (int j = 0; j < kWT; ++j) wd[j * kWT + lane] = (xin && j < lane) ? wcost(c, x0 + j, x, lamf) : inf;
-      __syncwarp();
+      const float* wd = c.tdiag;
       float prev = xin ? c.G[pst + x] : inf;  // layer i - 1 at this column
       for (int i = 2; i <= S; ++i) {
         float b = inf;
@@ -1045,12 +1084,14 @@ __device__ void approx_solve_wide(const WCtx& c, double lam, int refine, AOut* o
 constexpr int kWideApproxThreads = 512;
 
 // Dynamic shared memory of k_approx_wide: the three codes, then the tiled
-// sweep's staging, partial minima, block costs and diagonal block.
+// sweep's staging, partial minima, block costs, diagonal block and A-tile ends.
 __host__ __device__ inline size_t wide_smem_head(int S) { return (sizeof(int) * 3 * static_cast<size_t>(S) + 15) & ~size_t(15); }
 __host__ __device__ inline size_t wide_smem_bytes(int S) {
   const size_t kS = static_cast<size_t>(wide_tile_layers(S));
   const size_t nw = kWideApproxThreads / kWarp;
-  return wide_smem_head(S) + (kS ? sizeof(float) * (2 * nw * kWT * kS + nw * kWT * kWT + kWT * kWT) : 0);
+  return wide_smem_head(S) +
+         (kS ? sizeof(float) * (nw * kWA * kS + nw * kS * kWT + nw * kWA * kWT + kWT * kWT) + sizeof(WSide) * nw * kWA
+             : 0);
 }
 
 __global__ void __launch_bounds__(kWideApproxThreads, 1) k_approx_wide(ApproxArgs a) {
@@ -1074,9 +1115,10 @@ __global__ void __launch_bounds__(kWideApproxThreads, 1) k_approx_wide(ApproxArg
     const int kS = wide_tile_layers(S);
     unsigned char* ts = smem + wide_smem_head(S);
     c.tG = reinterpret_cast<float*>(ts);
-    c.tpart = c.tG + static_cast<size_t>(kNW) * kWT * kS;
+    c.tpart = c.tG + static_cast<size_t>(kNW) * kWA * kS;
     c.tw = c.tpart + static_cast<size_t>(kNW) * kS * kWT;
-    c.tdiag = c.tw + static_cast<size_t>(kNW) * kWT * kWT;
+    c.tdiag = c.tw + static_cast<size_t>(kNW) * kWA * kWT;
+    c.tside = reinterpret_cast<WSide*>(c.tdiag + kWT * kWT);
   }
   c.moved = &s_misc[0];
   c.msh = &s_misc[1];

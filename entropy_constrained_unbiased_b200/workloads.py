@@ -113,3 +113,15 @@ def make_inputs(w: Workload | str, rows: int | None = None, rank: int = 0) -> np
 def random_case(seed: int, n: int, d: int, dist: str = "normal") -> np.ndarray:
     """A seeded n x d test input of one family."""
     return draw(dist, np.random.default_rng([1000, seed]), n, d)
+
+
+def pinned_range_rows(seed: int, n: int, d: int, lo: float, hi: float) -> np.ndarray:
+    """n x d float32 rows, log-uniform between lo > 0 and hi with log-normal
+    jitter, clipped to [lo, hi] and holding lo and hi themselves, so that every
+    row covers exactly [lo, hi] (and has the same alphabet of the values
+    representable in a given format over that range)."""
+    rng = np.random.default_rng([2000, seed])
+    X = np.exp(rng.uniform(np.log(lo), np.log(hi), size=(n, d)) + 0.3 * rng.standard_normal((n, d)))
+    X = np.clip(X, lo, hi).astype(np.float32)
+    X[:, 0], X[:, 1] = np.float32(lo), np.float32(hi)
+    return X
