@@ -735,6 +735,7 @@ struct WCtx {
   int* sQ;
   int* moved;
   int* msh;
+  int* found;
 };
 
 __device__ __forceinline__ WSide wside(const WCtx& c, int k) {
@@ -773,18 +774,18 @@ __device__ __forceinline__ void wpair(const WCtx& c, int a, int e, double& V, do
 }
 
 // The layers' cost w(a, e) in fp32 (as the fp32 table path forms it).
-__device__ __forceinline__ float wcost_sides(const WCtx& c, const WSide& sa, const WSide& se, float lamf) {
+__device__ __forceinline__ float wcost_sides(double inv_d, const WSide& sa, const WSide& se, float lamf) {
   double V, R, L;
   wpair_sides(sa, se, V, R, L);
-  const float vt = static_cast<float>(V * c.inv_d);
-  const float qr = static_cast<float>(R * c.inv_d), ql = static_cast<float>(L * c.inv_d);
+  const float vt = static_cast<float>(V * inv_d);
+  const float qr = static_cast<float>(R * inv_d), ql = static_cast<float>(L * inv_d);
   const float hr = qr > 0.0f ? -qr * lg2_approx(qr) : 0.0f;
   const float hl = ql > 0.0f ? -ql * lg2_approx(ql) : 0.0f;
   return __fmaf_rn(lamf, hl + hr, vt);
 }
 
 __device__ __forceinline__ float wcost(const WCtx& c, int a, int e, float lamf) {
-  return wcost_sides(c, wside(c, a), wside(c, e), lamf);
+  return wcost_sides(c.inv_d, wside(c, a), wside(c, e), lamf);
 }
 
 // Direct fp64 sums over buckets a .. e-1, every operation rounded as written,
@@ -935,17 +936,24 @@ __host__ __device__ inline int wide_tile_layers(int S) {
 }
 
 template <int kS>
-__device__ __noinline__ void wide_layers_tiled(const WCtx& c, float lamf) {
+__device__ __noinline__ void wide_layers_tiled(const WCtx& cx, float lamf) {
+  // the context in registers: a reference would be re-read from local memory
+  // after every shared-memory store
+  const WCtx c = cx;
   const int p = c.p, S = c.S, pst = c.pst, tid = threadIdx.x, bd = blockDim.x;
   const int lane = lane_id(), warp = warp_id(), nw = bd / kWarp;
+  const double inv_d = c.inv_d;
+  float* __restrict__ G = c.G;
+  float* __restrict__ tpart = c.tpart;
+  float* __restrict__ tdiag = c.tdiag;
   const float inf = __int_as_float(0x7f800000);
   for (int i = 1; i <= S; ++i)
-    for (int x = tid; x < p; x += bd) c.G[i * pst + x] = (i == 1 && x == 0) ? 0.0f : inf;
+    for (int x = tid; x < p; x += bd) G[i * pst + x] = (i == 1 && x == 0) ? 0.0f : inf;
   __syncthreads();
-  float* gs = c.tG + static_cast<size_t>(warp) * kWA * kS;      // [kWA][kS]
-  float* ws = c.tw + static_cast<size_t>(warp) * kWA * kWT;      // [kWA][kWT]
-  float* part = c.tpart + static_cast<size_t>(warp) * kS * kWT;  // [kS][kWT]
-  WSide* as = c.tside + static_cast<size_t>(warp) * kWA;         // [kWA]
+  float* gs = c.tG + static_cast<size_t>(warp) * kWA * kS;    // [kWA][kS]
+  float* ws = c.tw + static_cast<size_t>(warp) * kWA * kWT;    // [kWA][kWT]
+  float* part = tpart + static_cast<size_t>(warp) * kS * kWT;  // [kS][kWT]
+  WSide* as = c.tside + static_cast<size_t>(warp) * kWA;       // [kWA]
   const int ntile = (p + kWT - 1) / kWT;
   for (int xt = 0; xt < ntile; ++xt) {
     const int x0 = xt * kWT, x = x0 + lane;
@@ -962,10 +970,10 @@ __device__ __noinline__ void wide_layers_tiled(const WCtx& c, float lamf) {
       if (lane < kWA) {
         as[lane] = wside(c, a0 + lane);
 #pragma unroll
-        for (int q = 0; q < kS; ++q) gs[lane * kS + q] = (q + 1 <= S - 1) ? c.G[(q + 1) * pst + a0 + lane] : inf;
+        for (int q = 0; q < kS; ++q) gs[lane * kS + q] = (q + 1 <= S - 1) ? G[(q + 1) * pst + a0 + lane] : inf;
       }
       __syncwarp();
-      for (int j = 0; j < kWA; ++j) ws[j * kWT + lane] = xin ? wcost_sides(c, as[j], xs, lamf) : 0.0f;
+      for (int j = 0; j < kWA; ++j) ws[j * kWT + lane] = xin ? wcost_sides(inv_d, as[j], xs, lamf) : 0.0f;
       __syncwarp();
       float best[kS];
 #pragma unroll
@@ -989,19 +997,19 @@ __device__ __noinline__ void wide_layers_tiled(const WCtx& c, float lamf) {
     }
     // the diagonal block's costs wd[j][lane] = w(x0 + j, x), +inf unless j < lane
     for (int j = warp; j < kWT; j += nw)
-      c.tdiag[j * kWT + lane] = (xin && j < lane) ? wcost_sides(c, wside(c, x0 + j), xs, lamf) : inf;
+      tdiag[j * kWT + lane] = (xin && j < lane) ? wcost_sides(inv_d, wside(c, x0 + j), xs, lamf) : inf;
     __syncthreads();
     if (warp == 0) {
-      const float* wd = c.tdiag;
-      float prev = xin ? c.G[pst + x] : inf;  // layer i - 1 at this column
+      const float* wd = tdiag;
+      float prev = xin ? G[pst + x] : inf;  // layer i - 1 at this column
       for (int i = 2; i <= S; ++i) {
         float b = inf;
-        for (int w = 0; w < nw; ++w) b = fminf(b, c.tpart[(static_cast<size_t>(w) * kS + (i - 2)) * kWT + lane]);
+        for (int w = 0; w < nw; ++w) b = fminf(b, tpart[(static_cast<size_t>(w) * kS + (i - 2)) * kWT + lane]);
         for (int j = 0; j < kWT; ++j) {
           const float gj = __shfl_sync(0xffffffffu, prev, j);
           b = fminf(b, __fadd_rn(gj, wd[j * kWT + lane]));
         }
-        if (xin) c.G[i * pst + x] = b;
+        if (xin) G[i * pst + x] = b;
         prev = b;
       }
     }
@@ -1046,36 +1054,41 @@ __device__ void approx_solve_wide(const WCtx& c, double lam, int refine, AOut* o
       }
     }
     warp_argmin(bv, bi);
-    int m;
-    if (bi == 0x7fffffff) {
-      m = 2;
-      if (lane == 0) {
-        c.sQ[0] = 0;
-        c.sQ[1] = p - 1;
-      }
-    } else {
-      m = bi;
-      int x = p - 1;
-      if (lane == 0) c.sQ[m - 1] = x;
-      for (int i = m; i >= 2; --i) {
-        const float target = c.G[i * c.pst + x];
-        const float* Gp = c.G + (i - 1) * c.pst;
-        int found = 0x7fffffff;
-        for (int base = i - 2; base < x && found == 0x7fffffff; base += kWarp) {
-          const int a = base + lane;
-          const bool hit = a < x && __fadd_rn(Gp[a], wcost(c, a, x, lamf)) == target;
-          const unsigned msk = __ballot_sync(0xffffffffu, hit);
-          if (msk) found = base + __ffs(msk) - 1;
-        }
-        if (found == 0x7fffffff) found = i - 2;  // not reached: the minimum is one of the sums
-        x = found;
-        if (lane == 0) c.sQ[i - 2] = x;
-      }
+    if (lane == 0) {
+      c.sQ[0] = 0;
+      c.sQ[1] = p - 1;  // no finite candidate (non-finite inputs): {P_0, P_{p-1}}
+      if (bi != 0x7fffffff) c.sQ[bi - 1] = p - 1;
+      *c.msh = (bi == 0x7fffffff) ? -2 : bi;
     }
-    if (lane == 0) *c.msh = m;
   }
   __syncthreads();
-  const int m = *c.msh;
+  // Recovery, all threads: at layer i the value before c_i = x is the smallest
+  // a < x whose sum G_{i-1}(a) + w(a, x) equals G_i(x) (the minimum is one of
+  // the sums, recomputed with the same operations).
+  const int mr = *c.msh;
+  if (mr > 0) {
+    int x = p - 1;
+    for (int i = mr; i >= 2; --i) {
+      const float target = c.G[i * c.pst + x];
+      const float* Gp = c.G + (i - 1) * c.pst;
+      if (tid == 0) *c.found = 0x7fffffff;
+      __syncthreads();
+      const WSide xs = wside(c, x);
+      for (int a = i - 2 + tid; a < x; a += bd) {
+        if (__fadd_rn(Gp[a], wcost_sides(c.inv_d, wside(c, a), xs, lamf)) == target) {
+          atomicMin(c.found, a);
+          break;
+        }
+      }
+      __syncthreads();
+      const int f = *c.found;
+      x = (f == 0x7fffffff) ? i - 2 : f;  // not reached: the minimum is one of the sums
+      if (tid == 0) c.sQ[i - 2] = x;
+      __syncthreads();  // every thread has read found before it is reset
+    }
+  }
+  __syncthreads();
+  const int m = mr > 0 ? mr : 2;
   if (refine > 0) wrefine(c, lam, m, refine);
   if (warp_id() == 0) wevaluate(c, lam, refine > 0, m, out);
   __syncthreads();
@@ -1085,7 +1098,9 @@ constexpr int kWideApproxThreads = 512;
 
 // Dynamic shared memory of k_approx_wide: the three codes, then the tiled
 // sweep's staging, partial minima, block costs, diagonal block and A-tile ends.
-__host__ __device__ inline size_t wide_smem_head(int S) { return (sizeof(int) * 3 * static_cast<size_t>(S) + 15) & ~size_t(15); }
+__host__ __device__ inline size_t wide_smem_head(int S) {
+  return (sizeof(int) * 3 * static_cast<size_t>(S) + 15) & ~size_t(15);
+}
 __host__ __device__ inline size_t wide_smem_bytes(int S) {
   const size_t kS = static_cast<size_t>(wide_tile_layers(S));
   const size_t nw = kWideApproxThreads / kWarp;
@@ -1098,7 +1113,7 @@ __global__ void __launch_bounds__(kWideApproxThreads, 1) k_approx_wide(ApproxArg
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ AOut s_out;
   __shared__ int s_flag;
-  __shared__ int s_misc[2];
+  __shared__ int s_misc[3];
   __shared__ double s_tot[6][kWideApproxThreads / kWarp];
   const int p = a.p, S = a.s, tid = threadIdx.x, lane = lane_id(), warp = warp_id();
   constexpr int kNW = kWideApproxThreads / kWarp;
@@ -1122,6 +1137,7 @@ __global__ void __launch_bounds__(kWideApproxThreads, 1) k_approx_wide(ApproxArg
   }
   c.moved = &s_misc[0];
   c.msh = &s_misc[1];
+  c.found = &s_misc[2];
   unsigned char* gs = a.scratch + static_cast<size_t>(blockIdx.x) * a.scratch_per_cta;
   auto take = [&gs](size_t bytes) {
     unsigned char* r = gs;
