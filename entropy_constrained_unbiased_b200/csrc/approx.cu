@@ -978,17 +978,25 @@ __device__ __noinline__ void wide_layers_tiled(const WCtx& cx, float lamf) {
       float best[kS];
 #pragma unroll
       for (int q = 0; q < kS; ++q) best[q] = part[q * kWT + lane];
+      // two rows at a time: eight relaxations are four packed additions and
+      // four three-input minima
 #pragma unroll 1
-      for (int j = 0; j < kWA; ++j) {
-        const float w = ws[j * kWT + lane];
-        const float4* g4 = reinterpret_cast<const float4*>(gs + j * kS);
+      for (int j = 0; j < kWA; j += 2) {
+        const float w0 = ws[j * kWT + lane], w1 = ws[(j + 1) * kWT + lane];
+        const float2 ww0 = make_float2(w0, w0), ww1 = make_float2(w1, w1);
+        const float4* g0 = reinterpret_cast<const float4*>(gs + j * kS);
+        const float4* g1 = reinterpret_cast<const float4*>(gs + (j + 1) * kS);
 #pragma unroll
         for (int q4 = 0; q4 < kS / 4; ++q4) {
-          const float4 g = g4[q4];
-          best[4 * q4 + 0] = fminf(best[4 * q4 + 0], __fadd_rn(g.x, w));
-          best[4 * q4 + 1] = fminf(best[4 * q4 + 1], __fadd_rn(g.y, w));
-          best[4 * q4 + 2] = fminf(best[4 * q4 + 2], __fadd_rn(g.z, w));
-          best[4 * q4 + 3] = fminf(best[4 * q4 + 3], __fadd_rn(g.w, w));
+          const float4 ga = g0[q4], gb = g1[q4];
+          const float2 a01 = add_f32x2(make_float2(ga.x, ga.y), ww0);
+          const float2 a23 = add_f32x2(make_float2(ga.z, ga.w), ww0);
+          const float2 b01 = add_f32x2(make_float2(gb.x, gb.y), ww1);
+          const float2 b23 = add_f32x2(make_float2(gb.z, gb.w), ww1);
+          best[4 * q4 + 0] = min3f(best[4 * q4 + 0], a01.x, b01.x);
+          best[4 * q4 + 1] = min3f(best[4 * q4 + 1], a01.y, b01.y);
+          best[4 * q4 + 2] = min3f(best[4 * q4 + 2], a23.x, b23.x);
+          best[4 * q4 + 3] = min3f(best[4 * q4 + 3], a23.y, b23.y);
         }
       }
 #pragma unroll
