@@ -302,24 +302,30 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
     t_ms = D.max_over_ranks(float(sum(step_ms)))
     D.barrier()
 
-    # e2e: same step through the C ABI with host buffers, copies inside the timed region
+    # e2e: same step through the C ABI with host buffers, copies inside the timed
+    # region: pinned input, the step's results read back into pinned buffers;
+    # one untimed pass (allocations), then as many timed steps as above
     Xpin = torch.from_numpy(X_host).pin_memory()
+    keys = ("Q1", "Q2", "theta") if w.mode == "budget" else ()
+    host_out = None
     e2e_ms = []
-    for k in range(max(1, min(args.steps, 3))):
+    for k in range(args.steps + 1):
         flush.fill_(k & 0xFF)
         torch.cuda.synchronize()
-        t0 = time.perf_counter()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         Xd = Xpin.to(dev, non_blocking=True)
         o2, idx2, hist2, H2 = step(Xd)
-        res = [idx2.to("cpu", non_blocking=True), H2.to("cpu", non_blocking=True)]
-        if w.mode == "budget":
-            res += [o2[k2].to("cpu", non_blocking=True) for k2 in ("Q1", "Q2", "theta")]
+        dev_out = [idx2, H2] + [o2[k2] for k2 in keys]
+        if host_out is None:
+            host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in dev_out]
+        for h, t in zip(host_out, dev_out):
+            h.copy_(t, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms.append(e0.elapsed_time(e1))
+        if k > 0:
+            e2e_ms.append(e0.elapsed_time(e1))
     bo = n * d + n * 8 + (n * s * 4 * 2 + n * 8 if w.mode == "budget" else 0)
 
     peaks = measured_peaks()
