@@ -726,11 +726,6 @@ struct WCtx {
   double* ab;
   double* bb;
   float* G;         // [(S+1) * pst] layers
-  float* tG;        // tiled layers: [warps][kWT][kS] staged layer values of an A-tile
-  float* tpart;     // [warps][kS][kWT] per-warp partial minima of an X-tile
-  float* tw;        // [warps][kWA][kWT] pair costs of a block
-  WSide* tside;     // [warps][kWA] the A-tile's ends of the pair terms
-  float* tdiag;     // [kWT][kWT] costs of the diagonal block
   double* fbuf;     // [warps][p] local costs of the refinement
   int* sQ;
   int* moved;
@@ -935,6 +930,21 @@ __host__ __device__ inline int wide_tile_layers(int S) {
   return S - 1 <= 8 ? 8 : (S - 1 <= 16 ? 16 : (S - 1 <= 32 ? 32 : 0));
 }
 
+constexpr int kWideApproxThreads = 512;
+
+// Dynamic shared memory of k_approx_wide: the three codes, then the tiled
+// sweep's staging, partial minima, block costs, diagonal block and A-tile ends.
+__host__ __device__ inline size_t wide_smem_head(int S) {
+  return (sizeof(int) * 3 * static_cast<size_t>(S) + 15) & ~size_t(15);
+}
+__host__ __device__ inline size_t wide_smem_bytes(int S) {
+  const size_t kS = static_cast<size_t>(wide_tile_layers(S));
+  const size_t nw = kWideApproxThreads / kWarp;
+  return wide_smem_head(S) +
+         (kS ? sizeof(float) * (nw * kWA * kS + nw * kS * kWT + nw * kWA * kWT + kWT * kWT) + sizeof(WSide) * nw * kWA
+             : 0);
+}
+
 template <int kS>
 __device__ __noinline__ void wide_layers_tiled(const WCtx& cx, float lamf) {
   // the context in registers: a reference would be re-read from local memory
@@ -944,16 +954,25 @@ __device__ __noinline__ void wide_layers_tiled(const WCtx& cx, float lamf) {
   const int lane = lane_id(), warp = warp_id(), nw = bd / kWarp;
   const double inv_d = c.inv_d;
   float* __restrict__ G = c.G;
-  float* __restrict__ tpart = c.tpart;
-  float* __restrict__ tdiag = c.tdiag;
+  // the tiles, carved here from the dynamic shared array (after the three
+  // codes) so that every access compiles to a shared-memory instruction:
+  // staged layer values [warps][kWA][kS], partial minima [warps][kS][kWT], block
+  // costs [warps][kWA][kWT], the diagonal block's costs [kWT][kWT], the A-tile
+  // ends [warps][kWA]
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* tG = reinterpret_cast<float*>(smem + wide_smem_head(S));
+  float* tpart = tG + static_cast<size_t>(nw) * kWA * kS;
+  float* tw = tpart + static_cast<size_t>(nw) * kS * kWT;
+  float* tdiag = tw + static_cast<size_t>(nw) * kWA * kWT;
+  WSide* tside = reinterpret_cast<WSide*>(tdiag + kWT * kWT);
   const float inf = __int_as_float(0x7f800000);
   for (int i = 1; i <= S; ++i)
     for (int x = tid; x < p; x += bd) G[i * pst + x] = (i == 1 && x == 0) ? 0.0f : inf;
   __syncthreads();
-  float* gs = c.tG + static_cast<size_t>(warp) * kWA * kS;    // [kWA][kS]
-  float* ws = c.tw + static_cast<size_t>(warp) * kWA * kWT;    // [kWA][kWT]
+  float* gs = tG + static_cast<size_t>(warp) * kWA * kS;       // [kWA][kS]
+  float* ws = tw + static_cast<size_t>(warp) * kWA * kWT;      // [kWA][kWT]
   float* part = tpart + static_cast<size_t>(warp) * kS * kWT;  // [kS][kWT]
-  WSide* as = c.tside + static_cast<size_t>(warp) * kWA;       // [kWA]
+  WSide* as = tside + static_cast<size_t>(warp) * kWA;         // [kWA]
   const int ntile = (p + kWT - 1) / kWT;
   for (int xt = 0; xt < ntile; ++xt) {
     const int x0 = xt * kWT, x = x0 + lane;
@@ -967,10 +986,11 @@ __device__ __noinline__ void wide_layers_tiled(const WCtx& cx, float lamf) {
       // are not read), then the block's costs ws[j][lane] = w(a0 + j, x); the
       // partial minima stay in shared memory between blocks so that the cost
       // evaluation has the registers
-      if (lane < kWA) {
-        as[lane] = wside(c, a0 + lane);
+      if (lane < kWA) as[lane] = wside(c, a0 + lane);
 #pragma unroll
-        for (int q = 0; q < kS; ++q) gs[lane * kS + q] = (q + 1 <= S - 1) ? G[(q + 1) * pst + a0 + lane] : inf;
+      for (int e = lane; e < kWA * kS; e += kWarp) {  // consecutive lanes, consecutive words
+        const int j = e / kS, q = e % kS;
+        gs[e] = (q + 1 <= S - 1) ? G[(q + 1) * pst + a0 + j] : inf;
       }
       __syncwarp();
       for (int j = 0; j < kWA; ++j) ws[j * kWT + lane] = xin ? wcost_sides(inv_d, as[j], xs, lamf) : 0.0f;
@@ -1102,21 +1122,6 @@ __device__ void approx_solve_wide(const WCtx& c, double lam, int refine, AOut* o
   __syncthreads();
 }
 
-constexpr int kWideApproxThreads = 512;
-
-// Dynamic shared memory of k_approx_wide: the three codes, then the tiled
-// sweep's staging, partial minima, block costs, diagonal block and A-tile ends.
-__host__ __device__ inline size_t wide_smem_head(int S) {
-  return (sizeof(int) * 3 * static_cast<size_t>(S) + 15) & ~size_t(15);
-}
-__host__ __device__ inline size_t wide_smem_bytes(int S) {
-  const size_t kS = static_cast<size_t>(wide_tile_layers(S));
-  const size_t nw = kWideApproxThreads / kWarp;
-  return wide_smem_head(S) +
-         (kS ? sizeof(float) * (nw * kWA * kS + nw * kS * kWT + nw * kWA * kWT + kWT * kWT) + sizeof(WSide) * nw * kWA
-             : 0);
-}
-
 __global__ void __launch_bounds__(kWideApproxThreads, 1) k_approx_wide(ApproxArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ AOut s_out;
@@ -1134,15 +1139,6 @@ __global__ void __launch_bounds__(kWideApproxThreads, 1) k_approx_wide(ApproxArg
   c.sQ = reinterpret_cast<int*>(smem);
   int* sQ1 = c.sQ + S;
   int* sQ2 = sQ1 + S;
-  {
-    const int kS = wide_tile_layers(S);
-    unsigned char* ts = smem + wide_smem_head(S);
-    c.tG = reinterpret_cast<float*>(ts);
-    c.tpart = c.tG + static_cast<size_t>(kNW) * kWA * kS;
-    c.tw = c.tpart + static_cast<size_t>(kNW) * kS * kWT;
-    c.tdiag = c.tw + static_cast<size_t>(kNW) * kWA * kWT;
-    c.tside = reinterpret_cast<WSide*>(c.tdiag + kWT * kWT);
-  }
   c.moved = &s_misc[0];
   c.msh = &s_misc[1];
   c.found = &s_misc[2];
