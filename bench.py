@@ -37,7 +37,7 @@ METRIC = "ECASQ DP (k,l,j) triples/s"  # the same string in both arms
 B200_SMS = 148
 
 # DRAM bytes (read + write) per k_dp launch per row, from one ncu capture of
-# k_dp on the first 296 rows of the weights workload (1.71 MB read, 1411 MB
+# k_dp on the first 296 rows of the weights workload (1.40 MB read, 1409 MB
 # written, almost all of it the stored DP layers written back from L2), scaled
 # by the rows of a launch. The figure belongs to the kernel source it was taken
 # on; it is dropped (null) when that source has changed since.
