@@ -133,3 +133,21 @@ def test_hirschberg_triple_count_matches_enumeration():
                 want += _pass_enum(p - 1 - code[hi], p - 1 - code[lo], hi - mid, False)
                 segs += [sg for sg in ((lo, mid), (mid + 1, hi)) if sg[1] - sg[0] - 1 >= 1]
             assert hirschberg_triples(code, p, s) == want, (p, s, code)
+
+
+def test_quantize_argument_checks_and_no_cpu_path():
+    """quantize() checks its arguments before any call and, without a GPU,
+    fails in the binding instead of computing anything on the CPU."""
+    import torch
+    from entropy_constrained_unbiased_b200 import ecasq
+    from entropy_constrained_unbiased_b200.pipeline import quantize
+    X = torch.zeros(1, 8)
+    with pytest.raises(ecasq.EcasqError):
+        quantize(X, 4, 2)
+    with pytest.raises(ecasq.EcasqError):
+        quantize(X, 4, 2, b=1.0, lam=0.1)
+    with pytest.raises(ecasq.EcasqError):
+        quantize(X, 4, 2, b=1.0, solver="other")
+    if not torch.cuda.is_available():
+        with pytest.raises(ecasq.EcasqError):
+            quantize(X, 4, 2, b=1.0)
