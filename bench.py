@@ -671,16 +671,19 @@ def measure_unit_peaks():
     return {k: v for k, v in out.items() if v > 0}
 
 
-def oracle_sample(w: W.Workload, budget_s: float):
-    """Time the fp64 oracle on a deterministic row sample of the workload."""
+def oracle_sample(w: W.Workload, budget_s: float, stages: bool = True):
+    """Time the fp64 oracle on a deterministic row sample of the workload: the
+    exact DP solves (the metric), then, on the same rows, the other stages of
+    the path (grid, bucketing, encoding with the solved codes, the
+    approximation), so that each GPU stage has the oracle's rate beside it."""
     from oracle import oracle as O
 
     rows = 1
     X = W.make_inputs(w, rows=64 if w.n >= 64 else w.n)
-    stride = max(1, X.shape[0] // 64)
     threads = O.threads()
     tps = triples_per_solve(w.p, w.s)
     done_rows, solves, t_tot = 0, 0, 0.0
+    codes = []
     while done_rows < X.shape[0] and t_tot < budget_s:
         take = min(max(rows, threads), X.shape[0] - done_rows)
         Xs = np.ascontiguousarray(X[done_rows:done_rows + take])
@@ -693,12 +696,47 @@ def oracle_sample(w: W.Workload, budget_s: float):
             solves += int(sum(2 if st[i] == 1 else (1 if lam_hi[i] == 0 else 2 + w.steps) for i in range(take)))
         else:
             lam = w.lambdas()[:take]
-            O.solve_batch(Xs, P, w.s, lam)
+            r = O.solve_batch(Xs, P, w.s, lam)
             solves += take * lam.shape[1]
         t_tot += time.perf_counter() - t0
+        codes.append(r)
         done_rows += take
-    return {"value": solves * tps / t_tot, "unit": "triples/s", "cores": threads, "kind": "oracle",
-            "sample": f"first {done_rows} rows of {w.n} ({solves} fp64 DP solves, {t_tot:.1f} s)"}
+    res = {"value": solves * tps / t_tot, "unit": "triples/s", "cores": threads, "kind": "oracle",
+           "sample": f"first {done_rows} rows of {w.n} ({solves} fp64 DP solves, {t_tot:.1f} s)"}
+    if not stages or done_rows == 0:
+        return res
+    Xs = np.ascontiguousarray(X[:done_rows])
+    entries = Xs.size
+    out = {}
+    t0 = time.perf_counter()
+    P, _ = O.grid_batch(Xs, w.p)
+    out["grid"] = {"entries_per_s": entries / (time.perf_counter() - t0), "cores": threads}
+    t0 = time.perf_counter()
+    for i in range(done_rows):
+        O.bucket(Xs[i], P[i])
+    out["bucket"] = {"entries_per_s": entries / (time.perf_counter() - t0), "cores": 1}
+    if w.mode == "budget":
+        cat = {k: np.concatenate([c[k] for c in codes]) for k in ("Q1", "m1", "Q2", "m2", "theta")}
+        t0 = time.perf_counter()
+        O.encode_batch(Xs, P, cat["Q1"], cat["m1"], w.s, w.seed_encode, cat["Q2"], cat["m2"], cat["theta"])
+    else:
+        Q = np.concatenate([c["Q"][:, 0, :] for c in codes])
+        m = np.concatenate([c["m"][:, 0] for c in codes])
+        t0 = time.perf_counter()
+        O.encode_batch(Xs, P, Q, m, w.s, w.seed_encode)
+    out["encode"] = {"entries_per_s": entries / (time.perf_counter() - t0), "cores": threads}
+    t0 = time.perf_counter()
+    if w.mode == "budget":
+        ra = O.solve_approx_budget_batch(Xs, P, w.s, w.b, w.steps)
+        n_ap = int(sum(1 if ra["lam_hi"][i] == 0 else 2 + w.steps for i in range(done_rows)))
+    else:
+        O.solve_approx_batch(Xs, P, w.s, w.lambdas()[:done_rows])
+        n_ap = done_rows * w.lambdas().shape[1]
+    t_ap = time.perf_counter() - t0
+    out["approx"] = {"relaxations_per_s": n_ap * relaxations_per_solve(w.p, w.s) / t_ap, "solves": n_ap,
+                     "cores": threads}
+    res["stages"] = out
+    return res
 
 
 def run_reference(args, w: W.Workload, rank: int, world: int):
@@ -708,11 +746,11 @@ def run_reference(args, w: W.Workload, rank: int, world: int):
         return None
     per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        oracle_sample(w, per_step / 4)
+        oracle_sample(w, per_step / 4, stages=False)
     vals = []
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        vals.append(oracle_sample(w, per_step))
+        vals.append(oracle_sample(w, per_step, stages=False))
     wall = time.perf_counter() - t0
     v = float(np.mean([x["value"] for x in vals]))
     cb = dict(vals[-1])
