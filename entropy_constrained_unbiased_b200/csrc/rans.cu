@@ -125,25 +125,42 @@ __device__ __forceinline__ int row_mode(int two_codes, const double* theta, int 
   return t >= 1.0 ? 0 : 1;
 }
 
+// A warp's two models (parts 0 and 1), in dynamic shared memory sized by s.
 struct WarpModel {
-  uint32_t f[2 * 256];
-  uint32_t cum[2 * 257];
   // floor(x / f) = umulhi64(x, rcp) for x < 2^32, f in [2, 2^15]:
   // rcp = ceil(2^47 / f) * 2^17; the product overestimates x/f by less than
   // x / 2^47 < 2^-15 <= 1/f, which never crosses the next integer.
-  unsigned long long rcp[2 * 256];
+  unsigned long long* rcp;  // [2s]
+  uint32_t* f;              // [2s]
+  uint32_t* cum;            // [2(s+1)]
 };
+
+// Bytes of one warp's models (16-byte multiple).
+__host__ __device__ inline size_t warp_model_bytes(int s) {
+  return (sizeof(unsigned long long) * 2 * s + sizeof(uint32_t) * 2 * s + sizeof(uint32_t) * 2 * (s + 1) + 15) &
+         ~size_t(15);
+}
+
+__device__ __forceinline__ WarpModel warp_model(unsigned char* base, int s, int warp) {
+  unsigned char* b = base + warp_model_bytes(s) * warp;
+  WarpModel m;
+  m.rcp = reinterpret_cast<unsigned long long*>(b);
+  m.f = reinterpret_cast<uint32_t*>(b + sizeof(unsigned long long) * 2 * s);
+  m.cum = m.f + 2 * s;
+  return m;
+}
 
 constexpr int kChunk = 32;  // steps staged at a time
 
-// Symbols and parts of kChunk steps, staged in shared memory so that the serial
-// state updates do not wait on global loads or on Philox.
+// The decoder's staged chunk: the parts of kChunk steps (so that the serial
+// state updates do not wait on Philox) and the decoded symbols, written back
+// to the row in one coalesced pass.
 struct WarpStage {
   uint8_t sym[kChunk * kWarp];
   uint32_t part[kChunk];  // bit j of word t: part of lane j at step t_lo + t
 };
 
-__device__ void model_reciprocals(WarpModel& m, int s) {
+__device__ void model_reciprocals(const WarpModel& m, int s) {
   for (int i = lane_id(); i < 2 * s; i += kWarp) {
     const unsigned long long f = m.f[i];
     m.rcp[i] = f >= 2 ? (((1ull << 47) + f - 1) / f) << 17 : 0ull;
@@ -151,24 +168,12 @@ __device__ void model_reciprocals(WarpModel& m, int s) {
   __syncwarp();
 }
 
-// Parts of steps t_lo .. t_hi-1 (lane j draws the 8 Philox blocks of step
-// t_lo + j), and, when xrow is given, their symbols.
-__device__ void stage_chunk(const uint8_t* __restrict__ xrow, int64_t d, int64_t base, int t_lo, int t_hi, uint32_t row,
-                            uint32_t k0, uint32_t k1, int mode, double th, WarpStage& st) {
+// Parts of steps t_lo .. t_hi-1 for the decoder (lane j draws the 8 Philox
+// blocks of step t_lo + j).
+__device__ void stage_chunk(int64_t base, int t_lo, int t_hi, uint32_t row, uint32_t k0, uint32_t k1, int mode,
+                            double th, WarpStage& st) {
   const int lane = lane_id();
   const int64_t e_lo = base + static_cast<int64_t>(t_lo) * kWarp;
-  if (xrow) {
-    // all 32 loads of a lane in flight before the first store
-    const int n_ent = (t_hi - t_lo) * kWarp;
-    uint8_t v[kChunk];
-#pragma unroll
-    for (int k = 0; k < kChunk; ++k) {
-      const int i = k * kWarp + lane;
-      v[k] = (i < n_ent && e_lo + i < d) ? xrow[e_lo + i] : 0;
-    }
-#pragma unroll
-    for (int k = 0; k < kChunk; ++k) st.sym[k * kWarp + lane] = v[k];
-  }
   if (lane < t_hi - t_lo) {
     uint32_t bits = mode == 1 ? 0xffffffffu : 0u;
     if (mode == 2) {
@@ -190,22 +195,84 @@ __device__ void stage_chunk(const uint8_t* __restrict__ xrow, int64_t d, int64_t
   __syncwarp();
 }
 
+// The encoder's staged chunk: per entry the index of its (part, symbol) pair,
+// part * s + symbol, into the packed model; per step the parts' bit word.
+struct EncStage {
+  uint16_t code[kChunk * kWarp];
+  uint32_t part[kChunk];
+};
+
+// Parts (lane j draws the 8 Philox blocks of step t_lo + j) and the pair
+// indices of steps t_lo .. t_hi-1. A symbol >= s sets *bad and is coded as
+// s - 1 (the row's status reports it).
+__device__ void stage_codes(const uint8_t* __restrict__ xrow, int64_t d, int64_t base, int t_lo, int t_hi,
+                            uint32_t row, uint32_t k0, uint32_t k1, int mode, double th, int s, EncStage& st,
+                            int* bad) {
+  const int lane = lane_id();
+  const int64_t e_lo = base + static_cast<int64_t>(t_lo) * kWarp;
+  const int n_ent = (t_hi - t_lo) * kWarp;
+  uint8_t v[kChunk];
+#pragma unroll
+  for (int k = 0; k < kChunk; ++k) {  // all 32 loads of a lane in flight first
+    const int i = k * kWarp + lane;
+    v[k] = (i < n_ent && e_lo + i < d) ? xrow[e_lo + i] : 0;
+  }
+  if (lane < t_hi - t_lo) {
+    uint32_t bits = mode == 1 ? 0xffffffffu : 0u;
+    if (mode == 2) {
+      const int64_t e0 = e_lo + static_cast<int64_t>(lane) * kWarp;
+      // u < theta with u = word * 2^-32 is word < ceil(theta * 2^32): theta * 2^32
+      // is exact in fp64 and the word is an integer.
+      const uint64_t cut = static_cast<uint64_t>(ceil(th * 0x1p32));
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        const uint4 w = Philox4x32::block(make_uint4(static_cast<uint32_t>((e0 >> 2) + b), row, 1u, 0u), k0, k1);
+        bits |= (static_cast<uint64_t>(w.x) < cut ? 0u : 1u) << (4 * b);
+        bits |= (static_cast<uint64_t>(w.y) < cut ? 0u : 1u) << (4 * b + 1);
+        bits |= (static_cast<uint64_t>(w.z) < cut ? 0u : 1u) << (4 * b + 2);
+        bits |= (static_cast<uint64_t>(w.w) < cut ? 0u : 1u) << (4 * b + 3);
+      }
+    }
+    st.part[lane] = bits;
+  }
+  __syncwarp();
+#pragma unroll
+  for (int k = 0; k < kChunk; ++k) {
+    const int i = k * kWarp + lane;
+    int sym = v[k];
+    if (i < n_ent && e_lo + i < d && sym >= s) {
+      *bad = 1;
+      sym = s - 1;
+    }
+    const int part = (k < t_hi - t_lo) ? static_cast<int>((st.part[k] >> lane) & 1u) : 0;
+    st.code[i] = static_cast<uint16_t>(part * s + sym);
+  }
+  __syncwarp();
+}
+
 __global__ void __launch_bounds__(kWarp * kWarpsPerBlock) k_rans_encode(
     const uint8_t* __restrict__ idx, const int64_t* __restrict__ hist, const double* __restrict__ theta,
     int two_codes, int n, int64_t d, int s, uint64_t seed, int64_t nseg, uint16_t* __restrict__ words,
     int32_t* __restrict__ seg_len, int32_t* __restrict__ status) {
-  __shared__ WarpModel sm[kWarpsPerBlock];
-  __shared__ WarpStage ss[kWarpsPerBlock];
+  extern __shared__ __align__(16) unsigned char rsm[];
+  __shared__ EncStage ss[kWarpsPerBlock];
   const int warp = warp_id(), lane = lane_id();
   const int64_t unit = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + warp;
   if (unit >= static_cast<int64_t>(n) * nseg) return;  // warp-uniform
   const int r = static_cast<int>(unit / nseg);
   const int64_t g = unit % nseg;
-  WarpModel& m = sm[warp];
-  WarpStage& st = ss[warp];
+  const WarpModel m = warp_model(rsm, s, warp);
+  EncStage& st = ss[warp];
   build_model(hist + static_cast<int64_t>(r) * 2 * s, s, m.f, m.cum);
   build_model(hist + static_cast<int64_t>(r) * 2 * s + s, s, m.f + s, m.cum + s + 1);
   model_reciprocals(m, s);
+  // pack each pair's frequency and cumulative start into one word of m.f:
+  // f | c << 16 (both below 2^16), so a step reads one word and the reciprocal
+  for (int i = lane_id(); i < 2 * s; i += kWarp) {
+    const int part = i >= s ? 1 : 0, sym = i - part * s;
+    m.f[i] |= m.cum[part * (s + 1) + sym] << 16;
+  }
+  __syncwarp();
   double th;
   const int mode = row_mode(two_codes, theta, r, &th);
   const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
@@ -220,24 +287,16 @@ __global__ void __launch_bounds__(kWarp * kWarpsPerBlock) k_rans_encode(
   for (int ch = (steps - 1) / kChunk; ch >= 0; --ch) {
     const int t_lo = ch * kChunk, t_hi = min(steps, t_lo + kChunk);
     __syncwarp();  // the previous chunk's reads are done
-    stage_chunk(xrow, d, base, t_lo, t_hi, static_cast<uint32_t>(r), k0, k1, mode, th, st);
+    stage_codes(xrow, d, base, t_lo, t_hi, static_cast<uint32_t>(r), k0, k1, mode, th, s, st, &bad);
     for (int t = t_hi - 1; t >= t_lo; --t) {
       const bool live = t * kWarp + lane < len32;
-      const int part = (st.part[t - t_lo] >> lane) & 1;
-      const int sym = st.sym[(t - t_lo) * kWarp + lane];
-      uint32_t f = 1, c = 0;
-      unsigned long long rc = 0;
-      if (live) {
-        if (sym < s) {
-          f = m.f[part * s + sym];
-          c = m.cum[part * (s + 1) + sym];
-          rc = m.rcp[part * s + sym];
-        }
-        if (sym >= s || f == 0) {
-          bad = 1;
-          f = 1;
-        }
-      }
+      const uint32_t code = st.code[(t - t_lo) * kWarp + lane];
+      const uint32_t fc = m.f[code];
+      const unsigned long long rc = m.rcp[code];
+      const uint32_t c = fc >> 16;
+      uint32_t f = fc & 0xFFFFu;
+      if (live && f == 0) bad = 1;
+      f = f == 0 ? 1u : f;
       // x >= 2^17 f  <=>  floor(x / 2^17) >= f
       const bool need = live && (x >> 17) >= f;
       const unsigned mask = __ballot_sync(0xffffffffu, need);
@@ -268,14 +327,14 @@ __global__ void __launch_bounds__(kWarp * kWarpsPerBlock) k_rans_decode(
     const uint16_t* __restrict__ words, const int32_t* __restrict__ seg_len, const int64_t* __restrict__ hist,
     const double* __restrict__ theta, int two_codes, int n, int64_t d, int s, uint64_t seed, int64_t nseg,
     uint8_t* __restrict__ idx, int32_t* __restrict__ status) {
-  __shared__ WarpModel sm[kWarpsPerBlock];
+  extern __shared__ __align__(16) unsigned char rsm[];
   __shared__ WarpStage ss[kWarpsPerBlock];
   const int warp = warp_id(), lane = lane_id();
   const int64_t unit = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + warp;
   if (unit >= static_cast<int64_t>(n) * nseg) return;  // warp-uniform
   const int r = static_cast<int>(unit / nseg);
   const int64_t g = unit % nseg;
-  WarpModel& m = sm[warp];
+  const WarpModel m = warp_model(rsm, s, warp);
   WarpStage& st = ss[warp];
   build_model(hist + static_cast<int64_t>(r) * 2 * s, s, m.f, m.cum);
   build_model(hist + static_cast<int64_t>(r) * 2 * s + s, s, m.f + s, m.cum + s + 1);
@@ -298,7 +357,7 @@ __global__ void __launch_bounds__(kWarp * kWarpsPerBlock) k_rans_decode(
   for (int ch = 0; ch * kChunk < steps && !bad; ++ch) {
     const int t_lo = ch * kChunk, t_hi = min(steps, t_lo + kChunk);
     __syncwarp();
-    stage_chunk(nullptr, d, base, t_lo, t_hi, static_cast<uint32_t>(r), k0, k1, mode, th, st);
+    stage_chunk(base, t_lo, t_hi, static_cast<uint32_t>(r), k0, k1, mode, th, st);
     for (int t = t_lo; t < t_hi; ++t) {
       const bool live = t * kWarp + lane < len32;
       const int part = (st.part[t - t_lo] >> lane) & 1;
@@ -355,7 +414,7 @@ cudaError_t launch_rans_encode(const uint8_t* idx, const int64_t* hist, const do
   const int64_t units = static_cast<int64_t>(n) * nseg;
   cudaMemsetAsync(status, 0, sizeof(int32_t) * n, st);
   const int64_t blocks = (units + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  k_rans_encode<<<static_cast<unsigned>(blocks), kWarp * kWarpsPerBlock, 0, st>>>(idx, hist, theta, two_codes, n, d,
+  k_rans_encode<<<static_cast<unsigned>(blocks), kWarp * kWarpsPerBlock, warp_model_bytes(s) * kWarpsPerBlock, st>>>(idx, hist, theta, two_codes, n, d,
                                                                                    s, seed, nseg, words, seg_len,
                                                                                    status);
   note_launch();
@@ -369,7 +428,7 @@ cudaError_t launch_rans_decode(const uint16_t* words, const int32_t* seg_len, co
   const int64_t units = static_cast<int64_t>(n) * nseg;
   cudaMemsetAsync(status, 0, sizeof(int32_t) * n, st);
   const int64_t blocks = (units + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  k_rans_decode<<<static_cast<unsigned>(blocks), kWarp * kWarpsPerBlock, 0, st>>>(words, seg_len, hist, theta,
+  k_rans_decode<<<static_cast<unsigned>(blocks), kWarp * kWarpsPerBlock, warp_model_bytes(s) * kWarpsPerBlock, st>>>(words, seg_len, hist, theta,
                                                                                    two_codes, n, d, s, seed, nseg, idx,
                                                                                    status);
   note_launch();
