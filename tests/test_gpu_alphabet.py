@@ -201,3 +201,29 @@ def test_approx_large_alphabet_code_sizes(E, O, wide, s):
             J_ib = mse + lam[r, t] * O.eval_raw_ib(X[r], vals)
             assert J_ib <= ref["J"][r, t] * (1 + 1e-5), (r, t, J_ib, ref["J"][r, t])
             assert g["objective"][r, t].item() == pytest.approx(J_ib, rel=1e-9)
+
+
+def test_approx_4097_value_alphabet_single_column_tail(E, O):
+    """A 4097-value BF16 alphabet (every BF16 value in [2^-16, 2^16]): the tiled
+    sweep's last X-tile holds one column (4097 = 128 x 32 + 1). One row at one
+    lambda (the oracle's O(p^2) tables take seconds here) against the oracle's
+    optimum, fp64 figures against its raw evaluation."""
+    X = W.pinned_range_rows(7, 1, 65536, 2.0 ** -16, 2.0 ** 16)
+    Xd = torch.from_numpy(X).cuda()
+    Pd, p_len, st = E.bf16_alphabet(Xd, 8192)
+    p = int(p_len[0].item())
+    assert p == 4097 and int(st.abs().sum()) == 0
+    P = Pd[:, :p].contiguous()
+    lam = np.var(X.astype(np.float64), axis=1)[:, None] * np.array([[0.01]])
+    s = 16
+    g = E.solve_approx(Xd, P, s, torch.from_numpy(lam).cuda())
+    assert int(g["status"].abs().sum()) == 0
+    Pn = P.cpu().numpy()
+    ref = O.solve_approx_batch(X, Pn, s, lam, refine=0)
+    Q, m = g["Q"].cpu().numpy(), g["Q_len"].cpu().numpy()
+    for t in range(lam.shape[1]):
+        vals = Pn[0][Q[0, t, : m[0, t]]]
+        mse, _, _ = O.eval_raw(X[0], vals)
+        J_ib = mse + lam[0, t] * O.eval_raw_ib(X[0], vals)
+        assert J_ib <= ref["J"][0, t] * (1 + 1e-5), (t, J_ib, ref["J"][0, t])
+        assert g["objective"][0, t].item() == pytest.approx(J_ib, rel=1e-9)
