@@ -522,6 +522,31 @@ int eo_encode(const float* x, int64_t d, const double* P, int p, const int32_t* 
   return 0;
 }
 
+// Reconstruction X^ of one encoded vector: entry j takes the value of its
+// index in the code its part used (the part drawn exactly as eo_encode draws
+// it), rounded to float32. E[X^] = X is the unbiasedness of §1 "O Problema
+// ECASQ". Returns -1 when an index lies outside its code.
+int eo_dequantize(const uint8_t* idx, int64_t d, const double* P, const int32_t* Q1, int m1,
+                  const int32_t* Q2, int m2, double theta, uint64_t seed, uint32_t v, float* out) {
+  const bool mix = Q2 && theta > 0.0 && theta < 1.0;
+  for (int64_t j = 0; j < d; ++j) {
+    int part;
+    if (!Q2) {
+      part = 0;
+    } else if (mix) {
+      double us = double(philox_word(seed, j, v, 1u)) * 0x1p-32;
+      part = (us < theta) ? 0 : 1;
+    } else {
+      part = (theta >= 1.0) ? 0 : 1;
+    }
+    const int32_t* q = part == 0 ? Q1 : Q2;
+    const int m = part == 0 ? m1 : m2;
+    if (idx[j] >= m) return -1;
+    out[j] = float(P[q[idx[j]]]);
+  }
+  return 0;
+}
+
 // Empirical entropy of the emitted indices: per part H_part = -sum c/d_part log2(c/d_part),
 // combined as (d_0 H_0 + d_1 H_1)/d.
 double eo_entropy(const int64_t* hist, int s) {
@@ -605,6 +630,18 @@ int eo_encode_batch(const float* X, int n, int64_t d, const double* P, int p, co
                           Q2 ? Q2 + int64_t(r) * s : nullptr, Q2 ? m2[r] : 0,
                           theta ? theta[r] : 0.0, s, seed, uint32_t(r), idx + int64_t(r) * d,
                           hist + int64_t(r) * 2 * s);
+  }
+  return eo_threads();
+}
+
+int eo_dequantize_batch(const uint8_t* idx, int n, int64_t d, const double* P, int p, const int32_t* Q1,
+                        const int32_t* m1, const int32_t* Q2, const int32_t* m2, const double* theta, int s,
+                        uint64_t seed, float* out, int32_t* status) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int r = 0; r < n; ++r) {
+    status[r] = eo_dequantize(idx + int64_t(r) * d, d, P + int64_t(r) * p, Q1 + int64_t(r) * s, m1[r],
+                              Q2 ? Q2 + int64_t(r) * s : nullptr, Q2 ? m2[r] : 0, theta ? theta[r] : 0.0, seed,
+                              uint32_t(r), out + int64_t(r) * d);
   }
   return eo_threads();
 }

@@ -52,6 +52,8 @@ def lib():
             "eo_encode_batch": (I, [f32p, I, I64, f64p, I, i32p, i32p, C.c_void_p, C.c_void_p, C.c_void_p,
                                     I, U64, u8p, i64p, i32p]),
             "eo_grid_batch": (I, [f32p, I, I64, I, f64p, i32p]),
+            "eo_dequantize_batch": (I, [u8p, I, I64, f64p, I, i32p, i32p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                        I, U64, f32p, i32p]),
             "eo_hib_tables": (D, [f64p, f64p, f64p, I, I64, i32p, I]),
             "eo_bf16_alphabet": (I, [f32p, I64, f64p, I]),
             "eo_rans_segment_words": (C.c_int64, []),
@@ -366,6 +368,31 @@ def encode_batch(X, P, Q1, m1, s, seed, Q2=None, m2=None, theta=None):
     lib().eo_encode_batch(X, n, d, P, p, Q1, m1, q2p, m2p, thp, s, C.c_uint64(seed), idx, hist, st)
     del keep
     return idx, hist, st
+
+
+def dequantize_batch(idx, P, Q1, m1, s, seed, Q2=None, m2=None, theta=None):
+    """X^ [n, d] float32 from the indices of encode_batch (same codes, seed and
+    theta); status -1 for a row with an index outside its code."""
+    idx = np.ascontiguousarray(idx, np.uint8)
+    n, d = idx.shape
+    P = _f64(P)
+    p = P.shape[1]
+    Q1 = np.ascontiguousarray(Q1, np.int32).reshape(n, s)
+    m1 = np.ascontiguousarray(m1, np.int32).reshape(n)
+    out = np.zeros((n, d), np.float32)
+    st = np.zeros(n, np.int32)
+    keep = []
+    if Q2 is not None:
+        Q2 = np.ascontiguousarray(Q2, np.int32).reshape(n, s)
+        m2 = np.ascontiguousarray(m2, np.int32).reshape(n)
+        th = _f64(theta).reshape(n)
+        keep = [Q2, m2, th]
+        q2p, m2p, thp = (a.ctypes.data_as(C.c_void_p) for a in keep)
+    else:
+        q2p = m2p = thp = None
+    lib().eo_dequantize_batch(idx, n, d, P, p, Q1, m1, q2p, m2p, thp, s, C.c_uint64(seed), out, st)
+    del keep
+    return out, st
 
 
 def encode_row(x, P_row, Q1, m1, s, seed, row, Q2=None, m2=0, theta=0.0):
