@@ -446,6 +446,16 @@ int ecasq_encode(const float* X, const double* P, int n, int64_t d, int p, int s
                                    static_cast<cudaStream_t>(stream)));
 }
 
+int ecasq_dequantize(const uint8_t* idx, const double* P, int n, int64_t d, int p, int s, const int32_t* Q1,
+                     const int32_t* Q1_len, const int32_t* Q2, const int32_t* Q2_len, const double* theta,
+                     uint64_t seed, float* Xhat, int32_t* status, void* stream) {
+  if (!idx || !P || !Q1 || !Q1_len || !Xhat || !status || !valid_sizes(n, d, p, 2, kMaxPWide) || s < 1 || s > 256)
+    return ECASQ_ERR_ARG;
+  if (Q2 && !Q2_len) return ECASQ_ERR_ARG;
+  return cuda_status(launch_dequantize(idx, P, n, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, seed, Xhat, status,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 int64_t ecasq_rans_segments(int64_t d) { return d >= 1 ? rans_segments(d) : 0; }
 int64_t ecasq_rans_segment_words(void) { return rans_segment_words(); }
 

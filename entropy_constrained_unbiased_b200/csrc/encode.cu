@@ -473,6 +473,127 @@ size_t encode_smem(int p, int s) {
 
 }  // namespace
 
+// ---- reconstruction X^ from the indices ---------------------------------------
+// X^[r][j] = P[r][Q_part[idx[r][j]]] rounded to float32, the part of entry j
+// drawn as k_encode draws it (§1 "O Problema ECASQ": the emitted value whose
+// expectation is the entry; §2.1: time-sharing). One CTA per (row, chunk of
+// kEncChunk entries); the codes' values sit in shared memory as float32 and
+// each thread handles aligned groups of four entries (one Philox block of the
+// part stream per group when the row mixes two codes).
+namespace {
+__global__ void __launch_bounds__(kEncThreads) k_dequantize(const uint8_t* __restrict__ idx,
+                                                           const double* __restrict__ Pall, int64_t d, int p, int s,
+                                                           const int32_t* __restrict__ Q1,
+                                                           const int32_t* __restrict__ Q1_len,
+                                                           const int32_t* __restrict__ Q2,
+                                                           const int32_t* __restrict__ Q2_len,
+                                                           const double* __restrict__ theta,
+                                                           const Philox4x32::RoundKeys K, float* __restrict__ out,
+                                                           int32_t* __restrict__ status) {
+  __shared__ float qv[2][256];
+  __shared__ int s_m[2];
+  __shared__ int s_bad;
+  const int r = blockIdx.y;
+  const bool has2 = (Q2 != nullptr);
+  const double th = (has2 && theta) ? theta[r] : 0.0;
+  const bool mix = has2 && th > 0.0 && th < 1.0;
+  const int fixed_part = (!has2 || th >= 1.0) ? 0 : 1;
+  if (threadIdx.x == 0) {
+    s_m[0] = Q1_len[r];
+    s_m[1] = has2 ? Q2_len[r] : 0;
+    s_bad = 0;
+  }
+  __syncthreads();
+  int bad = 0;
+  for (int k = threadIdx.x; k < 2 * 256; k += blockDim.x) {
+    const int part = k >> 8, t = k & 255;
+    const int32_t* Q = part == 0 ? Q1 : Q2;
+    float v = __int_as_float(0x7fc00000);  // no value: an index here is an error
+    if (Q && t < s && t < s_m[part]) {
+      const int32_t q = Q[static_cast<int64_t>(r) * s + t];
+      if (q >= 0 && q < p)
+        v = static_cast<float>(Pall[static_cast<int64_t>(r) * p + q]);
+      else
+        bad = 1;
+    }
+    qv[part][t] = v;
+  }
+  if (bad) s_bad = 1;
+  __syncthreads();
+  const int m0 = s_m[0], m1 = s_m[1];
+  // u < theta with u = word * 2^-32 is word <= ceil(theta * 2^32) - 1
+  const uint32_t th_last = mix ? static_cast<uint32_t>(static_cast<uint64_t>(ceil(th * 0x1p32)) - 1u) : 0u;
+  const int64_t beg = static_cast<int64_t>(blockIdx.x) * kEncChunk;
+  const int len = static_cast<int>((beg + kEncChunk < d ? beg + kEncChunk : d) - beg);
+  const uint8_t* ix = idx + static_cast<int64_t>(r) * d + beg;
+  float* o = out + static_cast<int64_t>(r) * d + beg;
+  const bool vec = ((reinterpret_cast<uintptr_t>(ix) & 3u) == 0) && ((reinterpret_cast<uintptr_t>(o) & 15u) == 0);
+  const uint32_t blk0 = static_cast<uint32_t>(static_cast<uint64_t>(beg) >> 2);
+  Philox4x32::RoundKeys rk;
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    rk.k0[i] = K.k0[i];
+    rk.k1[i] = K.k1[i];
+  }
+  // beg is a multiple of 4, so group g holds the entries of Philox block blk0 + g
+  for (int g = threadIdx.x; 4 * g < len; g += blockDim.x) {
+    const int j = 4 * g;
+    const int cnt = len - j < 4 ? len - j : 4;
+    uint32_t sel[4] = {0u, 0u, 0u, 0u};
+    if (mix) {
+      const uint4 w = Philox4x32::block(make_uint4(blk0 + static_cast<uint32_t>(g), static_cast<uint32_t>(r), 1u, 0u),
+                                        rk);
+      sel[0] = w.x;
+      sel[1] = w.y;
+      sel[2] = w.z;
+      sel[3] = w.w;
+    }
+    uint32_t iv[4] = {0u, 0u, 0u, 0u};
+    if (vec && cnt == 4) {
+      const uchar4 b = *reinterpret_cast<const uchar4*>(ix + j);
+      iv[0] = b.x;
+      iv[1] = b.y;
+      iv[2] = b.z;
+      iv[3] = b.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (e < cnt) iv[e] = ix[j + e];
+    }
+    float v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int part = mix ? (sel[e] <= th_last ? 0 : 1) : fixed_part;
+      bad |= (e < cnt) && static_cast<int>(iv[e]) >= (part == 0 ? m0 : m1);
+      v[e] = qv[part][iv[e]];
+    }
+    if (vec && cnt == 4) {
+      __stcs(reinterpret_cast<float4*>(o + j), make_float4(v[0], v[1], v[2], v[3]));
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (e < cnt) o[j + e] = v[e];
+    }
+  }
+  if (bad) s_bad = 1;
+  __syncthreads();
+  if (threadIdx.x == 0 && s_bad) atomicExch(status + r, kStatusRange);
+}
+}  // namespace
+
+cudaError_t launch_dequantize(const uint8_t* idx, const double* P, int n, int64_t d, int p, int s,
+                              const int32_t* Q1, const int32_t* Q1_len, const int32_t* Q2, const int32_t* Q2_len,
+                              const double* theta, uint64_t seed, float* Xhat, int32_t* status, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t) * n, st);
+  if (e != cudaSuccess) return e;
+  const int nc = static_cast<int>((d + kEncChunk - 1) / kEncChunk);
+  const Philox4x32::RoundKeys K =
+      Philox4x32::round_keys(static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
+  k_dequantize<<<dim3(nc, n), kEncThreads, 0, st>>>(idx, P, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, Xhat, status);
+  note_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_encode(const float* X, const double* P, int n, int64_t d, int p, int s,
                           const int32_t* Q1, const int32_t* Q1_len, const int32_t* Q2,
                           const int32_t* Q2_len, const double* theta, uint64_t seed, uint8_t* idx,

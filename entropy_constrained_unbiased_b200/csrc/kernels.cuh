@@ -167,5 +167,8 @@ cudaError_t launch_encode(const float* X, const double* P, int n, int64_t d, int
                           const int32_t* Q2_len, const double* theta, uint64_t seed, uint8_t* idx,
                           int64_t* hist, int32_t* status, cudaStream_t st);
 cudaError_t launch_entropy(const int64_t* hist, int n, int s, double* H, cudaStream_t st);
+cudaError_t launch_dequantize(const uint8_t* idx, const double* P, int n, int64_t d, int p, int s,
+                              const int32_t* Q1, const int32_t* Q1_len, const int32_t* Q2, const int32_t* Q2_len,
+                              const double* theta, uint64_t seed, float* Xhat, int32_t* status, cudaStream_t st);
 
 }  // namespace ecasq

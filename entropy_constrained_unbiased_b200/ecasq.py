@@ -22,8 +22,8 @@ EXPORTS = [
     "ecasq_solve", "ecasq_solve_stats", "ecasq_solve_budget", "ecasq_solve_budget_stats",
     "ecasq_approx_workspace_size", "ecasq_solve_approx", "ecasq_solve_approx_stats", "ecasq_solve_approx_budget",
     "ecasq_solve_approx_budget_stats",
-    "ecasq_encode", "ecasq_entropy", "ecasq_rans_segments", "ecasq_rans_segment_words", "ecasq_rans_encode",
-    "ecasq_rans_decode", "ecasq_status_string", "ecasq_launch_count",
+    "ecasq_encode", "ecasq_dequantize", "ecasq_entropy", "ecasq_rans_segments", "ecasq_rans_segment_words",
+    "ecasq_rans_encode", "ecasq_rans_decode", "ecasq_status_string", "ecasq_launch_count",
 ]
 
 
@@ -68,6 +68,7 @@ def load(path: str = LIB_PATH):
         "ecasq_solve_approx_budget_stats": (I, [P, P, P, P, I, I64, I, I, D, I] + [P] * 14 + [OP, P, SZ, P]),
         "ecasq_encode": (I, [P, P, I, I64, I, I, P, P, P, P, P, U64, P, P, P, P]),
         "ecasq_entropy": (I, [P, I, I, P, P]),
+        "ecasq_dequantize": (I, [P, P, I, I64, I, I, P, P, P, P, P, U64, P, P, P]),
         "ecasq_rans_segments": (I64, [I64]),
         "ecasq_rans_segment_words": (I64, []),
         "ecasq_rans_encode": (I, [P, P, P, I, I, I64, I, U64, P, P, P, P]),
@@ -397,6 +398,21 @@ def encode(X: torch.Tensor, P: torch.Tensor, s: int, Q1, Q1_len, seed: int, Q2=N
     _check(L.ecasq_encode(_ptr(X), _ptr(P), n, d, p, s, _ptr(Q1), _ptr(Q1_len), _ptr(Q2), _ptr(Q2_len), _ptr(theta),
                           C.c_uint64(seed), _ptr(idx), _ptr(hist), _ptr(st), _stream()), "ecasq_encode")
     return idx, hist, st
+
+
+def dequantize(idx: torch.Tensor, P: torch.Tensor, s: int, Q1, Q1_len, seed: int, Q2=None, Q2_len=None,
+               theta=None):
+    """X^ [n,d] float32 from the indices of encode (same codes, s, seed and theta), and status."""
+    L = _need_cuda()
+    _dev(idx, torch.uint8, "idx")
+    _dev(P, torch.float64, "P")
+    n, d = idx.shape
+    p = P.shape[1]
+    Xh = torch.empty((n, d), dtype=torch.float32, device=idx.device)
+    st = torch.empty(n, dtype=torch.int32, device=idx.device)
+    _check(L.ecasq_dequantize(_ptr(idx), _ptr(P), n, d, p, s, _ptr(Q1), _ptr(Q1_len), _ptr(Q2), _ptr(Q2_len),
+                              _ptr(theta), C.c_uint64(seed), _ptr(Xh), _ptr(st), _stream()), "ecasq_dequantize")
+    return Xh, st
 
 
 def entropy(hist: torch.Tensor):

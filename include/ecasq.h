@@ -272,6 +272,19 @@ int ecasq_encode(const float* X, const double* P, int n, int64_t d, int p, int s
                  const int32_t* Q2_len, const double* theta, uint64_t seed, uint8_t* idx,
                  int64_t* hist, int32_t* status, void* stream);
 
+/* Reconstruction X^ from the emitted indices (§1 "O Problema ECASQ": the
+ * quantized value of each entry, with E[X^] = X; §2.1: the time-sharing part
+ * drawn again from seed and theta exactly as ecasq_encode drew it):
+ * Xhat[r][j] = P[r][Q_part[r][idx[r][j]]] rounded to float32, with Q1, Q1_len,
+ * Q2, Q2_len, theta, s and seed as given to ecasq_encode. Xhat [n][d] float32
+ * (device, caller-owned). status[r] = ECASQ_ERR_RANGE when an index is not
+ * below its code's length (or a code holds an index outside P); that row's
+ * values are then unspecified. Asynchronous; allocates nothing. */
+int ecasq_dequantize(const uint8_t* idx, const double* P, int n, int64_t d, int p, int s,
+                     const int32_t* Q1, const int32_t* Q1_len, const int32_t* Q2,
+                     const int32_t* Q2_len, const double* theta, uint64_t seed, float* Xhat,
+                     int32_t* status, void* stream);
+
 /* Empirical entropy of the emitted indices from hist [n][2][s] (§1, H(X^)):
  * per part H_part = -sum c/d_part log2(c/d_part), combined as
  * (d_0 H_0 + d_1 H_1)/(d_0 + d_1). H [n] float64. */
