@@ -441,16 +441,20 @@ def run_ours(args, w: W.Workload, rank: int, world: int):
 
 def stage_figures(E, X, P, p, s, enc_args, stream, flush, hbm):
     """Device time of the uniform grid (min/max pass + grid), bucketing, the two
-    in one call, and encoding, each call alone after an L2 flush; algorithmic
-    bytes: 4 B/entry read for the grid, for bucketing and for the combined call,
-    4 B read + 1 B written for encoding (the histograms are fused)."""
+    in one call, encoding and the reconstruction, each call alone after an L2
+    flush; algorithmic bytes: 4 B/entry read for the grid, for bucketing and for
+    the combined call, 4 B read + 1 B written for encoding (the histograms are
+    fused), 1 B read + 4 B written for the reconstruction."""
     entries = X.numel()
+    idx, _, _ = E.encode(X, P, s, *enc_args)  # the reconstruction takes the encoder's arguments
     fns = {"grid": lambda: E.uniform_grid(X, p), "bucket": lambda: E.bucket(X, P),
-           "grid_bucket": lambda: E.grid_bucket(X, p), "encode": lambda: E.encode(X, P, s, *enc_args)}
+           "grid_bucket": lambda: E.grid_bucket(X, p), "encode": lambda: E.encode(X, P, s, *enc_args),
+           "dequantize": lambda: E.dequantize(idx, P, s, *enc_args)}
     out = {}
     # grid_bucket: the grid and bucketing in one call, one read of X (4 B/entry)
-    # when rows fit in shared memory, else the two passes above (8 B/entry)
-    for name, bpe in (("grid", 4), ("bucket", 4), ("grid_bucket", 4), ("encode", 5)):
+    # when rows fit in shared memory, else the two passes above (8 B/entry);
+    # dequantize: 1 B of index read and 4 B of X^ written per entry
+    for name, bpe in (("grid", 4), ("bucket", 4), ("grid_bucket", 4), ("encode", 5), ("dequantize", 5)):
         fns[name]()
         ms = device_ms(fns[name], stream, flush)
         gbs = entries * bpe / (ms * 1e-3) / 1e9

@@ -477,9 +477,9 @@ size_t encode_smem(int p, int s) {
 // X^[r][j] = P[r][Q_part[idx[r][j]]] rounded to float32, the part of entry j
 // drawn as k_encode draws it (§1 "O Problema ECASQ": the emitted value whose
 // expectation is the entry; §2.1: time-sharing). One CTA per (row, chunk of
-// kEncChunk entries); the codes' values sit in shared memory as float32 and
-// each thread handles aligned groups of four entries (one Philox block of the
-// part stream per group when the row mixes two codes).
+// kEncChunk entries); the codes' values sit in shared memory as float32; a
+// thread handles 16 entries at a time on 16-byte aligned rows, else four (one
+// Philox block of the part stream per four entries when the row mixes codes).
 namespace {
 __global__ void __launch_bounds__(kEncThreads) k_dequantize(const uint8_t* __restrict__ idx,
                                                            const double* __restrict__ Pall, int64_t d, int p, int s,
@@ -527,7 +527,6 @@ __global__ void __launch_bounds__(kEncThreads) k_dequantize(const uint8_t* __res
   const int len = static_cast<int>((beg + kEncChunk < d ? beg + kEncChunk : d) - beg);
   const uint8_t* ix = idx + static_cast<int64_t>(r) * d + beg;
   float* o = out + static_cast<int64_t>(r) * d + beg;
-  const bool vec = ((reinterpret_cast<uintptr_t>(ix) & 3u) == 0) && ((reinterpret_cast<uintptr_t>(o) & 15u) == 0);
   const uint32_t blk0 = static_cast<uint32_t>(static_cast<uint64_t>(beg) >> 2);
   Philox4x32::RoundKeys rk;
 #pragma unroll
@@ -535,45 +534,45 @@ __global__ void __launch_bounds__(kEncThreads) k_dequantize(const uint8_t* __res
     rk.k0[i] = K.k0[i];
     rk.k1[i] = K.k1[i];
   }
-  // beg is a multiple of 4, so group g holds the entries of Philox block blk0 + g
-  for (int g = threadIdx.x; 4 * g < len; g += blockDim.x) {
+  auto value = [&](uint32_t sel, uint32_t i) {
+    const int part = mix ? (sel <= th_last ? 0 : 1) : fixed_part;
+    bad |= static_cast<int>(i) >= (part == 0 ? m0 : m1);
+    return qv[part][i];
+  };
+  const bool vec16 = ((reinterpret_cast<uintptr_t>(ix) & 15u) == 0) && ((reinterpret_cast<uintptr_t>(o) & 15u) == 0);
+  int j16 = 0;
+  if (vec16) {
+    // 16 entries per thread and step: one 16-byte index load, four Philox
+    // blocks of the part stream (mixed rows), four 16-byte stores
+    const int n16 = len >> 4;
+    for (int g = threadIdx.x; g < n16; g += blockDim.x) {
+      const uint4 b16 = *reinterpret_cast<const uint4*>(ix + 16 * g);
+      const uint32_t w32[4] = {b16.x, b16.y, b16.z, b16.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 sel = make_uint4(0u, 0u, 0u, 0u);
+        if (mix)
+          sel = Philox4x32::block(
+              make_uint4(blk0 + static_cast<uint32_t>(4 * g + q), static_cast<uint32_t>(r), 1u, 0u), rk);
+        const float4 v = make_float4(value(sel.x, w32[q] & 0xFFu), value(sel.y, (w32[q] >> 8) & 0xFFu),
+                                     value(sel.z, (w32[q] >> 16) & 0xFFu), value(sel.w, w32[q] >> 24));
+        __stcs(reinterpret_cast<float4*>(o + 16 * g + 4 * q), v);
+      }
+    }
+    j16 = n16 << 4;
+  }
+  // the rest (rows off 16-byte alignment, the last < 16 entries) four at a
+  // time; beg and j16 are multiples of 4, so group g holds the entries of
+  // Philox block blk0 + g
+  for (int g = (j16 >> 2) + threadIdx.x; 4 * g < len; g += blockDim.x) {
     const int j = 4 * g;
     const int cnt = len - j < 4 ? len - j : 4;
-    uint32_t sel[4] = {0u, 0u, 0u, 0u};
-    if (mix) {
-      const uint4 w = Philox4x32::block(make_uint4(blk0 + static_cast<uint32_t>(g), static_cast<uint32_t>(r), 1u, 0u),
-                                        rk);
-      sel[0] = w.x;
-      sel[1] = w.y;
-      sel[2] = w.z;
-      sel[3] = w.w;
-    }
-    uint32_t iv[4] = {0u, 0u, 0u, 0u};
-    if (vec && cnt == 4) {
-      const uchar4 b = *reinterpret_cast<const uchar4*>(ix + j);
-      iv[0] = b.x;
-      iv[1] = b.y;
-      iv[2] = b.z;
-      iv[3] = b.w;
-    } else {
+    uint4 sel = make_uint4(0u, 0u, 0u, 0u);
+    if (mix) sel = Philox4x32::block(make_uint4(blk0 + static_cast<uint32_t>(g), static_cast<uint32_t>(r), 1u, 0u), rk);
+    const uint32_t sv[4] = {sel.x, sel.y, sel.z, sel.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (e < cnt) iv[e] = ix[j + e];
-    }
-    float v[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int part = mix ? (sel[e] <= th_last ? 0 : 1) : fixed_part;
-      bad |= (e < cnt) && static_cast<int>(iv[e]) >= (part == 0 ? m0 : m1);
-      v[e] = qv[part][iv[e]];
-    }
-    if (vec && cnt == 4) {
-      __stcs(reinterpret_cast<float4*>(o + j), make_float4(v[0], v[1], v[2], v[3]));
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (e < cnt) o[j + e] = v[e];
-    }
+    for (int e = 0; e < 4; ++e)
+      if (e < cnt) o[j + e] = value(sv[e], ix[j + e]);
   }
   if (bad) s_bad = 1;
   __syncthreads();

@@ -8,7 +8,8 @@ gist.science/pt/paper/2608.18147, §1 "O Problema ECASQ" and §2):
 - the solver: exact or approximate, at a fixed λ or under an entropy budget
   with two-way time-sharing;
 - stochastic-rounding encoding;
-- the empirical entropy of the indices.
+- the empirical entropy of the indices;
+- on request (`Quantized.dequantize`), the reconstruction X^.
 
 Every step runs in the library's kernels; this module only chooses the calls
 and passes tensors between them. There is no CPU path.
@@ -34,6 +35,16 @@ class Quantized:
     Q2_len: torch.Tensor | None = None
     theta: torch.Tensor | None = None    # [n] share of the entries coded with Q1
     stats: dict = field(default_factory=dict)  # the solver's fp64 figures (mse, H, lambda, ...)
+    seed: int = 0
+
+    def dequantize(self) -> torch.Tensor:
+        """X^ [n, d] float32: each entry's value in the code its part used."""
+        s = self.Q1.shape[1]
+        Xh, st = E.dequantize(self.idx, self.P, s, self.Q1, self.Q1_len, self.seed, self.Q2, self.Q2_len,
+                              self.theta)
+        if int(st.abs().sum()) != 0:
+            raise E.EcasqError(f"reconstruction rejected rows: {st.nonzero().flatten().tolist()[:8]}")
+        return Xh
 
 
 def quantize(X: torch.Tensor, p: int, s: int, *, b: float | None = None, lam: float | None = None,
@@ -69,7 +80,7 @@ def quantize(X: torch.Tensor, p: int, s: int, *, b: float | None = None, lam: fl
             g = E.solve_approx_budget_stats(cnt, A, B, P, d, s, b, refine=refine, steps=steps, fp64=fp64)
         idx, hist, est = E.encode(X, P, s, g["Q1"], g["Q1_len"], seed, g["Q2"], g["Q2_len"], g["theta"])
         out = Quantized(P=P, Q1=g["Q1"], Q1_len=g["Q1_len"], Q2=g["Q2"], Q2_len=g["Q2_len"], theta=g["theta"],
-                        idx=idx, hist=hist, H_emp=E.entropy(hist))
+                        idx=idx, hist=hist, H_emp=E.entropy(hist), seed=seed)
         skip = ("Q1", "Q1_len", "Q2", "Q2_len", "theta")
     else:
         lam_t = torch.full((n, 1), float(lam), dtype=torch.float64, device=X.device)
@@ -80,7 +91,7 @@ def quantize(X: torch.Tensor, p: int, s: int, *, b: float | None = None, lam: fl
         Q1 = g["Q"][:, 0, :].contiguous()
         Q1_len = g["Q_len"][:, 0].contiguous()
         idx, hist, est = E.encode(X, P, s, Q1, Q1_len, seed)
-        out = Quantized(P=P, Q1=Q1, Q1_len=Q1_len, idx=idx, hist=hist, H_emp=E.entropy(hist))
+        out = Quantized(P=P, Q1=Q1, Q1_len=Q1_len, idx=idx, hist=hist, H_emp=E.entropy(hist), seed=seed)
         skip = ("Q", "Q_len")
     if int(est.abs().sum()) != 0:
         raise E.EcasqError(f"encoding rejected rows: {est.nonzero().flatten().tolist()[:8]}")

@@ -44,6 +44,8 @@ def test_quantize_budget_matches_the_calls(E, O, solver):
     _eq(q.hist, hist)
     _eq(q.H_emp, E.entropy(hist))
     assert set(q.stats) >= {"status", "mse1", "mse2", "H1", "H2"}
+    Xh, _ = E.dequantize(idx, P, s, g["Q1"], g["Q1_len"], seed, g["Q2"], g["Q2_len"], g["theta"])
+    _eq(q.dequantize(), Xh)
     # the time-shared indices against the oracle's encoder
     Pn, gn = P.cpu().numpy(), {k: v.cpu().numpy() for k, v in g.items()}
     io, ho, so = O.encode_batch(X, Pn, gn["Q1"], gn["Q1_len"], s, seed, gn["Q2"], gn["Q2_len"], gn["theta"])
