@@ -177,6 +177,11 @@ def test_approx_budget_and_encode_large_alphabet(E, O, wide):
     assert np.all(so == 0)
     np.testing.assert_array_equal(idx.cpu().numpy(), io)
     np.testing.assert_array_equal(hist.cpu().numpy(), ho)
+    # and the reconstruction on the large alphabet
+    Xh, sd = E.dequantize(idx, P, s, g["Q1"], g["Q1_len"], 7, g["Q2"], g["Q2_len"], g["theta"])
+    ref, sr = O.dequantize_batch(io, Pn, gn["Q1"], gn["Q1_len"], s, 7, gn["Q2"], gn["Q2_len"], gn["theta"])
+    assert int(sd.abs().sum()) == 0 and np.all(sr == 0)
+    np.testing.assert_array_equal(Xh.cpu().numpy(), ref)
 
 
 @pytest.mark.parametrize("s", [6, 24, 40])
