@@ -112,6 +112,8 @@ GRID_BUCKET_CASES = [  # (dist, n, d, p): one-read path (aligned, d <= 16384, p 
     ("normal", 2, 1, 16),
     ("grad", 3, 20000, 128),
     ("mixture", 3, 5000, 256),
+    ("laplace", 2, 70001, 257),   # long rows: the persistent bucketing kernel
+    ("normal", 2, 9000, 1000),    # beyond 512 values: bucketing by bisection
 ]
 
 
