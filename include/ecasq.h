@@ -35,8 +35,9 @@
  *   - Limits: 2 <= s <= 255 (s > p is treated as s = p), 1 <= d <= 2^31 - 1,
  *     n >= 1; 2 <= p <= 512 for the exact solver (ecasq_solve*,
  *     ecasq_workspace_size), 2 <= p <= 65536 for the grid, bucketing,
- *     encoding and the approximation (large alphabets, e.g. every BF16 value of
- *     a range; above 512 values the approximation runs fp32 layers only).
+ *     encoding, the reconstruction and the approximation (large alphabets, e.g.
+ *     every BF16 value of a range; above 512 values the approximation runs fp32
+ *     layers only).
  *   - Entropies are in bits per entry; the MSE is the per-entry mean
  *     (1/d) * sum (q_hi - x)(x - q_lo); the objective is MSE + lambda * H.
  */
