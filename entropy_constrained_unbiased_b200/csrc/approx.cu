@@ -37,6 +37,9 @@
 //     in the order of a direct sum with every operation rounded as written (no
 //     contraction), so every decision is taken on the same values as a plain
 //     fp64 statement of the method.
+// Alphabets beyond 512 values (k_approx_wide, further down) keep O(p) prefix
+// sums instead of the tables and evaluate each pair cost once per solve in a
+// tiled sweep that relaxes all layers with it.
 #include <cuda_runtime.h>
 
 #include <cstdint>
