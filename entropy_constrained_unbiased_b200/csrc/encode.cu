@@ -249,8 +249,8 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
       const uint32_t rw[4] = {ru.x, ru.y, ru.z, ru.w};
       const uint32_t sel[4] = {su.x, su.y, su.z, su.w};
       int part[4];
-      uint32_t packed = 0;
-      unsigned okm = 0;
+      uint32_t ob[4];
+      bool allok = true;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         part[e] = kMix ? (sel[e] <= th_last ? 0 : 1) : fixed_part;
@@ -269,13 +269,23 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
         const double prod = __dmul_rn(static_cast<double>(rw[e]), rec.y);
         const int out = t + ((prod < y) ? 1 : 0);
         red_shared_inc(wh_base + 4u * static_cast<uint32_t>(ok ? part[e] * s + out : trash));
-        packed |= static_cast<uint32_t>(out & 0xFF) << (8 * e);
-        okm |= ok ? (1u << e) : 0u;
+        ob[e] = static_cast<uint32_t>(out);
+        allok = allok && ok;
       }
-      if (okm != 0xFu) {
+      // bytes 0 of ob[0..3] into one word (out <= 255 on the fast path)
+      uint32_t packed = __byte_perm(__byte_perm(ob[0], ob[1], 0x0040), __byte_perm(ob[2], ob[3], 0x0040), 0x5410);
+      if (!allok) {
+        // the rare entries off the fast path: redo the test and code them exactly
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          if (!(okm & (1u << e))) {
+          const float gf = fmaf(xv[e], s_f, c_f);
+          const float tf = __fadd_rn(__fadd_rn(gf, -0.5f), 12582912.0f);
+          const float kf = __fsub_rn(tf, 12582912.0f);
+          const int k = __float_as_int(tf) - 0x4B400000;
+          const bool kin = static_cast<unsigned>(k) <= pm2;
+          const int t = tmap[part[e] * p + (kin ? k : 0)];
+          const bool ok = kin && fabsf((gf - kf) - 0.5f) < lim && t != 255;
+          if (!ok) {
             const int out = enc_fix1(&S, xv[e], rw[e], part[e]);
             packed = (packed & ~(0xFFu << (8 * e))) | (static_cast<uint32_t>(out) << (8 * e));
           }
