@@ -224,6 +224,10 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
   const int nf = vec ? (len >> 2) : 0;  // full float4 groups on the vector path
   const uint32_t wh_base = smem_addr(sh + warp_id() * nbins);
   const int trash = 2 * s;
+  // histogram word addresses: part 1's bins, the fixed part's, the trash bin
+  const uint32_t wh_p1 = wh_base + 4u * static_cast<uint32_t>(s);
+  const uint32_t wh_fixed = wh_base + 4u * static_cast<uint32_t>(fixed_part * s);
+  const uint32_t wh_trash = wh_base + 4u * static_cast<uint32_t>(trash);
   const uint32_t blk0 = static_cast<uint32_t>(static_cast<uint64_t>(beg) >> 2);
   Philox4x32::RoundKeys rk;
 #pragma unroll
@@ -268,7 +272,8 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
         const double y = __dsub_rn(static_cast<double>(xv[e]), rec.x);
         const double prod = __dmul_rn(static_cast<double>(rw[e]), rec.y);
         const int out = t + ((prod < y) ? 1 : 0);
-        red_shared_inc(wh_base + 4u * static_cast<uint32_t>(ok ? part[e] * s + out : trash));
+        const uint32_t hb = kMix ? (part[e] ? wh_p1 : wh_base) : wh_fixed;
+        red_shared_inc(ok ? hb + 4u * static_cast<uint32_t>(out) : wh_trash);
         ob[e] = static_cast<uint32_t>(out);
         allok = allok && ok;
       }
