@@ -23,7 +23,8 @@ namespace {
 
 constexpr int kEncThreads = 256;
 constexpr int kEncWarps = kEncThreads / kWarp;
-constexpr int64_t kEncChunk = 32768;  // entries per CTA (multiple of 4)
+constexpr int64_t kEncChunk = 65536;  // entries per encoder CTA (multiple of 4)
+constexpr int64_t kDeqChunk = 32768;  // entries per reconstruction CTA (multiple of 4)
 
 // Per-CTA state of the encoder in shared memory: the row's alphabet, both
 // codes, and the per-bucket records of the fast path.
@@ -492,7 +493,7 @@ size_t encode_smem(int p, int s) {
 // X^[r][j] = P[r][Q_part[idx[r][j]]] rounded to float32, the part of entry j
 // drawn as k_encode draws it (§1 "O Problema ECASQ": the emitted value whose
 // expectation is the entry; §2.1: time-sharing). One CTA per (row, chunk of
-// kEncChunk entries); the codes' values sit in shared memory as float32; a
+// kDeqChunk entries); the codes' values sit in shared memory as float32; a
 // thread handles 16 entries at a time on 16-byte aligned rows, else four (one
 // Philox block of the part stream per four entries when the row mixes codes).
 namespace {
@@ -538,8 +539,8 @@ __global__ void __launch_bounds__(kEncThreads) k_dequantize(const uint8_t* __res
   const int m0 = s_m[0], m1 = s_m[1];
   // u < theta with u = word * 2^-32 is word <= ceil(theta * 2^32) - 1
   const uint32_t th_last = mix ? static_cast<uint32_t>(static_cast<uint64_t>(ceil(th * 0x1p32)) - 1u) : 0u;
-  const int64_t beg = static_cast<int64_t>(blockIdx.x) * kEncChunk;
-  const int len = static_cast<int>((beg + kEncChunk < d ? beg + kEncChunk : d) - beg);
+  const int64_t beg = static_cast<int64_t>(blockIdx.x) * kDeqChunk;
+  const int len = static_cast<int>((beg + kDeqChunk < d ? beg + kDeqChunk : d) - beg);
   const uint8_t* ix = idx + static_cast<int64_t>(r) * d + beg;
   float* o = out + static_cast<int64_t>(r) * d + beg;
   const uint32_t blk0 = static_cast<uint32_t>(static_cast<uint64_t>(beg) >> 2);
@@ -600,7 +601,7 @@ cudaError_t launch_dequantize(const uint8_t* idx, const double* P, int n, int64_
                               const double* theta, uint64_t seed, float* Xhat, int32_t* status, cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t) * n, st);
   if (e != cudaSuccess) return e;
-  const int nc = static_cast<int>((d + kEncChunk - 1) / kEncChunk);
+  const int nc = static_cast<int>((d + kDeqChunk - 1) / kDeqChunk);
   const Philox4x32::RoundKeys K =
       Philox4x32::round_keys(static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
   k_dequantize<<<dim3(nc, n), kEncThreads, 0, st>>>(idx, P, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, Xhat, status);

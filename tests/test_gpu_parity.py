@@ -304,7 +304,7 @@ def test_budget_matches_oracle(E, O, case, fp64):
 
 # -- encoder -------------------------------------------------------------------------
 
-@pytest.mark.parametrize("d", [1, 3, 1024, 4099, 40000])
+@pytest.mark.parametrize("d", [1, 3, 1024, 4099, 40000, 140003])  # 140003: three encoder chunks, ragged
 def test_encode_bit_exact_single_code(E, O, d):
     X = _case(30, 3, d, "laplace")
     P, _ = O.grid_batch(X, 32)
@@ -321,9 +321,9 @@ def test_encode_bit_exact_single_code(E, O, d):
         assert H[r] == pytest.approx(O.entropy(ho[r], 6), rel=1e-12, abs=1e-15)
 
 
-@pytest.mark.parametrize("seed", [1, 2**40 + 12345])
-def test_encode_bit_exact_time_shared(E, O, seed):
-    X = _case(31, 4, 20001, "student_t")
+@pytest.mark.parametrize("seed,d", [(1, 20001), (2**40 + 12345, 20001), (5, 131077)])
+def test_encode_bit_exact_time_shared(E, O, seed, d):
+    X = _case(31, 4, d, "student_t")
     P, _ = O.grid_batch(X, 64)
     ref = O.solve_budget_batch(X, P, 10, 2.3, 30)
     args = [ref["Q1"], ref["m1"], ref["Q2"], ref["m2"], ref["theta"]]
