@@ -140,11 +140,11 @@ def dp_traffic(w):
 SPIN_CYCLES = 4_000_000  # about 2 ms of GPU clock
 
 
-def device_ms(fn, stream, flush, reps=3):
-    """Mean device time (ms) of the launches fn makes, each rep after an L2
-    flush. A spin kernel queued before the first event keeps the stream busy
-    while the host allocates and enqueues fn, so host overhead between the two
-    events is not counted."""
+def device_ms(fn, stream, flush, reps=3, stat="mean"):
+    """Mean (or median) device time (ms) of the launches fn makes, each rep
+    after an L2 flush. A spin kernel queued before the first event keeps the
+    stream busy while the host allocates and enqueues fn, so host overhead
+    between the two events is not counted."""
     import torch
 
     a = torch.cuda.Event(enable_timing=True)
@@ -158,7 +158,7 @@ def device_ms(fn, stream, flush, reps=3):
         b.record(stream)
         torch.cuda.synchronize()
         out.append(a.elapsed_time(b))
-    return float(np.mean(out))
+    return float(np.median(out) if stat == "median" else np.mean(out))
 
 
 def measured_peaks():
@@ -463,10 +463,12 @@ def stage_figures(E, X, P, p, s, enc_args, stream, flush, hbm):
     return out
 
 
-def dp_figure(E, w: W.Workload, cnt, A, B, P, stream, flush, mufu_peak, reps=2):
+def dp_figure(E, w: W.Workload, cnt, A, B, P, stream, flush, mufu_peak, reps=3):
     """Device time of one exact-solver call on a workload's bucket statistics
-    (L2 flushed before each call) and its triples/s against the MUFU peak.
-    Hirschberg's recovery passes are work the triple count leaves out."""
+    (L2 flushed before each call; the median of the reps, so that one
+    disturbed call does not move the figure) and its triples/s against the
+    MUFU peak. Hirschberg's recovery passes are work the triple count leaves
+    out."""
     import torch
 
     if w.mode == "budget":
@@ -479,7 +481,7 @@ def dp_figure(E, w: W.Workload, cnt, A, B, P, stream, flush, mufu_peak, reps=2):
             return E.solve_stats(cnt, A, B, P, w.d, w.s, lam, hirschberg=w.hirschberg)
     out = call()
     torch.cuda.synchronize()
-    ms = device_ms(call, stream, flush, reps=reps)
+    ms = device_ms(call, stream, flush, reps=reps, stat="median")
     ns = solves_done(w, out)
     tps = triples_per_solve(w.p, w.s)
     ach = ns * tps / (ms * 1e-3)

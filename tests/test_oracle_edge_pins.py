@@ -433,6 +433,32 @@ def _one_iteration(V, R, L, d, lam, Q, cls_of):
     return Q
 
 
+def test_refinement_search_stays_inside_the_open_interval():
+    """A value searches (c_{t-1}, c_{t+1}) only: it never lands on a neighbour,
+    also where the local cost still falls at the interval's right end (cases
+    of that kind are required to occur, so the check has teeth)."""
+    right_end = 0
+    for seed in range(200):
+        rng = np.random.default_rng(1000 + seed)
+        x = (rng.standard_normal(400) * rng.uniform(0.5, 2.0)).astype(np.float32)
+        P, _ = O.uniform_grid(x, 32)
+        cnt, A, B, _ = O.bucket(x, P)
+        V, R, L = O.tables(cnt, A, B, P)
+        lam = float(rng.uniform(0.01, 0.3)) * float(np.var(x.astype(np.float64)))
+        Q, _ = O.approx_dp(V, R, L, 8, x.size, lam)
+        Q = np.asarray(Q, np.int32)
+        for t in range(1, Q.size - 1):
+            lo, hi = int(Q[t - 1]) + 1, int(Q[t + 1]) - 1
+            if hi - lo < 1:
+                continue
+            c = O.refine_point(V, R, L, x.size, lam, Q, t)
+            assert lo <= c <= hi, (seed, t, c, lo, hi)
+            f = [O.refine_local(V, R, L, x.size, lam, Q, t, k) for k in (hi - 1, hi)]
+            if f[1] < f[0]:
+                right_end += 1
+    assert right_end >= 3
+
+
 def test_refinement_classes_run_in_position_order():
     """Q_c = {t : (t - 1) mod 3 = c} over the interior positions 1 .. m-2, so Q0
     holds position 1; one iteration runs Q0, Q1, Q2. Checked on cases where
