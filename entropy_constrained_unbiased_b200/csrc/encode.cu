@@ -23,7 +23,8 @@ namespace {
 
 constexpr int kEncThreads = 256;
 constexpr int kEncWarps = kEncThreads / kWarp;
-constexpr int64_t kEncChunk = 65536;  // entries per encoder CTA (multiple of 4)
+constexpr int64_t kEncChunk = 65536;    // entries per encoder CTA on grids that fill the GPU
+constexpr int64_t kEncMinChunk = 4096;  // fewest entries per encoder CTA
 constexpr int64_t kDeqChunk = 32768;  // entries per reconstruction CTA (multiple of 4)
 
 // Per-CTA state of the encoder in shared memory: the row's alphabet, both
@@ -71,6 +72,9 @@ __device__ __forceinline__ int enc_exact(EncRow& S, float xf, int part, uint32_t
 // Exact code of one entry that the fast path did not decide, with its
 // histogram count; kept out of line (scalar arguments, so that the fast loop
 // keeps its values in registers) so that the fast loop carries none of it.
+// One instance per kernel (kTag): a callee shared by two kernels gets a
+// calling convention fitted to neither, and the fast loop spills more.
+template <int kTag>
 __device__ __noinline__ int enc_fix1(EncRow* S, float x, uint32_t word, int part) {
   const int out = enc_exact(*S, x, part, word);
   red_shared_inc(smem_addr(S->hist + warp_id() * (2 * S->s + 1) + part * S->s + out));
@@ -85,14 +89,14 @@ __device__ __noinline__ int enc_fix1(EncRow* S, float x, uint32_t word, int part
 // interval and w' = (q_{t+1} - q_t) 2^-32; with u = word 2^-32 (both scalings
 // exact) u (q_{t+1} - q_t) = word w' as real numbers, so the product is
 // taken as word * w' in one rounding.
-template <bool kMix>
+template <bool kMix, int kTag>
 __device__ __forceinline__ void encode_row(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d,
                                            int p, int s, const int32_t* __restrict__ Q1,
                                            const int32_t* __restrict__ Q1_len, const int32_t* __restrict__ Q2,
                                            const int32_t* __restrict__ Q2_len, const double* __restrict__ theta,
                                            const Philox4x32::RoundKeys& K, uint8_t* __restrict__ idx,
                                            unsigned long long* __restrict__ hist, int32_t* __restrict__ status,
-                                           unsigned char* smem, EncRow& S, int& s_wexact) {
+                                           int64_t chunk, unsigned char* smem, EncRow& S, int& s_wexact) {
   const int r = blockIdx.y;
   const int nbins = 2 * s + 1;
   double2* sR = reinterpret_cast<double2*>(smem);                          // [2][p] (q_t, w') per bucket
@@ -217,8 +221,8 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
   // sel is an integer, so it is sel < ceil(theta * 2^32), i.e. sel <= cut - 1
   // (cut >= 1 whenever theta > 0).
   const uint32_t th_last = mix ? static_cast<uint32_t>(static_cast<uint64_t>(ceil(th * 0x1p32)) - 1u) : 0u;
-  const int64_t beg = static_cast<int64_t>(blockIdx.x) * kEncChunk;
-  const int len = static_cast<int>((beg + kEncChunk < d ? beg + kEncChunk : d) - beg);
+  const int64_t beg = static_cast<int64_t>(blockIdx.x) * chunk;
+  const int len = static_cast<int>((beg + chunk < d ? beg + chunk : d) - beg);
   const float* x = X + static_cast<int64_t>(r) * d + beg;
   uint8_t* o = idx + static_cast<int64_t>(r) * d + beg;
   const bool vec = ((reinterpret_cast<uintptr_t>(x) & 15u) == 0) && ((reinterpret_cast<uintptr_t>(o) & 3u) == 0);
@@ -292,7 +296,7 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
           const int t = tmap[part[e] * p + (kin ? k : 0)];
           const bool ok = kin && fabsf((gf - kf) - 0.5f) < lim && t != 255;
           if (!ok) {
-            const int out = enc_fix1(&S, xv[e], rw[e], part[e]);
+            const int out = enc_fix1<kTag>(&S, xv[e], rw[e], part[e]);
             packed = (packed & ~(0xFFu << (8 * e))) | (static_cast<uint32_t>(out) << (8 * e));
           }
         }
@@ -319,7 +323,7 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
     for (int e = 0; e < 4; ++e) {
       if (e < cnt) {
         const int part = mix ? (sel[e] <= th_last ? 0 : 1) : fixed_part;
-        o[j + e] = static_cast<uint8_t>(enc_fix1(&S, xv[e], rw[e], part));
+        o[j + e] = static_cast<uint8_t>(enc_fix1<kTag>(&S, xv[e], rw[e], part));
       }
     }
   }
@@ -346,9 +350,31 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
   __shared__ int s_wexact;
   const double th = (Q2 != nullptr && theta) ? theta[blockIdx.y] : 0.0;
   if (Q2 != nullptr && th > 0.0 && th < 1.0)
-    encode_row<true>(X, Pall, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, idx, hist, status, smem, S, s_wexact);
+    encode_row<true, 0>(X, Pall, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, idx, hist, status, kEncChunk, smem, S,
+                     s_wexact);
   else
-    encode_row<false>(X, Pall, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, idx, hist, status, smem, S, s_wexact);
+    encode_row<false, 0>(X, Pall, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, idx, hist, status, kEncChunk, smem, S,
+                      s_wexact);
+}
+
+// k_encode with chunks of `chunk` entries (a multiple of 4, below kEncChunk),
+// for grids of few or short rows that kEncChunk would leave part-empty.
+__global__ void __launch_bounds__(kEncThreads, 5)
+k_encode_chunked(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d, int p, int s,
+                 const int32_t* __restrict__ Q1, const int32_t* __restrict__ Q1_len,
+                 const int32_t* __restrict__ Q2, const int32_t* __restrict__ Q2_len,
+                 const double* __restrict__ theta, const Philox4x32::RoundKeys K, uint8_t* __restrict__ idx,
+                 unsigned long long* __restrict__ hist, int32_t* __restrict__ status, int64_t chunk) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ EncRow S;
+  __shared__ int s_wexact;
+  const double th = (Q2 != nullptr && theta) ? theta[blockIdx.y] : 0.0;
+  if (Q2 != nullptr && th > 0.0 && th < 1.0)
+    encode_row<true, 1>(X, Pall, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, idx, hist, status, chunk, smem, S,
+                     s_wexact);
+  else
+    encode_row<false, 1>(X, Pall, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, idx, hist, status, chunk, smem, S,
+                      s_wexact);
 }
 
 // Encoder for large alphabets (p > 512): no per-bucket tables; the interval of
@@ -359,7 +385,8 @@ __global__ void __launch_bounds__(kEncThreads)
 k_encode_code(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d, int p, int s,
               const int32_t* __restrict__ Q1, const int32_t* __restrict__ Q1_len, const int32_t* __restrict__ Q2,
               const int32_t* __restrict__ Q2_len, const double* __restrict__ theta, const Philox4x32::RoundKeys K,
-              uint8_t* __restrict__ idx, unsigned long long* __restrict__ hist, int32_t* __restrict__ status) {
+              uint8_t* __restrict__ idx, unsigned long long* __restrict__ hist, int32_t* __restrict__ status,
+              int64_t chunk) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ int s_m[2];
   __shared__ int s_bad;
@@ -402,8 +429,8 @@ k_encode_code(const float* __restrict__ X, const double* __restrict__ Pall, int6
     return;
   }
   const uint32_t th_last = mix ? static_cast<uint32_t>(static_cast<uint64_t>(ceil(th * 0x1p32)) - 1u) : 0u;
-  const int64_t beg = static_cast<int64_t>(blockIdx.x) * kEncChunk;
-  const int len = static_cast<int>((beg + kEncChunk < d ? beg + kEncChunk : d) - beg);
+  const int64_t beg = static_cast<int64_t>(blockIdx.x) * chunk;
+  const int len = static_cast<int>((beg + chunk < d ? beg + chunk : d) - beg);
   const float* x = X + static_cast<int64_t>(r) * d + beg;
   uint8_t* o = idx + static_cast<int64_t>(r) * d + beg;
   const uint32_t blk0 = static_cast<uint32_t>(static_cast<uint64_t>(beg) >> 2);
@@ -480,6 +507,20 @@ __global__ void k_entropy(const int64_t* __restrict__ hist, int n, int s, double
     tot += dp;
   }
   if (lane_id() == 0) H[r] = tot > 0.0 ? acc / tot : 0.0;
+}
+
+// Entries per encoder CTA: kEncChunk, unless the n * ceil(d / kEncChunk) CTAs
+// would leave resident slots empty (few or short rows); then ceil(resident / n)
+// chunks per row, each a multiple of 4 (a Philox block serves four entries, and
+// chunk starts stay 16-byte aligned on aligned rows) and at least
+// kEncMinChunk. Smaller chunks on full grids only add per-CTA setups.
+int64_t encode_chunk(int n, int64_t d, int64_t resident) {
+  const int64_t d4 = (d + 3) & ~int64_t(3);
+  if (d4 == 0) return kEncChunk;
+  if (static_cast<int64_t>(n) * ((d4 + kEncChunk - 1) / kEncChunk) >= resident) return kEncChunk;
+  const int64_t k = (resident + n - 1) / n;
+  const int64_t chunk = (((d4 + k - 1) / k) + 3) & ~int64_t(3);
+  return chunk < kEncMinChunk ? kEncMinChunk : (chunk > kEncChunk ? kEncChunk : chunk);
 }
 
 size_t encode_smem(int p, int s) {
@@ -617,17 +658,30 @@ cudaError_t launch_encode(const float* X, const double* P, int n, int64_t d, int
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(status, 0, sizeof(int32_t) * n, st);
   if (e != cudaSuccess) return e;
-  const int nc = static_cast<int>((d + kEncChunk - 1) / kEncChunk);
   const size_t smem = encode_smem(p, s);
+  const size_t sm2 = sizeof(double) * 2 * s + sizeof(unsigned int) * kEncWarps * 2 * s;
   const Philox4x32::RoundKeys K =
       Philox4x32::round_keys(static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
+  int dev = 0, sms = 0, per_sm = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  e = (p > kMaxP) ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_encode_code, kEncThreads, sm2)
+                  : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_encode, kEncThreads, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t chunk = encode_chunk(n, d, static_cast<int64_t>(sms) * (per_sm > 0 ? per_sm : 1));
+  const int nc = static_cast<int>((d + chunk - 1) / chunk);
   if (p > kMaxP) {
-    const size_t sm2 = sizeof(double) * 2 * s + sizeof(unsigned int) * kEncWarps * 2 * s;
     k_encode_code<<<dim3(nc, n), kEncThreads, sm2, st>>>(X, P, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, idx,
-                                                         reinterpret_cast<unsigned long long*>(hist), status);
-  } else {
+                                                         reinterpret_cast<unsigned long long*>(hist), status, chunk);
+  } else if (chunk == kEncChunk) {
     k_encode<<<dim3(nc, n), kEncThreads, smem, st>>>(X, P, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, idx,
                                                       reinterpret_cast<unsigned long long*>(hist), status);
+  } else {
+    k_encode_chunked<<<dim3(nc, n), kEncThreads, smem, st>>>(X, P, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K,
+                                                              idx, reinterpret_cast<unsigned long long*>(hist),
+                                                              status, chunk);
   }
   note_launch();
   return cudaGetLastError();
