@@ -14,6 +14,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -25,6 +26,7 @@ constexpr int kEncThreads = 256;
 constexpr int kEncWarps = kEncThreads / kWarp;
 constexpr int64_t kEncChunk = 65536;    // entries per encoder CTA on grids that fill the GPU
 constexpr int64_t kEncMinChunk = 4096;  // fewest entries per encoder CTA
+constexpr int kEncCtasPerSm = 5;         // resident encoder CTAs per SM (48 registers a thread)
 constexpr int64_t kDeqChunk = 32768;  // entries per reconstruction CTA (multiple of 4)
 
 // Per-CTA state of the encoder in shared memory: the row's alphabet, both
@@ -340,7 +342,7 @@ __device__ __forceinline__ void encode_row(const float* __restrict__ X, const do
 
 // One CTA per (row, chunk of kEncChunk entries); rows coded with two codes
 // (0 < theta < 1) and rows coded with one take separate specialisations.
-__global__ void __launch_bounds__(kEncThreads, 5)
+__global__ void __launch_bounds__(kEncThreads, kEncCtasPerSm)
 k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d, int p, int s,
          const int32_t* __restrict__ Q1, const int32_t* __restrict__ Q1_len, const int32_t* __restrict__ Q2,
          const int32_t* __restrict__ Q2_len, const double* __restrict__ theta, const Philox4x32::RoundKeys K,
@@ -359,7 +361,7 @@ k_encode(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d
 
 // k_encode with chunks of `chunk` entries (a multiple of 4, below kEncChunk),
 // for grids of few or short rows that kEncChunk would leave part-empty.
-__global__ void __launch_bounds__(kEncThreads, 5)
+__global__ void __launch_bounds__(kEncThreads, kEncCtasPerSm)
 k_encode_chunked(const float* __restrict__ X, const double* __restrict__ Pall, int64_t d, int p, int s,
                  const int32_t* __restrict__ Q1, const int32_t* __restrict__ Q1_len,
                  const int32_t* __restrict__ Q2, const int32_t* __restrict__ Q2_len,
@@ -662,15 +664,19 @@ cudaError_t launch_encode(const float* X, const double* P, int n, int64_t d, int
   const size_t sm2 = sizeof(double) * 2 * s + sizeof(unsigned int) * kEncWarps * 2 * s;
   const Philox4x32::RoundKeys K =
       Philox4x32::round_keys(static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
-  int dev = 0, sms = 0, per_sm = 0;
+  // resident CTAs: the SM count (read once per device) x the 5 CTAs per SM
+  // that k_encode's launch bounds ask for
+  static std::once_flag once[64];
+  static int sm_count[64];
+  int dev = 0;
   e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
-  e = (p > kMaxP) ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_encode_code, kEncThreads, sm2)
-                  : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_encode, kEncThreads, smem);
-  if (e != cudaSuccess) return e;
-  const int64_t chunk = encode_chunk(n, d, static_cast<int64_t>(sms) * (per_sm > 0 ? per_sm : 1));
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::call_once(once[dev], [dev]() {
+    if (cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sm_count[dev] = 0;
+  });
+  const int64_t resident = static_cast<int64_t>(sm_count[dev] > 0 ? sm_count[dev] : 1) * kEncCtasPerSm;
+  const int64_t chunk = encode_chunk(n, d, resident);
   const int nc = static_cast<int>((d + chunk - 1) / chunk);
   if (p > kMaxP) {
     k_encode_code<<<dim3(nc, n), kEncThreads, sm2, st>>>(X, P, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, idx,
