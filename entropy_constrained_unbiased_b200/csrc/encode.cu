@@ -27,7 +27,8 @@ constexpr int kEncWarps = kEncThreads / kWarp;
 constexpr int64_t kEncChunk = 65536;    // entries per encoder CTA on grids that fill the GPU
 constexpr int64_t kEncMinChunk = 4096;  // fewest entries per encoder CTA
 constexpr int kEncCtasPerSm = 5;         // resident encoder CTAs per SM (48 registers a thread)
-constexpr int64_t kDeqChunk = 32768;  // entries per reconstruction CTA (multiple of 4)
+constexpr int64_t kDeqChunk = 32768;  // entries per reconstruction CTA on grids that fill the GPU
+constexpr int kDeqCtasPerSm = 8;      // resident reconstruction CTAs per SM
 
 // Per-CTA state of the encoder in shared memory: the row's alphabet, both
 // codes, and the per-bucket records of the fast path.
@@ -511,18 +512,19 @@ __global__ void k_entropy(const int64_t* __restrict__ hist, int n, int s, double
   if (lane_id() == 0) H[r] = tot > 0.0 ? acc / tot : 0.0;
 }
 
-// Entries per encoder CTA: kEncChunk, unless the n * ceil(d / kEncChunk) CTAs
-// would leave resident slots empty (few or short rows); then ceil(resident / n)
-// chunks per row, each a multiple of 4 (a Philox block serves four entries, and
-// chunk starts stay 16-byte aligned on aligned rows) and at least
-// kEncMinChunk. Smaller chunks on full grids only add per-CTA setups.
-int64_t encode_chunk(int n, int64_t d, int64_t resident) {
-  const int64_t d4 = (d + 3) & ~int64_t(3);
-  if (d4 == 0) return kEncChunk;
-  if (static_cast<int64_t>(n) * ((d4 + kEncChunk - 1) / kEncChunk) >= resident) return kEncChunk;
-  const int64_t k = (resident + n - 1) / n;
-  const int64_t chunk = (((d4 + k - 1) / k) + 3) & ~int64_t(3);
-  return chunk < kEncMinChunk ? kEncMinChunk : (chunk > kEncChunk ? kEncChunk : chunk);
+// SM count of the current device, read once per device.
+cudaError_t device_sms(int* sms) {
+  static std::once_flag once[64];
+  static int count[64];
+  int dev = 0;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::call_once(once[dev], [dev]() {
+    if (cudaDeviceGetAttribute(&count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) count[dev] = 0;
+  });
+  *sms = count[dev] > 0 ? count[dev] : 1;
+  return cudaSuccess;
 }
 
 size_t encode_smem(int p, int s) {
@@ -540,6 +542,7 @@ size_t encode_smem(int p, int s) {
 // thread handles 16 entries at a time on 16-byte aligned rows, else four (one
 // Philox block of the part stream per four entries when the row mixes codes).
 namespace {
+template <bool kFixed>
 __global__ void __launch_bounds__(kEncThreads) k_dequantize(const uint8_t* __restrict__ idx,
                                                            const double* __restrict__ Pall, int64_t d, int p, int s,
                                                            const int32_t* __restrict__ Q1,
@@ -548,7 +551,8 @@ __global__ void __launch_bounds__(kEncThreads) k_dequantize(const uint8_t* __res
                                                            const int32_t* __restrict__ Q2_len,
                                                            const double* __restrict__ theta,
                                                            const Philox4x32::RoundKeys K, float* __restrict__ out,
-                                                           int32_t* __restrict__ status) {
+                                                           int32_t* __restrict__ status, int64_t chunk_arg) {
+  const int64_t chunk = kFixed ? kDeqChunk : chunk_arg;  // entries of this CTA's chunk
   __shared__ float qv[2][256];
   __shared__ int s_m[2];
   __shared__ int s_bad;
@@ -582,8 +586,8 @@ __global__ void __launch_bounds__(kEncThreads) k_dequantize(const uint8_t* __res
   const int m0 = s_m[0], m1 = s_m[1];
   // u < theta with u = word * 2^-32 is word <= ceil(theta * 2^32) - 1
   const uint32_t th_last = mix ? static_cast<uint32_t>(static_cast<uint64_t>(ceil(th * 0x1p32)) - 1u) : 0u;
-  const int64_t beg = static_cast<int64_t>(blockIdx.x) * kDeqChunk;
-  const int len = static_cast<int>((beg + kDeqChunk < d ? beg + kDeqChunk : d) - beg);
+  const int64_t beg = static_cast<int64_t>(blockIdx.x) * chunk;
+  const int len = static_cast<int>((beg + chunk < d ? beg + chunk : d) - beg);
   const uint8_t* ix = idx + static_cast<int64_t>(r) * d + beg;
   float* o = out + static_cast<int64_t>(r) * d + beg;
   const uint32_t blk0 = static_cast<uint32_t>(static_cast<uint64_t>(beg) >> 2);
@@ -644,10 +648,20 @@ cudaError_t launch_dequantize(const uint8_t* idx, const double* P, int n, int64_
                               const double* theta, uint64_t seed, float* Xhat, int32_t* status, cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t) * n, st);
   if (e != cudaSuccess) return e;
-  const int nc = static_cast<int>((d + kDeqChunk - 1) / kDeqChunk);
+  // resident CTAs: the SM count x 8 (256 threads of 32 registers)
+  int sms = 1;
+  e = device_sms(&sms);
+  if (e != cudaSuccess) return e;
+  const int64_t chunk = fill_chunk(n, d, static_cast<int64_t>(sms) * kDeqCtasPerSm, kDeqChunk, 16, kEncMinChunk);
+  const int nc = static_cast<int>((d + chunk - 1) / chunk);
   const Philox4x32::RoundKeys K =
       Philox4x32::round_keys(static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
-  k_dequantize<<<dim3(nc, n), kEncThreads, 0, st>>>(idx, P, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, Xhat, status);
+  if (chunk == kDeqChunk)
+    k_dequantize<true><<<dim3(nc, n), kEncThreads, 0, st>>>(idx, P, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, Xhat,
+                                                             status, chunk);
+  else
+    k_dequantize<false><<<dim3(nc, n), kEncThreads, 0, st>>>(idx, P, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K,
+                                                              Xhat, status, chunk);
   note_launch();
   return cudaGetLastError();
 }
@@ -664,19 +678,12 @@ cudaError_t launch_encode(const float* X, const double* P, int n, int64_t d, int
   const size_t sm2 = sizeof(double) * 2 * s + sizeof(unsigned int) * kEncWarps * 2 * s;
   const Philox4x32::RoundKeys K =
       Philox4x32::round_keys(static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
-  // resident CTAs: the SM count (read once per device) x the 5 CTAs per SM
-  // that k_encode's launch bounds ask for
-  static std::once_flag once[64];
-  static int sm_count[64];
-  int dev = 0;
-  e = cudaGetDevice(&dev);
+  // resident CTAs: the SM count x the 5 CTAs per SM that k_encode's launch
+  // bounds ask for
+  int sms = 1;
+  e = device_sms(&sms);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  std::call_once(once[dev], [dev]() {
-    if (cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sm_count[dev] = 0;
-  });
-  const int64_t resident = static_cast<int64_t>(sm_count[dev] > 0 ? sm_count[dev] : 1) * kEncCtasPerSm;
-  const int64_t chunk = encode_chunk(n, d, resident);
+  const int64_t chunk = fill_chunk(n, d, static_cast<int64_t>(sms) * kEncCtasPerSm, kEncChunk, 4, kEncMinChunk);
   const int nc = static_cast<int>((d + chunk - 1) / chunk);
   if (p > kMaxP) {
     k_encode_code<<<dim3(nc, n), kEncThreads, sm2, st>>>(X, P, d, p, s, Q1, Q1_len, Q2, Q2_len, theta, K, idx,

@@ -193,6 +193,7 @@ constexpr int kBucketThreads = 256;
 constexpr int kBucketSub = 8192;          // entries between two folds of the shared counters
 constexpr int kBucketSubsPerCta = 8;      // 65536 entries per CTA
 constexpr int kBucketOwn = 2;             // buckets owned per thread (p - 1 <= 511)
+constexpr int kBucketCtasPerSm = 3;       // resident k_bucket CTAs per SM
 constexpr int kHotW = 48;                 // buckets with one counter per lane
 constexpr int kLimbBlock = kHotW * kWarp + kMaxP;  // words per limb: [kHotW][32] lane counters, then [kMaxP]
 constexpr int kLimbBits = 18;
@@ -254,6 +255,9 @@ __device__ __forceinline__ void bucket_add(uint32_t cnt_base, uint32_t limb_base
 // + eta_k, 0, 1); other rows: v = min((x - P_k)/D_k, 1). Kept out of line: on
 // uniform rows it runs only for groups holding an entry within 2^-20 bucket
 // widths of a grid point.
+// One instance per kernel (kTag): a callee shared by two kernels gets a calling
+// convention fitted to neither.
+template <int kTag>
 __device__ __noinline__ void bucket_exact(BucketRow* S, const float* xv, int cnt) {
   const int lane = lane_id();
   for (int e = 0; e < cnt; ++e) {
@@ -306,9 +310,12 @@ __device__ __noinline__ void bucket_exact(BucketRow* S, const float* xv, int cnt
 // owner thread every 8192 entries (8192 limbs of at most 2^18 stay below 2^32);
 // a lane counter receives at most 2048 entries per CTA and is summed once at
 // the end. Each CTA adds its totals to the row's 64-bit sums in global memory.
-__global__ void __launch_bounds__(kBucketThreads, 3)
+// kFixed: chunks of kBucketSub * kBucketSubsPerCta entries; else `chunk_arg`
+// entries (a multiple of 4, smaller), for grids of few or short rows.
+template <bool kFixed>
+__global__ void __launch_bounds__(kBucketThreads, kBucketCtasPerSm)
 k_bucket(const float* __restrict__ X, int64_t d, const double* __restrict__ Pall, int p, int fb,
-         unsigned long long* __restrict__ acc, int32_t* __restrict__ flag) {
+         unsigned long long* __restrict__ acc, int32_t* __restrict__ flag, int64_t chunk_arg) {
   __shared__ unsigned int sc[kMaxP];                 // counts (every bucket)
   __shared__ unsigned int sl[4 * kLimbBlock];       // limbs: [4][kLimbBlock]
   __shared__ unsigned int spre[kMaxP + 1];           // sample counts, then their prefix sums
@@ -362,7 +369,7 @@ k_bucket(const float* __restrict__ X, int64_t d, const double* __restrict__ Pall
   const bool fastg = uni && fabs(c0) <= kFmaOffsetMax;
 
   const float* x = X + static_cast<int64_t>(r) * d;
-  const int64_t chunk = static_cast<int64_t>(kBucketSub) * kBucketSubsPerCta;
+  const int64_t chunk = kFixed ? static_cast<int64_t>(kBucketSub) * kBucketSubsPerCta : chunk_arg;
   const int64_t beg = static_cast<int64_t>(blockIdx.x) * chunk;
   const int len = static_cast<int>((beg + chunk < d ? beg + chunk : d) - beg);
   const float* xc = x + beg;
@@ -490,7 +497,7 @@ k_bucket(const float* __restrict__ X, int64_t d, const double* __restrict__ Pall
 #pragma unroll
           for (int e = 0; e < 4; ++e) bucket_add(sc_base, sl_base, k[e], v[e], hot0, lane, twoF, twoH);
         } else {
-          bucket_exact(&S, xv, 4);
+          bucket_exact<kFixed ? 0 : 1>(&S, xv, 4);
         }
       }
     }
@@ -502,7 +509,7 @@ k_bucket(const float* __restrict__ X, int64_t d, const double* __restrict__ Pall
     if (threadIdx.x < h || (threadIdx.x >= 4 && threadIdx.x - 4 + tail0 < len)) {
       const int i = threadIdx.x < h ? threadIdx.x : tail0 + threadIdx.x - 4;
       const float xv[1] = {__ldcs(xc + i)};
-      bucket_exact(&S, xv, 1);
+      bucket_exact<kFixed ? 0 : 1>(&S, xv, 1);
     }
   }
   fold();
@@ -1197,10 +1204,14 @@ cudaError_t launch_bucket(const float* X, const double* P, int n, int64_t d, int
     if (e != cudaSuccess) return e;
     k_bucket_wide<<<sms, kWideThreads, kWideSmem, st>>>(X, n, d, P, p, fb, acc, flag);
   } else {
-    const int64_t chunk = static_cast<int64_t>(kBucketSub) * kBucketSubsPerCta;
+    const int64_t full = static_cast<int64_t>(kBucketSub) * kBucketSubsPerCta;
+    const int64_t chunk = fill_chunk(n, d, static_cast<int64_t>(sms) * kBucketCtasPerSm, full, 4, 4096);
     const int nc = static_cast<int>((d + chunk - 1) / chunk);
     // 37 KB of static and at most 10 KB of dynamic shared memory (p = 512): no attribute needed
-    k_bucket<<<dim3(nc, n), kBucketThreads, bucket_smem_bytes(p), st>>>(X, d, P, p, fb, acc, flag);
+    if (chunk == full)
+      k_bucket<true><<<dim3(nc, n), kBucketThreads, bucket_smem_bytes(p), st>>>(X, d, P, p, fb, acc, flag, chunk);
+    else
+      k_bucket<false><<<dim3(nc, n), kBucketThreads, bucket_smem_bytes(p), st>>>(X, d, P, p, fb, acc, flag, chunk);
   }
   note_launch();
   k_bucket_finish<<<n, 256, 0, st>>>(acc, P, p, fb, flag, cnt, A, B, status);

@@ -161,6 +161,19 @@ cudaError_t launch_rans_decode(const uint16_t* words, const int32_t* seg_len, co
                                int two_codes, int n, int64_t d, int s, uint64_t seed, uint8_t* idx, int32_t* status,
                                cudaStream_t st);
 
+// Entries per CTA for kernels that take rows in chunks: `full`, unless the
+// n * ceil(d / full) CTAs would leave some of the `resident` CTA slots empty
+// (few or short rows); then ceil(resident / n) chunks per row, each a multiple
+// of `align` (a power of two) and at least `min_chunk`. Smaller chunks on
+// grids that already fill the GPU only add per-CTA setups.
+inline int64_t fill_chunk(int n, int64_t d, int64_t resident, int64_t full, int64_t align, int64_t min_chunk) {
+  if (d <= 0) return full;
+  if (static_cast<int64_t>(n) * ((d + full - 1) / full) >= resident) return full;
+  const int64_t k = (resident + n - 1) / n;
+  const int64_t chunk = (((d + k - 1) / k) + align - 1) & ~(align - 1);
+  return chunk < min_chunk ? min_chunk : (chunk > full ? full : chunk);
+}
+
 // ---- encoder (encode.cu) ----
 cudaError_t launch_encode(const float* X, const double* P, int n, int64_t d, int p, int s,
                           const int32_t* Q1, const int32_t* Q1_len, const int32_t* Q2,
