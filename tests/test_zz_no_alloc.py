@@ -64,3 +64,30 @@ def test_noalloc_rejects_sizes_beyond_the_fixed_scratch(E):
                                 C.c_void_p(out.data_ptr()), C.c_void_p(out.data_ptr()), C.c_void_p(out.data_ptr()),
                                 C.c_void_p(st.data_ptr()), C.c_void_p(0))
     assert rc == E.ERR_WORKSPACE
+
+
+def test_noalloc_capacity_boundary_at_p128(E):
+    """The fixed 8 MiB scratch must hold round256(24 n (p - 1)) + round256(4 n)
+    bytes: at p = 128, n = 2748 rows need 8,387,072 bytes and fit, n = 2749
+    need 8,390,144 and are refused without a launch."""
+    def need(n, p):
+        r = lambda b: (b + 255) // 256 * 256
+        return r(24 * n * (p - 1)) + r(4 * n)
+    assert need(2748, 128) <= 8 << 20 < need(2749, 128)
+    X = W.random_case(73, 2748, 64, "normal")
+    Xd = torch.from_numpy(X).cuda()
+    P = _grid(X, 128)
+    c1, A1, B1, s1 = E.bucket_noalloc(Xd, P)
+    c0, A0, B0, s0 = E.bucket(Xd, P)
+    torch.cuda.synchronize()
+    assert int(s1.abs().sum()) == 0 and torch.equal(c1, c0)
+    np.testing.assert_allclose(A1.cpu().numpy(), A0.cpu().numpy(), rtol=1e-9, atol=0)
+    L = E.load()
+    X2 = torch.zeros((2749, 64), dtype=torch.float32, device="cuda")
+    P2 = torch.zeros((2749, 128), dtype=torch.float64, device="cuda")
+    out = torch.zeros(8, dtype=torch.float64, device="cuda")
+    st = torch.zeros(2749, dtype=torch.int32, device="cuda")
+    rc = L.ecasq_bucket_noalloc(C.c_void_p(X2.data_ptr()), C.c_void_p(P2.data_ptr()), 2749, 64, 128,
+                                C.c_void_p(out.data_ptr()), C.c_void_p(out.data_ptr()), C.c_void_p(out.data_ptr()),
+                                C.c_void_p(st.data_ptr()), C.c_void_p(0))
+    assert rc == E.ERR_WORKSPACE
