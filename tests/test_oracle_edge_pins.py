@@ -483,3 +483,40 @@ def test_refinement_classes_run_in_position_order():
         if found == 3:
             break
     assert found == 3
+
+
+# -- accuracy of the oracle's sums and the BF16 alphabet's statuses ---------------------
+
+def test_bucket_sums_are_compensated():
+    """A_k and B_k are sums of the fp64 terms y = x - P_k and y^2 over about
+    66,000 entries per bucket. Compensated summation keeps them within
+    3 eps sum|y| of the correctly rounded sum (math.fsum of the same terms);
+    plain summation drifts by about sqrt(n) eps, far beyond that bound."""
+    import math
+    rng = np.random.default_rng(90)
+    x = rng.standard_normal(200000).astype(np.float32)
+    P, st = O.uniform_grid(x, 4)
+    assert st == 0
+    cnt, A, B, st = O.bucket(x, P)
+    assert st == 0
+    xd = x.astype(np.float64)
+    k = np.clip(np.searchsorted(P[:-1], xd, side="right") - 1, 0, P.size - 2)
+    eps = np.finfo(np.float64).eps
+    for b in range(P.size - 1):
+        y = xd[k == b] - P[b]
+        assert cnt[b] == y.size
+        for got, terms in ((A[b], y), (B[b], y * y)):
+            exact = math.fsum(terms.tolist())
+            bound = 3 * eps * float(np.abs(terms).sum())
+            assert abs(got - exact) <= bound, (b, got, exact, bound)
+
+
+def test_bf16_alphabet_status_values():
+    """A non-finite entry, and an entry above the largest finite BF16 value
+    (so that no BF16 value >= max X exists), give ECASQ_ERR_RANGE."""
+    P = np.zeros(16)
+    for bad in (np.float32("nan"), np.float32(np.finfo(np.float32).max)):
+        x = np.array([0.5, bad, -1.0], np.float32)
+        assert O.lib().eo_bf16_alphabet(x, x.size, P, P.size) == ERR_RANGE
+    x = np.array([0.5, -1.0], np.float32)
+    assert O.lib().eo_bf16_alphabet(x, x.size, P, P.size) > 0
