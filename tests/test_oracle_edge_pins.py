@@ -520,3 +520,33 @@ def test_bf16_alphabet_status_values():
         assert O.lib().eo_bf16_alphabet(x, x.size, P, P.size) == ERR_RANGE
     x = np.array([0.5, -1.0], np.float32)
     assert O.lib().eo_bf16_alphabet(x, x.size, P, P.size) > 0
+
+
+def test_budget_bisection_runs_the_given_number_of_steps():
+    """The lambda bracket starts as [0, (P_{p-1} - P_0)^2] and halves once per
+    step, so after `steps` steps lambda_hi - lambda_lo is that width x
+    2^-steps (up to the rounding of the midpoints, about 2^-23 relative), for
+    the exact and the approximate budget drivers, wherever the budget binds."""
+    X, P = _distinct_rows(95, 3, 700, 24)
+    for steps in (12, 30):
+        for out in (O.solve_budget_batch(X, P, 6, 1.6, steps),
+                    O.solve_approx_budget_batch(X, P, 6, 1.6, steps, refine=0)):
+            for r in range(3):
+                assert out["status"][r] == 0 and 0.0 < out["theta"][r] < 1.0
+                width = (P[r, -1] - P[r, 0]) ** 2 * 2.0 ** -steps
+                assert out["lam_hi"][r] - out["lam_lo"][r] == pytest.approx(width, rel=1e-5)
+
+
+def test_rans_truncated_stream_is_an_argument_error():
+    """A segment length that drops renormalisation words leaves the decoder
+    short of words: ECASQ_ERR_ARG."""
+    d = 16384
+    idx = np.zeros((1, d), np.uint8)
+    hist = np.zeros((1, 2, 2), np.int64)
+    hist[0, 0] = [1, 1]
+    words, seg_len, st = O.rans_encode(idx, hist, 1)
+    assert st[0] == 0 and seg_len[0, 0] == 32 * 32 + 64
+    bad = seg_len.copy()
+    bad[0, 0] = 64 + 100
+    _, st2 = O.rans_decode(words, bad, d, hist, 1)
+    assert st2[0] == ERR_ARG
